@@ -1,0 +1,253 @@
+/*
+ * libomq — OmniQuant fake-quantized linear calibration step on NVIDIA B200 (sm_100a).
+ *
+ * Sources (web pages, cited by title and section):
+ *   [ICLR] "【ICLR 2024】OmniQuant: Omnidirectionally Calibrated Quantization for Large
+ *          Language Models" (onecrewdev.com paper reading), sections 框架 (block-wise
+ *          objective), LWC (W_q, h, z), LET (Y = [(X-δ)⊘s][s⊙W] + [B+δW]), 实验证据
+ *          (AdamW, learning rates, per-channel / g128 weights, per-token activations).
+ *   [AFF]  "LLM quantization tutorial" (devpress.csdn.net), section 2.2: affine
+ *          (scale, zero-point) quantization.
+ *   [EDGE] "OmniQuant：端侧大模型低比特量化的新思路与实战" (bjdmk.com.cn), section 2.2:
+ *          the straight-through estimator.
+ *
+ * Notation. A linear layer Y = X W^T + B in PyTorch layout: W is [N, K] (N output rows,
+ * K input channels), X is [M, K] (M tokens), Y is [M, N]. This is the paper's X W with
+ * W_paper = W^T. s and δ have one entry per input channel (column of W, channel of X).
+ * LWC groups are contiguous runs of `group` elements along K inside one row of W
+ * (group == K is "per output channel"). Q = 2^bits - 1.
+ *
+ * Conventions for every entry point:
+ *   - Memory. Every tensor pointer is a caller-owned DEVICE buffer, row-major and dense,
+ *     16-byte aligned. Scalars are passed by value. The library allocates no device memory:
+ *     scratch comes from a caller-provided workspace whose size omq_*_workspace_bytes
+ *     reports.
+ *   - Asynchrony. Work is enqueued on `stream` (0 = legacy default stream); calls return
+ *     after validation and launch, before the GPU finishes.
+ *   - Errors. Arguments are validated on the host before anything is launched; a rejected
+ *     call returns a non-zero omq_status and enqueues nothing. A launch failure returns
+ *     OMQ_ERR_CUDA (the CUDA code is kept in omq_last_cuda_error()). No call aborts, throws
+ *     or traps. Kernels that wait on barriers give up after a bounded time and raise a
+ *     device error flag that omq_sync_check() reports as OMQ_ERR_TIMEOUT.
+ *   - Dtypes. W and X (and their fake-quant copies, and dY) are OMQ_BF16 or OMQ_F32;
+ *     all learnable parameters, scales, gradients and losses are float32.
+ *   - Rounding. round() is round-half-to-even. h, z and codes follow one fixed binary32
+ *     operation order (no fused multiply-add, IEEE division):
+ *        W~ = W*s;  h = max(((g*M) - (b*m)) / Q, 1e-8);  z = -round((b*m)/h)
+ *        code = clamp(round(W~/h) + z, 0, Q);  W^ = (code - z)*h
+ *     with g = sigmoid(γ), b = sigmoid(β) evaluated in binary64 and rounded once.
+ */
+#ifndef OMQ_H_
+#define OMQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* omq_stream_t;   /* a cudaStream_t */
+
+typedef enum {
+  OMQ_OK = 0,
+  OMQ_ERR_NULL = 1,         /* a required pointer is NULL */
+  OMQ_ERR_SHAPE = 2,        /* a size is non-positive, too large, or not divisible as required */
+  OMQ_ERR_DTYPE = 3,        /* unsupported dtype or dtype combination */
+  OMQ_ERR_ALIGN = 4,        /* a pointer is not 16-byte aligned */
+  OMQ_ERR_BITS = 5,         /* bits / abits out of range */
+  OMQ_ERR_WORKSPACE = 6,    /* workspace NULL or smaller than required */
+  OMQ_ERR_CUDA = 7,         /* a CUDA call failed; see omq_last_cuda_error() */
+  OMQ_ERR_UNSUPPORTED = 8,  /* valid request this build does not implement */
+  OMQ_ERR_TIMEOUT = 9       /* a kernel's bounded barrier wait expired (device flag) */
+} omq_status;
+
+typedef enum { OMQ_F32 = 0, OMQ_BF16 = 1 } omq_dtype;
+
+/* Per-group (or per-token) range record written by the quantizers and read by the
+ * backward: the group's max and min of the quantized values, and how many elements
+ * attain each (ties share the range's gradient equally). */
+typedef struct {
+  float vmax;
+  float vmin;
+  int32_t nmax;
+  int32_t nmin;
+} omq_range;
+
+/* Static description of a status code. Never NULL. */
+const char* omq_status_str(int status);
+/* CUDA error code (cudaError_t value) of the last OMQ_ERR_CUDA on this host thread. */
+int omq_last_cuda_error(void);
+/* Library version, major*10000 + minor*100 + patch. */
+int omq_version(void);
+/* Synchronize `stream`, then report and clear the device error flag raised by a kernel
+ * whose bounded wait expired: OMQ_ERR_TIMEOUT if it was set, OMQ_ERR_CUDA if the
+ * synchronization failed, OMQ_OK otherwise. */
+omq_status omq_sync_check(omq_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
+ * omq_lwc_quant — weight side of the step: LET weight scaling, then Learnable Weight
+ * Clipping fake-quantization ([ICLR] sections LET and LWC).
+ *
+ *   W~[n,k] = W[n,k] * s[k]                                   (s == NULL: s = 1)
+ *   per group (n, j):  M = max W~, m = min W~ over the group's `group` elements,
+ *                      g = sigmoid(gamma_logit[n,j]), b = sigmoid(beta_logit[n,j]),
+ *                      h = (g*M - b*m)/Q, z = -round(b*m/h)
+ *   code[n,k] = clamp(round(W~/h) + z, 0, Q);   W_hat[n,k] = (code - z)*h
+ *
+ * W [N,K] in `wdt`; gamma_logit, beta_logit [N, K/group] float32; s [K] float32 or NULL.
+ * Outputs: W_hat [N,K] in `hat_dt` (bf16 holds the binary32 value rounded to nearest
+ * even); h [N, K/group] float32; z [N, K/group] int32; codes [N,K] uint8 or NULL;
+ * grp_range [N, K/group] or NULL (needed by omq_fq_linear_bwd).
+ * Requires K % group == 0, group % 8 == 0, bits in {2,3,4,8}.
+ * ------------------------------------------------------------------------------------ */
+omq_status omq_lwc_quant(const void* W, omq_dtype wdt, int64_t N, int64_t K, int64_t group,
+                         int bits, const float* gamma_logit, const float* beta_logit,
+                         const float* s, void* W_hat, omq_dtype hat_dt, float* h, int32_t* z,
+                         uint8_t* codes, omq_range* grp_range, omq_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
+ * omq_let_apply — activation side of the step ([ICLR] section LET; per-token activation
+ * quantization, section 实验证据).
+ *
+ *   X~[m,k] = (X[m,k] - delta[k]) / s[k]          (s == NULL: 1; delta == NULL: 0)
+ *   abits < 16: per token m, MinMax affine fake-quant of row X~[m,:] with
+ *               h_a = (max - min)/(2^abits - 1), z_a = -round(min/h_a),
+ *               Xq = (clamp(round(X~/h_a) + z_a, 0, 2^abits-1) - z_a) * h_a
+ *   abits == 16: Xq = X~ (h_a, z_a, tok_range are not written and may be NULL)
+ *   B_tilde[n] = B[n] + sum_k W[n,k] delta[k]      (computed when B_tilde != NULL;
+ *                                                   B == NULL means 0; uses the original W)
+ *
+ * X [M,K] in `xdt`; Xq [M,K] in `xq_dt`; h_a [M] float32, z_a [M] int32, tok_range [M].
+ * W [N,K] in `wdt` is read only for B_tilde. abits in {2,3,4,6,8,16}.
+ * ------------------------------------------------------------------------------------ */
+omq_status omq_let_apply(const void* X, omq_dtype xdt, int64_t M, int64_t K, const float* s,
+                         const float* delta, int abits, void* Xq, omq_dtype xq_dt, float* h_a,
+                         int32_t* z_a, omq_range* tok_range, const void* W, omq_dtype wdt,
+                         int64_t N, const float* B, float* B_tilde, omq_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
+ * omq_fq_linear_fwd — fake-quantized linear forward and reconstruction loss
+ * ([ICLR] section LET: Y = Q_a(X~) Q_w(W~) + B~; section 框架: the reconstruction
+ * objective, taken as the mean squared error).
+ *
+ *   Y[m,n] = sum_k Xq[m,k] W_hat[n,k] + B_tilde[n]      (B_tilde == NULL: 0)
+ *   if Y_ref != NULL:  loss = mean over M*N of (Y - Y_ref)^2     (device float32 scalar)
+ *                      dY[m,n] = 2 (Y - Y_ref) / (M N)           (stored in `dt`)
+ *
+ * Xq [M,K], W_hat [N,K] in `dt`; Y_ref, Y [M,N] float32. Y may be NULL (not stored);
+ * with Y_ref == NULL, `loss` and `dY` must be NULL and Y must not be.
+ * bf16 operands run on the tcgen05 tensor cores with float32 accumulation; float32
+ * operands on CUDA cores in float32. K % 8 == 0 and N % 8 == 0.
+ * Workspace: omq_fwd_workspace_bytes(M, N, K).
+ * ------------------------------------------------------------------------------------ */
+omq_status omq_fq_linear_fwd(const void* Xq, const void* W_hat, omq_dtype dt, int64_t M,
+                             int64_t N, int64_t K, const float* B_tilde, const float* Y_ref,
+                             float* Y, void* dY, float* loss, void* workspace, size_t ws_bytes,
+                             omq_stream_t stream);
+size_t omq_fwd_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/* ------------------------------------------------------------------------------------
+ * omq_fq_linear_bwd — straight-through backward of the step ([EDGE] section 2.2; the
+ * formulas of [ICLR] sections LWC and LET differentiated as written).
+ *
+ *   dW_hat = dY^T Xq,  dXq = dY W_hat,  dB~ = sum_m dY[m,:]
+ *   Per LWC group, u = W~/h, c = code:
+ *     in range (0 <= round(u)+z <= Q): dW_hat/dW~ = 1, dW_hat/dh = round(u) - u, dW_hat/dz = 0
+ *     clipped:                          dW_hat/dW~ = 0, dW_hat/dh = c - z,        dW_hat/dz = -h
+ *   and the chain through h = (g M - b m)/Q and z = -round(b m / h) into g, b and the
+ *   group's max / min elements (ties split equally). Same rule per token for Q_a (g=b=1).
+ *   d_gamma_logit = dL/dg * g(1-g), d_beta_logit = dL/db * b(1-b)
+ *   d_s[k]     = sum_n dW~[n,k] W[n,k] - sum_m dX~[m,k] X~[m,k] / s[k]
+ *   d_delta[k] = -sum_m dX~[m,k] / s[k] + sum_n dB~[n] W[n,k]
+ *
+ * Outputs that are NULL are skipped; d_s and d_delta need s, delta and X (LET learnable).
+ * All reductions run in a fixed order: results are bitwise reproducible run to run.
+ * Workspace: omq_bwd_workspace_bytes(M, N, K, group).
+ * ------------------------------------------------------------------------------------ */
+typedef struct {
+  int64_t M, N, K, group;
+  int bits, abits;
+  omq_dtype dt;                   /* dtype of X, W, Xq, W_hat and dY */
+  const void* X;                  /* [M,K]   needed for d_s / d_delta */
+  const void* W;                  /* [N,K] */
+  const float* s;                 /* [K] or NULL (LET off) */
+  const float* delta;             /* [K] or NULL */
+  const float* gamma_logit;       /* [N, K/group] */
+  const float* beta_logit;        /* [N, K/group] */
+  const void* Xq;                 /* [M,K] forward GEMM operand */
+  const void* W_hat;              /* [N,K] forward GEMM operand */
+  const float* h;                 /* [N, K/group] from omq_lwc_quant */
+  const int32_t* z;               /* [N, K/group] */
+  const omq_range* grp_range;     /* [N, K/group] */
+  const float* h_a;               /* [M] from omq_let_apply (abits < 16) */
+  const int32_t* z_a;             /* [M] */
+  const omq_range* tok_range;     /* [M] */
+  const void* dY;                 /* [M,N] from omq_fq_linear_fwd */
+  float* d_gamma_logit;           /* [N, K/group] or NULL */
+  float* d_beta_logit;            /* [N, K/group] or NULL */
+  float* d_s;                     /* [K] or NULL */
+  float* d_delta;                 /* [K] or NULL */
+  float* d_B_tilde;               /* [N] or NULL */
+} omq_bwd_args;
+
+omq_status omq_fq_linear_bwd(const omq_bwd_args* args, void* workspace, size_t ws_bytes,
+                             omq_stream_t stream);
+size_t omq_bwd_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t group);
+
+/* ------------------------------------------------------------------------------------
+ * omq_adamw_step — one AdamW update ([ICLR] section 实验证据: AdamW, zero weight decay,
+ * lr 5e-3 for the LWC logits and 1e-2 for s, δ), elementwise over n float32 values:
+ *   p *= 1 - lr*wd;  m = b1 m + (1-b1) g;  v = b2 v + (1-b2) g^2
+ *   p -= lr/(1-b1^step) * m / (sqrt(v)/sqrt(1-b2^step) + eps)          (step >= 1)
+ * ------------------------------------------------------------------------------------ */
+omq_status omq_adamw_step(float* param, const float* grad, float* m, float* v, int64_t n,
+                          float lr, float beta1, float beta2, float eps, float weight_decay,
+                          int64_t step, omq_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
+ * omq_fold_pack — fold the learned parameters into deployable integer weights
+ * ([ICLR] section 框架: the learned transforms fold back into the weights).
+ * codes as in omq_lwc_quant, packed row-major: element k of a row goes to byte
+ * k*bits/8 at bit offset (k*bits) mod 8, least-significant bits first.
+ * packed [N, K*bits/8] uint8; h, z [N, K/group]. bits in {2,4,8} (3: OMQ_ERR_UNSUPPORTED).
+ * ------------------------------------------------------------------------------------ */
+omq_status omq_fold_pack(const void* W, omq_dtype wdt, int64_t N, int64_t K, int64_t group,
+                         int bits, const float* gamma_logit, const float* beta_logit,
+                         const float* s, uint8_t* packed, float* h, int32_t* z,
+                         omq_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
+ * omq_calib_step — one whole calibration step on one stream: omq_let_apply (when LET is
+ * on or abits < 16), omq_lwc_quant, omq_fq_linear_fwd, omq_fq_linear_bwd, then AdamW on
+ * the logits (lr_lwc) and, with LET, on s and delta (lr_let). `step` counts from 1.
+ * All buffers are caller-owned device memory; Xq may alias X only when LET is off and
+ * abits == 16 (then X is the GEMM operand as is). Workspace:
+ * omq_step_workspace_bytes(M, N, K, group).
+ * ------------------------------------------------------------------------------------ */
+typedef struct {
+  int64_t M, N, K, group;
+  int bits, abits, let;           /* let != 0: s, delta learnable */
+  omq_dtype dt;
+  const void* X; const void* W; const float* B; const float* Y_ref;
+  float* gamma_logit; float* beta_logit; float* s; float* delta;     /* learnable */
+  float* m_gamma; float* v_gamma; float* m_beta; float* v_beta;      /* AdamW moments */
+  float* m_s; float* v_s; float* m_delta; float* v_delta;
+  void* Xq; void* W_hat; float* B_tilde;                             /* step buffers */
+  float* h; int32_t* z; omq_range* grp_range;
+  float* h_a; int32_t* z_a; omq_range* tok_range;
+  void* dY;
+  float* d_gamma_logit; float* d_beta_logit; float* d_s; float* d_delta;
+  float* loss;                    /* device scalar */
+  float lr_lwc, lr_let;
+  int64_t step;
+} omq_step_args;
+
+omq_status omq_calib_step(const omq_step_args* args, void* workspace, size_t ws_bytes,
+                          omq_stream_t stream);
+size_t omq_step_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t group);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* OMQ_H_ */

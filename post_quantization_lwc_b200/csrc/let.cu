@@ -1,0 +1,167 @@
+// Activation side of the step ("【ICLR 2024】OmniQuant: ...", section LET and the
+// per-token activation quantizer of section 实验证据):
+//   X~ = (X - delta) / s                       (one HBM pass, 16-byte vector accesses)
+//   per token: MinMax affine fake-quant of the row X~[m, :]   (one block per token,
+//     row staged in shared memory, warp-shuffle + shared-memory reductions)
+//   B~ = B + W delta                            (one warp per output row)
+#include <float.h>
+
+#include "omq_internal.cuh"
+
+namespace omq {
+
+__device__ __forceinline__ void let8(const LetParams& p, int64_t off, int64_t col, float (&v)[8]) {
+  load8(p.X, off, p.xdt, v);
+  float sv[8], dv[8];
+  if (p.s) {
+    const float4* q = reinterpret_cast<const float4*>(p.s + col);
+    const float4 a = q[0], b = q[1];
+    sv[0] = a.x; sv[1] = a.y; sv[2] = a.z; sv[3] = a.w; sv[4] = b.x; sv[5] = b.y; sv[6] = b.z; sv[7] = b.w;
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) sv[i] = 1.f;
+  }
+  if (p.d) {
+    const float4* q = reinterpret_cast<const float4*>(p.d + col);
+    const float4 a = q[0], b = q[1];
+    dv[0] = a.x; dv[1] = a.y; dv[2] = a.z; dv[3] = a.w; dv[4] = b.x; dv[5] = b.y; dv[6] = b.z; dv[7] = b.w;
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) dv[i] = 0.f;
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __fdiv_rn(__fsub_rn(v[i], dv[i]), sv[i]);
+}
+
+__global__ void __launch_bounds__(256) let_elem_kernel(LetParams p) {
+  const int64_t chunks = p.M * p.K / 8;
+  for (int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; c < chunks;
+       c += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t off = c * 8;
+    float v[8];
+    let8(p, off, off % p.K, v);
+    store8(p.Xq, off, p.xq_dt, v);
+  }
+}
+
+__global__ void __launch_bounds__(256) act_quant_kernel(LetParams p) {
+  extern __shared__ float row[];   // K floats: X~[m, :]
+  __shared__ float smf[64];
+  __shared__ int smi[64];
+  const int chunks = static_cast<int>(p.K / 8);
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int64_t m = blockIdx.x; m < p.M; m += gridDim.x) {
+    const int64_t base = m * p.K;
+    float vmax = -FLT_MAX, vmin = FLT_MAX;
+    for (int c = threadIdx.x; c < chunks; c += blockDim.x) {
+      float v[8];
+      let8(p, base + c * 8, c * 8, v);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        row[c * 8 + i] = v[i];
+        vmax = fmaxf(vmax, v[i]);
+        vmin = fminf(vmin, v[i]);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+      vmin = fminf(vmin, __shfl_xor_sync(0xffffffffu, vmin, o));
+    }
+    __syncthreads();
+    if (lane == 0) { smf[w] = vmax; smf[32 + w] = vmin; }
+    __syncthreads();
+    vmax = smf[0];
+    vmin = smf[32];
+    for (int i = 1; i < nw; ++i) { vmax = fmaxf(vmax, smf[i]); vmin = fminf(vmin, smf[32 + i]); }
+    int nmax = 0, nmin = 0;
+    for (int c = threadIdx.x; c < chunks; c += blockDim.x)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) { nmax += row[c * 8 + i] == vmax; nmin += row[c * 8 + i] == vmin; }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      nmax += __shfl_xor_sync(0xffffffffu, nmax, o);
+      nmin += __shfl_xor_sync(0xffffffffu, nmin, o);
+    }
+    if (lane == 0) { smi[w] = nmax; smi[32 + w] = nmin; }
+    __syncthreads();
+    nmax = 0;
+    nmin = 0;
+    for (int i = 0; i < nw; ++i) { nmax += smi[i]; nmin += smi[32 + i]; }
+    // gamma = beta = 1: h = (M - m)/Q, z = -round(m/h)
+    const GroupQ q = group_params(1.f, 1.f, vmax, vmin, p.Qa);
+    const float hinv = __frcp_rn(q.h);
+    for (int c = threadIdx.x; c < chunks; c += blockDim.x) {
+      float o[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float lvl = __fadd_rn(round_quotient(row[c * 8 + i], q.h, hinv), q.z);
+        const float cc = fminf(fmaxf(lvl, 0.f), p.Qa);
+        o[i] = __fmul_rn(__fsub_rn(cc, q.z), q.h);
+      }
+      store8(p.Xq, base + c * 8, p.xq_dt, o);
+    }
+    if (threadIdx.x == 0) {
+      if (p.h_a) p.h_a[m] = q.h;
+      if (p.z_a) p.z_a[m] = z_to_i32(q.z);
+      if (p.range) p.range[m] = omq_range{vmax, vmin, nmax, nmin};
+    }
+    __syncthreads();
+  }
+}
+
+// B~[n] = B[n] + sum_k W[n,k] delta[k]  (one warp per row; lanes stride 8-element chunks)
+__global__ void __launch_bounds__(256) let_bias_kernel(const void* W, omq_dtype wdt, int64_t N,
+                                                       int64_t K, const float* delta,
+                                                       const float* B, float* Bt) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp_g = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t n_warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t n = warp_g; n < N; n += n_warps) {
+    float acc = 0.f;
+    if (delta) {
+      for (int64_t c = lane; c < K / 8; c += 32) {
+        float v[8];
+        load8(W, n * K + c * 8, wdt, v);
+        const float4* q = reinterpret_cast<const float4*>(delta + c * 8);
+        const float4 a = q[0], b = q[1];
+        acc += v[0] * a.x + v[1] * a.y + v[2] * a.z + v[3] * a.w + v[4] * b.x + v[5] * b.y +
+               v[6] * b.z + v[7] * b.w;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    }
+    if (lane == 0) Bt[n] = (B ? B[n] : 0.f) + acc;
+  }
+}
+
+omq_status launch_let(const LetParams& p, int abits, cudaStream_t stream) {
+  const int sms = num_sms();
+  if (abits >= 16) {
+    const int64_t chunks = p.M * p.K / 8;
+    const int64_t want = ceil_div(chunks, 256);
+    const unsigned grid = static_cast<unsigned>(want < int64_t(sms) * 16 ? want : int64_t(sms) * 16);
+    let_elem_kernel<<<grid, 256, 0, stream>>>(p);
+    return launch_status();
+  }
+  const size_t smem = static_cast<size_t>(p.K) * sizeof(float);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(act_quant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) { set_cuda_error(e); return OMQ_ERR_CUDA; }
+  }
+  const unsigned grid = static_cast<unsigned>(p.M < int64_t(sms) * 8 ? p.M : int64_t(sms) * 8);
+  act_quant_kernel<<<grid, 256, smem, stream>>>(p);
+  return launch_status();
+}
+
+omq_status launch_let_bias(const void* W, omq_dtype wdt, int64_t N, int64_t K, const float* delta,
+                           const float* B, float* Bt, cudaStream_t stream) {
+  const int sms = num_sms();
+  const int64_t want = ceil_div(N, 8);
+  const unsigned grid = static_cast<unsigned>(want < int64_t(sms) * 16 ? want : int64_t(sms) * 16);
+  let_bias_kernel<<<grid, 256, 0, stream>>>(W, wdt, N, K, delta, B, Bt);
+  return launch_status();
+}
+
+}  // namespace omq

@@ -1,0 +1,411 @@
+// The libomq C ABI: host-side validation, workspace layout and launch sequencing of the
+// fake-quantized linear calibration step. Nothing here allocates device memory.
+#include <cstdio>
+#include <mutex>
+#include <vector>
+
+#include "omq_internal.cuh"
+
+namespace omq {
+
+namespace {
+thread_local int t_last_cuda_error = 0;
+
+constexpr int64_t kMaxGroupLarge = 16384;   // group staged in shared memory (per group / row)
+constexpr int64_t kMaxDim = (int64_t(1) << 31) - 1;
+constexpr int kRowsSmallW = 64;             // rows per block, weight STE, group <= 256
+constexpr int kRowsLargeW = 16;             // rows per block, weight STE, larger groups
+constexpr int kRowsX = 16;                  // tokens per block, activation STE
+constexpr int kRowsColsum = 64;             // rows per block of the dY column sums
+
+size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
+
+bool small_group(int64_t g) { return g <= 256 && (g & (g - 1)) == 0; }
+
+int64_t rows_per_block_w(int64_t group) { return small_group(group) ? kRowsSmallW : kRowsLargeW; }
+
+struct BwdLayout {
+  size_t dbt_part, dbt, dwhat, dxq, part_ws, part_wd, part_xs, part_xd, total;
+  int64_t rb_colsum, rb_w, rb_x;
+};
+
+BwdLayout bwd_layout(int64_t M, int64_t N, int64_t K, int64_t group) {
+  BwdLayout L{};
+  L.rb_colsum = ceil_div(M, kRowsColsum);
+  L.rb_w = ceil_div(N, rows_per_block_w(group));
+  L.rb_x = ceil_div(M, kRowsX);
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off += align256(bytes); return o; };
+  L.dbt_part = take(sizeof(float) * L.rb_colsum * N);
+  L.dbt = take(sizeof(float) * N);
+  L.dwhat = take(sizeof(float) * N * K);
+  L.dxq = take(sizeof(float) * M * K);
+  L.part_ws = take(sizeof(float) * L.rb_w * K);
+  L.part_wd = take(sizeof(float) * L.rb_w * K);
+  L.part_xs = take(sizeof(float) * L.rb_x * K);
+  L.part_xd = take(sizeof(float) * L.rb_x * K);
+  L.total = off;
+  return L;
+}
+
+size_t fwd_bytes(int64_t M, int64_t N) {
+  int64_t t = gemm_bf16_tc_tiles(M, N);
+  int64_t t2 = gemm_f32_simt_tiles(M, N);
+  return align256(sizeof(float) * static_cast<size_t>(t > t2 ? t : t2));
+}
+
+template <class T>
+T* at(void* base, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(base) + off);
+}
+
+bool dtype_ok(omq_dtype d) { return d == OMQ_F32 || d == OMQ_BF16; }
+bool wbits_ok(int b) { return b == 2 || b == 3 || b == 4 || b == 8; }
+bool abits_ok(int b) { return b == 2 || b == 3 || b == 4 || b == 6 || b == 8 || b == 16; }
+bool a16(const void* p) { return p == nullptr || aligned16(p); }
+
+#define OMQ_TRY(expr)                 \
+  do {                                \
+    omq_status _s = (expr);           \
+    if (_s != OMQ_OK) return _s;      \
+  } while (0)
+
+omq_status check_lwc(const void* W, omq_dtype wdt, int64_t N, int64_t K, int64_t group, int bits,
+                     const float* gl, const float* bl, const float* s, omq_dtype hat_dt,
+                     const void* W_hat, const void* codes, const void* h, const void* z) {
+  if (!W || !gl || !bl || !h || !z) return OMQ_ERR_NULL;
+  if (!dtype_ok(wdt) || !dtype_ok(hat_dt)) return OMQ_ERR_DTYPE;
+  if (!wbits_ok(bits)) return OMQ_ERR_BITS;
+  if (N < 1 || K < 8 || group < 8 || N > kMaxDim || K > kMaxDim) return OMQ_ERR_SHAPE;
+  if (group % 8 || K % group) return OMQ_ERR_SHAPE;
+  if (!small_group(group) && group > kMaxGroupLarge) return OMQ_ERR_SHAPE;
+  if (!a16(W) || !a16(W_hat) || !a16(codes) || !a16(s)) return OMQ_ERR_ALIGN;
+  return OMQ_OK;
+}
+
+}  // namespace
+
+void set_cuda_error(cudaError_t e) { t_last_cuda_error = static_cast<int>(e); }
+
+omq_status launch_status() {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_cuda_error(e);
+    return OMQ_ERR_CUDA;
+  }
+  return OMQ_OK;
+}
+
+int num_sms() {
+  static std::mutex mu;
+  static std::vector<int> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  std::lock_guard<std::mutex> lk(mu);
+  if (static_cast<int>(cache.size()) <= dev) cache.resize(dev + 1, 0);
+  if (cache[dev] == 0) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cache[dev] = n > 0 ? n : 148;
+  }
+  return cache[dev];
+}
+
+}  // namespace omq
+
+using namespace omq;
+
+extern "C" {
+
+const char* omq_status_str(int status) {
+  switch (status) {
+    case OMQ_OK: return "ok";
+    case OMQ_ERR_NULL: return "required pointer is NULL";
+    case OMQ_ERR_SHAPE: return "invalid shape";
+    case OMQ_ERR_DTYPE: return "unsupported dtype";
+    case OMQ_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case OMQ_ERR_BITS: return "bit width out of range";
+    case OMQ_ERR_WORKSPACE: return "workspace missing or too small";
+    case OMQ_ERR_CUDA: return "CUDA error";
+    case OMQ_ERR_UNSUPPORTED: return "unsupported configuration";
+    case OMQ_ERR_TIMEOUT: return "device barrier wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int omq_last_cuda_error(void) { return t_last_cuda_error; }
+
+int omq_version(void) { return 10000; }
+
+omq_status omq_sync_check(omq_stream_t stream) {
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) {
+    set_cuda_error(e);
+    return OMQ_ERR_CUDA;
+  }
+  unsigned flag = 0;
+  e = take_device_error(&flag);
+  if (e != cudaSuccess) {
+    set_cuda_error(e);
+    return OMQ_ERR_CUDA;
+  }
+  return flag ? OMQ_ERR_TIMEOUT : OMQ_OK;
+}
+
+omq_status omq_lwc_quant(const void* W, omq_dtype wdt, int64_t N, int64_t K, int64_t group,
+                         int bits, const float* gamma_logit, const float* beta_logit,
+                         const float* s, void* W_hat, omq_dtype hat_dt, float* h, int32_t* z,
+                         uint8_t* codes, omq_range* grp_range, omq_stream_t stream) {
+  OMQ_TRY(check_lwc(W, wdt, N, K, group, bits, gamma_logit, beta_logit, s, hat_dt, W_hat, codes,
+                    h, z));
+  LwcParams p{W, wdt, N, K, group, K / group, static_cast<float>((1 << bits) - 1), gamma_logit,
+              beta_logit, s, W_hat, hat_dt, h, z, codes, grp_range, nullptr, bits};
+  return launch_lwc(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+omq_status omq_fold_pack(const void* W, omq_dtype wdt, int64_t N, int64_t K, int64_t group,
+                         int bits, const float* gamma_logit, const float* beta_logit,
+                         const float* s, uint8_t* packed, float* h, int32_t* z,
+                         omq_stream_t stream) {
+  if (!packed) return OMQ_ERR_NULL;
+  OMQ_TRY(check_lwc(W, wdt, N, K, group, bits, gamma_logit, beta_logit, s, OMQ_F32, nullptr,
+                    packed, h, z));
+  if (bits == 3) return OMQ_ERR_UNSUPPORTED;
+  LwcParams p{W, wdt, N, K, group, K / group, static_cast<float>((1 << bits) - 1), gamma_logit,
+              beta_logit, s, nullptr, OMQ_F32, h, z, nullptr, nullptr, packed, bits};
+  return launch_lwc(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+omq_status omq_let_apply(const void* X, omq_dtype xdt, int64_t M, int64_t K, const float* s,
+                         const float* delta, int abits, void* Xq, omq_dtype xq_dt, float* h_a,
+                         int32_t* z_a, omq_range* tok_range, const void* W, omq_dtype wdt,
+                         int64_t N, const float* B, float* B_tilde, omq_stream_t stream) {
+  if (!X || !Xq) return OMQ_ERR_NULL;
+  if (!dtype_ok(xdt) || !dtype_ok(xq_dt)) return OMQ_ERR_DTYPE;
+  if (!abits_ok(abits)) return OMQ_ERR_BITS;
+  if (M < 1 || K < 8 || K % 8 || M > kMaxDim || K > kMaxDim) return OMQ_ERR_SHAPE;
+  if (abits < 16 && K > 49152) return OMQ_ERR_SHAPE;
+  if (!a16(X) || !a16(Xq) || !a16(s) || !a16(delta)) return OMQ_ERR_ALIGN;
+  if (B_tilde) {
+    if (delta && !W) return OMQ_ERR_NULL;
+    if (N < 1 || N > kMaxDim) return OMQ_ERR_SHAPE;
+    if (delta && !dtype_ok(wdt)) return OMQ_ERR_DTYPE;
+    if (!a16(W)) return OMQ_ERR_ALIGN;
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  LetParams p{X, xdt, M, K, s, delta, static_cast<float>((1 << (abits < 16 ? abits : 1)) - 1), Xq,
+              xq_dt, h_a, z_a, tok_range};
+  OMQ_TRY(launch_let(p, abits, st));
+  if (B_tilde) OMQ_TRY(launch_let_bias(W, wdt, N, K, delta, B, B_tilde, st));
+  return OMQ_OK;
+}
+
+size_t omq_fwd_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  (void)K;
+  if (M < 1 || N < 1) return 0;
+  return fwd_bytes(M, N);
+}
+
+static omq_status run_gemm(omq_dtype dt, const GemmOperand& A, const GemmOperand& B, int64_t rows,
+                           int64_t cols, int64_t depth, const GemmEpilogue& epi, int64_t* tiles,
+                           cudaStream_t st) {
+  if (dt == OMQ_BF16) return gemm_bf16_tc(A, B, rows, cols, depth, epi, tiles, st);
+  return gemm_f32_simt(A, B, rows, cols, depth, epi, tiles, st);
+}
+
+omq_status omq_fq_linear_fwd(const void* Xq, const void* W_hat, omq_dtype dt, int64_t M,
+                             int64_t N, int64_t K, const float* B_tilde, const float* Y_ref,
+                             float* Y, void* dY, float* loss, void* workspace, size_t ws_bytes,
+                             omq_stream_t stream) {
+  if (!Xq || !W_hat) return OMQ_ERR_NULL;
+  if (!dtype_ok(dt)) return OMQ_ERR_DTYPE;
+  if (M < 1 || N < 8 || K < 8 || N % 8 || K % 8 || M > kMaxDim || N > kMaxDim || K > kMaxDim)
+    return OMQ_ERR_SHAPE;
+  if (Y_ref) {
+    if (!dY) return OMQ_ERR_NULL;
+  } else {
+    if (!Y) return OMQ_ERR_NULL;
+    if (dY || loss) return OMQ_ERR_NULL;
+  }
+  if (!a16(Xq) || !a16(W_hat) || !a16(B_tilde) || !a16(Y_ref) || !a16(Y) || !a16(dY))
+    return OMQ_ERR_ALIGN;
+  if (Y_ref && (!workspace || ws_bytes < fwd_bytes(M, N))) return OMQ_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  GemmOperand A{Xq, K, false}, B{W_hat, K, false};
+  GemmEpilogue epi{};
+  epi.bias = B_tilde;
+  if (Y_ref) {
+    epi.kind = Epi::MseLoss;
+    epi.out = Y;
+    epi.y_ref = Y_ref;
+    epi.dy = dY;
+    epi.dy_dt = dt;
+    epi.dy_scale = static_cast<float>(2.0 / (static_cast<double>(M) * static_cast<double>(N)));
+    epi.loss_partials = static_cast<float*>(workspace);
+  } else {
+    epi.kind = Epi::StoreF32;
+    epi.out = Y;
+  }
+  int64_t tiles = 0;
+  OMQ_TRY(run_gemm(dt, A, B, M, N, K, epi, &tiles, st));
+  if (Y_ref && loss)
+    OMQ_TRY(launch_loss_finalize(epi.loss_partials, tiles,
+                                 1.0 / (static_cast<double>(M) * static_cast<double>(N)), loss, st));
+  return OMQ_OK;
+}
+
+size_t omq_bwd_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t group) {
+  if (M < 1 || N < 1 || K < 1 || group < 1) return 0;
+  return bwd_layout(M, N, K, group).total;
+}
+
+omq_status omq_fq_linear_bwd(const omq_bwd_args* a, void* workspace, size_t ws_bytes,
+                             omq_stream_t stream) {
+  if (!a) return OMQ_ERR_NULL;
+  const int64_t M = a->M, N = a->N, K = a->K, G = a->group;
+  if (!a->W || !a->Xq || !a->W_hat || !a->h || !a->z || !a->grp_range || !a->dY ||
+      !a->gamma_logit || !a->beta_logit)
+    return OMQ_ERR_NULL;
+  if (!dtype_ok(a->dt)) return OMQ_ERR_DTYPE;
+  if (!wbits_ok(a->bits) || !abits_ok(a->abits)) return OMQ_ERR_BITS;
+  if (M < 1 || N < 8 || K < 8 || G < 8 || N % 8 || K % 8 || G % 8 || K % G || M > kMaxDim ||
+      N > kMaxDim || K > kMaxDim)
+    return OMQ_ERR_SHAPE;
+  if (!small_group(G) && G > kMaxGroupLarge) return OMQ_ERR_SHAPE;
+  const bool need_let = a->d_s || a->d_delta;
+  if (need_let) {
+    if (!a->X || !a->s || !a->delta) return OMQ_ERR_NULL;
+    if (2 * K * sizeof(float) > 200 * 1024) return OMQ_ERR_SHAPE;
+    if (a->abits < 16 && (!a->h_a || !a->z_a || !a->tok_range)) return OMQ_ERR_NULL;
+  }
+  if (!a16(a->X) || !a16(a->W) || !a16(a->s) || !a16(a->delta) || !a16(a->Xq) ||
+      !a16(a->W_hat) || !a16(a->dY))
+    return OMQ_ERR_ALIGN;
+  const BwdLayout L = bwd_layout(M, N, K, G);
+  if (!workspace || ws_bytes < L.total) return OMQ_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+
+  float* dbt_part = at<float>(workspace, L.dbt_part);
+  float* dbt = a->d_B_tilde ? a->d_B_tilde : at<float>(workspace, L.dbt);
+  float* dwhat = at<float>(workspace, L.dwhat);
+  float* dxq = at<float>(workspace, L.dxq);
+  float* part_ws = at<float>(workspace, L.part_ws);
+  float* part_wd = at<float>(workspace, L.part_wd);
+  float* part_xs = at<float>(workspace, L.part_xs);
+  float* part_xd = at<float>(workspace, L.part_xd);
+
+  // dB~ = column sums of dY (needed for d_delta, or when asked for)
+  if (a->d_delta || a->d_B_tilde) {
+    OMQ_TRY(launch_colsum(a->dY, a->dt, M, N, kRowsColsum, dbt_part, st));
+    OMQ_TRY(launch_reduce_cols(dbt_part, L.rb_colsum, nullptr, 0, N, dbt, st));
+  }
+  // dW^ = dY^T Xq   [N, K]
+  {
+    GemmOperand A{a->dY, N, true}, B{a->Xq, K, true};
+    GemmEpilogue epi{};
+    epi.kind = Epi::StoreF32;
+    epi.out = dwhat;
+    OMQ_TRY(run_gemm(a->dt, A, B, N, K, M, epi, nullptr, st));
+  }
+  // weight-side STE: d gamma / d beta logits and the W-side LET column partials
+  {
+    SteWParams p{a->W, a->dt, N, K, G, K / G, static_cast<float>((1 << a->bits) - 1),
+                 a->s, a->gamma_logit, a->beta_logit, a->h, a->z,
+                 a->grp_range, dwhat, a->d_delta ? dbt : nullptr, a->d_gamma_logit,
+                 a->d_beta_logit, a->d_s ? part_ws : nullptr, a->d_delta ? part_wd : nullptr,
+                 static_cast<int>(rows_per_block_w(G))};
+    OMQ_TRY(launch_ste_w(p, st));
+  }
+  if (!need_let) return OMQ_OK;
+  // dXq = dY W^   [M, K]
+  {
+    GemmOperand A{a->dY, N, false}, B{a->W_hat, K, true};
+    GemmEpilogue epi{};
+    epi.kind = Epi::StoreF32;
+    epi.out = dxq;
+    OMQ_TRY(run_gemm(a->dt, A, B, M, K, N, epi, nullptr, st));
+  }
+  {
+    SteXParams p{a->X, a->dt, M, K,
+                 static_cast<float>((1 << (a->abits < 16 ? a->abits : 1)) - 1),
+                 a->abits < 16 ? 1 : 0, a->s, a->delta, a->h_a, a->z_a, a->tok_range, dxq, part_xs,
+                 part_xd, kRowsX};
+    OMQ_TRY(launch_ste_x(p, st));
+  }
+  if (a->d_s) OMQ_TRY(launch_reduce_cols(part_ws, L.rb_w, part_xs, L.rb_x, K, a->d_s, st));
+  if (a->d_delta) OMQ_TRY(launch_reduce_cols(part_wd, L.rb_w, part_xd, L.rb_x, K, a->d_delta, st));
+  return OMQ_OK;
+}
+
+omq_status omq_adamw_step(float* param, const float* grad, float* m, float* v, int64_t n, float lr,
+                          float beta1, float beta2, float eps, float weight_decay, int64_t step,
+                          omq_stream_t stream) {
+  if (n < 0) return OMQ_ERR_SHAPE;
+  if (n == 0) return OMQ_OK;
+  if (!param || !grad || !m || !v) return OMQ_ERR_NULL;
+  if (step < 1) return OMQ_ERR_SHAPE;
+  return launch_adamw(param, grad, m, v, n, lr, beta1, beta2, eps, weight_decay, step,
+                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t omq_step_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t group) {
+  if (M < 1 || N < 1 || K < 1 || group < 1) return 0;
+  return fwd_bytes(M, N) + bwd_layout(M, N, K, group).total;
+}
+
+omq_status omq_calib_step(const omq_step_args* a, void* workspace, size_t ws_bytes,
+                          omq_stream_t stream) {
+  if (!a) return OMQ_ERR_NULL;
+  const int64_t M = a->M, N = a->N, K = a->K, G = a->group;
+  if (!a->X || !a->W || !a->Y_ref || !a->gamma_logit || !a->beta_logit || !a->W_hat || !a->h ||
+      !a->z || !a->grp_range || !a->dY || !a->d_gamma_logit || !a->d_beta_logit || !a->loss ||
+      !a->m_gamma || !a->v_gamma || !a->m_beta || !a->v_beta)
+    return OMQ_ERR_NULL;
+  if (M < 1 || N < 1 || K < 1 || G < 1) return OMQ_ERR_SHAPE;
+  if (a->step < 1) return OMQ_ERR_SHAPE;
+  const bool let = a->let != 0;
+  const bool need_act = let || a->abits < 16;
+  if (let && (!a->s || !a->delta || !a->d_s || !a->d_delta || !a->m_s || !a->v_s || !a->m_delta ||
+              !a->v_delta || !a->B_tilde))
+    return OMQ_ERR_NULL;
+  if (need_act && (!a->Xq || a->Xq == a->X)) return OMQ_ERR_NULL;
+  if (a->abits < 16 && (!a->h_a || !a->z_a || !a->tok_range)) return OMQ_ERR_NULL;
+  const size_t fwd_ws = fwd_bytes(M, N);
+  if (!workspace || ws_bytes < omq_step_workspace_bytes(M, N, K, G)) return OMQ_ERR_WORKSPACE;
+  const void* Xq = need_act ? a->Xq : a->X;
+  const float* Bt = let ? a->B_tilde : a->B;
+  if (need_act) {
+    OMQ_TRY(omq_let_apply(a->X, a->dt, M, K, let ? a->s : nullptr, let ? a->delta : nullptr,
+                          a->abits, a->Xq, a->dt, a->h_a, a->z_a, a->tok_range, a->W, a->dt, N,
+                          a->B, let ? a->B_tilde : nullptr, stream));
+  }
+  OMQ_TRY(omq_lwc_quant(a->W, a->dt, N, K, G, a->bits, a->gamma_logit, a->beta_logit,
+                        let ? a->s : nullptr, a->W_hat, a->dt, a->h, a->z, nullptr, a->grp_range,
+                        stream));
+  OMQ_TRY(omq_fq_linear_fwd(Xq, a->W_hat, a->dt, M, N, K, Bt, a->Y_ref, nullptr, a->dY, a->loss,
+                            workspace, fwd_ws, stream));
+  omq_bwd_args b{};
+  b.M = M; b.N = N; b.K = K; b.group = G; b.bits = a->bits; b.abits = a->abits; b.dt = a->dt;
+  b.X = a->X; b.W = a->W; b.s = let ? a->s : nullptr; b.delta = let ? a->delta : nullptr;
+  b.gamma_logit = a->gamma_logit; b.beta_logit = a->beta_logit;
+  b.Xq = Xq; b.W_hat = a->W_hat; b.h = a->h; b.z = a->z; b.grp_range = a->grp_range;
+  b.h_a = a->h_a; b.z_a = a->z_a; b.tok_range = a->tok_range; b.dY = a->dY;
+  b.d_gamma_logit = a->d_gamma_logit; b.d_beta_logit = a->d_beta_logit;
+  b.d_s = let ? a->d_s : nullptr; b.d_delta = let ? a->d_delta : nullptr;
+  OMQ_TRY(omq_fq_linear_bwd(&b, static_cast<char*>(workspace) + fwd_ws, ws_bytes - fwd_ws,
+                            stream));
+  const int64_t ng = N * (K / G);
+  OMQ_TRY(omq_adamw_step(a->gamma_logit, a->d_gamma_logit, a->m_gamma, a->v_gamma, ng, a->lr_lwc,
+                         0.9f, 0.999f, 1e-8f, 0.f, a->step, stream));
+  OMQ_TRY(omq_adamw_step(a->beta_logit, a->d_beta_logit, a->m_beta, a->v_beta, ng, a->lr_lwc,
+                         0.9f, 0.999f, 1e-8f, 0.f, a->step, stream));
+  if (let) {
+    OMQ_TRY(omq_adamw_step(a->s, a->d_s, a->m_s, a->v_s, K, a->lr_let, 0.9f, 0.999f, 1e-8f, 0.f,
+                           a->step, stream));
+    OMQ_TRY(omq_adamw_step(a->delta, a->d_delta, a->m_delta, a->v_delta, K, a->lr_let, 0.9f,
+                           0.999f, 1e-8f, 0.f, a->step, stream));
+  }
+  return OMQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,235 @@
+// Internal declarations shared by the libomq translation units: launch helpers, the
+// device error flag, bf16 conversion, the clipping-strength sigmoid and the binary32
+// encoder arithmetic (one fixed operation order, no contraction).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include <cmath>
+
+#include "../../include/omq.h"
+
+namespace omq {
+
+// Raised (bitwise OR) by kernels whose bounded barrier waits expired; read by
+// omq_sync_check(). Bit values say which wait gave up. The flag lives in gemm_tc.cu (the
+// only translation unit with barrier waits); the host reads and clears it through this call.
+enum : unsigned { DEV_ERR_TMA_WAIT = 1u, DEV_ERR_MMA_WAIT = 2u, DEV_ERR_EPI_WAIT = 4u };
+cudaError_t take_device_error(unsigned* flag);
+
+constexpr float H_FLOOR = 1e-8f;          // floor of the quantization step h
+constexpr int Z_LIMIT = 1 << 30;          // |z| stored as int32 is clamped to this
+
+// ---- element access --------------------------------------------------------------------
+__device__ __forceinline__ float load_elem(const void* p, int64_t i, omq_dtype dt) {
+  if (dt == OMQ_BF16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[i]);
+  return reinterpret_cast<const float*>(p)[i];
+}
+__device__ __forceinline__ void store_elem(void* p, int64_t i, float v, omq_dtype dt) {
+  if (dt == OMQ_BF16) reinterpret_cast<__nv_bfloat16*>(p)[i] = __float2bfloat16_rn(v);
+  else reinterpret_cast<float*>(p)[i] = v;
+}
+// 8 consecutive elements (16 B of bf16 or 32 B of f32) starting at a multiple of 8.
+__device__ __forceinline__ void load8(const void* p, int64_t i, omq_dtype dt, float (&v)[8]) {
+  if (dt == OMQ_BF16) {
+    uint4 raw = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(p) + i);
+    const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float2 f = __bfloat1622float2(b2[j]);
+      v[2 * j] = f.x;
+      v[2 * j + 1] = f.y;
+    }
+  } else {
+    const float4* q = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p) + i);
+    float4 a = q[0], b = q[1];
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+}
+__device__ __forceinline__ void store8(void* p, int64_t i, omq_dtype dt, const float (&v)[8]) {
+  if (dt == OMQ_BF16) {
+    uint4 raw;
+    __nv_bfloat162* b2 = reinterpret_cast<__nv_bfloat162*>(&raw);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) b2[j] = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
+    *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p) + i) = raw;
+  } else {
+    float4* q = reinterpret_cast<float4*>(reinterpret_cast<float*>(p) + i);
+    q[0] = make_float4(v[0], v[1], v[2], v[3]);
+    q[1] = make_float4(v[4], v[5], v[6], v[7]);
+  }
+}
+
+// ---- encoder arithmetic ----------------------------------------------------------------
+// Clipping strength in [0, 1] from its logit: evaluated in binary64, rounded once.
+__device__ __forceinline__ float strength(float logit) {
+  return __double2float_rn(1.0 / (1.0 + exp(-static_cast<double>(logit))));
+}
+
+struct GroupQ {
+  float h;       // step (floored)
+  float z;       // zero point, integral
+  bool active;   // unfloored h >= H_FLOOR (h's gradient reaches g, b, max, min)
+};
+
+// h = max(((g*M) - (b*m)) / Q, 1e-8);  z = -round((b*m) / h)
+__device__ __forceinline__ GroupQ group_params(float g, float b, float vmax, float vmin, float Q) {
+  float hr = __fdiv_rn(__fsub_rn(__fmul_rn(g, vmax), __fmul_rn(b, vmin)), Q);
+  GroupQ r;
+  r.active = hr >= H_FLOOR;
+  r.h = r.active ? hr : H_FLOOR;
+  r.z = -rintf(__fdiv_rn(__fmul_rn(b, vmin), r.h));
+  return r;
+}
+
+// round(v / h) with v / h the correctly rounded binary32 quotient.
+//
+// The quotient matters only through round(). With hinv = 1/h correctly rounded, the
+// product v*hinv differs from v/h by at most 2^-23 |v/h| (two roundings), i.e. below
+// 2.5e-4 while |v*hinv| < 2048. round() of the product therefore equals round() of the
+// quotient unless the product lies within 1e-3 of a half-integer; in that case, and for
+// large quotients, the IEEE division itself is taken. The result is bitwise the level an
+// exact-division implementation produces, at the cost of a multiply in almost all cases.
+__device__ __forceinline__ float round_quotient(float v, float h, float hinv) {
+  float ua = __fmul_rn(v, hinv);
+  if (fabsf(ua) >= 2048.f || fabsf(ua - floorf(ua) - 0.5f) < 1e-3f) ua = __fdiv_rn(v, h);
+  return rintf(ua);
+}
+
+__device__ __forceinline__ int32_t z_to_i32(float z) {
+  float c = fminf(fmaxf(z, -static_cast<float>(Z_LIMIT)), static_cast<float>(Z_LIMIT));
+  return static_cast<int32_t>(c);
+}
+
+// ---- host-side helpers ------------------------------------------------------------------
+void set_cuda_error(cudaError_t e);
+omq_status launch_status();          // checks cudaGetLastError after a launch
+int num_sms();
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---- GEMM front ends (gemm_tc.cu / gemm_simt.cu) -----------------------------------------
+// C[i, j] = sum_k A(i, k) * B(j, k) for i < rows, j < cols, k < depth.
+// An operand is "K-major" when A(i, k) = A[i*ld + k] and "MN-major" when A(i, k) = A[k*ld + i].
+struct GemmOperand {
+  const void* ptr;
+  int64_t ld;         // elements between consecutive rows of the stored matrix
+  bool mn_major;
+};
+
+enum class Epi { StoreF32 = 0, MseLoss = 1 };
+
+struct GemmEpilogue {
+  Epi kind;
+  float* out;              // StoreF32: [rows, cols] fp32 (ld = cols); MseLoss: Y or NULL
+  const float* bias;       // per column j, or NULL
+  const float* y_ref;      // MseLoss: [rows, cols]
+  void* dy;                // MseLoss: [rows, cols] in dy_dt
+  omq_dtype dy_dt;
+  float dy_scale;          // 2 / (rows * cols)
+  float* loss_partials;    // MseLoss: one per CTA tile (fixed order)
+};
+
+// bf16 operands on tcgen05 (sm_100a). Returns the number of CTA tiles launched.
+omq_status gemm_bf16_tc(const GemmOperand& A, const GemmOperand& B, int64_t rows, int64_t cols,
+                        int64_t depth, const GemmEpilogue& epi, int64_t* n_tiles,
+                        cudaStream_t stream);
+int64_t gemm_bf16_tc_tiles(int64_t rows, int64_t cols);
+// f32 operands on CUDA cores.
+omq_status gemm_f32_simt(const GemmOperand& A, const GemmOperand& B, int64_t rows, int64_t cols,
+                         int64_t depth, const GemmEpilogue& epi, int64_t* n_tiles,
+                         cudaStream_t stream);
+int64_t gemm_f32_simt_tiles(int64_t rows, int64_t cols);
+
+
+// ---- kernel parameter blocks and launchers (lwc.cu, let.cu, ste.cu) --------------------
+struct LwcParams {
+  const void* W;
+  omq_dtype wdt;
+  int64_t N, K, G, ng;
+  float Q;
+  const float* gl;
+  const float* bl;
+  const float* s;
+  void* W_hat;
+  omq_dtype hat_dt;
+  float* h;
+  int32_t* z;
+  uint8_t* codes;
+  omq_range* range;
+  uint8_t* packed;
+  int bits;
+};
+
+struct LetParams {
+  const void* X;
+  omq_dtype xdt;
+  int64_t M, K;
+  const float* s;
+  const float* d;
+  float Qa;
+  void* Xq;
+  omq_dtype xq_dt;
+  float* h_a;
+  int32_t* z_a;
+  omq_range* range;
+};
+
+struct SteWParams {
+  const void* W;
+  omq_dtype wdt;
+  int64_t N, K, G, ng;
+  float Q;
+  const float* s;
+  const float* gl;
+  const float* bl;
+  const float* h;
+  const int32_t* z;
+  const omq_range* range;
+  const float* dWhat;   // [N,K] fp32
+  const float* dBt;     // [N] or NULL
+  float* d_gl;
+  float* d_bl;
+  float* part_s;        // [row blocks, K] or NULL: sum_n dW~[n,k] W[n,k]
+  float* part_d;        // [row blocks, K] or NULL: sum_n dB~[n] W[n,k]
+  int rows_per_block;
+};
+
+struct SteXParams {
+  const void* X;
+  omq_dtype xdt;
+  int64_t M, K;
+  float Qa;
+  int quantized;        // abits < 16
+  const float* s;
+  const float* d;
+  const float* h_a;
+  const int32_t* z_a;
+  const omq_range* range;
+  const float* dXq;     // [M,K] fp32
+  float* part_s;        // [row blocks, K]: -sum_m dX~ X~ / s
+  float* part_d;        // [row blocks, K]: -sum_m dX~ / s
+  int rows_per_block;
+};
+
+omq_status launch_lwc(const LwcParams& p, cudaStream_t stream);
+omq_status launch_let(const LetParams& p, int abits, cudaStream_t stream);
+omq_status launch_let_bias(const void* W, omq_dtype wdt, int64_t N, int64_t K, const float* delta,
+                           const float* B, float* Bt, cudaStream_t stream);
+omq_status launch_ste_w(const SteWParams& p, cudaStream_t stream);
+omq_status launch_ste_x(const SteXParams& p, cudaStream_t stream);
+omq_status launch_colsum(const void* A, omq_dtype dt, int64_t rows, int64_t cols, int R,
+                         float* part, cudaStream_t stream);
+omq_status launch_reduce_cols(const float* p0, int64_t r0n, const float* p1, int64_t r1n,
+                              int64_t cols, float* out, cudaStream_t stream);
+omq_status launch_loss_finalize(const float* part, int64_t n, double inv_count, float* loss,
+                                cudaStream_t stream);
+omq_status launch_adamw(float* p, const float* g, float* m, float* v, int64_t n, float lr,
+                        float b1, float b2, float eps, float wd, int64_t step,
+                        cudaStream_t stream);
+
+}  // namespace omq

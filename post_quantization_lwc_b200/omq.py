@@ -1,0 +1,361 @@
+"""ctypes binding of libomq (include/omq.h): argument marshalling only.
+
+PyTorch tensors supply device memory and the current stream; every computation runs in the
+library's CUDA kernels. Importing this module loads ``libomq.so`` from the package
+directory and raises ImportError when it is missing: there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libomq.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"libomq.so is not built ({LIB_PATH}); run "
+                      "`python -m post_quantization_lwc_b200.build`")
+_lib = ctypes.CDLL(LIB_PATH)
+
+OMQ_F32, OMQ_BF16 = 0, 1
+STATUS = {0: "OMQ_OK", 1: "OMQ_ERR_NULL", 2: "OMQ_ERR_SHAPE", 3: "OMQ_ERR_DTYPE",
+          4: "OMQ_ERR_ALIGN", 5: "OMQ_ERR_BITS", 6: "OMQ_ERR_WORKSPACE", 7: "OMQ_ERR_CUDA",
+          8: "OMQ_ERR_UNSUPPORTED", 9: "OMQ_ERR_TIMEOUT"}
+
+# every symbol declared in include/omq.h
+EXPORTS = ("omq_status_str", "omq_last_cuda_error", "omq_version", "omq_sync_check",
+           "omq_lwc_quant", "omq_let_apply", "omq_fq_linear_fwd", "omq_fwd_workspace_bytes",
+           "omq_fq_linear_bwd", "omq_bwd_workspace_bytes", "omq_adamw_step", "omq_fold_pack",
+           "omq_calib_step", "omq_step_workspace_bytes")
+
+_p = ctypes.c_void_p
+_i64 = ctypes.c_int64
+_i32 = ctypes.c_int
+_f32 = ctypes.c_float
+_sz = ctypes.c_size_t
+
+
+class OmqError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = _lib.omq_status_str(status).decode()
+        extra = f" (cuda error {_lib.omq_last_cuda_error()})" if status == 7 else ""
+        super().__init__(f"{where}: {STATUS.get(status, status)}: {msg}{extra}")
+
+
+class BwdArgs(ctypes.Structure):
+    _fields_ = [("M", _i64), ("N", _i64), ("K", _i64), ("group", _i64), ("bits", _i32),
+                ("abits", _i32), ("dt", _i32),
+                ("X", _p), ("W", _p), ("s", _p), ("delta", _p), ("gamma_logit", _p),
+                ("beta_logit", _p), ("Xq", _p), ("W_hat", _p), ("h", _p), ("z", _p),
+                ("grp_range", _p), ("h_a", _p), ("z_a", _p), ("tok_range", _p), ("dY", _p),
+                ("d_gamma_logit", _p), ("d_beta_logit", _p), ("d_s", _p), ("d_delta", _p),
+                ("d_B_tilde", _p)]
+
+
+class StepArgs(ctypes.Structure):
+    _fields_ = [("M", _i64), ("N", _i64), ("K", _i64), ("group", _i64), ("bits", _i32),
+                ("abits", _i32), ("let", _i32), ("dt", _i32),
+                ("X", _p), ("W", _p), ("B", _p), ("Y_ref", _p),
+                ("gamma_logit", _p), ("beta_logit", _p), ("s", _p), ("delta", _p),
+                ("m_gamma", _p), ("v_gamma", _p), ("m_beta", _p), ("v_beta", _p),
+                ("m_s", _p), ("v_s", _p), ("m_delta", _p), ("v_delta", _p),
+                ("Xq", _p), ("W_hat", _p), ("B_tilde", _p),
+                ("h", _p), ("z", _p), ("grp_range", _p),
+                ("h_a", _p), ("z_a", _p), ("tok_range", _p),
+                ("dY", _p),
+                ("d_gamma_logit", _p), ("d_beta_logit", _p), ("d_s", _p), ("d_delta", _p),
+                ("loss", _p), ("lr_lwc", _f32), ("lr_let", _f32), ("step", _i64)]
+
+
+def _sig(name, res, args):
+    f = getattr(_lib, name)
+    f.restype = res
+    f.argtypes = args
+
+
+_sig("omq_status_str", ctypes.c_char_p, [_i32])
+_sig("omq_last_cuda_error", _i32, [])
+_sig("omq_version", _i32, [])
+_sig("omq_sync_check", _i32, [_p])
+_sig("omq_lwc_quant", _i32, [_p, _i32, _i64, _i64, _i64, _i32, _p, _p, _p, _p, _i32, _p, _p, _p,
+                             _p, _p])
+_sig("omq_let_apply", _i32, [_p, _i32, _i64, _i64, _p, _p, _i32, _p, _i32, _p, _p, _p, _p, _i32,
+                             _i64, _p, _p, _p])
+_sig("omq_fq_linear_fwd", _i32, [_p, _p, _i32, _i64, _i64, _i64, _p, _p, _p, _p, _p, _p, _sz, _p])
+_sig("omq_fwd_workspace_bytes", _sz, [_i64, _i64, _i64])
+_sig("omq_fq_linear_bwd", _i32, [ctypes.POINTER(BwdArgs), _p, _sz, _p])
+_sig("omq_bwd_workspace_bytes", _sz, [_i64, _i64, _i64, _i64])
+_sig("omq_adamw_step", _i32, [_p, _p, _p, _p, _i64, _f32, _f32, _f32, _f32, _f32, _i64, _p])
+_sig("omq_fold_pack", _i32, [_p, _i32, _i64, _i64, _i64, _i32, _p, _p, _p, _p, _p, _p, _p])
+_sig("omq_calib_step", _i32, [ctypes.POINTER(StepArgs), _p, _sz, _p])
+_sig("omq_step_workspace_bytes", _sz, [_i64, _i64, _i64, _i64])
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise OmqError(status, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return OMQ_BF16
+    if t.dtype == torch.float32:
+        return OMQ_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _tdt(code: int):
+    return torch.bfloat16 if code == OMQ_BF16 else torch.float32
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dev(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def version() -> int:
+    return _lib.omq_version()
+
+
+def sync_check(stream=None):
+    _check(_lib.omq_sync_check(_stream(stream)), "omq_sync_check")
+
+
+def new_range(n: int, device) -> torch.Tensor:
+    """Storage for omq_range records (16 bytes each) as an int32 [n, 4] tensor."""
+    return torch.empty(n, 4, dtype=torch.int32, device=device)
+
+
+def range_fields(r: torch.Tensor):
+    """(vmax, vmin, nmax, nmin) views of an omq_range tensor."""
+    return r[:, 0].view(torch.float32), r[:, 1].view(torch.float32), r[:, 2], r[:, 3]
+
+
+# ---------------------------------------------------------------------------- primitives
+
+def lwc_quant(W, gamma_logit, beta_logit, bits, group, s=None, hat_dtype=None, codes=False,
+              stream=None):
+    """omq_lwc_quant. Returns dict(W_hat, h, z, codes, grp_range)."""
+    _dev(W, gamma_logit, beta_logit, s)
+    N, K = W.shape
+    ng = K // group
+    dev = W.device
+    W_hat = torch.empty(N, K, dtype=hat_dtype or W.dtype, device=dev)
+    h = torch.empty(N, ng, dtype=torch.float32, device=dev)
+    z = torch.empty(N, ng, dtype=torch.int32, device=dev)
+    c = torch.empty(N, K, dtype=torch.uint8, device=dev) if codes else None
+    rg = new_range(N * ng, dev)
+    _check(_lib.omq_lwc_quant(_ptr(W), _dt(W), N, K, group, bits, _ptr(gamma_logit),
+                              _ptr(beta_logit), _ptr(s), _ptr(W_hat), _dt(W_hat), _ptr(h), _ptr(z),
+                              _ptr(c), _ptr(rg), _stream(stream)), "omq_lwc_quant")
+    return dict(W_hat=W_hat, h=h, z=z, codes=c, grp_range=rg)
+
+
+def let_apply(X, abits, s=None, delta=None, xq_dtype=None, W=None, B=None, want_bias=False,
+              stream=None):
+    """omq_let_apply. Returns dict(Xq, h_a, z_a, tok_range, B_tilde)."""
+    _dev(X, s, delta, W, B)
+    M, K = X.shape
+    dev = X.device
+    Xq = torch.empty(M, K, dtype=xq_dtype or X.dtype, device=dev)
+    q = abits < 16
+    h_a = torch.empty(M, dtype=torch.float32, device=dev) if q else None
+    z_a = torch.empty(M, dtype=torch.int32, device=dev) if q else None
+    tr = new_range(M, dev) if q else None
+    N = W.shape[0] if W is not None else (B.shape[0] if B is not None else 0)
+    Bt = torch.empty(N, dtype=torch.float32, device=dev) if want_bias else None
+    _check(_lib.omq_let_apply(_ptr(X), _dt(X), M, K, _ptr(s), _ptr(delta), abits, _ptr(Xq),
+                              _dt(Xq), _ptr(h_a), _ptr(z_a), _ptr(tr), _ptr(W),
+                              _dt(W) if W is not None else 0, N, _ptr(B), _ptr(Bt),
+                              _stream(stream)), "omq_let_apply")
+    return dict(Xq=Xq, h_a=h_a, z_a=z_a, tok_range=tr, B_tilde=Bt)
+
+
+def fwd_workspace_bytes(M, N, K) -> int:
+    return _lib.omq_fwd_workspace_bytes(M, N, K)
+
+
+def fq_linear_fwd(Xq, W_hat, B_tilde=None, Y_ref=None, want_Y=True, workspace=None,
+                  stream=None):
+    """omq_fq_linear_fwd. Returns dict(Y, dY, loss)."""
+    _dev(Xq, W_hat, B_tilde, Y_ref)
+    M, K = Xq.shape
+    N = W_hat.shape[0]
+    dev = Xq.device
+    Y = torch.empty(M, N, dtype=torch.float32, device=dev) if (want_Y or Y_ref is None) else None
+    dY = torch.empty(M, N, dtype=Xq.dtype, device=dev) if Y_ref is not None else None
+    loss = torch.empty(1, dtype=torch.float32, device=dev) if Y_ref is not None else None
+    nbytes = fwd_workspace_bytes(M, N, K)
+    if workspace is None and Y_ref is not None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    _check(_lib.omq_fq_linear_fwd(_ptr(Xq), _ptr(W_hat), _dt(Xq), M, N, K, _ptr(B_tilde),
+                                  _ptr(Y_ref), _ptr(Y), _ptr(dY), _ptr(loss), _ptr(workspace),
+                                  0 if workspace is None else workspace.numel(), _stream(stream)),
+           "omq_fq_linear_fwd")
+    return dict(Y=Y, dY=dY, loss=loss)
+
+
+def bwd_workspace_bytes(M, N, K, group) -> int:
+    return _lib.omq_bwd_workspace_bytes(M, N, K, group)
+
+
+def fq_linear_bwd(*, X, W, gamma_logit, beta_logit, Xq, W_hat, h, z, grp_range, dY, bits, group,
+                  abits=16, s=None, delta=None, h_a=None, z_a=None, tok_range=None,
+                  want_let=False, want_dBt=False, workspace=None, stream=None):
+    """omq_fq_linear_bwd. Returns dict(d_gamma_logit, d_beta_logit, d_s, d_delta, d_B_tilde)."""
+    _dev(X, W, gamma_logit, beta_logit, Xq, W_hat, h, z, grp_range, dY, s, delta)
+    M, K = Xq.shape
+    N = W.shape[0]
+    dev = W.device
+    f = lambda *shape: torch.empty(*shape, dtype=torch.float32, device=dev)
+    out = dict(d_gamma_logit=f(N, K // group), d_beta_logit=f(N, K // group),
+               d_s=f(K) if want_let else None, d_delta=f(K) if want_let else None,
+               d_B_tilde=f(N) if want_dBt else None)
+    a = BwdArgs(M=M, N=N, K=K, group=group, bits=bits, abits=abits, dt=_dt(Xq),
+                X=_ptr(X), W=_ptr(W), s=_ptr(s), delta=_ptr(delta), gamma_logit=_ptr(gamma_logit),
+                beta_logit=_ptr(beta_logit), Xq=_ptr(Xq), W_hat=_ptr(W_hat), h=_ptr(h), z=_ptr(z),
+                grp_range=_ptr(grp_range), h_a=_ptr(h_a), z_a=_ptr(z_a), tok_range=_ptr(tok_range),
+                dY=_ptr(dY), d_gamma_logit=_ptr(out["d_gamma_logit"]),
+                d_beta_logit=_ptr(out["d_beta_logit"]), d_s=_ptr(out["d_s"]),
+                d_delta=_ptr(out["d_delta"]), d_B_tilde=_ptr(out["d_B_tilde"]))
+    if workspace is None:
+        workspace = torch.empty(bwd_workspace_bytes(M, N, K, group), dtype=torch.uint8, device=dev)
+    _check(_lib.omq_fq_linear_bwd(ctypes.byref(a), _ptr(workspace), workspace.numel(),
+                                  _stream(stream)), "omq_fq_linear_bwd")
+    return out
+
+
+def adamw_step(param, grad, m, v, lr, step, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0,
+               stream=None):
+    """omq_adamw_step (in place on param, m, v)."""
+    _dev(param, grad, m, v)
+    _check(_lib.omq_adamw_step(_ptr(param), _ptr(grad), _ptr(m), _ptr(v), param.numel(), lr, beta1,
+                               beta2, eps, weight_decay, step, _stream(stream)), "omq_adamw_step")
+
+
+def fold_pack(W, gamma_logit, beta_logit, bits, group, s=None, stream=None):
+    """omq_fold_pack. Returns (packed uint8 [N, K*bits/8], h, z)."""
+    _dev(W, gamma_logit, beta_logit, s)
+    N, K = W.shape
+    dev = W.device
+    packed = torch.empty(N, K * bits // 8, dtype=torch.uint8, device=dev)
+    h = torch.empty(N, K // group, dtype=torch.float32, device=dev)
+    z = torch.empty(N, K // group, dtype=torch.int32, device=dev)
+    _check(_lib.omq_fold_pack(_ptr(W), _dt(W), N, K, group, bits, _ptr(gamma_logit),
+                              _ptr(beta_logit), _ptr(s), _ptr(packed), _ptr(h), _ptr(z),
+                              _stream(stream)), "omq_fold_pack")
+    return packed, h, z
+
+
+def step_workspace_bytes(M, N, K, group) -> int:
+    return _lib.omq_step_workspace_bytes(M, N, K, group)
+
+
+# ---------------------------------------------------------------------------- whole step
+
+@dataclasses.dataclass
+class LinearCalibration:
+    """Device buffers of one linear layer's calibration, driven by omq_calib_step.
+
+    Holds W, the learnable parameters with their AdamW moments, the step's intermediate
+    buffers and the workspace; ``step(X, Y_ref)`` runs one whole calibration step on the
+    current stream (LET, LWC, forward + loss, STE backward, AdamW).
+    """
+    M: int
+    N: int
+    K: int
+    group: int
+    bits: int
+    abits: int
+    let: bool
+    dtype: torch.dtype
+    device: torch.device
+    lr_lwc: float = 5e-3
+    lr_let: float = 1e-2
+
+    def __post_init__(self):
+        dev, M, N, K = self.device, self.M, self.N, self.K
+        ng = K // self.group
+        f = lambda *shape: torch.zeros(*shape, dtype=torch.float32, device=dev)
+        self.W = torch.empty(N, K, dtype=self.dtype, device=dev)
+        self.B = f(N)
+        self.gamma_logit, self.beta_logit = f(N, ng), f(N, ng)
+        self.s, self.delta = f(K), f(K)
+        self.moments = {k: (f(*shape), f(*shape)) for k, shape in
+                        (("gamma", (N, ng)), ("beta", (N, ng)), ("s", (K,)), ("delta", (K,)))}
+        need_act = self.let or self.abits < 16
+        self.Xq = torch.empty(M, K, dtype=self.dtype, device=dev) if need_act else None
+        self.W_hat = torch.empty(N, K, dtype=self.dtype, device=dev)
+        self.B_tilde = f(N)
+        self.h = f(N, ng)
+        self.z = torch.zeros(N, ng, dtype=torch.int32, device=dev)
+        self.grp_range = new_range(N * ng, dev)
+        q = self.abits < 16
+        self.h_a = f(M) if q else None
+        self.z_a = torch.zeros(M, dtype=torch.int32, device=dev) if q else None
+        self.tok_range = new_range(M, dev) if q else None
+        self.dY = torch.empty(M, N, dtype=self.dtype, device=dev)
+        self.d_gamma, self.d_beta = f(N, ng), f(N, ng)
+        self.d_s, self.d_delta = f(K), f(K)
+        self.loss = f(1)
+        self.workspace = torch.empty(step_workspace_bytes(M, N, K, self.group), dtype=torch.uint8,
+                                     device=dev)
+        self.t = 0
+
+    def load(self, W, gamma_logit, beta_logit, s=None, delta=None, B=None):
+        self.W.copy_(W)
+        self.gamma_logit.copy_(gamma_logit)
+        self.beta_logit.copy_(beta_logit)
+        if s is not None:
+            self.s.copy_(s)
+        if delta is not None:
+            self.delta.copy_(delta)
+        if B is not None:
+            self.B.copy_(B)
+        for m, v in self.moments.values():
+            m.zero_()
+            v.zero_()
+        self.t = 0
+
+    def args(self, X, Y_ref) -> StepArgs:
+        mo = self.moments
+        return StepArgs(
+            M=self.M, N=self.N, K=self.K, group=self.group, bits=self.bits, abits=self.abits,
+            let=1 if self.let else 0, dt=_dt(self.W), X=_ptr(X), W=_ptr(self.W), B=_ptr(self.B),
+            Y_ref=_ptr(Y_ref), gamma_logit=_ptr(self.gamma_logit), beta_logit=_ptr(self.beta_logit),
+            s=_ptr(self.s), delta=_ptr(self.delta),
+            m_gamma=_ptr(mo["gamma"][0]), v_gamma=_ptr(mo["gamma"][1]),
+            m_beta=_ptr(mo["beta"][0]), v_beta=_ptr(mo["beta"][1]),
+            m_s=_ptr(mo["s"][0]), v_s=_ptr(mo["s"][1]),
+            m_delta=_ptr(mo["delta"][0]), v_delta=_ptr(mo["delta"][1]),
+            Xq=_ptr(self.Xq), W_hat=_ptr(self.W_hat), B_tilde=_ptr(self.B_tilde), h=_ptr(self.h),
+            z=_ptr(self.z), grp_range=_ptr(self.grp_range), h_a=_ptr(self.h_a), z_a=_ptr(self.z_a),
+            tok_range=_ptr(self.tok_range), dY=_ptr(self.dY), d_gamma_logit=_ptr(self.d_gamma),
+            d_beta_logit=_ptr(self.d_beta), d_s=_ptr(self.d_s), d_delta=_ptr(self.d_delta),
+            loss=_ptr(self.loss), lr_lwc=self.lr_lwc, lr_let=self.lr_let, step=self.t)
+
+    def step(self, X, Y_ref, stream=None):
+        _dev(X, Y_ref)
+        self.t += 1
+        a = self.args(X, Y_ref)
+        _check(_lib.omq_calib_step(ctypes.byref(a), _ptr(self.workspace), self.workspace.numel(),
+                                   _stream(stream)), "omq_calib_step")
+        return self.loss
+
+    def reference_output(self, X, stream=None):
+        """Y* = X W^T + B with the library's own GEMM (computed once, outside the step)."""
+        return fq_linear_fwd(X, self.W, B_tilde=self.B, stream=stream)["Y"]
