@@ -1,0 +1,410 @@
+#!/usr/bin/env python
+"""Benchmark: OmniQuant fake-quantized linear calibration steps per second on B200.
+
+A step is one pass of the whole hot path over one calibration batch: LET (activation and
+weight side), LWC fake-quant of the weight, per-token activation fake-quant (when
+configured), the tcgen05 forward GEMM with the fused bias / MSE / dY epilogue, the
+straight-through backward (dW^ and dXq GEMMs, STE reductions, LET gradients) and the AdamW
+update, all through one omq_calib_step call on one stream. Inputs are synthetic and
+resident in HBM when the timed region starts (they follow the LLaMA-7B q_proj shape by
+default: 2048 tokens x 4096 -> 4096, W4A16, group 128, LET learnable).
+
+One process per GPU (torchrun for N > 1): each rank calibrates its own independent layer
+(different seed), with no collective on the data path; the timed region is bracketed by a
+barrier and device synchronisation and its length is the maximum over ranks.
+
+Also printed on the same JSON line: the roofline of the dominant kernel (the tcgen05 GEMM,
+timed with CUDA events around its launches inside the timed region), the CPU oracle timed
+on the host as a reported baseline, an end-to-end figure through the same C ABI with the
+step's inputs copied from pinned host memory inside the timed region, and the SM clocks
+sampled during the timed region.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl reference]
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fake-quant linear fwd+bwd calib steps/s; TFLOP/s & GB/s as % of roofline"
+UNIT = "steps/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="llama7b_qproj_w4a16g128")
+    ap.add_argument("--impl", default="omq", choices=["omq", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in ("gemm_tc.cu", "gemm_epilogue.cuh", "omq_internal.cuh"):
+        with open(os.path.join(ROOT, "post_quantization_lwc_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch of the GEMM kernel from a committed ncu summary, when the kernel
+    source has not changed since the counters were taken; otherwise None."""
+    path = os.path.join(ROOT, "profiles", "gemm_tc_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    if rec.get("source_sha") != kernel_source_hash():
+        return None
+    return rec.get("bytes_per_launch", {}).get(workload)
+
+
+def step_flops(cfg) -> int:
+    """Dense contractions of one step: forward, dW^ and (LET learnable) dXq GEMMs."""
+    n_gemm = 3 if cfg.let else 2
+    return n_gemm * 2 * cfg.m_tokens * cfg.n_out * cfg.k_in
+
+
+def phase_bytes(cfg) -> dict:
+    """Compulsory DRAM bytes of the HBM-bound phases (inputs read once, outputs written once)."""
+    es = 4 if cfg.dtype == "f32" else 2
+    M, N, K, ng = cfg.m_tokens, cfg.n_out, cfg.k_in, cfg.n_groups
+    act = cfg.let or cfg.abits < 16
+    out = {
+        "lwc": 2 * es * N * K + N * ng * (4 + 4 + 4 + 4 + 16) + 4 * K,
+        "ste_w": es * N * K + 4 * N * K + N * ng * (4 + 4 + 4 + 4 + 16 + 4 + 4),
+        "dbias": es * M * N if cfg.let else 0,
+    }
+    if act:
+        out["let"] = 2 * es * M * K + (es * N * K if cfg.let else 0)
+    if cfg.let:
+        out["ste_x"] = es * M * K + 4 * M * K
+    return out
+
+
+class ClockSampler(threading.Thread):
+    """Polls NVML for the SM clock and the clock-event reasons while running."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, index: int, period_s: float = 0.005):
+        super().__init__(daemon=True)
+        self.period = period_s
+        self.samples = []
+        self.reasons = 0
+        self.ok = False
+        self._halt = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.nv = None
+
+    def run(self):
+        if not self.ok:
+            return
+        while not self._halt.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= int(self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def stop(self):
+        self._halt.set()
+        self.join(timeout=2)
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": getattr(self, "max_mhz", None), "reasons": [],
+                    "samples": 0}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": [n for b, n in self.REASONS.items() if self.reasons & b and b != 0x1],
+                "samples": len(self.samples)}
+
+
+def workload_config(cfg):
+    return {"workload": cfg.name, "M_tokens": cfg.m_tokens, "K_in": cfg.k_in, "N_out": cfg.n_out,
+            "group": cfg.group, "bits": cfg.bits, "abits": cfg.abits, "let": cfg.let,
+            "storage": cfg.dtype}
+
+
+# ----------------------------------------------------------------------------- oracle (CPU)
+
+def oracle_sample(cfg, inp, rows: int | None):
+    """A bounded sample of the workload for the CPU oracle: the first `rows` output rows
+    (the whole layer when None). Returns numpy inputs and the fraction of the layer."""
+    import numpy as np
+
+    from oracle import omniquant as om
+    from post_quantization_lwc_b200 import synth
+    X = synth.as_f32_numpy(inp.X)
+    W = synth.as_f32_numpy(inp.W)
+    n = cfg.n_out if rows is None else rows
+    W = np.ascontiguousarray(W[:n])
+    Yref = om.reference_output(X, W, inp.B.numpy()[:n]).astype(np.float32)
+    return dict(X=X, W=W, B=inp.B.numpy()[:n], Yref=Yref, gl=inp.gamma_logit.numpy()[:n],
+                bl=inp.beta_logit.numpy()[:n], s=inp.s.numpy(), d=inp.delta.numpy()), n / cfg.n_out
+
+
+def oracle_steps(cfg, smp, steps: int):
+    from oracle import omniquant as om
+    return om.calibrate(smp["X"], smp["W"], smp["B"], smp["Yref"], smp["gl"], smp["bl"], smp["s"],
+                        smp["d"], cfg.bits, cfg.group, cfg.abits, cfg.let, steps)
+
+
+def blas_threads() -> int:
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        return max([i.get("num_threads", 1) for i in info if i.get("user_api") == "blas"] or [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(cfg, inp, budget_s: float = 20.0):
+    """Time the oracle (as it stands) on the host: whole steps of the full layer while they
+    fit the budget, else a row sample scaled to the layer."""
+    smp, frac = oracle_sample(cfg, inp, None)
+    t0 = time.perf_counter()
+    oracle_steps(cfg, smp, 1)
+    t1 = time.perf_counter() - t0
+    steps = max(1, min(5, int(budget_s / max(t1, 1e-3)) - 1))
+    t0 = time.perf_counter()
+    oracle_steps(cfg, smp, steps)
+    dt = time.perf_counter() - t0
+    return {"value": steps * frac / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{steps} whole calibration step(s) of the full {cfg.name} layer "
+                      f"(numpy binary64 oracle, after one untimed step), {dt:.1f} s"}
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def run_reference(args, cfg, rank: int, world: int):
+    if rank != 0:
+        return 0
+    from post_quantization_lwc_b200 import synth
+    inp = synth.make_inputs(cfg)
+    smp, frac = oracle_sample(cfg, inp, None)
+    t0 = time.perf_counter()
+    oracle_steps(cfg, smp, 1)
+    t1 = time.perf_counter() - t0
+    total = (args.steps + args.warmup) * t1
+    rows = None
+    if total > 150.0:   # keep the whole run within a few minutes: sample output rows
+        rows = max(8, int(cfg.n_out * 150.0 / total) // 8 * 8)
+        smp, frac = oracle_sample(cfg, inp, rows)
+    if args.warmup > 1:
+        oracle_steps(cfg, smp, args.warmup - 1)
+    t0 = time.perf_counter()
+    oracle_steps(cfg, smp, args.steps)
+    dt = time.perf_counter() - t0
+    value = args.steps * frac / dt
+    sample = (f"whole {cfg.name} layer per step" if rows is None else
+              f"first {rows} of {cfg.n_out} output rows per step, throughput scaled by "
+              f"{cfg.n_out}/{rows}")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / value,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {**workload_config(cfg), "parallelism": "host cores"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- libomq arm
+
+def run_omq(args, cfg, rank: int, world: int, local_rank: int):
+    import torch
+    import torch.distributed as dist
+
+    from post_quantization_lwc_b200 import omq, synth
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    import dataclasses
+    my_cfg = dataclasses.replace(cfg, seed=cfg.seed + 1000 * rank) if rank else cfg
+    inp = synth.make_inputs(my_cfg)
+    dt = torch.float32 if cfg.dtype == "f32" else torch.bfloat16
+    lc = omq.LinearCalibration(M=cfg.m_tokens, N=cfg.n_out, K=cfg.k_in, group=cfg.group,
+                               bits=cfg.bits, abits=cfg.abits, let=cfg.let, dtype=dt, device=dev)
+    lc.load(inp.W.to(dev), inp.gamma_logit.to(dev), inp.beta_logit.to(dev), s=inp.s.to(dev),
+            delta=inp.delta.to(dev), B=inp.B.to(dev))
+    X = inp.X.to(dev).contiguous()
+    Yref = lc.reference_output(X).contiguous()
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        lc.step(X, Yref)
+    torch.cuda.synchronize()
+    omq.sync_check()
+
+    timer = omq.PhaseTimer(args.steps)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev.index)
+    barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    n0 = omq.launch_count()
+    ev0.record()
+    for i in range(args.steps):
+        lc.step(X, Yref, events=timer.sets[i])
+    ev1.record()
+    torch.cuda.synchronize()
+    n1 = omq.launch_count()
+    sampler.stop()
+    barrier()
+    omq.sync_check()
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    phases = timer.mean_ms()
+    last_loss = float(lc.loss.item())
+
+    # end to end through the same C ABI: each step's X and Y* come from pinned host memory
+    e2e = None
+    if not args.no_e2e:
+        Xh = inp.X.pin_memory()
+        Yh = Yref.cpu().pin_memory()
+        lh = torch.empty(1, dtype=torch.float32).pin_memory()
+        Xd, Yd = torch.empty_like(X), torch.empty_like(Yref)
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            Xd.copy_(Xh, non_blocking=True)
+            Yd.copy_(Yh, non_blocking=True)
+            lc.step(Xd, Yd)
+            lh.copy_(lc.loss, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        barrier()
+        ems = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([ems], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        e2e = {"value": world * args.steps / (ems / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": Xh.numel() * Xh.element_size() + Yh.numel() * Yh.element_size(),
+               "d2h_bytes_per_step": 4}
+
+    if rank != 0:
+        return 0
+
+    peaks, peak_src = load_peaks()
+    value = world * args.steps / (ms / 1e3)
+    gemm_keys = [k for k in ("fwd_gemm", "dw_gemm", "dx_gemm") if phases[k] > 0.0005]
+    gemm_ms = sum(phases[k] for k in gemm_keys) / len(gemm_keys)
+    gemm_flops = 2 * cfg.m_tokens * cfg.n_out * cfg.k_in
+    achieved = gemm_flops / (gemm_ms * 1e-3) / 1e12
+    timed_s = ms / 1e3
+    peak_key = "bf16_tflops" if timed_s < 1.0 else "bf16_tflops_sustained"
+    peak = float(peaks.get(peak_key, FALLBACK_PEAKS[peak_key]))
+    pbytes = phase_bytes(cfg)
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    phase_report = {}
+    for k in omq.PHASES:
+        entry = {"us": round(phases[k] * 1e3, 2)}
+        if k in pbytes and phases[k] > 0.0005 and pbytes[k] > 0:
+            gbs = pbytes[k] / (phases[k] * 1e-3) / 1e9
+            entry.update({"gbs": round(gbs, 1), "hbm_frac": round(gbs / hbm, 3)})
+        if k in gemm_keys:
+            tf = gemm_flops / (phases[k] * 1e-3) / 1e12
+            entry.update({"tflops": round(tf, 1), "tc_frac": round(tf / peak, 3)})
+        phase_report[k] = entry
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if cfg.dtype == "bf16" else "f32",
+        "data": "synthetic (seeded LLaMA-shaped weights and outlier-channel activations)",
+        "config": {**workload_config(cfg),
+                   "l2": "no flush: the step's working set (W, W^, X, Xq, Y*, dY, dW^, dXq) "
+                         "exceeds the 126 MB L2",
+                   "parallelism": f"replicas x{world} (one independent layer per GPU)"},
+        "tflops": step_flops(cfg) * value / 1e12,
+        "roofline": {"bound": "tensor", "kernel": "gemm_tc_kernel", "achieved": achieved,
+                     "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "traffic": recorded_traffic(cfg.name),
+                     "peak_source": f"{peak_key} of {peak_src}",
+                     "per_launch": f"2*M*N*K = {gemm_flops / 1e9:.1f} GFLOP over the average "
+                                   f"duration of the {len(gemm_keys)} GEMM launches per step"},
+        "phases": phase_report,
+        "loss": last_loss,
+        "gpu_launches": int(n1 - n0),
+        "clocks": sampler.summary(),
+    }
+    if e2e is not None:
+        line["e2e"] = e2e
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg, inp)
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    from post_quantization_lwc_b200 import synth
+    cfg = synth.CONFIGS[args.config]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, cfg, rank, world)
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        return run_omq(args, cfg, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -221,10 +221,28 @@ omq_status omq_fold_pack(const void* W, omq_dtype wdt, int64_t N, int64_t K, int
  * omq_calib_step — one whole calibration step on one stream: omq_let_apply (when LET is
  * on or abits < 16), omq_lwc_quant, omq_fq_linear_fwd, omq_fq_linear_bwd, then AdamW on
  * the logits (lr_lwc) and, with LET, on s and delta (lr_let). `step` counts from 1.
- * All buffers are caller-owned device memory; Xq may alias X only when LET is off and
- * abits == 16 (then X is the GEMM operand as is). Workspace:
- * omq_step_workspace_bytes(M, N, K, group).
+ * All buffers are caller-owned device memory. When LET is off and abits == 16, X itself is
+ * the GEMM operand and Xq is not used. Workspace: omq_step_workspace_bytes(M, N, K, group).
+ *
+ * Per-phase timing: `events` is NULL or an array of OMQ_PH_COUNT + 1 cudaEvent_t (passed
+ * as void*). Event i is recorded on `stream` when phase i starts and event OMQ_PH_COUNT
+ * when the step ends; phases that do not run are recorded back to back (zero length).
  * ------------------------------------------------------------------------------------ */
+enum {
+  OMQ_PH_LET = 0,       /* omq_let_apply: X~, per-token act quant, B~ */
+  OMQ_PH_LWC,           /* omq_lwc_quant */
+  OMQ_PH_FWD_GEMM,      /* forward GEMM with the bias / MSE / dY epilogue */
+  OMQ_PH_LOSS,          /* loss reduction */
+  OMQ_PH_DBIAS,         /* dB~ = column sums of dY */
+  OMQ_PH_DW_GEMM,       /* dW^ = dY^T Xq */
+  OMQ_PH_STE_W,         /* weight-side STE and LWC parameter gradients */
+  OMQ_PH_DX_GEMM,       /* dXq = dY W^ */
+  OMQ_PH_STE_X,         /* activation-side STE and LET column partials */
+  OMQ_PH_LET_REDUCE,    /* d_s, d_delta reductions */
+  OMQ_PH_ADAMW,         /* parameter updates */
+  OMQ_PH_COUNT
+};
+
 typedef struct {
   int64_t M, N, K, group;
   int bits, abits, let;           /* let != 0: s, delta learnable */
@@ -241,11 +259,16 @@ typedef struct {
   float* loss;                    /* device scalar */
   float lr_lwc, lr_let;
   int64_t step;
+  void* const* events;            /* NULL, or OMQ_PH_COUNT + 1 cudaEvent_t */
 } omq_step_args;
 
 omq_status omq_calib_step(const omq_step_args* args, void* workspace, size_t ws_bytes,
                           omq_stream_t stream);
 size_t omq_step_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t group);
+
+/* Number of kernels this library has launched in this process (all threads, all devices),
+ * counted on the host at each launch. */
+uint64_t omq_launch_count(void);
 
 #ifdef __cplusplus
 }

@@ -1,5 +1,6 @@
 // The libomq C ABI: host-side validation, workspace layout and launch sequencing of the
 // fake-quantized linear calibration step. Nothing here allocates device memory.
+#include <atomic>
 #include <cstdio>
 #include <mutex>
 #include <vector>
@@ -70,6 +71,21 @@ bool a16(const void* p) { return p == nullptr || aligned16(p); }
     if (_s != OMQ_OK) return _s;      \
   } while (0)
 
+// Optional per-phase event recording of omq_calib_step (see OMQ_PH_* in omq.h).
+struct Phases {
+  void* const* ev = nullptr;
+  cudaStream_t st = nullptr;
+  omq_status mark(int i) const {
+    if (!ev) return OMQ_OK;
+    cudaError_t e = cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), st);
+    if (e != cudaSuccess) {
+      t_last_cuda_error = static_cast<int>(e);
+      return OMQ_ERR_CUDA;
+    }
+    return OMQ_OK;
+  }
+};
+
 omq_status check_lwc(const void* W, omq_dtype wdt, int64_t N, int64_t K, int64_t group, int bits,
                      const float* gl, const float* bl, const float* s, omq_dtype hat_dt,
                      const void* W_hat, const void* codes, const void* h, const void* z) {
@@ -87,7 +103,10 @@ omq_status check_lwc(const void* W, omq_dtype wdt, int64_t N, int64_t K, int64_t
 
 void set_cuda_error(cudaError_t e) { t_last_cuda_error = static_cast<int>(e); }
 
+static std::atomic<uint64_t> g_launches{0};
+
 omq_status launch_status() {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_cuda_error(e);
@@ -213,10 +232,10 @@ static omq_status run_gemm(omq_dtype dt, const GemmOperand& A, const GemmOperand
   return gemm_f32_simt(A, B, rows, cols, depth, epi, tiles, st);
 }
 
-omq_status omq_fq_linear_fwd(const void* Xq, const void* W_hat, omq_dtype dt, int64_t M,
-                             int64_t N, int64_t K, const float* B_tilde, const float* Y_ref,
-                             float* Y, void* dY, float* loss, void* workspace, size_t ws_bytes,
-                             omq_stream_t stream) {
+static omq_status fwd_impl(const void* Xq, const void* W_hat, omq_dtype dt, int64_t M, int64_t N,
+                           int64_t K, const float* B_tilde, const float* Y_ref, float* Y, void* dY,
+                           float* loss, void* workspace, size_t ws_bytes, omq_stream_t stream,
+                           const Phases& ph) {
   if (!Xq || !W_hat) return OMQ_ERR_NULL;
   if (!dtype_ok(dt)) return OMQ_ERR_DTYPE;
   if (M < 1 || N < 8 || K < 8 || N % 8 || K % 8 || M > kMaxDim || N > kMaxDim || K > kMaxDim)
@@ -247,11 +266,21 @@ omq_status omq_fq_linear_fwd(const void* Xq, const void* W_hat, omq_dtype dt, in
     epi.out = Y;
   }
   int64_t tiles = 0;
+  OMQ_TRY(ph.mark(OMQ_PH_FWD_GEMM));
   OMQ_TRY(run_gemm(dt, A, B, M, N, K, epi, &tiles, st));
+  OMQ_TRY(ph.mark(OMQ_PH_LOSS));
   if (Y_ref && loss)
     OMQ_TRY(launch_loss_finalize(epi.loss_partials, tiles,
                                  1.0 / (static_cast<double>(M) * static_cast<double>(N)), loss, st));
   return OMQ_OK;
+}
+
+omq_status omq_fq_linear_fwd(const void* Xq, const void* W_hat, omq_dtype dt, int64_t M,
+                             int64_t N, int64_t K, const float* B_tilde, const float* Y_ref,
+                             float* Y, void* dY, float* loss, void* workspace, size_t ws_bytes,
+                             omq_stream_t stream) {
+  return fwd_impl(Xq, W_hat, dt, M, N, K, B_tilde, Y_ref, Y, dY, loss, workspace, ws_bytes, stream,
+                  Phases{});
 }
 
 size_t omq_bwd_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t group) {
@@ -259,8 +288,8 @@ size_t omq_bwd_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t group) {
   return bwd_layout(M, N, K, group).total;
 }
 
-omq_status omq_fq_linear_bwd(const omq_bwd_args* a, void* workspace, size_t ws_bytes,
-                             omq_stream_t stream) {
+static omq_status bwd_impl(const omq_bwd_args* a, void* workspace, size_t ws_bytes,
+                           omq_stream_t stream, const Phases& ph) {
   if (!a) return OMQ_ERR_NULL;
   const int64_t M = a->M, N = a->N, K = a->K, G = a->group;
   if (!a->W || !a->Xq || !a->W_hat || !a->h || !a->z || !a->grp_range || !a->dY ||
@@ -295,11 +324,13 @@ omq_status omq_fq_linear_bwd(const omq_bwd_args* a, void* workspace, size_t ws_b
   float* part_xd = at<float>(workspace, L.part_xd);
 
   // dB~ = column sums of dY (needed for d_delta, or when asked for)
+  OMQ_TRY(ph.mark(OMQ_PH_DBIAS));
   if (a->d_delta || a->d_B_tilde) {
     OMQ_TRY(launch_colsum(a->dY, a->dt, M, N, kRowsColsum, dbt_part, st));
     OMQ_TRY(launch_reduce_cols(dbt_part, L.rb_colsum, nullptr, 0, N, dbt, st));
   }
   // dW^ = dY^T Xq   [N, K]
+  OMQ_TRY(ph.mark(OMQ_PH_DW_GEMM));
   {
     GemmOperand A{a->dY, N, true}, B{a->Xq, K, true};
     GemmEpilogue epi{};
@@ -308,6 +339,7 @@ omq_status omq_fq_linear_bwd(const omq_bwd_args* a, void* workspace, size_t ws_b
     OMQ_TRY(run_gemm(a->dt, A, B, N, K, M, epi, nullptr, st));
   }
   // weight-side STE: d gamma / d beta logits and the W-side LET column partials
+  OMQ_TRY(ph.mark(OMQ_PH_STE_W));
   {
     SteWParams p{a->W, a->dt, N, K, G, K / G, static_cast<float>((1 << a->bits) - 1),
                  a->s, a->gamma_logit, a->beta_logit, a->h, a->z,
@@ -316,7 +348,11 @@ omq_status omq_fq_linear_bwd(const omq_bwd_args* a, void* workspace, size_t ws_b
                  static_cast<int>(rows_per_block_w(G))};
     OMQ_TRY(launch_ste_w(p, st));
   }
-  if (!need_let) return OMQ_OK;
+  OMQ_TRY(ph.mark(OMQ_PH_DX_GEMM));
+  if (!need_let) {
+    OMQ_TRY(ph.mark(OMQ_PH_STE_X));
+    return ph.mark(OMQ_PH_LET_REDUCE);
+  }
   // dXq = dY W^   [M, K]
   {
     GemmOperand A{a->dY, N, false}, B{a->W_hat, K, true};
@@ -325,6 +361,7 @@ omq_status omq_fq_linear_bwd(const omq_bwd_args* a, void* workspace, size_t ws_b
     epi.out = dxq;
     OMQ_TRY(run_gemm(a->dt, A, B, M, K, N, epi, nullptr, st));
   }
+  OMQ_TRY(ph.mark(OMQ_PH_STE_X));
   {
     SteXParams p{a->X, a->dt, M, K,
                  static_cast<float>((1 << (a->abits < 16 ? a->abits : 1)) - 1),
@@ -332,9 +369,15 @@ omq_status omq_fq_linear_bwd(const omq_bwd_args* a, void* workspace, size_t ws_b
                  part_xd, kRowsX};
     OMQ_TRY(launch_ste_x(p, st));
   }
+  OMQ_TRY(ph.mark(OMQ_PH_LET_REDUCE));
   if (a->d_s) OMQ_TRY(launch_reduce_cols(part_ws, L.rb_w, part_xs, L.rb_x, K, a->d_s, st));
   if (a->d_delta) OMQ_TRY(launch_reduce_cols(part_wd, L.rb_w, part_xd, L.rb_x, K, a->d_delta, st));
   return OMQ_OK;
+}
+
+omq_status omq_fq_linear_bwd(const omq_bwd_args* a, void* workspace, size_t ws_bytes,
+                             omq_stream_t stream) {
+  return bwd_impl(a, workspace, ws_bytes, stream, Phases{});
 }
 
 omq_status omq_adamw_step(float* param, const float* grad, float* m, float* v, int64_t n, float lr,
@@ -374,16 +417,19 @@ omq_status omq_calib_step(const omq_step_args* a, void* workspace, size_t ws_byt
   if (!workspace || ws_bytes < omq_step_workspace_bytes(M, N, K, G)) return OMQ_ERR_WORKSPACE;
   const void* Xq = need_act ? a->Xq : a->X;
   const float* Bt = let ? a->B_tilde : a->B;
+  Phases ph{a->events, reinterpret_cast<cudaStream_t>(stream)};
+  OMQ_TRY(ph.mark(OMQ_PH_LET));
   if (need_act) {
     OMQ_TRY(omq_let_apply(a->X, a->dt, M, K, let ? a->s : nullptr, let ? a->delta : nullptr,
                           a->abits, a->Xq, a->dt, a->h_a, a->z_a, a->tok_range, a->W, a->dt, N,
                           a->B, let ? a->B_tilde : nullptr, stream));
   }
+  OMQ_TRY(ph.mark(OMQ_PH_LWC));
   OMQ_TRY(omq_lwc_quant(a->W, a->dt, N, K, G, a->bits, a->gamma_logit, a->beta_logit,
                         let ? a->s : nullptr, a->W_hat, a->dt, a->h, a->z, nullptr, a->grp_range,
                         stream));
-  OMQ_TRY(omq_fq_linear_fwd(Xq, a->W_hat, a->dt, M, N, K, Bt, a->Y_ref, nullptr, a->dY, a->loss,
-                            workspace, fwd_ws, stream));
+  OMQ_TRY(fwd_impl(Xq, a->W_hat, a->dt, M, N, K, Bt, a->Y_ref, nullptr, a->dY, a->loss, workspace,
+                   fwd_ws, stream, ph));
   omq_bwd_args b{};
   b.M = M; b.N = N; b.K = K; b.group = G; b.bits = a->bits; b.abits = a->abits; b.dt = a->dt;
   b.X = a->X; b.W = a->W; b.s = let ? a->s : nullptr; b.delta = let ? a->delta : nullptr;
@@ -392,8 +438,8 @@ omq_status omq_calib_step(const omq_step_args* a, void* workspace, size_t ws_byt
   b.h_a = a->h_a; b.z_a = a->z_a; b.tok_range = a->tok_range; b.dY = a->dY;
   b.d_gamma_logit = a->d_gamma_logit; b.d_beta_logit = a->d_beta_logit;
   b.d_s = let ? a->d_s : nullptr; b.d_delta = let ? a->d_delta : nullptr;
-  OMQ_TRY(omq_fq_linear_bwd(&b, static_cast<char*>(workspace) + fwd_ws, ws_bytes - fwd_ws,
-                            stream));
+  OMQ_TRY(bwd_impl(&b, static_cast<char*>(workspace) + fwd_ws, ws_bytes - fwd_ws, stream, ph));
+  OMQ_TRY(ph.mark(OMQ_PH_ADAMW));
   const int64_t ng = N * (K / G);
   OMQ_TRY(omq_adamw_step(a->gamma_logit, a->d_gamma_logit, a->m_gamma, a->v_gamma, ng, a->lr_lwc,
                          0.9f, 0.999f, 1e-8f, 0.f, a->step, stream));
@@ -405,7 +451,9 @@ omq_status omq_calib_step(const omq_step_args* a, void* workspace, size_t ws_byt
     OMQ_TRY(omq_adamw_step(a->delta, a->d_delta, a->m_delta, a->v_delta, K, a->lr_let, 0.9f,
                            0.999f, 1e-8f, 0.f, a->step, stream));
   }
-  return OMQ_OK;
+  return ph.mark(OMQ_PH_COUNT);
 }
+
+uint64_t omq_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 }  // extern "C"

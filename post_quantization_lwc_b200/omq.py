@@ -29,7 +29,7 @@ STATUS = {0: "OMQ_OK", 1: "OMQ_ERR_NULL", 2: "OMQ_ERR_SHAPE", 3: "OMQ_ERR_DTYPE"
 EXPORTS = ("omq_status_str", "omq_last_cuda_error", "omq_version", "omq_sync_check",
            "omq_lwc_quant", "omq_let_apply", "omq_fq_linear_fwd", "omq_fwd_workspace_bytes",
            "omq_fq_linear_bwd", "omq_bwd_workspace_bytes", "omq_adamw_step", "omq_fold_pack",
-           "omq_calib_step", "omq_step_workspace_bytes")
+           "omq_calib_step", "omq_step_workspace_bytes", "omq_launch_count")
 
 _p = ctypes.c_void_p
 _i64 = ctypes.c_int64
@@ -68,7 +68,13 @@ class StepArgs(ctypes.Structure):
                 ("h_a", _p), ("z_a", _p), ("tok_range", _p),
                 ("dY", _p),
                 ("d_gamma_logit", _p), ("d_beta_logit", _p), ("d_s", _p), ("d_delta", _p),
-                ("loss", _p), ("lr_lwc", _f32), ("lr_let", _f32), ("step", _i64)]
+                ("loss", _p), ("lr_lwc", _f32), ("lr_let", _f32), ("step", _i64),
+                ("events", _p)]
+
+
+# phases of omq_calib_step (OMQ_PH_* in include/omq.h), in order
+PHASES = ("let", "lwc", "fwd_gemm", "loss", "dbias", "dw_gemm", "ste_w", "dx_gemm", "ste_x",
+          "let_reduce", "adamw")
 
 
 def _sig(name, res, args):
@@ -93,6 +99,7 @@ _sig("omq_adamw_step", _i32, [_p, _p, _p, _p, _i64, _f32, _f32, _f32, _f32, _f32
 _sig("omq_fold_pack", _i32, [_p, _i32, _i64, _i64, _i64, _i32, _p, _p, _p, _p, _p, _p, _p])
 _sig("omq_calib_step", _i32, [ctypes.POINTER(StepArgs), _p, _sz, _p])
 _sig("omq_step_workspace_bytes", _sz, [_i64, _i64, _i64, _i64])
+_sig("omq_launch_count", ctypes.c_uint64, [])
 
 
 def _check(status: int, where: str):
@@ -129,6 +136,11 @@ def _dev(*ts):
 
 def version() -> int:
     return _lib.omq_version()
+
+
+def launch_count() -> int:
+    """Kernels launched by the library so far in this process."""
+    return int(_lib.omq_launch_count())
 
 
 def sync_check(stream=None):
@@ -348,10 +360,15 @@ class LinearCalibration:
             d_beta_logit=_ptr(self.d_beta), d_s=_ptr(self.d_s), d_delta=_ptr(self.d_delta),
             loss=_ptr(self.loss), lr_lwc=self.lr_lwc, lr_let=self.lr_let, step=self.t)
 
-    def step(self, X, Y_ref, stream=None):
+    def step(self, X, Y_ref, stream=None, events=None):
+        """One calibration step. ``events``: None, or len(PHASES) + 1 timing-enabled
+        torch.cuda.Event objects recorded at the phase boundaries (see PhaseTimer)."""
         _dev(X, Y_ref)
         self.t += 1
         a = self.args(X, Y_ref)
+        if events is not None:
+            arr = (ctypes.c_void_p * (len(PHASES) + 1))(*[e.cuda_event for e in events])
+            a.events = ctypes.cast(arr, ctypes.c_void_p)
         _check(_lib.omq_calib_step(ctypes.byref(a), _ptr(self.workspace), self.workspace.numel(),
                                    _stream(stream)), "omq_calib_step")
         return self.loss
@@ -359,3 +376,24 @@ class LinearCalibration:
     def reference_output(self, X, stream=None):
         """Y* = X W^T + B with the library's own GEMM (computed once, outside the step)."""
         return fq_linear_fwd(X, self.W, B_tilde=self.B, stream=stream)["Y"]
+
+
+class PhaseTimer:
+    """Per-step sets of CUDA events for omq_calib_step's phase boundaries."""
+
+    def __init__(self, n_steps: int):
+        self.sets = []
+        for _ in range(n_steps):
+            evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(PHASES) + 1)]
+            for e in evs:          # create the underlying cudaEvent_t now
+                e.record()
+            self.sets.append(evs)
+        torch.cuda.synchronize()
+
+    def mean_ms(self):
+        """Average duration of each phase over the recorded steps (call after a sync)."""
+        tot = [0.0] * len(PHASES)
+        for evs in self.sets:
+            for i in range(len(PHASES)):
+                tot[i] += evs[i].elapsed_time(evs[i + 1])
+        return {p: t / len(self.sets) for p, t in zip(PHASES, tot)}

@@ -21,7 +21,7 @@ def omq():
 
 def header_functions():
     text = open(HEADER).read()
-    return sorted(set(re.findall(r"^\s*(?:omq_status|const char\*|int|size_t)\s+(omq_\w+)\(",
+    return sorted(set(re.findall(r"^\s*(?:omq_status|const char\*|int|size_t|uint64_t)\s+(omq_\w+)\(",
                                  text, re.M)))
 
 

@@ -172,16 +172,30 @@ def test_calib_step_through_one_call(omq, cuda_device, case):
     assert abs(loss.item() - r.loss) <= (1e-4 if case.dtype == "f32" else 2e-2) * r.loss
     ok, e = close(_np(lc.d_gamma), r.d_gamma_logit, case.dtype)
     assert ok, e
-    # AdamW step 1 moves every logit by lr * g / (|g| + eps): +-lr where |g| >> eps
-    gl_new, _, _ = om.adamw_step(p.gl.numpy(), r.d_gamma_logit, 0, 0, 1, om.LR_LWC)
-    big = np.abs(r.d_gamma_logit) > 1e-4 * np.abs(r.d_gamma_logit).max()
-    assert np.abs(_np(lc.gamma_logit)[big] - gl_new[big]).max() <= 1e-5
+    # AdamW step 1 moves a parameter by lr * g / (|g| + eps): about lr * sign(g) once |g| >> eps.
+    # Two gradients g1 = g, g2 = g (1 + r) of the same sign give moves that differ by about
+    # lr * eps * |r| / |g|: below 1e-10 for |g| > 1e-6, so there the updates agree to 1e-5
+    # (binary32 rounding of the parameter) unless the sign differs. bf16 GEMM operands bound
+    # the gradient's error in norm (2e-2 of ||g||), not per element, so the sign is only
+    # reliable well above the noise: elements with |g| > 0.1 rms(g) must agree (99%). The
+    # AdamW arithmetic itself is pinned separately; this checks the step's wiring.
+    def check_update(new_gpu, old, grad_oracle, lr):
+        moved = _np(new_gpu) - old
+        assert np.abs(moved).max() <= lr * 1.0001
+        want, _, _ = om.adamw_step(old, grad_oracle, 0, 0, 1, lr)
+        rms = np.sqrt(np.mean(np.square(grad_oracle)))
+        big = np.abs(grad_oracle) > max(1e-6, 0.1 * rms)
+        assert big.any()
+        agree = np.abs(_np(new_gpu)[big] - want[big]) <= 1e-5
+        assert agree.mean() >= 0.99
+
+    check_update(lc.gamma_logit, p.gl.numpy(), r.d_gamma_logit, om.LR_LWC)
+    check_update(lc.beta_logit, p.bl.numpy(), r.d_beta_logit, om.LR_LWC)
     if case.let:
         ok, e = close(_np(lc.d_s), r.d_s, case.dtype)
         assert ok, e
-        s_new, _, _ = om.adamw_step(p.s.numpy(), r.d_s, 0, 0, 1, om.LR_LET)
-        big = np.abs(r.d_s) > 1e-3 * np.abs(r.d_s).max()
-        assert np.abs(_np(lc.s)[big] - s_new[big]).max() <= 1e-5
+        check_update(lc.s, p.s.numpy(), r.d_s, om.LR_LET)
+        check_update(lc.delta, p.delta.numpy(), r.d_delta, om.LR_LET)
 
 
 @pytest.mark.parametrize("case", [c for c in SMALL_CASES if c.bits in (2, 4, 8)],
