@@ -148,6 +148,30 @@ omq_status omq_fq_linear_fwd(const void* Xq, const void* W_hat, omq_dtype dt, in
 size_t omq_fwd_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /* ------------------------------------------------------------------------------------
+ * omq_fq_linear_fwd_noalloc — omq_fq_linear_fwd (with the loss) for callers that cannot
+ * supply device scratch memory. The paper has no counterpart: this is a library convenience.
+ *
+ * Some hosts own every device allocation and give a plug-in library no way to obtain
+ * scratch (a framework with its own memory pool and no allocation hook, or a runtime that
+ * forbids device allocation after start-up). For them this call keeps its scratch (one
+ * float per output tile) in a fixed array compiled into the library and allocates nothing.
+ * Arguments are those of omq_fq_linear_fwd without the workspace; Y_ref, dY and loss are
+ * required, Y may be NULL.
+ *   - Limit: ceil(M/128)*ceil(N/256) (bf16) or ceil(M/64)*ceil(N/64) (float32) must not
+ *     exceed 16384; larger problems return OMQ_ERR_SHAPE and launch nothing.
+ *   - The array (64 KiB) is held on every GPU that loads the library until the process exits.
+ *   - All calls on a device share it and it keeps the last call's contents; each call writes
+ *     every slot it reads first, so nothing needs clearing. Calls that overlap on the GPU
+ *     (unordered streams) race on it: order them on one stream.
+ *   - The first call on a device looks up the array's address with that device current; make
+ *     that first call before any stream capture begins.
+ * ------------------------------------------------------------------------------------ */
+omq_status omq_fq_linear_fwd_noalloc(const void* Xq, const void* W_hat, omq_dtype dt, int64_t M,
+                                     int64_t N, int64_t K, const float* B_tilde,
+                                     const float* Y_ref, float* Y, void* dY, float* loss,
+                                     omq_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
  * omq_fq_linear_bwd — straight-through backward of the step ([EDGE] section 2.2; the
  * formulas of [ICLR] sections LWC and LET differentiated as written).
  *

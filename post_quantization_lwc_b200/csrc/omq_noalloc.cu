@@ -1,0 +1,102 @@
+// omq_fq_linear_fwd_noalloc: the fake-quantized linear forward and loss of
+// omq_fq_linear_fwd, for callers that cannot supply device scratch memory.
+//
+// Who needs it: some hosts own every device allocation themselves. Examples are a framework
+// that routes all device memory through its own pool and gives plug-ins no allocation hook,
+// or a runtime that forbids device allocation once it has started. Such a host cannot call
+// cudaMalloc for this library's workspace and has no workspace of its own to lend. This entry
+// point keeps its scratch (one float per output tile: the partial sums of the squared error)
+// in a fixed array compiled into the library. The caller still passes every input and output
+// buffer, and the call allocates nothing.
+//
+// Limits and sharing:
+//   - The array holds kNoAllocTiles partial sums. A problem needs ceil(M/128) * ceil(N/256)
+//     of them on the bf16 tensor-core path, or ceil(M/64) * ceil(N/64) on the float32 path;
+//     larger problems are rejected with OMQ_ERR_SHAPE before anything is launched.
+//   - Every GPU that loads the library holds the array (64 KiB) until the process exits.
+//   - All calls on a device share the one array, and it keeps the last call's contents.
+//     Each call writes every slot it reads before reading it, so nothing needs clearing.
+//     Calls whose work overlaps on the GPU (different streams with no ordering between them)
+//     race on the array and may return a wrong loss; order such calls on one stream.
+//   - The first call on each device looks up the array's device address with that device
+//     current (cudaGetSymbolAddress) and keeps it; make that first call before any stream
+//     capture begins.
+#include <mutex>
+
+#include "omq_internal.cuh"
+
+namespace omq {
+namespace {
+
+constexpr int64_t kNoAllocTiles = 16384;
+constexpr int kMaxDevices = 64;
+
+static __device__ __align__(256) float g_noalloc_loss_partials[kNoAllocTiles];
+
+std::mutex g_noalloc_mu;
+float* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the fixed scratch array for the current device (looked up once).
+omq_status noalloc_scratch(float** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    set_cuda_error(e);
+    return OMQ_ERR_CUDA;
+  }
+  if (dev < 0 || dev >= kMaxDevices) return OMQ_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_loss_partials);
+    if (e != cudaSuccess || p == nullptr) {
+      set_cuda_error(e != cudaSuccess ? e : cudaErrorInvalidSymbol);
+      return OMQ_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = static_cast<float*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return OMQ_OK;
+}
+
+}  // namespace
+}  // namespace omq
+
+using namespace omq;
+
+extern "C" omq_status omq_fq_linear_fwd_noalloc(const void* Xq, const void* W_hat, omq_dtype dt,
+                                                int64_t M, int64_t N, int64_t K,
+                                                const float* B_tilde, const float* Y_ref,
+                                                float* Y, void* dY, float* loss,
+                                                omq_stream_t stream) {
+  if (!Xq || !W_hat || !Y_ref || !dY || !loss) return OMQ_ERR_NULL;
+  if (dt != OMQ_F32 && dt != OMQ_BF16) return OMQ_ERR_DTYPE;
+  const int64_t kMax = (int64_t(1) << 31) - 1;
+  if (M < 1 || N < 8 || K < 8 || N % 8 || K % 8 || M > kMax || N > kMax || K > kMax)
+    return OMQ_ERR_SHAPE;
+  if (!aligned16(Xq) || !aligned16(W_hat) || !aligned16(Y_ref) || !aligned16(dY) ||
+      (B_tilde && !aligned16(B_tilde)) || (Y && !aligned16(Y)))
+    return OMQ_ERR_ALIGN;
+  const int64_t tiles = dt == OMQ_BF16 ? gemm_bf16_tc_tiles(M, N) : gemm_f32_simt_tiles(M, N);
+  if (tiles > kNoAllocTiles) return OMQ_ERR_SHAPE;
+  float* partials = nullptr;
+  omq_status st = noalloc_scratch(&partials);
+  if (st != OMQ_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  GemmOperand A{Xq, K, false}, B{W_hat, K, false};
+  GemmEpilogue epi{};
+  epi.kind = Epi::MseLoss;
+  epi.bias = B_tilde;
+  epi.out = Y;
+  epi.y_ref = Y_ref;
+  epi.dy = dY;
+  epi.dy_dt = dt;
+  epi.dy_scale = static_cast<float>(2.0 / (static_cast<double>(M) * static_cast<double>(N)));
+  epi.loss_partials = partials;
+  int64_t launched = 0;
+  st = dt == OMQ_BF16 ? gemm_bf16_tc(A, B, M, N, K, epi, &launched, s)
+                      : gemm_f32_simt(A, B, M, N, K, epi, &launched, s);
+  if (st != OMQ_OK) return st;
+  return launch_loss_finalize(partials, launched,
+                              1.0 / (static_cast<double>(M) * static_cast<double>(N)), loss, s);
+}

@@ -29,7 +29,8 @@ STATUS = {0: "OMQ_OK", 1: "OMQ_ERR_NULL", 2: "OMQ_ERR_SHAPE", 3: "OMQ_ERR_DTYPE"
 EXPORTS = ("omq_status_str", "omq_last_cuda_error", "omq_version", "omq_sync_check",
            "omq_lwc_quant", "omq_let_apply", "omq_fq_linear_fwd", "omq_fwd_workspace_bytes",
            "omq_fq_linear_bwd", "omq_bwd_workspace_bytes", "omq_adamw_step", "omq_fold_pack",
-           "omq_calib_step", "omq_step_workspace_bytes", "omq_launch_count")
+           "omq_calib_step", "omq_step_workspace_bytes", "omq_launch_count",
+           "omq_fq_linear_fwd_noalloc")
 
 _p = ctypes.c_void_p
 _i64 = ctypes.c_int64
@@ -100,6 +101,7 @@ _sig("omq_fold_pack", _i32, [_p, _i32, _i64, _i64, _i64, _i32, _p, _p, _p, _p, _
 _sig("omq_calib_step", _i32, [ctypes.POINTER(StepArgs), _p, _sz, _p])
 _sig("omq_step_workspace_bytes", _sz, [_i64, _i64, _i64, _i64])
 _sig("omq_launch_count", ctypes.c_uint64, [])
+_sig("omq_fq_linear_fwd_noalloc", _i32, [_p, _p, _i32, _i64, _i64, _i64, _p, _p, _p, _p, _p, _p])
 
 
 def _check(status: int, where: str):
@@ -218,6 +220,23 @@ def fq_linear_fwd(Xq, W_hat, B_tilde=None, Y_ref=None, want_Y=True, workspace=No
                                   _ptr(Y_ref), _ptr(Y), _ptr(dY), _ptr(loss), _ptr(workspace),
                                   0 if workspace is None else workspace.numel(), _stream(stream)),
            "omq_fq_linear_fwd")
+    return dict(Y=Y, dY=dY, loss=loss)
+
+
+def fq_linear_fwd_noalloc(Xq, W_hat, Y_ref, B_tilde=None, want_Y=True, stream=None):
+    """omq_fq_linear_fwd_noalloc: the forward with its loss for hosts that cannot lend the
+    library device scratch; the scratch is a fixed array inside the library (see omq.h).
+    Returns dict(Y, dY, loss)."""
+    _dev(Xq, W_hat, B_tilde, Y_ref)
+    M, K = Xq.shape
+    N = W_hat.shape[0]
+    dev = Xq.device
+    Y = torch.empty(M, N, dtype=torch.float32, device=dev) if want_Y else None
+    dY = torch.empty(M, N, dtype=Xq.dtype, device=dev)
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    _check(_lib.omq_fq_linear_fwd_noalloc(_ptr(Xq), _ptr(W_hat), _dt(Xq), M, N, K, _ptr(B_tilde),
+                                          _ptr(Y_ref), _ptr(Y), _ptr(dY), _ptr(loss),
+                                          _stream(stream)), "omq_fq_linear_fwd_noalloc")
     return dict(Y=Y, dY=dY, loss=loss)
 
 
