@@ -335,7 +335,7 @@ def run_omq(args, cfg, rank: int, world: int, local_rank: int):
 
     peaks, peak_src = load_peaks()
     value = world * args.steps / (ms / 1e3)
-    gemm_keys = [k for k in ("fwd_gemm", "dw_gemm", "dx_gemm") if phases[k] > 0.0005]
+    gemm_keys = ["fwd_gemm", "dw_gemm"] + (["dx_gemm"] if cfg.let else [])
     gemm_ms = sum(phases[k] for k in gemm_keys) / len(gemm_keys)
     gemm_flops = 2 * cfg.m_tokens * cfg.n_out * cfg.k_in
     achieved = gemm_flops / (gemm_ms * 1e-3) / 1e12

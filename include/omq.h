@@ -62,7 +62,11 @@ typedef enum {
   OMQ_ERR_TIMEOUT = 9       /* a kernel's bounded barrier wait expired (device flag) */
 } omq_status;
 
-typedef enum { OMQ_F32 = 0, OMQ_BF16 = 1 } omq_dtype;
+/* Element types. W and X may be stored as F32, BF16 or F16. The GEMM operands (Xq, W_hat
+ * and the residual dY) are F32 (CUDA-core path) or F16 / BF16 (tensor-core path); F16 keeps
+ * 3 more mantissa bits than BF16 at the same speed and is the default of omq_calib_step
+ * for 16-bit storage, its range (|x| < 65504) being ample for LET-scaled activations. */
+typedef enum { OMQ_F32 = 0, OMQ_BF16 = 1, OMQ_F16 = 2 } omq_dtype;
 
 /* Per-group (or per-token) range record written by the quantizers and read by the
  * backward: the group's max and min of the quantized values, and how many elements
@@ -133,11 +137,13 @@ omq_status omq_let_apply(const void* X, omq_dtype xdt, int64_t M, int64_t K, con
  *
  *   Y[m,n] = sum_k Xq[m,k] W_hat[n,k] + B_tilde[n]      (B_tilde == NULL: 0)
  *   if Y_ref != NULL:  loss = mean over M*N of (Y - Y_ref)^2     (device float32 scalar)
- *                      dY[m,n] = 2 (Y - Y_ref) / (M N)           (stored in `dt`)
+ *                      dY[m,n] = Y - Y_ref, the residual, stored in `dt`; the loss
+ *                      gradient is dL/dY = 2 dY / (M N), a factor omq_fq_linear_bwd applies
+ *                      (the residual keeps its precision in a 16-bit type)
  *
  * Xq [M,K], W_hat [N,K] in `dt`; Y_ref, Y [M,N] float32. Y may be NULL (not stored);
  * with Y_ref == NULL, `loss` and `dY` must be NULL and Y must not be.
- * bf16 operands run on the tcgen05 tensor cores with float32 accumulation; float32
+ * 16-bit operands run on the tcgen05 tensor cores with float32 accumulation; float32
  * operands on CUDA cores in float32. K % 8 == 0 and N % 8 == 0.
  * Workspace: omq_fwd_workspace_bytes(M, N, K).
  * ------------------------------------------------------------------------------------ */
@@ -157,7 +163,7 @@ size_t omq_fwd_workspace_bytes(int64_t M, int64_t N, int64_t K);
  * float per output tile) in a fixed array compiled into the library and allocates nothing.
  * Arguments are those of omq_fq_linear_fwd without the workspace; Y_ref, dY and loss are
  * required, Y may be NULL.
- *   - Limit: ceil(M/128)*ceil(N/256) (bf16) or ceil(M/64)*ceil(N/64) (float32) must not
+ *   - Limit: ceil(M/128)*ceil(N/256) (16-bit operands) or ceil(M/64)*ceil(N/64) (float32) must not
  *     exceed 16384; larger problems return OMQ_ERR_SHAPE and launch nothing.
  *   - The array (64 KiB) is held on every GPU that loads the library until the process exits.
  *   - All calls on a device share it and it keeps the last call's contents; each call writes
@@ -175,7 +181,8 @@ omq_status omq_fq_linear_fwd_noalloc(const void* Xq, const void* W_hat, omq_dtyp
  * omq_fq_linear_bwd — straight-through backward of the step ([EDGE] section 2.2; the
  * formulas of [ICLR] sections LWC and LET differentiated as written).
  *
- *   dW_hat = dY^T Xq,  dXq = dY W_hat,  dB~ = sum_m dY[m,:]
+ *   with G = 2 dY / (M N) the loss gradient (dY the forward's residual):
+ *   dW_hat = G^T Xq,  dXq = G W_hat,  dB~ = sum_m G[m,:]
  *   Per LWC group, u = W~/h, c = code:
  *     in range (0 <= round(u)+z <= Q): dW_hat/dW~ = 1, dW_hat/dh = round(u) - u, dW_hat/dz = 0
  *     clipped:                          dW_hat/dW~ = 0, dW_hat/dh = c - z,        dW_hat/dz = -h
@@ -192,7 +199,8 @@ omq_status omq_fq_linear_fwd_noalloc(const void* Xq, const void* W_hat, omq_dtyp
 typedef struct {
   int64_t M, N, K, group;
   int bits, abits;
-  omq_dtype dt;                   /* dtype of X, W, Xq, W_hat and dY */
+  omq_dtype dt;                   /* storage dtype of X and W */
+  omq_dtype op_dt;                /* dtype of the GEMM operands Xq, W_hat and dY */
   const void* X;                  /* [M,K]   needed for d_s / d_delta */
   const void* W;                  /* [N,K] */
   const float* s;                 /* [K] or NULL (LET off) */
@@ -270,7 +278,9 @@ enum {
 typedef struct {
   int64_t M, N, K, group;
   int bits, abits, let;           /* let != 0: s, delta learnable */
-  omq_dtype dt;
+  omq_dtype dt;                   /* storage dtype of X and W */
+  omq_dtype op_dt;                /* GEMM operand dtype of Xq, W_hat, dY (F16 for 16-bit
+                                     storage, F32 for F32 storage) */
   const void* X; const void* W; const float* B; const float* Y_ref;
   float* gamma_logit; float* beta_logit; float* s; float* delta;     /* learnable */
   float* m_gamma; float* v_gamma; float* m_beta; float* v_beta;      /* AdamW moments */

@@ -1,10 +1,11 @@
 // Per-element GEMM epilogues shared by the tcgen05 and CUDA-core GEMMs.
 //
-// StoreF32: out[i, j] = acc (+ bias[j]).
+// StoreF32: out[i, j] = out_scale * acc (+ bias[j]).
 // MseLoss : the fake-quant forward's tail ("Y = Q_a(X~) Q_w(W~) + B~", then the squared
 //           reconstruction error against the full-precision output):
-//           Y = acc + bias[j]; optionally stored; diff = Y - Y_ref;
-//           loss partial += diff^2; dY = diff * 2/(rows*cols).
+//           Y = acc + bias[j]; optionally stored; R = Y - Y_ref written as the residual
+//           (the loss gradient is 2 R / (rows cols), applied by the backward);
+//           loss partial += R^2.
 #pragma once
 
 #include "omq_internal.cuh"
@@ -14,30 +15,32 @@ namespace omq {
 __device__ __forceinline__ void epi_element(const GemmEpilogue& e, int64_t i, int64_t j,
                                             int64_t cols, float acc, float& lsum) {
   const int64_t o = i * cols + j;
-  float y = acc + (e.bias ? e.bias[j] : 0.f);
   if (e.kind == Epi::StoreF32) {
-    e.out[o] = y;
+    e.out[o] = e.out_scale * acc + (e.bias ? e.bias[j] : 0.f);
     return;
   }
+  const float y = acc + (e.bias ? e.bias[j] : 0.f);
   if (e.out) e.out[o] = y;
-  float d = y - e.y_ref[o];
+  const float d = y - e.y_ref[o];
   lsum += d * d;
-  store_elem(e.dy, o, d * e.dy_scale, e.dy_dt);
+  store_elem(e.dy, o, d, e.dy_dt);
 }
 
 // 8 consecutive columns j0..j0+7 of row i, all in range, j0 % 8 == 0, cols % 8 == 0.
 __device__ __forceinline__ void epi_vec8(const GemmEpilogue& e, int64_t i, int64_t j0,
                                          int64_t cols, const float (&acc)[8], float& lsum) {
   const int64_t o = i * cols + j0;
+  const float sc = e.kind == Epi::StoreF32 ? e.out_scale : 1.f;
   float y[8];
   if (e.bias) {
     const float4* bp = reinterpret_cast<const float4*>(e.bias + j0);
     float4 b0 = bp[0], b1 = bp[1];
-    y[0] = acc[0] + b0.x; y[1] = acc[1] + b0.y; y[2] = acc[2] + b0.z; y[3] = acc[3] + b0.w;
-    y[4] = acc[4] + b1.x; y[5] = acc[5] + b1.y; y[6] = acc[6] + b1.z; y[7] = acc[7] + b1.w;
+    y[0] = sc * acc[0] + b0.x; y[1] = sc * acc[1] + b0.y; y[2] = sc * acc[2] + b0.z;
+    y[3] = sc * acc[3] + b0.w; y[4] = sc * acc[4] + b1.x; y[5] = sc * acc[5] + b1.y;
+    y[6] = sc * acc[6] + b1.z; y[7] = sc * acc[7] + b1.w;
   } else {
 #pragma unroll
-    for (int t = 0; t < 8; ++t) y[t] = acc[t];
+    for (int t = 0; t < 8; ++t) y[t] = sc * acc[t];
   }
   if (e.kind == Epi::StoreF32) {
     store8(e.out, o, OMQ_F32, y);
@@ -46,14 +49,13 @@ __device__ __forceinline__ void epi_vec8(const GemmEpilogue& e, int64_t i, int64
   if (e.out) store8(e.out, o, OMQ_F32, y);
   float r[8];
   load8(e.y_ref, o, OMQ_F32, r);
-  float dy[8];
+  float d[8];
 #pragma unroll
   for (int t = 0; t < 8; ++t) {
-    float d = y[t] - r[t];
-    lsum += d * d;
-    dy[t] = d * e.dy_scale;
+    d[t] = y[t] - r[t];
+    lsum += d[t] * d[t];
   }
-  store8(e.dy, o, e.dy_dt, dy);
+  store8(e.dy, o, e.dy_dt, d);
 }
 
 }  // namespace omq

@@ -1,13 +1,16 @@
 // bf16 x bf16 -> fp32 GEMM on the 5th-generation tensor cores (tcgen05, sm_100a).
 //
-// C[i, j] = sum_k A(i, k) B(j, k), one 128 x BN output tile per CTA, accumulator in TMEM.
-// Warp roles (192 threads):
+// C[i, j] = sum_k A(i, k) B(j, k) over 128 x BN output tiles, persistent: one CTA per SM
+// walks tiles t, t + grid, t + 2 grid, ... Warp roles (192 threads):
 //   warp 0      TMA producer: one elected lane streams A and B k-blocks into a STAGES-deep
 //               shared-memory ring (128-byte swizzle), completing "full" mbarriers.
-//   warp 1      allocates TMEM; one lane issues tcgen05.mma (M=128, N=BN, K=16) per k-slice
-//               and tcgen05.commit's each stage back to its "empty" mbarrier.
-//   warps 2..5  epilogue: tcgen05.ld 32 lanes x 32 columns at a time, fused epilogue
-//               (bias, MSE loss, dY) and global stores.
+//   warp 1      allocates TMEM for two accumulators (2 x BN columns); one lane issues
+//               tcgen05.mma (M=128, N=BN, K=16) per k-slice, tcgen05.commit's each stage back
+//               to its "empty" mbarrier and each finished tile to its accumulator's "full"
+//               mbarrier. It starts a tile as soon as the epilogue has released the other
+//               accumulator, so tile i+1's MMAs run while tile i is being stored.
+//   warps 2..5  epilogue: tcgen05.ld 32 lanes x 32 columns at a time, fused epilogue (bias,
+//               MSE loss, dY) and global stores; then release the accumulator.
 // Operands may be K-major (row of the stored matrix runs along k) or MN-major (row runs
 // along i / j), so the three contractions of the step read X, W and dY in their natural
 // layouts without transposed copies:
@@ -15,7 +18,8 @@
 //   dW^       dW = dY^T Xq  : A = dY [M,N] MN-major,       B = Xq [M,K] MN-major
 //   dXq       dX = dY W^    : A = dY [M,N] K-major,        B = W^ [N,K] MN-major
 // Every mbarrier wait is bounded in time; on expiry the kernel raises the device error
-// flag, skips its remaining work, and still releases its TMEM.
+// flag, every role stops, outstanding copies and MMAs are drained (bounded), and the TMEM
+// is released.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -59,6 +63,9 @@ __device__ __forceinline__ void fence_mbar_init() {
 __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   uint32_t ok;
@@ -152,10 +159,12 @@ __device__ __forceinline__ uint64_t operand_desc(uint32_t base, bool mn_major, i
   return smem_desc(base + kk * 32, 16, 1024);
 }
 
-// Instruction descriptor of kind::f16: D fp32 (bits 4-5 = 1), A and B bf16 (bits 7-9,
-// 10-12 = 1), A / B major (bits 15, 16), N >> 3 (bits 17-22), M >> 4 (bits 24-28).
-__host__ __device__ constexpr uint32_t instr_desc(int m, int n, bool a_mn, bool b_mn) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(a_mn) << 15) |
+// Instruction descriptor of kind::f16: D fp32 (bits 4-5 = 1), A and B format (bits 7-9,
+// 10-12: 0 = f16, 1 = bf16; always the same for both), A / B major (bits 15, 16), N >> 3
+// (bits 17-22), M >> 4 (bits 24-28).
+__host__ __device__ constexpr uint32_t instr_desc(int m, int n, bool a_mn, bool b_mn,
+                                                  uint32_t fmt) {
+  return (1u << 4) | (fmt << 7) | (fmt << 10) | (static_cast<uint32_t>(a_mn) << 15) |
          (static_cast<uint32_t>(b_mn) << 16) | (static_cast<uint32_t>(n >> 3) << 17) |
          (static_cast<uint32_t>(m >> 4) << 24);
 }
@@ -166,32 +175,38 @@ struct Layout {
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
+  // barriers: full[S], empty[S], acc_full[2], acc_empty[2], drain; then tmem slot, abort
+  // flag, the epilogue's per-warp loss partials [2][4] and arrival counters [2]
+  static constexpr int FULL = 0, EMPTY = 8 * STAGES, ACCF = 16 * STAGES, ACCE = ACCF + 16,
+                       DRAIN = ACCE + 16, SLOT = DRAIN + 8, ABORT = SLOT + 4, RED = ABORT + 4,
+                       CNT = RED + 32;
   static constexpr int SMEM_BYTES = 1024 /*align slack*/ + BAR_OFF + 256;
+  static constexpr uint32_t TMEM_COLS = 2 * BN;
 };
 
 template <int BN, int STAGES>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   int a_mn, int b_mn, int64_t rows, int64_t cols, int64_t depth,
-                   GemmEpilogue epi, int tiles_n) {
+                   int a_mn, int b_mn, uint32_t fmt, int64_t rows, int64_t cols, int64_t depth,
+                   GemmEpilogue epi, int tiles_n, int num_tiles) {
   using L = Layout<BN, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t bar_full = sbase + L::BAR_OFF;          // STAGES x 8 bytes
-  const uint32_t bar_empty = bar_full + STAGES * 8;       // STAGES x 8 bytes
-  const uint32_t bar_acc = bar_empty + STAGES * 8;        // 8 bytes
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::BAR_OFF + STAGES * 16 + 8);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::BAR_OFF + STAGES * 16 + 12);
-  float* red = reinterpret_cast<float*>(smem + L::BAR_OFF + STAGES * 16 + 16);   // 4 floats
+  uint8_t* ctl = smem + L::BAR_OFF;
+  const uint32_t bar_full = sbase + L::BAR_OFF + L::FULL;
+  const uint32_t bar_empty = sbase + L::BAR_OFF + L::EMPTY;
+  const uint32_t bar_accf = sbase + L::BAR_OFF + L::ACCF;
+  const uint32_t bar_acce = sbase + L::BAR_OFF + L::ACCE;
+  const uint32_t bar_drain = sbase + L::BAR_OFF + L::DRAIN;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctl + L::SLOT);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(ctl + L::ABORT);
+  volatile float* red = reinterpret_cast<volatile float*>(ctl + L::RED);     // [2][4]
+  int* cnt = reinterpret_cast<int*>(ctl + L::CNT);                           // [2]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int tm = blockIdx.x / tiles_n;
-  const int tn = blockIdx.x % tiles_n;
-  const int64_t row0 = static_cast<int64_t>(tm) * BM;
-  const int64_t col0 = static_cast<int64_t>(tn) * BN;
   const int nk = static_cast<int>((depth + BK - 1) / BK);
 
   if (threadIdx.x == 0) {
@@ -199,14 +214,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(bar_full + 8 * s, 1);
       mbar_init(bar_empty + 8 * s, 1);
     }
-    mbar_init(bar_acc, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_accf + 8 * b, 1);
+      mbar_init(bar_acce + 8 * b, 4);   // one arrival per epilogue warp
+      cnt[b] = 0;
+    }
+    mbar_init(bar_drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(tmem_slot)),
-                 "r"(BN));
+                 "r"(L::TMEM_COLS));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   tc_fence_before();
@@ -216,71 +236,101 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (warp == 0 && lane == 0) {
     // ---------------- TMA producer
-    int issued = 0;
+    int it = 0;
     bool ok = true;
-    for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % STAGES;
-      const uint32_t ph = (kb / STAGES) & 1;
-      if (!mbar_wait(bar_empty + 8 * s, ph ^ 1, DEV_ERR_TMA_WAIT)) { ok = false; break; }
-      const uint32_t a_dst = sbase + s * L::STAGE_BYTES;
-      const uint32_t b_dst = a_dst + L::A_BYTES;
-      const uint32_t full = bar_full + 8 * s;
-      mbar_expect_tx(full, L::STAGE_BYTES);
-      const int k0 = kb * BK;
-      if (a_mn) {
-        for (int c = 0; c < BM / 64; ++c)
-          tma_load_2d(a_dst + c * 8192, &tmA, full, static_cast<int>(row0) + 64 * c, k0);
-      } else {
-        tma_load_2d(a_dst, &tmA, full, k0, static_cast<int>(row0));
+    for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+      const int row0 = (t / tiles_n) * BM;
+      const int col0 = (t % tiles_n) * BN;
+      for (int kb = 0; kb < nk; ++kb, ++it) {
+        const int s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1;
+        if (*abort_flag || !mbar_wait(bar_empty + 8 * s, ph ^ 1, DEV_ERR_TMA_WAIT)) {
+          ok = false;
+          break;
+        }
+        const uint32_t a_dst = sbase + s * L::STAGE_BYTES;
+        const uint32_t b_dst = a_dst + L::A_BYTES;
+        const uint32_t full = bar_full + 8 * s;
+        mbar_expect_tx(full, L::STAGE_BYTES);
+        const int k0 = kb * BK;
+        if (a_mn) {
+          for (int c = 0; c < BM / 64; ++c) tma_load_2d(a_dst + c * 8192, &tmA, full, row0 + 64 * c, k0);
+        } else {
+          tma_load_2d(a_dst, &tmA, full, k0, row0);
+        }
+        if (b_mn) {
+          for (int c = 0; c < BN / 64; ++c) tma_load_2d(b_dst + c * 8192, &tmB, full, col0 + 64 * c, k0);
+        } else {
+          tma_load_2d(b_dst, &tmB, full, k0, col0);
+        }
       }
-      if (b_mn) {
-        for (int c = 0; c < BN / 64; ++c)
-          tma_load_2d(b_dst + c * 8192, &tmB, full, static_cast<int>(col0) + 64 * c, k0);
-      } else {
-        tma_load_2d(b_dst, &tmB, full, k0, static_cast<int>(col0));
-      }
-      ++issued;
     }
     if (!ok) {
       *abort_flag = 1;
       // let the copies already in flight land before the CTA can exit
-      for (int kb = issued - STAGES < 0 ? 0 : issued - STAGES; kb < issued; ++kb)
-        mbar_wait(bar_full + 8 * (kb % STAGES), (kb / STAGES) & 1, DEV_ERR_TMA_WAIT);
+      for (int j = it - STAGES < 0 ? 0 : it - STAGES; j < it; ++j)
+        mbar_wait(bar_full + 8 * (j % STAGES), (j / STAGES) & 1, DEV_ERR_TMA_WAIT);
     }
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer
-    const uint32_t idesc = instr_desc(BM, BN, a_mn != 0, b_mn != 0);
+    const uint32_t idesc = instr_desc(BM, BN, a_mn != 0, b_mn != 0, fmt);
+    int it = 0, lt = 0;
     bool ok = true;
-    for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % STAGES;
-      const uint32_t ph = (kb / STAGES) & 1;
-      if (!mbar_wait(bar_full + 8 * s, ph, DEV_ERR_MMA_WAIT)) { ok = false; break; }
-      tc_fence_after();
-      const uint32_t a_base = sbase + s * L::STAGE_BYTES;
-      const uint32_t b_base = a_base + L::A_BYTES;
-#pragma unroll
-      for (int kk = 0; kk < BK / UMMA_K; ++kk) {
-        umma_bf16(tmem, operand_desc(a_base, a_mn != 0, kk), operand_desc(b_base, b_mn != 0, kk),
-                  idesc, (kb | kk) != 0 ? 1u : 0u);
+    for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++lt) {
+      const int buf = lt & 1;
+      if (*abort_flag || !mbar_wait(bar_acce + 8 * buf, ((lt >> 1) & 1) ^ 1, DEV_ERR_MMA_WAIT)) {
+        ok = false;
+        break;
       }
-      umma_commit(bar_empty + 8 * s);
+      tc_fence_after();
+      const uint32_t d = tmem + static_cast<uint32_t>(buf * BN);
+      for (int kb = 0; kb < nk; ++kb, ++it) {
+        const int s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1;
+        if (*abort_flag || !mbar_wait(bar_full + 8 * s, ph, DEV_ERR_MMA_WAIT)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a_base = sbase + s * L::STAGE_BYTES;
+        const uint32_t b_base = a_base + L::A_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < BK / UMMA_K; ++kk) {
+          umma_bf16(d, operand_desc(a_base, a_mn != 0, kk), operand_desc(b_base, b_mn != 0, kk),
+                    idesc, (kb | kk) != 0 ? 1u : 0u);
+        }
+        umma_commit(bar_empty + 8 * s);
+      }
+      if (!ok) break;
+      umma_commit(bar_accf + 8 * buf);
     }
     if (!ok) *abort_flag = 1;
-    umma_commit(bar_acc);   // arrives once every MMA issued above has completed
+    // every MMA issued above has completed once this commit arrives
+    umma_commit(bar_drain);
+    mbar_wait(bar_drain, 0, DEV_ERR_MMA_WAIT);
   } else if (warp >= 2) {
     // ---------------- epilogue
     const int quad = warp & 3;                       // TMEM lanes 32*quad .. 32*quad+31
-    const int64_t row = row0 + quad * 32 + lane;
-    float lsum = 0.f;
-    // one lane polls; the decision is broadcast so the warp-wide tcgen05.ld stays uniform
-    int go = 0;
-    if (lane == 0) go = (mbar_wait(bar_acc, 0, DEV_ERR_EPI_WAIT) && *abort_flag == 0) ? 1 : 0;
-    go = __shfl_sync(0xffffffffu, go, 0);
-    tc_fence_after();
-    if (go) {
+    int lt = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++lt) {
+      const int buf = lt & 1;
+      // one lane polls; the decision is broadcast so the warp-wide tcgen05.ld stays uniform
+      int go = 0;
+      if (lane == 0)
+        go = (mbar_wait(bar_accf + 8 * buf, (lt >> 1) & 1, DEV_ERR_EPI_WAIT) && *abort_flag == 0)
+                 ? 1 : 0;
+      go = __shfl_sync(0xffffffffu, go, 0);
+      tc_fence_after();
+      if (!go) break;
+      const int64_t row0 = static_cast<int64_t>(t / tiles_n) * BM;
+      const int64_t col0 = static_cast<int64_t>(t % tiles_n) * BN;
+      const int64_t row = row0 + quad * 32 + lane;
+      float lsum = 0.f;
+      const uint32_t tbase = tmem + (static_cast<uint32_t>(quad * 32) << 16) +
+                             static_cast<uint32_t>(buf * BN);
       for (int ch = 0; ch < BN / 32; ++ch) {
         uint32_t r[32];
-        tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + ch * 32, r);
+        tmem_ld32(tbase + ch * 32, r);
         tmem_ld_wait();
         const int64_t cbase = col0 + ch * 32;
         if (row < rows && cbase < cols) {
@@ -289,30 +339,45 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int v = 0; v < 4; ++v) {
               float acc[8];
 #pragma unroll
-              for (int t = 0; t < 8; ++t) acc[t] = __uint_as_float(r[v * 8 + t]);
+              for (int q = 0; q < 8; ++q) acc[q] = __uint_as_float(r[v * 8 + q]);
               epi_vec8(epi, row, cbase + v * 8, cols, acc, lsum);
             }
           } else {
 #pragma unroll
-            for (int t = 0; t < 32; ++t)
-              if (cbase + t < cols) epi_element(epi, row, cbase + t, cols, __uint_as_float(r[t]), lsum);
+            for (int q = 0; q < 32; ++q)
+              if (cbase + q < cols) epi_element(epi, row, cbase + q, cols, __uint_as_float(r[q]), lsum);
           }
         }
       }
-    }
-    if (epi.kind == Epi::MseLoss) {
+      if (epi.kind == Epi::MseLoss) {
+        // per-tile partial: the last of the four warps adds the warps' sums in a fixed order.
+        // red[buf] / cnt[buf] are next touched two tiles later, which cannot start before all
+        // four warps have released this accumulator below.
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
-      if (lane == 0) red[quad] = lsum;
+        for (int off = 16; off > 0; off >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
+        if (lane == 0) {
+          red[buf * 4 + quad] = lsum;
+          __threadfence_block();
+          if (atomicAdd(&cnt[buf], 1) == 3) {
+            __threadfence_block();
+            epi.loss_partials[t] = ((red[buf * 4 + 0] + red[buf * 4 + 1]) + red[buf * 4 + 2]) +
+                                   red[buf * 4 + 3];
+            cnt[buf] = 0;
+          }
+        }
+      }
+      // the accumulator has been read: hand it back to the MMA warp
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_acce + 8 * buf);
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (epi.kind == Epi::MseLoss && threadIdx.x == 0)
-    epi.loss_partials[blockIdx.x] = ((red[0] + red[1]) + red[2]) + red[3];
   if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(BN));
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(L::TMEM_COLS));
   }
 }
 
@@ -334,8 +399,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // Tensor map of one operand. K-major: stored [n_rows, depth] -> dims {depth, n_rows},
 // box {64, box_rows}. MN-major: stored [depth, n_rows] -> dims {n_rows, depth}, box {64, 64}.
-bool make_map(CUtensorMap* map, const GemmOperand& op, int64_t n_rows, int64_t depth,
-              int box_rows) {
+bool make_map(CUtensorMap* map, omq_dtype dt, const GemmOperand& op, int64_t n_rows,
+              int64_t depth, int box_rows) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2];
@@ -353,7 +418,9 @@ bool make_map(CUtensorMap* map, const GemmOperand& op, int64_t n_rows, int64_t d
   }
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(op.ld) * 2};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(op.ptr), dims,
+  const CUtensorMapDataType ty =
+      dt == OMQ_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  CUresult r = fn(map, ty, 2, const_cast<void*>(op.ptr), dims,
                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -364,16 +431,17 @@ constexpr int kStages = 4;
 
 }  // namespace tc
 
-int64_t gemm_bf16_tc_tiles(int64_t rows, int64_t cols) {
+int64_t gemm_tc_tiles(int64_t rows, int64_t cols) {
   return ceil_div(rows, tc::BM) * ceil_div(cols, tc::kBN);
 }
 
-omq_status gemm_bf16_tc(const GemmOperand& A, const GemmOperand& B, int64_t rows, int64_t cols,
-                        int64_t depth, const GemmEpilogue& epi, int64_t* n_tiles,
-                        cudaStream_t stream) {
+omq_status gemm_tc(omq_dtype dt, const GemmOperand& A, const GemmOperand& B, int64_t rows,
+                   int64_t cols, int64_t depth, const GemmEpilogue& epi, int64_t* n_tiles,
+                   cudaStream_t stream) {
   using namespace tc;
+  if (dt != OMQ_BF16 && dt != OMQ_F16) return OMQ_ERR_DTYPE;
   CUtensorMap ma, mb;
-  if (!make_map(&ma, A, rows, depth, BM) || !make_map(&mb, B, cols, depth, kBN)) {
+  if (!make_map(&ma, dt, A, rows, depth, BM) || !make_map(&mb, dt, B, cols, depth, kBN)) {
     set_cuda_error(cudaErrorInvalidValue);
     return OMQ_ERR_CUDA;
   }
@@ -391,9 +459,11 @@ omq_status gemm_bf16_tc(const GemmOperand& A, const GemmOperand& B, int64_t rows
     set_cuda_error(attr_err);
     return OMQ_ERR_CUDA;
   }
-  kern<<<static_cast<unsigned>(tiles), NUM_THREADS, smem, stream>>>(
-      ma, mb, A.mn_major ? 1 : 0, B.mn_major ? 1 : 0, rows, cols, depth, epi,
-      static_cast<int>(tiles_n));
+  const int64_t sms = num_sms();
+  const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);
+  kern<<<grid, NUM_THREADS, smem, stream>>>(ma, mb, A.mn_major ? 1 : 0, B.mn_major ? 1 : 0,
+                                            dt == OMQ_F16 ? 0u : 1u, rows, cols, depth, epi,
+                                            static_cast<int>(tiles_n), static_cast<int>(tiles));
   return launch_status();
 }
 

@@ -33,14 +33,24 @@ __device__ __forceinline__ void let8(const LetParams& p, int64_t off, int64_t co
   for (int i = 0; i < 8; ++i) v[i] = __fdiv_rn(__fsub_rn(v[i], dv[i]), sv[i]);
 }
 
+// U chunks of 8 per thread per iteration, all loaded before any is converted.
+template <int U>
 __global__ void __launch_bounds__(256) let_elem_kernel(LetParams p) {
   const int64_t chunks = p.M * p.K / 8;
-  for (int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; c < chunks;
-       c += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t off = c * 8;
-    float v[8];
-    let8(p, off, off % p.K, v);
-    store8(p.Xq, off, p.xq_dt, v);
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t c0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; c0 < chunks;
+       c0 += stride * U) {
+    float v[U][8];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t c = c0 + u * stride;
+      if (c < chunks) let8(p, c * 8, (c * 8) % p.K, v[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t c = c0 + u * stride;
+      if (c < chunks) store8(p.Xq, c * 8, p.xq_dt, v[u]);
+    }
   }
 }
 
@@ -120,6 +130,7 @@ __global__ void __launch_bounds__(256) let_bias_kernel(const void* W, omq_dtype 
   for (int64_t n = warp_g; n < N; n += n_warps) {
     float acc = 0.f;
     if (delta) {
+#pragma unroll 4
       for (int64_t c = lane; c < K / 8; c += 32) {
         float v[8];
         load8(W, n * K + c * 8, wdt, v);
@@ -139,9 +150,9 @@ omq_status launch_let(const LetParams& p, int abits, cudaStream_t stream) {
   const int sms = num_sms();
   if (abits >= 16) {
     const int64_t chunks = p.M * p.K / 8;
-    const int64_t want = ceil_div(chunks, 256);
-    const unsigned grid = static_cast<unsigned>(want < int64_t(sms) * 16 ? want : int64_t(sms) * 16);
-    let_elem_kernel<<<grid, 256, 0, stream>>>(p);
+    const int64_t want = ceil_div(chunks, 256 * 4);
+    const unsigned grid = static_cast<unsigned>(want < int64_t(sms) * 8 ? want : int64_t(sms) * 8);
+    let_elem_kernel<4><<<grid, 256, 0, stream>>>(p);
     return launch_status();
   }
   const size_t smem = static_cast<size_t>(p.K) * sizeof(float);

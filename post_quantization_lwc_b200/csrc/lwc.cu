@@ -30,7 +30,7 @@ __device__ __forceinline__ void encode8(const LwcParams& p, int64_t off, const f
     const float lvl = __fadd_rn(round_quotient(v[i], q.h, hinv), q.z);
     const float cc = fminf(fmaxf(lvl, 0.f), p.Q);
     deq[i] = __fmul_rn(__fsub_rn(cc, q.z), q.h);
-    c[i] = static_cast<uint32_t>(cc);
+    c[i] = small_uint(cc);
   }
   if (p.W_hat) store8(p.W_hat, off, p.hat_dt, deq);
   if (p.codes) {
@@ -72,51 +72,80 @@ __device__ __forceinline__ void load_scaled8(const LwcParams& p, int64_t off, in
   }
 }
 
-template <int LPG>
+// Launch shape shared by the small-group kernels: grid (256-column segments, row blocks of
+// rows_per_block rows); a warp covers one row of the segment (lane = 8 columns, one 16-byte
+// load of bf16), the 8 warps of a block take every 8th row, U rows per iteration. A lane's
+// columns, and so its group within the row, stay fixed: no index division in the loop.
+constexpr int kLwcRows = 64;
+
+template <int LPG, int U>
 __global__ void __launch_bounds__(256) lwc_small_kernel(LwcParams p) {
-  constexpr int SPW = 32 / LPG;
-  const int lane = threadIdx.x & 31;
+  constexpr int GPW = 32 / LPG;   // groups per segment
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int sub = lane / LPG, lig = lane % LPG;
-  const int64_t warp_g = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t n_warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-  const int64_t total = p.N * p.ng;
-  for (int64_t base = warp_g * SPW; base < total; base += n_warps * SPW) {
-    const int64_t gi = base + sub;
-    const bool valid = gi < total;
-    const int64_t n = valid ? gi / p.ng : 0, j = valid ? gi % p.ng : 0;
-    const int64_t col = j * p.G + lig * 8;
-    const int64_t off = n * p.K + col;
-    float v[8];
-    if (valid) {
-      load_scaled8(p, off, col, v);
-    } else {
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * 256 + lane * 8;
+  const bool cvalid = c0 < p.K;
+  const int64_t j = c0 / (LPG * 8);                        // this lane's group in the row
+  // lane t evaluates the strength of group (segment's first + t/2), gamma for even t
+  const int64_t jt = static_cast<int64_t>(blockIdx.x) * GPW + (lane >> 1);
+  const bool tvalid = lane < 2 * GPW && jt < p.ng;
+  const float* logit = (lane & 1) ? p.bl : p.gl;
+  float sv[8];
+  if (p.s && cvalid) {
+    const float4* sp = reinterpret_cast<const float4*>(p.s + c0);
+    const float4 s0 = sp[0], s1 = sp[1];
+    sv[0] = s0.x; sv[1] = s0.y; sv[2] = s0.z; sv[3] = s0.w;
+    sv[4] = s1.x; sv[5] = s1.y; sv[6] = s1.z; sv[7] = s1.w;
+  }
+  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * kLwcRows;
+  const int64_t r1 = min(p.N, r0 + kLwcRows);
+  for (int64_t nb = r0 + w; nb < r1; nb += 8 * U) {
+    float v[U][8], st[U];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) v[i] = 0.f;
+    for (int u = 0; u < U; ++u) {
+      const int64_t n = nb + 8 * u;
+      if (n < r1 && cvalid) {
+        load8(p.W, n * p.K + c0, p.wdt, v[u]);
+        if (p.s) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) v[u][i] = __fmul_rn(v[u][i], sv[i]);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[u][i] = 0.f;
+      }
+      st[u] = (n < r1 && tvalid) ? strength(logit[n * p.ng + jt]) : 1.f;
     }
-    float vmax = v[0], vmin = v[0];
 #pragma unroll
-    for (int i = 1; i < 8; ++i) { vmax = fmaxf(vmax, v[i]); vmin = fminf(vmin, v[i]); }
+    for (int u = 0; u < U; ++u) {
+      const int64_t n = nb + 8 * u;
+      float vmax = v[u][0], vmin = v[u][0];
 #pragma unroll
-    for (int o = LPG / 2; o > 0; o >>= 1) {
-      vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
-      vmin = fminf(vmin, __shfl_xor_sync(0xffffffffu, vmin, o));
-    }
-    int nmax = 0, nmin = 0;
+      for (int i = 1; i < 8; ++i) { vmax = fmaxf(vmax, v[u][i]); vmin = fminf(vmin, v[u][i]); }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) { nmax += v[i] == vmax; nmin += v[i] == vmin; }
+      for (int o = LPG / 2; o > 0; o >>= 1) {
+        vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+        vmin = fminf(vmin, __shfl_xor_sync(0xffffffffu, vmin, o));
+      }
+      int nmax = 0, nmin = 0;
 #pragma unroll
-    for (int o = LPG / 2; o > 0; o >>= 1) {
-      nmax += __shfl_xor_sync(0xffffffffu, nmax, o);
-      nmin += __shfl_xor_sync(0xffffffffu, nmin, o);
-    }
-    if (!valid) continue;
-    const float g = strength(p.gl[gi]), b = strength(p.bl[gi]);
-    const GroupQ q = group_params(g, b, vmax, vmin, p.Q);
-    encode8(p, off, v, q);
-    if (lig == 0) {
-      if (p.h) p.h[gi] = q.h;
-      if (p.z) p.z[gi] = z_to_i32(q.z);
-      if (p.range) p.range[gi] = omq_range{vmax, vmin, nmax, nmin};
+      for (int i = 0; i < 8; ++i) { nmax += v[u][i] == vmax; nmin += v[u][i] == vmin; }
+#pragma unroll
+      for (int o = LPG / 2; o > 0; o >>= 1) {
+        nmax += __shfl_xor_sync(0xffffffffu, nmax, o);
+        nmin += __shfl_xor_sync(0xffffffffu, nmin, o);
+      }
+      const float g = __shfl_sync(0xffffffffu, st[u], 2 * sub);
+      const float b = __shfl_sync(0xffffffffu, st[u], 2 * sub + 1);
+      if (n >= r1 || !cvalid) continue;
+      const GroupQ q = group_params(g, b, vmax, vmin, p.Q);
+      encode8(p, n * p.K + c0, v[u], q);
+      if (lig == 0) {
+        const int64_t gi = n * p.ng + j;
+        if (p.h) p.h[gi] = q.h;
+        if (p.z) p.z[gi] = z_to_i32(q.z);
+        if (p.range) p.range[gi] = omq_range{vmax, vmin, nmax, nmin};
+      }
     }
   }
 }
@@ -156,11 +185,13 @@ __global__ void __launch_bounds__(256) lwc_large_kernel(LwcParams p) {
   extern __shared__ float buf[];   // G floats: the scaled group
   __shared__ float smf[64];
   __shared__ int smi[64];
+  __shared__ float sgb[2];         // the group's strengths (read after the reductions' syncs)
   const int64_t total = p.N * p.ng;
   const int chunks = static_cast<int>(p.G / 8);
   for (int64_t gi = blockIdx.x; gi < total; gi += gridDim.x) {
     const int64_t n = gi / p.ng, j = gi % p.ng;
     const int64_t base = n * p.K + j * p.G;
+    if (threadIdx.x < 2) sgb[threadIdx.x] = strength(threadIdx.x ? p.bl[gi] : p.gl[gi]);
     float vmax = -FLT_MAX, vmin = FLT_MAX;
     for (int c = threadIdx.x; c < chunks; c += blockDim.x) {
       float v[8];
@@ -178,8 +209,7 @@ __global__ void __launch_bounds__(256) lwc_large_kernel(LwcParams p) {
 #pragma unroll
       for (int i = 0; i < 8; ++i) { nmax += buf[c * 8 + i] == vmax; nmin += buf[c * 8 + i] == vmin; }
     block_sum2i(nmax, nmin, smi);
-    const float g = strength(p.gl[gi]), b = strength(p.bl[gi]);
-    const GroupQ q = group_params(g, b, vmax, vmin, p.Q);
+    const GroupQ q = group_params(sgb[0], sgb[1], vmax, vmin, p.Q);
     for (int c = threadIdx.x; c < chunks; c += blockDim.x) {
       float v[8];
 #pragma unroll
@@ -198,18 +228,16 @@ __global__ void __launch_bounds__(256) lwc_large_kernel(LwcParams p) {
 omq_status launch_lwc(const LwcParams& p, cudaStream_t stream) {
   const int64_t total = p.N * p.ng;
   const int sms = num_sms();
-  if (p.G <= 256 && (p.G & (p.G - 1)) == 0) {
-    const int lpg = static_cast<int>(p.G / 8);
-    const int64_t groups_per_block = 8 * (32 / lpg);
-    const int64_t want = ceil_div(total, groups_per_block);
-    const unsigned grid = static_cast<unsigned>(want < int64_t(sms) * 16 ? want : int64_t(sms) * 16);
-    switch (lpg) {
-      case 1: lwc_small_kernel<1><<<grid, 256, 0, stream>>>(p); break;
-      case 2: lwc_small_kernel<2><<<grid, 256, 0, stream>>>(p); break;
-      case 4: lwc_small_kernel<4><<<grid, 256, 0, stream>>>(p); break;
-      case 8: lwc_small_kernel<8><<<grid, 256, 0, stream>>>(p); break;
-      case 16: lwc_small_kernel<16><<<grid, 256, 0, stream>>>(p); break;
-      default: lwc_small_kernel<32><<<grid, 256, 0, stream>>>(p); break;
+  if (small_group(p.G)) {
+    constexpr int U = 4;
+    dim3 grid(static_cast<unsigned>(ceil_div(p.K, 256)),
+              static_cast<unsigned>(ceil_div(p.N, kLwcRows)));
+    switch (p.G / 8) {
+      case 2: lwc_small_kernel<2, U><<<grid, 256, 0, stream>>>(p); break;
+      case 4: lwc_small_kernel<4, U><<<grid, 256, 0, stream>>>(p); break;
+      case 8: lwc_small_kernel<8, U><<<grid, 256, 0, stream>>>(p); break;
+      case 16: lwc_small_kernel<16, U><<<grid, 256, 0, stream>>>(p); break;
+      default: lwc_small_kernel<32, U><<<grid, 256, 0, stream>>>(p); break;
     }
     return launch_status();
   }

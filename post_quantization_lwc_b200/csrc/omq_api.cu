@@ -14,19 +14,17 @@ thread_local int t_last_cuda_error = 0;
 
 constexpr int64_t kMaxGroupLarge = 16384;   // group staged in shared memory (per group / row)
 constexpr int64_t kMaxDim = (int64_t(1) << 31) - 1;
-constexpr int kRowsSmallW = 64;             // rows per block, weight STE, group <= 256
+constexpr int kRowsSmallW = 128;            // rows per block, weight STE, lane-parallel groups
 constexpr int kRowsLargeW = 16;             // rows per block, weight STE, larger groups
-constexpr int kRowsX = 16;                  // tokens per block, activation STE
+constexpr int kRowsX = 64;                  // tokens per block, activation STE column sums
 constexpr int kRowsColsum = 64;             // rows per block of the dY column sums
 
 size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
 
-bool small_group(int64_t g) { return g <= 256 && (g & (g - 1)) == 0; }
-
 int64_t rows_per_block_w(int64_t group) { return small_group(group) ? kRowsSmallW : kRowsLargeW; }
 
 struct BwdLayout {
-  size_t dbt_part, dbt, dwhat, dxq, part_ws, part_wd, part_xs, part_xd, total;
+  size_t dbt_part, dbt, dwhat, dxq, part_ws, part_wd, part_xs, part_xd, rowstat, total;
   int64_t rb_colsum, rb_w, rb_x;
 };
 
@@ -45,12 +43,13 @@ BwdLayout bwd_layout(int64_t M, int64_t N, int64_t K, int64_t group) {
   L.part_wd = take(sizeof(float) * L.rb_w * K);
   L.part_xs = take(sizeof(float) * L.rb_x * K);
   L.part_xd = take(sizeof(float) * L.rb_x * K);
+  L.rowstat = take(sizeof(float) * 2 * M);
   L.total = off;
   return L;
 }
 
 size_t fwd_bytes(int64_t M, int64_t N) {
-  int64_t t = gemm_bf16_tc_tiles(M, N);
+  int64_t t = gemm_tc_tiles(M, N);
   int64_t t2 = gemm_f32_simt_tiles(M, N);
   return align256(sizeof(float) * static_cast<size_t>(t > t2 ? t : t2));
 }
@@ -60,7 +59,7 @@ T* at(void* base, size_t off) {
   return reinterpret_cast<T*>(static_cast<char*>(base) + off);
 }
 
-bool dtype_ok(omq_dtype d) { return d == OMQ_F32 || d == OMQ_BF16; }
+bool dtype_ok(omq_dtype d) { return d == OMQ_F32 || d == OMQ_BF16 || d == OMQ_F16; }
 bool wbits_ok(int b) { return b == 2 || b == 3 || b == 4 || b == 8; }
 bool abits_ok(int b) { return b == 2 || b == 3 || b == 4 || b == 6 || b == 8 || b == 16; }
 bool a16(const void* p) { return p == nullptr || aligned16(p); }
@@ -228,8 +227,8 @@ size_t omq_fwd_workspace_bytes(int64_t M, int64_t N, int64_t K) {
 static omq_status run_gemm(omq_dtype dt, const GemmOperand& A, const GemmOperand& B, int64_t rows,
                            int64_t cols, int64_t depth, const GemmEpilogue& epi, int64_t* tiles,
                            cudaStream_t st) {
-  if (dt == OMQ_BF16) return gemm_bf16_tc(A, B, rows, cols, depth, epi, tiles, st);
-  return gemm_f32_simt(A, B, rows, cols, depth, epi, tiles, st);
+  if (dt == OMQ_F32) return gemm_f32_simt(A, B, rows, cols, depth, epi, tiles, st);
+  return gemm_tc(dt, A, B, rows, cols, depth, epi, tiles, st);
 }
 
 static omq_status fwd_impl(const void* Xq, const void* W_hat, omq_dtype dt, int64_t M, int64_t N,
@@ -259,11 +258,11 @@ static omq_status fwd_impl(const void* Xq, const void* W_hat, omq_dtype dt, int6
     epi.y_ref = Y_ref;
     epi.dy = dY;
     epi.dy_dt = dt;
-    epi.dy_scale = static_cast<float>(2.0 / (static_cast<double>(M) * static_cast<double>(N)));
     epi.loss_partials = static_cast<float*>(workspace);
   } else {
     epi.kind = Epi::StoreF32;
     epi.out = Y;
+    epi.out_scale = 1.f;
   }
   int64_t tiles = 0;
   OMQ_TRY(ph.mark(OMQ_PH_FWD_GEMM));
@@ -295,11 +294,13 @@ static omq_status bwd_impl(const omq_bwd_args* a, void* workspace, size_t ws_byt
   if (!a->W || !a->Xq || !a->W_hat || !a->h || !a->z || !a->grp_range || !a->dY ||
       !a->gamma_logit || !a->beta_logit)
     return OMQ_ERR_NULL;
-  if (!dtype_ok(a->dt)) return OMQ_ERR_DTYPE;
+  if (!dtype_ok(a->dt) || !dtype_ok(a->op_dt)) return OMQ_ERR_DTYPE;
   if (!wbits_ok(a->bits) || !abits_ok(a->abits)) return OMQ_ERR_BITS;
   if (M < 1 || N < 8 || K < 8 || G < 8 || N % 8 || K % 8 || G % 8 || K % G || M > kMaxDim ||
       N > kMaxDim || K > kMaxDim)
     return OMQ_ERR_SHAPE;
+  // the loss gradient is 2 R / (M N) for the forward's residual R
+  const float gscale = static_cast<float>(2.0 / (static_cast<double>(M) * static_cast<double>(N)));
   if (!small_group(G) && G > kMaxGroupLarge) return OMQ_ERR_SHAPE;
   const bool need_let = a->d_s || a->d_delta;
   if (need_let) {
@@ -326,17 +327,18 @@ static omq_status bwd_impl(const omq_bwd_args* a, void* workspace, size_t ws_byt
   // dB~ = column sums of dY (needed for d_delta, or when asked for)
   OMQ_TRY(ph.mark(OMQ_PH_DBIAS));
   if (a->d_delta || a->d_B_tilde) {
-    OMQ_TRY(launch_colsum(a->dY, a->dt, M, N, kRowsColsum, dbt_part, st));
-    OMQ_TRY(launch_reduce_cols(dbt_part, L.rb_colsum, nullptr, 0, N, dbt, st));
+    OMQ_TRY(launch_colsum(a->dY, a->op_dt, M, N, kRowsColsum, dbt_part, st));
+    OMQ_TRY(launch_reduce_cols(dbt_part, L.rb_colsum, nullptr, 0, N, gscale, dbt, st));
   }
-  // dW^ = dY^T Xq   [N, K]
+  // dW^ = G^T Xq   [N, K]
   OMQ_TRY(ph.mark(OMQ_PH_DW_GEMM));
   {
     GemmOperand A{a->dY, N, true}, B{a->Xq, K, true};
     GemmEpilogue epi{};
     epi.kind = Epi::StoreF32;
     epi.out = dwhat;
-    OMQ_TRY(run_gemm(a->dt, A, B, N, K, M, epi, nullptr, st));
+    epi.out_scale = gscale;
+    OMQ_TRY(run_gemm(a->op_dt, A, B, N, K, M, epi, nullptr, st));
   }
   // weight-side STE: d gamma / d beta logits and the W-side LET column partials
   OMQ_TRY(ph.mark(OMQ_PH_STE_W));
@@ -353,25 +355,27 @@ static omq_status bwd_impl(const omq_bwd_args* a, void* workspace, size_t ws_byt
     OMQ_TRY(ph.mark(OMQ_PH_STE_X));
     return ph.mark(OMQ_PH_LET_REDUCE);
   }
-  // dXq = dY W^   [M, K]
+  // dXq = G W^   [M, K]
   {
     GemmOperand A{a->dY, N, false}, B{a->W_hat, K, true};
     GemmEpilogue epi{};
     epi.kind = Epi::StoreF32;
     epi.out = dxq;
-    OMQ_TRY(run_gemm(a->dt, A, B, M, K, N, epi, nullptr, st));
+    epi.out_scale = gscale;
+    OMQ_TRY(run_gemm(a->op_dt, A, B, M, K, N, epi, nullptr, st));
   }
   OMQ_TRY(ph.mark(OMQ_PH_STE_X));
   {
     SteXParams p{a->X, a->dt, M, K,
                  static_cast<float>((1 << (a->abits < 16 ? a->abits : 1)) - 1),
-                 a->abits < 16 ? 1 : 0, a->s, a->delta, a->h_a, a->z_a, a->tok_range, dxq, part_xs,
-                 part_xd, kRowsX};
+                 a->abits < 16 ? 1 : 0, a->s, a->delta, a->h_a, a->z_a, a->tok_range, dxq,
+                 at<float>(workspace, L.rowstat), part_xs, part_xd, kRowsX};
     OMQ_TRY(launch_ste_x(p, st));
   }
   OMQ_TRY(ph.mark(OMQ_PH_LET_REDUCE));
-  if (a->d_s) OMQ_TRY(launch_reduce_cols(part_ws, L.rb_w, part_xs, L.rb_x, K, a->d_s, st));
-  if (a->d_delta) OMQ_TRY(launch_reduce_cols(part_wd, L.rb_w, part_xd, L.rb_x, K, a->d_delta, st));
+  if (a->d_s) OMQ_TRY(launch_reduce_cols(part_ws, L.rb_w, part_xs, L.rb_x, K, 1.f, a->d_s, st));
+  if (a->d_delta)
+    OMQ_TRY(launch_reduce_cols(part_wd, L.rb_w, part_xd, L.rb_x, K, 1.f, a->d_delta, st));
   return OMQ_OK;
 }
 
@@ -387,7 +391,8 @@ omq_status omq_adamw_step(float* param, const float* grad, float* m, float* v, i
   if (n == 0) return OMQ_OK;
   if (!param || !grad || !m || !v) return OMQ_ERR_NULL;
   if (step < 1) return OMQ_ERR_SHAPE;
-  return launch_adamw(param, grad, m, v, n, lr, beta1, beta2, eps, weight_decay, step,
+  const AdamSeg seg{param, grad, m, v, n, lr};
+  return launch_adamw(&seg, 1, beta1, beta2, eps, weight_decay, step,
                       reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -407,7 +412,9 @@ omq_status omq_calib_step(const omq_step_args* a, void* workspace, size_t ws_byt
   if (M < 1 || N < 1 || K < 1 || G < 1) return OMQ_ERR_SHAPE;
   if (a->step < 1) return OMQ_ERR_SHAPE;
   const bool let = a->let != 0;
-  const bool need_act = let || a->abits < 16;
+  if (!dtype_ok(a->dt) || !dtype_ok(a->op_dt)) return OMQ_ERR_DTYPE;
+  // X itself is the GEMM operand only without LET, activation quantization or conversion
+  const bool need_act = let || a->abits < 16 || a->op_dt != a->dt;
   if (let && (!a->s || !a->delta || !a->d_s || !a->d_delta || !a->m_s || !a->v_s || !a->m_delta ||
               !a->v_delta || !a->B_tilde))
     return OMQ_ERR_NULL;
@@ -421,17 +428,18 @@ omq_status omq_calib_step(const omq_step_args* a, void* workspace, size_t ws_byt
   OMQ_TRY(ph.mark(OMQ_PH_LET));
   if (need_act) {
     OMQ_TRY(omq_let_apply(a->X, a->dt, M, K, let ? a->s : nullptr, let ? a->delta : nullptr,
-                          a->abits, a->Xq, a->dt, a->h_a, a->z_a, a->tok_range, a->W, a->dt, N,
-                          a->B, let ? a->B_tilde : nullptr, stream));
+                          a->abits, a->Xq, a->op_dt, a->h_a, a->z_a, a->tok_range, a->W, a->dt,
+                          N, a->B, let ? a->B_tilde : nullptr, stream));
   }
   OMQ_TRY(ph.mark(OMQ_PH_LWC));
   OMQ_TRY(omq_lwc_quant(a->W, a->dt, N, K, G, a->bits, a->gamma_logit, a->beta_logit,
-                        let ? a->s : nullptr, a->W_hat, a->dt, a->h, a->z, nullptr, a->grp_range,
-                        stream));
-  OMQ_TRY(fwd_impl(Xq, a->W_hat, a->dt, M, N, K, Bt, a->Y_ref, nullptr, a->dY, a->loss, workspace,
-                   fwd_ws, stream, ph));
+                        let ? a->s : nullptr, a->W_hat, a->op_dt, a->h, a->z, nullptr,
+                        a->grp_range, stream));
+  OMQ_TRY(fwd_impl(Xq, a->W_hat, a->op_dt, M, N, K, Bt, a->Y_ref, nullptr, a->dY, a->loss,
+                   workspace, fwd_ws, stream, ph));
   omq_bwd_args b{};
   b.M = M; b.N = N; b.K = K; b.group = G; b.bits = a->bits; b.abits = a->abits; b.dt = a->dt;
+  b.op_dt = a->op_dt;
   b.X = a->X; b.W = a->W; b.s = let ? a->s : nullptr; b.delta = let ? a->delta : nullptr;
   b.gamma_logit = a->gamma_logit; b.beta_logit = a->beta_logit;
   b.Xq = Xq; b.W_hat = a->W_hat; b.h = a->h; b.z = a->z; b.grp_range = a->grp_range;
@@ -441,16 +449,13 @@ omq_status omq_calib_step(const omq_step_args* a, void* workspace, size_t ws_byt
   OMQ_TRY(bwd_impl(&b, static_cast<char*>(workspace) + fwd_ws, ws_bytes - fwd_ws, stream, ph));
   OMQ_TRY(ph.mark(OMQ_PH_ADAMW));
   const int64_t ng = N * (K / G);
-  OMQ_TRY(omq_adamw_step(a->gamma_logit, a->d_gamma_logit, a->m_gamma, a->v_gamma, ng, a->lr_lwc,
-                         0.9f, 0.999f, 1e-8f, 0.f, a->step, stream));
-  OMQ_TRY(omq_adamw_step(a->beta_logit, a->d_beta_logit, a->m_beta, a->v_beta, ng, a->lr_lwc,
-                         0.9f, 0.999f, 1e-8f, 0.f, a->step, stream));
-  if (let) {
-    OMQ_TRY(omq_adamw_step(a->s, a->d_s, a->m_s, a->v_s, K, a->lr_let, 0.9f, 0.999f, 1e-8f, 0.f,
-                           a->step, stream));
-    OMQ_TRY(omq_adamw_step(a->delta, a->d_delta, a->m_delta, a->v_delta, K, a->lr_let, 0.9f,
-                           0.999f, 1e-8f, 0.f, a->step, stream));
-  }
+  const AdamSeg segs[kMaxAdamSegs] = {
+      {a->gamma_logit, a->d_gamma_logit, a->m_gamma, a->v_gamma, ng, a->lr_lwc},
+      {a->beta_logit, a->d_beta_logit, a->m_beta, a->v_beta, ng, a->lr_lwc},
+      {a->s, a->d_s, a->m_s, a->v_s, K, a->lr_let},
+      {a->delta, a->d_delta, a->m_delta, a->v_delta, K, a->lr_let}};
+  OMQ_TRY(launch_adamw(segs, let ? 4 : 2, 0.9f, 0.999f, 1e-8f, 0.f, a->step,
+                       reinterpret_cast<cudaStream_t>(stream)));
   return ph.mark(OMQ_PH_COUNT);
 }
 

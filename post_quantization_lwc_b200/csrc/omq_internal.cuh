@@ -5,6 +5,7 @@
 
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 #include <cmath>
@@ -25,13 +26,15 @@ constexpr int Z_LIMIT = 1 << 30;          // |z| stored as int32 is clamped to t
 // ---- element access --------------------------------------------------------------------
 __device__ __forceinline__ float load_elem(const void* p, int64_t i, omq_dtype dt) {
   if (dt == OMQ_BF16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[i]);
+  if (dt == OMQ_F16) return __half2float(reinterpret_cast<const __half*>(p)[i]);
   return reinterpret_cast<const float*>(p)[i];
 }
 __device__ __forceinline__ void store_elem(void* p, int64_t i, float v, omq_dtype dt) {
   if (dt == OMQ_BF16) reinterpret_cast<__nv_bfloat16*>(p)[i] = __float2bfloat16_rn(v);
+  else if (dt == OMQ_F16) reinterpret_cast<__half*>(p)[i] = __float2half_rn(v);
   else reinterpret_cast<float*>(p)[i] = v;
 }
-// 8 consecutive elements (16 B of bf16 or 32 B of f32) starting at a multiple of 8.
+// 8 consecutive elements (16 B of a 16-bit type or 32 B of f32) starting at a multiple of 8.
 __device__ __forceinline__ void load8(const void* p, int64_t i, omq_dtype dt, float (&v)[8]) {
   if (dt == OMQ_BF16) {
     uint4 raw = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(p) + i);
@@ -39,6 +42,15 @@ __device__ __forceinline__ void load8(const void* p, int64_t i, omq_dtype dt, fl
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       float2 f = __bfloat1622float2(b2[j]);
+      v[2 * j] = f.x;
+      v[2 * j + 1] = f.y;
+    }
+  } else if (dt == OMQ_F16) {
+    uint4 raw = *reinterpret_cast<const uint4*>(reinterpret_cast<const __half*>(p) + i);
+    const __half2* h2 = reinterpret_cast<const __half2*>(&raw);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float2 f = __half22float2(h2[j]);
       v[2 * j] = f.x;
       v[2 * j + 1] = f.y;
     }
@@ -56,6 +68,12 @@ __device__ __forceinline__ void store8(void* p, int64_t i, omq_dtype dt, const f
 #pragma unroll
     for (int j = 0; j < 4; ++j) b2[j] = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
     *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p) + i) = raw;
+  } else if (dt == OMQ_F16) {
+    uint4 raw;
+    __half2* h2 = reinterpret_cast<__half2*>(&raw);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) h2[j] = __floats2half2_rn(v[2 * j], v[2 * j + 1]);
+    *reinterpret_cast<uint4*>(reinterpret_cast<__half*>(p) + i) = raw;
   } else {
     float4* q = reinterpret_cast<float4*>(reinterpret_cast<float*>(p) + i);
     q[0] = make_float4(v[0], v[1], v[2], v[3]);
@@ -85,18 +103,35 @@ __device__ __forceinline__ GroupQ group_params(float g, float b, float vmax, flo
   return r;
 }
 
+// Round to nearest, ties to even, for |x| < 2^22, with two additions: x + 1.5*2^23 lands in
+// [2^23, 2^24) where the spacing of binary32 is 1, so the addition itself rounds x to an
+// integer in round-to-nearest-even mode, and the subtraction is exact. Same result as rintf,
+// on the FMA pipe.
+__device__ __forceinline__ float rne_small(float x) {
+  return __fsub_rn(__fadd_rn(x, 12582912.f), 12582912.f);
+}
+
 // round(v / h) with v / h the correctly rounded binary32 quotient.
 //
 // The quotient matters only through round(). With hinv = 1/h correctly rounded, the
 // product v*hinv differs from v/h by at most 2^-23 |v/h| (two roundings), i.e. below
-// 2.5e-4 while |v*hinv| < 2048. round() of the product therefore equals round() of the
-// quotient unless the product lies within 1e-3 of a half-integer; in that case, and for
-// large quotients, the IEEE division itself is taken. The result is bitwise the level an
-// exact-division implementation produces, at the cost of a multiply in almost all cases.
+// 2.5e-4 while |v*hinv| < 2048. If the product's distance to its nearest integer r is at
+// most 0.499, the quotient lies within 0.49925 of r and rounds to r as well; otherwise (the
+// product within 1e-3 of a half-integer) and for large quotients the IEEE division itself is
+// taken. The result is bitwise the level an exact-division implementation produces.
 __device__ __forceinline__ float round_quotient(float v, float h, float hinv) {
-  float ua = __fmul_rn(v, hinv);
-  if (fabsf(ua) >= 2048.f || fabsf(ua - floorf(ua) - 0.5f) < 1e-3f) ua = __fdiv_rn(v, h);
-  return rintf(ua);
+  const float ua = __fmul_rn(v, hinv);
+  if (fabsf(ua) < 2048.f) {
+    const float r = rne_small(ua);
+    if (fabsf(__fsub_rn(ua, r)) <= 0.499f) return r;
+  }
+  return rintf(__fdiv_rn(v, h));
+}
+
+// Integer value of an integral binary32 c in [0, 2^23): adding 2^23 leaves c in the low
+// mantissa bits.
+__device__ __forceinline__ uint32_t small_uint(float c) {
+  return __float_as_uint(__fadd_rn(c, 8388608.f)) & 0x7FFFFFu;
 }
 
 __device__ __forceinline__ int32_t z_to_i32(float z) {
@@ -110,6 +145,9 @@ omq_status launch_status();          // checks cudaGetLastError after a launch
 int num_sms();
 
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+// Groups handled lane-parallel inside a warp (16 to 256 elements, power of two); other group
+// lengths take the block-per-group kernels.
+inline bool small_group(int64_t g) { return g >= 16 && g <= 256 && (g & (g - 1)) == 0; }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // ---- GEMM front ends (gemm_tc.cu / gemm_simt.cu) -----------------------------------------
@@ -128,17 +166,18 @@ struct GemmEpilogue {
   float* out;              // StoreF32: [rows, cols] fp32 (ld = cols); MseLoss: Y or NULL
   const float* bias;       // per column j, or NULL
   const float* y_ref;      // MseLoss: [rows, cols]
-  void* dy;                // MseLoss: [rows, cols] in dy_dt
+  void* dy;                // MseLoss: [rows, cols] residual in dy_dt
   omq_dtype dy_dt;
-  float dy_scale;          // 2 / (rows * cols)
-  float* loss_partials;    // MseLoss: one per CTA tile (fixed order)
+  float out_scale;         // StoreF32: out = out_scale * acc (+ bias)
+  float* loss_partials;    // MseLoss: one per output tile (fixed order)
 };
 
-// bf16 operands on tcgen05 (sm_100a). Returns the number of CTA tiles launched.
-omq_status gemm_bf16_tc(const GemmOperand& A, const GemmOperand& B, int64_t rows, int64_t cols,
-                        int64_t depth, const GemmEpilogue& epi, int64_t* n_tiles,
-                        cudaStream_t stream);
-int64_t gemm_bf16_tc_tiles(int64_t rows, int64_t cols);
+// 16-bit operands (BF16 or F16, both the same type) on tcgen05 (sm_100a). Reports the
+// number of output tiles (loss partial slots).
+omq_status gemm_tc(omq_dtype dt, const GemmOperand& A, const GemmOperand& B, int64_t rows,
+                   int64_t cols, int64_t depth, const GemmEpilogue& epi, int64_t* n_tiles,
+                   cudaStream_t stream);
+int64_t gemm_tc_tiles(int64_t rows, int64_t cols);
 // f32 operands on CUDA cores.
 omq_status gemm_f32_simt(const GemmOperand& A, const GemmOperand& B, int64_t rows, int64_t cols,
                          int64_t depth, const GemmEpilogue& epi, int64_t* n_tiles,
@@ -211,10 +250,22 @@ struct SteXParams {
   const int32_t* z_a;
   const omq_range* range;
   const float* dXq;     // [M,K] fp32
+  float* rowstat;       // [M, 2] scratch: gradient share of each token's max / min element
   float* part_s;        // [row blocks, K]: -sum_m dX~ X~ / s
   float* part_d;        // [row blocks, K]: -sum_m dX~ / s
   int rows_per_block;
 };
+
+// One parameter tensor of a fused AdamW launch.
+struct AdamSeg {
+  float* p;
+  const float* g;
+  float* m;
+  float* v;
+  int64_t n;
+  float lr;
+};
+constexpr int kMaxAdamSegs = 4;
 
 omq_status launch_lwc(const LwcParams& p, cudaStream_t stream);
 omq_status launch_let(const LetParams& p, int abits, cudaStream_t stream);
@@ -225,11 +276,10 @@ omq_status launch_ste_x(const SteXParams& p, cudaStream_t stream);
 omq_status launch_colsum(const void* A, omq_dtype dt, int64_t rows, int64_t cols, int R,
                          float* part, cudaStream_t stream);
 omq_status launch_reduce_cols(const float* p0, int64_t r0n, const float* p1, int64_t r1n,
-                              int64_t cols, float* out, cudaStream_t stream);
+                              int64_t cols, float scale, float* out, cudaStream_t stream);
 omq_status launch_loss_finalize(const float* part, int64_t n, double inv_count, float* loss,
                                 cudaStream_t stream);
-omq_status launch_adamw(float* p, const float* g, float* m, float* v, int64_t n, float lr,
-                        float b1, float b2, float eps, float wd, int64_t step,
-                        cudaStream_t stream);
+omq_status launch_adamw(const AdamSeg* segs, int nseg, float b1, float b2, float eps, float wd,
+                        int64_t step, cudaStream_t stream);
 
 }  // namespace omq

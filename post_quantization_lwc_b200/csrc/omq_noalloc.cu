@@ -11,7 +11,7 @@
 //
 // Limits and sharing:
 //   - The array holds kNoAllocTiles partial sums. A problem needs ceil(M/128) * ceil(N/256)
-//     of them on the bf16 tensor-core path, or ceil(M/64) * ceil(N/64) on the float32 path;
+//     of them on the 16-bit tensor-core path, or ceil(M/64) * ceil(N/64) on the float32 path;
 //     larger problems are rejected with OMQ_ERR_SHAPE before anything is launched.
 //   - Every GPU that loads the library holds the array (64 KiB) until the process exits.
 //   - All calls on a device share the one array, and it keeps the last call's contents.
@@ -70,14 +70,14 @@ extern "C" omq_status omq_fq_linear_fwd_noalloc(const void* Xq, const void* W_ha
                                                 float* Y, void* dY, float* loss,
                                                 omq_stream_t stream) {
   if (!Xq || !W_hat || !Y_ref || !dY || !loss) return OMQ_ERR_NULL;
-  if (dt != OMQ_F32 && dt != OMQ_BF16) return OMQ_ERR_DTYPE;
+  if (dt != OMQ_F32 && dt != OMQ_BF16 && dt != OMQ_F16) return OMQ_ERR_DTYPE;
   const int64_t kMax = (int64_t(1) << 31) - 1;
   if (M < 1 || N < 8 || K < 8 || N % 8 || K % 8 || M > kMax || N > kMax || K > kMax)
     return OMQ_ERR_SHAPE;
   if (!aligned16(Xq) || !aligned16(W_hat) || !aligned16(Y_ref) || !aligned16(dY) ||
       (B_tilde && !aligned16(B_tilde)) || (Y && !aligned16(Y)))
     return OMQ_ERR_ALIGN;
-  const int64_t tiles = dt == OMQ_BF16 ? gemm_bf16_tc_tiles(M, N) : gemm_f32_simt_tiles(M, N);
+  const int64_t tiles = dt != OMQ_F32 ? gemm_tc_tiles(M, N) : gemm_f32_simt_tiles(M, N);
   if (tiles > kNoAllocTiles) return OMQ_ERR_SHAPE;
   float* partials = nullptr;
   omq_status st = noalloc_scratch(&partials);
@@ -91,11 +91,10 @@ extern "C" omq_status omq_fq_linear_fwd_noalloc(const void* Xq, const void* W_ha
   epi.y_ref = Y_ref;
   epi.dy = dY;
   epi.dy_dt = dt;
-  epi.dy_scale = static_cast<float>(2.0 / (static_cast<double>(M) * static_cast<double>(N)));
   epi.loss_partials = partials;
   int64_t launched = 0;
-  st = dt == OMQ_BF16 ? gemm_bf16_tc(A, B, M, N, K, epi, &launched, s)
-                      : gemm_f32_simt(A, B, M, N, K, epi, &launched, s);
+  st = dt != OMQ_F32 ? gemm_tc(dt, A, B, M, N, K, epi, &launched, s)
+                     : gemm_f32_simt(A, B, M, N, K, epi, &launched, s);
   if (st != OMQ_OK) return st;
   return launch_loss_finalize(partials, launched,
                               1.0 / (static_cast<double>(M) * static_cast<double>(N)), loss, s);

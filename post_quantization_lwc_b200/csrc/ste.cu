@@ -12,9 +12,11 @@
 // rounding passes gradients straight through, "OmniQuant：端侧大模型低比特量化的新思路与实战"
 // section 2.2.)
 //
-// LET gradients are column sums over rows; every kernel writes per-(row block, column)
-// partial sums which reduce_cols_kernel adds in a fixed order, so results are bitwise
-// reproducible (no floating-point atomics).
+// The in-range / clipped decisions repeat the forward's binary32 arithmetic exactly; the
+// gradient values use a fast binary32 sigmoid for g and b. LET gradients are column sums
+// over rows: kernels write per-(row block, column) partial sums that reduce_cols_kernel adds
+// in a fixed order, so results are bitwise reproducible (no floating-point atomics). The
+// memory-bound kernels issue the loads of several rows before computing on any of them.
 #include "omq_internal.cuh"
 
 namespace omq {
@@ -36,6 +38,19 @@ __device__ __forceinline__ GroupGrad group_grad(float Gh, float Gz, float g, flo
   return r;
 }
 
+// Clipping strength used in gradient values (never in an integer decision).
+__device__ __forceinline__ float strength_value(float logit) {
+  return 1.f / (1.f + __expf(-logit));
+}
+
+// Whether h's own gradient reaches g, b and the range: the stored h is max(h_raw, floor),
+// so h above the floor means h == h_raw; at the floor h_raw is recomputed exactly.
+__device__ __forceinline__ bool h_active(float h, float gl, float bl, float vmax, float vmin,
+                                         float Q) {
+  if (h > H_FLOOR) return true;
+  return group_params(strength(gl), strength(bl), vmax, vmin, Q).active;
+}
+
 // Per-element STE pieces for 8 values: in-range mask and the G_h / G_z contributions.
 __device__ __forceinline__ void ste8(const float (&v)[8], const float (&dq)[8], float h,
                                      float z, float Q, bool (&inr)[8], float& Gh, float& Gz) {
@@ -52,6 +67,16 @@ __device__ __forceinline__ void ste8(const float (&v)[8], const float (&dq)[8], 
   }
 }
 
+__device__ __forceinline__ void in_range8(const float (&v)[8], float h, float z, float Q,
+                                          bool (&inr)[8]) {
+  const float hinv = __frcp_rn(h);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float lvl = __fadd_rn(round_quotient(v[i], h, hinv), z);
+    inr[i] = lvl >= 0.f && lvl <= Q;
+  }
+}
+
 __device__ __forceinline__ void load_f8(const float* p, int64_t off, float (&v)[8]) {
   const float4* q = reinterpret_cast<const float4*>(p + off);
   const float4 a = q[0], b = q[1];
@@ -59,85 +84,113 @@ __device__ __forceinline__ void load_f8(const float* p, int64_t off, float (&v)[
 }
 
 // ------------------------------------------------------------------ weight side, G <= 256
-// grid (n_groups, row blocks); a sub-warp of G/8 lanes walks the rows of its block.
-template <int LPG>
-__global__ void __launch_bounds__(256) ste_w_small_kernel(SteWParams p) {
-  constexpr int SPW = 32 / LPG;
-  constexpr int NSUB = 8 * SPW;
-  __shared__ float red_s[NSUB * LPG * 8];
-  __shared__ float red_d[NSUB * LPG * 8];
-  const int lane = threadIdx.x & 31;
-  const int sw = (threadIdx.x >> 5) * SPW + lane / LPG;
+// grid (256-column segments, row blocks); a warp covers one row of the segment (lane = 8
+// columns; G/8 lanes per group), the 8 warps take every 8th row, U rows per iteration. A
+// lane's columns (and so its column partial sums) stay fixed; the warps' partials are added
+// in shared memory in warp order at the end.
+template <int LPG, int U>
+__global__ void __launch_bounds__(256, 2) ste_w_small_kernel(SteWParams p) {
+  __shared__ float red_s[8][256];
+  __shared__ float red_d[8][256];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int lig = lane % LPG;
-  const int64_t j = blockIdx.x;
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * 256 + lane * 8;
+  const bool cvalid = c0 < p.K;
+  const int64_t j = c0 / (LPG * 8);
   const int64_t rb = blockIdx.y;
   const int64_t r0 = rb * p.rows_per_block;
   const int64_t r1 = min(p.N, r0 + p.rows_per_block);
-  const int64_t col = j * p.G + lig * 8;
   float acc_s[8] = {}, acc_d[8] = {};
   float sv[8];
-  if (p.s) load_f8(p.s, col, sv);
-  // rows are visited in lockstep by all sub-warps of a warp (shuffles need full warps)
-  for (int64_t nb = r0; nb < r1; nb += NSUB) {
-    const int64_t n = nb + sw;
-    const bool valid = n < r1;
-    const int64_t gi = (valid ? n : r0) * p.ng + j;
-    const int64_t off = (valid ? n : r0) * p.K + col;
-    float w[8], wt[8], dq[8];
-    load8(p.W, off, p.wdt, w);
+  if (p.s && cvalid) {
+    load_f8(p.s, c0, sv);
+  } else {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) wt[i] = p.s ? __fmul_rn(w[i], sv[i]) : w[i];
-    load_f8(p.dWhat, off, dq);
-    const float h = p.h[gi];
-    const float z = static_cast<float>(p.z[gi]);
-    const omq_range rg = p.range[gi];
-    bool inr[8];
-    float Gh = 0.f, Gz = 0.f;
-    ste8(wt, dq, h, z, p.Q, inr, Gh, Gz);
+    for (int i = 0; i < 8; ++i) sv[i] = 1.f;
+  }
+  for (int64_t nb = r0 + w; nb < r1; nb += 8 * U) {
+    float wv[U][8], dq[U][8], h[U], z[U], glv[U], blv[U];
+    omq_range rg[U];
 #pragma unroll
-    for (int o = LPG / 2; o > 0; o >>= 1) {
-      Gh += __shfl_xor_sync(0xffffffffu, Gh, o);
-      Gz += __shfl_xor_sync(0xffffffffu, Gz, o);
-    }
-    if (!valid) continue;
-    const float g = strength(p.gl[gi]), b = strength(p.bl[gi]);
-    const bool active = group_params(g, b, rg.vmax, rg.vmin, p.Q).active;
-    const GroupGrad gg = group_grad(Gh, Gz, g, b, h, rg.vmax, rg.vmin, p.Q, active);
-    if (lig == 0) {
-      if (p.d_gl) p.d_gl[gi] = gg.dg * g * (1.f - g);
-      if (p.d_bl) p.d_bl[gi] = gg.db * b * (1.f - b);
-    }
-    if (p.part_s) {
-      const float eM = gg.dM / static_cast<float>(rg.nmax), em = gg.dm / static_cast<float>(rg.nmin);
+    for (int u = 0; u < U; ++u) {
+      const int64_t n = nb + 8 * u;
+      if (n < r1 && cvalid) {
+        const int64_t gi = n * p.ng + j;
+        load8(p.W, n * p.K + c0, p.wdt, wv[u]);
+        load_f8(p.dWhat, n * p.K + c0, dq[u]);
+        h[u] = p.h[gi];
+        z[u] = static_cast<float>(p.z[gi]);
+        rg[u] = p.range[gi];
+        glv[u] = p.gl[gi];
+        blv[u] = p.bl[gi];
+      } else {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        float dwt = inr[i] ? dq[i] : 0.f;
-        if (wt[i] == rg.vmax) dwt += eM;
-        if (wt[i] == rg.vmin) dwt += em;
-        acc_s[i] += dwt * w[i];
+        for (int i = 0; i < 8; ++i) { wv[u][i] = 0.f; dq[u][i] = 0.f; }
+        h[u] = 1.f;
+        z[u] = 0.f;
+        rg[u] = omq_range{0.f, 0.f, 1, 1};
+        glv[u] = 0.f;
+        blv[u] = 0.f;
       }
     }
-    if (p.part_d) {
-      const float db_n = p.dBt[n];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc_d[i] += db_n * w[i];
+    for (int u = 0; u < U; ++u) {
+      const int64_t n = nb + 8 * u;
+      float wt[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) wt[i] = p.s ? __fmul_rn(wv[u][i], sv[i]) : wv[u][i];
+      bool inr[8];
+      float Gh = 0.f, Gz = 0.f;
+      ste8(wt, dq[u], h[u], z[u], p.Q, inr, Gh, Gz);
+#pragma unroll
+      for (int o = LPG / 2; o > 0; o >>= 1) {
+        Gh += __shfl_xor_sync(0xffffffffu, Gh, o);
+        Gz += __shfl_xor_sync(0xffffffffu, Gz, o);
+      }
+      if (n >= r1 || !cvalid) continue;
+      const float g = strength_value(glv[u]), b = strength_value(blv[u]);
+      const bool active = h_active(h[u], glv[u], blv[u], rg[u].vmax, rg[u].vmin, p.Q);
+      const GroupGrad gg = group_grad(Gh, Gz, g, b, h[u], rg[u].vmax, rg[u].vmin, p.Q, active);
+      if (lig == 0) {
+        const int64_t gi = n * p.ng + j;
+        if (p.d_gl) p.d_gl[gi] = gg.dg * g * (1.f - g);
+        if (p.d_bl) p.d_bl[gi] = gg.db * b * (1.f - b);
+      }
+      if (p.part_s) {
+        const float eM = gg.dM / static_cast<float>(rg[u].nmax);
+        const float em = gg.dm / static_cast<float>(rg[u].nmin);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          float dwt = inr[i] ? dq[u][i] : 0.f;
+          if (wt[i] == rg[u].vmax) dwt += eM;
+          if (wt[i] == rg[u].vmin) dwt += em;
+          acc_s[i] += dwt * wv[u][i];
+        }
+      }
+      if (p.part_d) {
+        const float db_n = p.dBt[n];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc_d[i] += db_n * wv[u][i];
+      }
     }
   }
   if (!p.part_s && !p.part_d) return;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    red_s[sw * LPG * 8 + lig * 8 + i] = acc_s[i];
-    red_d[sw * LPG * 8 + lig * 8 + i] = acc_d[i];
+    red_s[w][lane * 8 + i] = acc_s[i];
+    red_d[w][lane * 8 + i] = acc_d[i];
   }
   __syncthreads();
-  for (int c = threadIdx.x; c < LPG * 8; c += blockDim.x) {
+  const int64_t col = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
+  if (col < p.K) {
     float a = 0.f, d = 0.f;
-    for (int q = 0; q < NSUB; ++q) {
-      a += red_s[q * LPG * 8 + c];
-      d += red_d[q * LPG * 8 + c];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      a += red_s[q][threadIdx.x];
+      d += red_d[q][threadIdx.x];
     }
-    if (p.part_s) p.part_s[rb * p.K + j * p.G + c] = a;
-    if (p.part_d) p.part_d[rb * p.K + j * p.G + c] = d;
+    if (p.part_s) p.part_s[rb * p.K + col] = a;
+    if (p.part_d) p.part_d[rb * p.K + col] = d;
   }
 }
 
@@ -192,8 +245,9 @@ __global__ void __launch_bounds__(256) ste_w_large_kernel(SteWParams p) {
       ste8(w, dq, h, z, p.Q, inr, Gh, Gz);
     }
     block_sum2(Gh, Gz, sm);
-    const float g = strength(p.gl[gi]), b = strength(p.bl[gi]);
-    const bool active = group_params(g, b, rg.vmax, rg.vmin, p.Q).active;
+    const float glv = p.gl[gi], blv = p.bl[gi];
+    const float g = strength_value(glv), b = strength_value(blv);
+    const bool active = h_active(h, glv, blv, rg.vmax, rg.vmin, p.Q);
     const GroupGrad gg = group_grad(Gh, Gz, g, b, h, rg.vmax, rg.vmin, p.Q, active);
     if (threadIdx.x == 0) {
       if (p.d_gl) p.d_gl[gi] = gg.dg * g * (1.f - g);
@@ -216,8 +270,7 @@ __global__ void __launch_bounds__(256) ste_w_large_kernel(SteWParams p) {
       }
       load_f8(p.dWhat, base + c * 8, dq);
       bool inr[8];
-      float dummy_h = 0.f, dummy_z = 0.f;
-      ste8(wt, dq, h, z, p.Q, inr, dummy_h, dummy_z);
+      in_range8(wt, h, z, p.Q, inr);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         float dwt = inr[i] ? dq[i] : 0.f;
@@ -238,115 +291,209 @@ __global__ void __launch_bounds__(256) ste_w_large_kernel(SteWParams p) {
 }
 
 // ------------------------------------------------------------------ activation side
-// grid (row blocks); one group per token row (K columns), g = b = 1, no parameters.
-__global__ void __launch_bounds__(256) ste_x_kernel(SteXParams p) {
-  extern __shared__ float acc[];   // 2 * K floats
+__device__ __forceinline__ void xtilde8(const SteXParams& p, int64_t off, const float (&sv)[8],
+                                        const float (&dv)[8], float (&v)[8]) {
+  load8(p.X, off, p.xdt, v);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __fdiv_rn(__fsub_rn(v[i], dv[i]), sv[i]);
+}
+
+__device__ __forceinline__ void let_vectors(const SteXParams& p, int64_t col, float (&sv)[8],
+                                            float (&dv)[8]) {
+  if (p.s) {
+    load_f8(p.s, col, sv);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) sv[i] = 1.f;
+  }
+  if (p.d) {
+    load_f8(p.d, col, dv);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) dv[i] = 0.f;
+  }
+}
+
+// Per token (quantized activations): the gradient share of the token's max and min elements,
+// from the token's G_h and G_z sums (g = b = 1).
+__global__ void __launch_bounds__(256) ste_x_rowstat_kernel(SteXParams p) {
   __shared__ float sm[64];
-  float* acc_s = acc;
-  float* acc_d = acc + p.K;
-  const int64_t rb = blockIdx.x;
-  const int64_t r0 = rb * p.rows_per_block, r1 = min(p.M, r0 + p.rows_per_block);
   const int chunks = static_cast<int>(p.K / 8);
-  for (int c = threadIdx.x; c < chunks; c += blockDim.x)
-#pragma unroll
-    for (int i = 0; i < 8; ++i) { acc_s[c * 8 + i] = 0.f; acc_d[c * 8 + i] = 0.f; }
-
-  auto xt8 = [&](int64_t off, int64_t col, float (&v)[8], float (&sv)[8]) {
-    load8(p.X, off, p.xdt, v);
-    float dv[8];
-    if (p.s) load_f8(p.s, col, sv); else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) sv[i] = 1.f;
-    }
-    if (p.d) load_f8(p.d, col, dv); else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) dv[i] = 0.f;
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = __fdiv_rn(__fsub_rn(v[i], dv[i]), sv[i]);
-  };
-
-  for (int64_t m = r0; m < r1; ++m) {
+  for (int64_t m = blockIdx.x; m < p.M; m += gridDim.x) {
     const int64_t base = m * p.K;
-    float eM = 0.f, em = 0.f, h = 1.f, z = 0.f;
-    omq_range rg{0.f, 0.f, 1, 1};
-    if (p.quantized) {
-      h = p.h_a[m];
-      z = static_cast<float>(p.z_a[m]);
-      rg = p.range[m];
-      float Gh = 0.f, Gz = 0.f;
-      for (int c = threadIdx.x; c < chunks; c += blockDim.x) {
-        float v[8], sv[8], dq[8];
-        xt8(base + c * 8, c * 8, v, sv);
-        load_f8(p.dXq, base + c * 8, dq);
-        bool inr[8];
-        ste8(v, dq, h, z, p.Qa, inr, Gh, Gz);
-      }
-      block_sum2(Gh, Gz, sm);
+    const float h = p.h_a[m];
+    const float z = static_cast<float>(p.z_a[m]);
+    float Gh = 0.f, Gz = 0.f;
+    for (int c = threadIdx.x; c < chunks; c += blockDim.x) {
+      float sv[8], dv[8], v[8], dq[8];
+      let_vectors(p, c * 8, sv, dv);
+      xtilde8(p, base + c * 8, sv, dv, v);
+      load_f8(p.dXq, base + c * 8, dq);
+      bool inr[8];
+      ste8(v, dq, h, z, p.Qa, inr, Gh, Gz);
+    }
+    block_sum2(Gh, Gz, sm);
+    if (threadIdx.x == 0) {
+      const omq_range rg = p.range[m];
       const bool active = group_params(1.f, 1.f, rg.vmax, rg.vmin, p.Qa).active;
       const GroupGrad gg = group_grad(Gh, Gz, 1.f, 1.f, h, rg.vmax, rg.vmin, p.Qa, active);
-      eM = gg.dM / static_cast<float>(rg.nmax);
-      em = gg.dm / static_cast<float>(rg.nmin);
+      p.rowstat[2 * m] = gg.dM / static_cast<float>(rg.nmax);
+      p.rowstat[2 * m + 1] = gg.dm / static_cast<float>(rg.nmin);
     }
-    for (int c = threadIdx.x; c < chunks; c += blockDim.x) {
-      float v[8], sv[8], dq[8];
-      xt8(base + c * 8, c * 8, v, sv);
-      load_f8(p.dXq, base + c * 8, dq);
-      float dxt[8];
-      if (p.quantized) {
-        bool inr[8];
-        float dh = 0.f, dz = 0.f;
-        ste8(v, dq, h, z, p.Qa, inr, dh, dz);
+  }
+}
+
+// Column partials over row blocks: part_s[rb, k] = -sum_m dX~ X~ / s, part_d[rb, k] =
+// -sum_m dX~ / s. grid (column segments of 256, row blocks); each warp covers the segment
+// for every 8th row (lane = 8 columns), U rows per iteration.
+template <int U>
+__global__ void __launch_bounds__(256, 2) ste_x_cols_kernel(SteXParams p) {
+  __shared__ float red_s[8][256];
+  __shared__ float red_d[8][256];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * 256 + lane * 8;
+  const bool cvalid = c0 < p.K;
+  const int64_t rb = blockIdx.y;
+  const int64_t r0 = rb * p.rows_per_block, r1 = min(p.M, r0 + p.rows_per_block);
+  float sv[8], dv[8], rs[8];
+  let_vectors(p, cvalid ? c0 : 0, sv, dv);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          dxt[i] = inr[i] ? dq[i] : 0.f;
-          if (v[i] == rg.vmax) dxt[i] += eM;
-          if (v[i] == rg.vmin) dxt[i] += em;
-        }
+  for (int i = 0; i < 8; ++i) rs[i] = 1.f / sv[i];
+  float acc_s[8] = {}, acc_d[8] = {};
+  for (int64_t mb = r0 + w; mb < r1; mb += 8 * U) {
+    float v[U][8], dq[U][8];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t m = mb + 8 * u;
+      if (m < r1 && cvalid) {
+        load8(p.X, m * p.K + c0, p.xdt, v[u]);
+        load_f8(p.dXq, m * p.K + c0, dq[u]);
       } else {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) dxt[i] = dq[i];
+        for (int i = 0; i < 8; ++i) { v[u][i] = 0.f; dq[u][i] = 0.f; }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t m = mb + 8 * u;
+      if (m >= r1 || !cvalid) continue;
+      float dxt[8];
+      if (p.quantized) {
+        // the in-range decisions need X~ exactly as the forward computed it
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[u][i] = __fdiv_rn(__fsub_rn(v[u][i], dv[i]), sv[i]);
+        const omq_range rg = p.range[m];
+        bool inr[8];
+        in_range8(v[u], p.h_a[m], static_cast<float>(p.z_a[m]), p.Qa, inr);
+        const float eM = p.rowstat[2 * m], em = p.rowstat[2 * m + 1];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          dxt[i] = inr[i] ? dq[u][i] : 0.f;
+          if (v[u][i] == rg.vmax) dxt[i] += eM;
+          if (v[u][i] == rg.vmin) dxt[i] += em;
+        }
+      } else {
+        // values only: X~ through the reciprocal of s
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          v[u][i] = (v[u][i] - dv[i]) * rs[i];
+          dxt[i] = dq[u][i];
+        }
       }
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const float q = dxt[i] / sv[i];
-        acc_s[c * 8 + i] -= q * v[i];
-        acc_d[c * 8 + i] -= q;
+        const float q = dxt[i] * rs[i];
+        acc_s[i] += q * v[u][i];
+        acc_d[i] += q;
       }
     }
   }
-  for (int c = threadIdx.x; c < chunks; c += blockDim.x)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      p.part_s[rb * p.K + c * 8 + i] = acc_s[c * 8 + i];
-      p.part_d[rb * p.K + c * 8 + i] = acc_d[c * 8 + i];
+  for (int i = 0; i < 8; ++i) {
+    red_s[w][lane * 8 + i] = acc_s[i];
+    red_d[w][lane * 8 + i] = acc_d[i];
+  }
+  __syncthreads();
+  const int64_t col = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
+  if (col < p.K) {
+    float a = 0.f, d = 0.f;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      a += red_s[q][threadIdx.x];
+      d += red_d[q][threadIdx.x];
     }
+    p.part_s[rb * p.K + col] = -a;
+    p.part_d[rb * p.K + col] = -d;
+  }
 }
 
 // ------------------------------------------------------------------ column sums
-// part[rb, j] = sum over rows rb*R .. rb*R+R-1 of A[i, j]  (A [rows, cols] in dt)
+// part[rb, j] = sum of A[i, j] over the rows of row block rb (A [rows, cols] in dt, cols % 8
+// == 0). Same launch shape as ste_x_cols_kernel.
+template <int U>
 __global__ void __launch_bounds__(256) colsum_kernel(const void* A, omq_dtype dt, int64_t rows,
                                                      int64_t cols, int R, float* part) {
-  const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  __shared__ float red[8][256];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * 256 + lane * 8;
+  const bool cvalid = c0 < cols;
   const int64_t rb = blockIdx.y;
-  if (j >= cols) return;
   const int64_t r0 = rb * R, r1 = min(rows, r0 + R);
-  float a = 0.f;
-  for (int64_t i = r0; i < r1; ++i) a += load_elem(A, i * cols + j, dt);
-  part[rb * cols + j] = a;
+  float acc[8] = {};
+  for (int64_t mb = r0 + w; mb < r1; mb += 8 * U) {
+    float v[U][8];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t m = mb + 8 * u;
+      if (m < r1 && cvalid) {
+        load8(A, m * cols + c0, dt, v[u]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[u][i] = 0.f;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] += v[u][i];
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) red[w][lane * 8 + i] = acc[i];
+  __syncthreads();
+  const int64_t col = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
+  if (col < cols) {
+    float a = 0.f;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) a += red[q][threadIdx.x];
+    part[rb * cols + col] = a;
+  }
 }
 
-// out[j] = sum_r p0[r, j] (+ sum_r p1[r, j]), binary64 accumulation in row order.
+// out[j] = scale * (sum_r p0[r, j] (+ sum_r p1[r, j])), binary64 accumulation in a fixed
+// order: 8 warps take every 8th row of 32 consecutive columns, then combine in warp order.
 __global__ void __launch_bounds__(256) reduce_cols_kernel(const float* p0, int64_t r0n,
                                                           const float* p1, int64_t r1n,
-                                                          int64_t cols, float* out) {
-  const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (j >= cols) return;
+                                                          int64_t cols, float scale, float* out) {
+  __shared__ double red[8][32];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int64_t j = static_cast<int64_t>(blockIdx.x) * 32 + lane;
   double a = 0.0;
-  for (int64_t r = 0; r < r0n; ++r) a += p0[r * cols + j];
-  if (p1)
-    for (int64_t r = 0; r < r1n; ++r) a += p1[r * cols + j];
-  out[j] = static_cast<float>(a);
+  if (j < cols) {
+#pragma unroll 4
+    for (int64_t r = w; r < r0n; r += 8) a += p0[r * cols + j];
+    if (p1) {
+#pragma unroll 4
+      for (int64_t r = w; r < r1n; r += 8) a += p1[r * cols + j];
+    }
+  }
+  red[w][lane] = a;
+  __syncthreads();
+  if (w == 0 && j < cols) {
+    double t = 0.0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) t += red[q][lane];
+    out[j] = static_cast<float>(t * static_cast<double>(scale));
+  }
 }
 
 // loss = (sum of per-tile partials) / count, binary64, fixed order.
@@ -364,19 +511,24 @@ __global__ void __launch_bounds__(256) loss_finalize_kernel(const float* part, i
   if (threadIdx.x == 0) *loss = static_cast<float>(sm[0] * inv_count);
 }
 
-__global__ void __launch_bounds__(256) adamw_kernel(float* p, const float* g, float* m, float* v,
-                                                    int64_t n, float lr, float b1, float b2,
-                                                    float eps, float wd, float bc1, float bc2_sqrt) {
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+struct AdamSegs {
+  AdamSeg s[kMaxAdamSegs];
+};
+
+// AdamW over up to four parameter tensors in one launch (blockIdx.y selects the tensor).
+__global__ void __launch_bounds__(256) adamw_kernel(AdamSegs segs, float b1, float b2, float eps,
+                                                    float wd, float bc1, float bc2_sqrt) {
+  const AdamSeg sg = segs.s[blockIdx.y];
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < sg.n;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const float gi = g[i];
-    float pi = p[i] * (1.f - lr * wd);
-    const float mi = b1 * m[i] + (1.f - b1) * gi;
-    const float vi = b2 * v[i] + (1.f - b2) * gi * gi;
-    pi -= (lr / bc1) * mi / (sqrtf(vi) / bc2_sqrt + eps);
-    p[i] = pi;
-    m[i] = mi;
-    v[i] = vi;
+    const float gi = sg.g[i];
+    float pi = sg.p[i] * (1.f - sg.lr * wd);
+    const float mi = b1 * sg.m[i] + (1.f - b1) * gi;
+    const float vi = b2 * sg.v[i] + (1.f - b2) * gi * gi;
+    pi -= (sg.lr / bc1) * mi / (sqrtf(vi) / bc2_sqrt + eps);
+    sg.p[i] = pi;
+    sg.m[i] = mi;
+    sg.v[i] = vi;
   }
 }
 
@@ -384,18 +536,18 @@ __global__ void __launch_bounds__(256) adamw_kernel(float* p, const float* g, fl
 
 omq_status launch_ste_w(const SteWParams& p, cudaStream_t stream) {
   const int64_t rbs = ceil_div(p.N, p.rows_per_block);
-  dim3 grid(static_cast<unsigned>(p.ng), static_cast<unsigned>(rbs));
-  if (p.G <= 256 && (p.G & (p.G - 1)) == 0) {
+  if (small_group(p.G)) {
+    dim3 grid(static_cast<unsigned>(ceil_div(p.K, 256)), static_cast<unsigned>(rbs));
     switch (p.G / 8) {
-      case 1: ste_w_small_kernel<1><<<grid, 256, 0, stream>>>(p); break;
-      case 2: ste_w_small_kernel<2><<<grid, 256, 0, stream>>>(p); break;
-      case 4: ste_w_small_kernel<4><<<grid, 256, 0, stream>>>(p); break;
-      case 8: ste_w_small_kernel<8><<<grid, 256, 0, stream>>>(p); break;
-      case 16: ste_w_small_kernel<16><<<grid, 256, 0, stream>>>(p); break;
-      default: ste_w_small_kernel<32><<<grid, 256, 0, stream>>>(p); break;
+      case 2: ste_w_small_kernel<2, 2><<<grid, 256, 0, stream>>>(p); break;
+      case 4: ste_w_small_kernel<4, 2><<<grid, 256, 0, stream>>>(p); break;
+      case 8: ste_w_small_kernel<8, 2><<<grid, 256, 0, stream>>>(p); break;
+      case 16: ste_w_small_kernel<16, 2><<<grid, 256, 0, stream>>>(p); break;
+      default: ste_w_small_kernel<32, 2><<<grid, 256, 0, stream>>>(p); break;
     }
     return launch_status();
   }
+  dim3 grid(static_cast<unsigned>(p.ng), static_cast<unsigned>(rbs));
   const size_t smem = 2 * static_cast<size_t>(p.G) * sizeof(float);
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(ste_w_large_kernel,
@@ -408,28 +560,30 @@ omq_status launch_ste_w(const SteWParams& p, cudaStream_t stream) {
 }
 
 omq_status launch_ste_x(const SteXParams& p, cudaStream_t stream) {
-  const int64_t rbs = ceil_div(p.M, p.rows_per_block);
-  const size_t smem = 2 * static_cast<size_t>(p.K) * sizeof(float);
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(ste_x_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) { set_cuda_error(e); return OMQ_ERR_CUDA; }
+  if (p.quantized) {
+    const int sms = num_sms();
+    const unsigned grid = static_cast<unsigned>(p.M < int64_t(sms) * 8 ? p.M : int64_t(sms) * 8);
+    ste_x_rowstat_kernel<<<grid, 256, 0, stream>>>(p);
+    const omq_status st = launch_status();
+    if (st != OMQ_OK) return st;
   }
-  ste_x_kernel<<<static_cast<unsigned>(rbs), 256, smem, stream>>>(p);
+  dim3 grid(static_cast<unsigned>(ceil_div(p.K, 256)),
+            static_cast<unsigned>(ceil_div(p.M, p.rows_per_block)));
+  ste_x_cols_kernel<2><<<grid, 256, 0, stream>>>(p);
   return launch_status();
 }
 
 omq_status launch_colsum(const void* A, omq_dtype dt, int64_t rows, int64_t cols, int R,
                          float* part, cudaStream_t stream) {
   dim3 grid(static_cast<unsigned>(ceil_div(cols, 256)), static_cast<unsigned>(ceil_div(rows, R)));
-  colsum_kernel<<<grid, 256, 0, stream>>>(A, dt, rows, cols, R, part);
+  colsum_kernel<4><<<grid, 256, 0, stream>>>(A, dt, rows, cols, R, part);
   return launch_status();
 }
 
 omq_status launch_reduce_cols(const float* p0, int64_t r0n, const float* p1, int64_t r1n,
-                              int64_t cols, float* out, cudaStream_t stream) {
-  reduce_cols_kernel<<<static_cast<unsigned>(ceil_div(cols, 256)), 256, 0, stream>>>(
-      p0, r0n, p1, r1n, cols, out);
+                              int64_t cols, float scale, float* out, cudaStream_t stream) {
+  reduce_cols_kernel<<<static_cast<unsigned>(ceil_div(cols, 32)), 256, 0, stream>>>(
+      p0, r0n, p1, r1n, cols, scale, out);
   return launch_status();
 }
 
@@ -439,17 +593,23 @@ omq_status launch_loss_finalize(const float* part, int64_t n, double inv_count, 
   return launch_status();
 }
 
-omq_status launch_adamw(float* p, const float* g, float* m, float* v, int64_t n, float lr,
-                        float b1, float b2, float eps, float wd, int64_t step,
-                        cudaStream_t stream) {
+omq_status launch_adamw(const AdamSeg* segs, int nseg, float b1, float b2, float eps, float wd,
+                        int64_t step, cudaStream_t stream) {
+  if (nseg < 1 || nseg > kMaxAdamSegs) return OMQ_ERR_SHAPE;
+  AdamSegs s{};
+  int64_t nmax = 0;
+  for (int i = 0; i < nseg; ++i) {
+    s.s[i] = segs[i];
+    nmax = segs[i].n > nmax ? segs[i].n : nmax;
+  }
   const double bc1 = 1.0 - std::pow(static_cast<double>(b1), static_cast<double>(step));
   const double bc2 = 1.0 - std::pow(static_cast<double>(b2), static_cast<double>(step));
-  const int64_t want = ceil_div(n, 256);
   const int sms = num_sms();
-  const unsigned grid = static_cast<unsigned>(want < int64_t(sms) * 8 ? want : int64_t(sms) * 8);
-  adamw_kernel<<<grid > 0 ? grid : 1, 256, 0, stream>>>(p, g, m, v, n, lr, b1, b2, eps, wd,
-                                                        static_cast<float>(bc1),
-                                                        static_cast<float>(std::sqrt(bc2)));
+  const int64_t want = ceil_div(nmax, 256);
+  const unsigned gx = static_cast<unsigned>(want < int64_t(sms) * 4 ? want : int64_t(sms) * 4);
+  dim3 grid(gx > 0 ? gx : 1, static_cast<unsigned>(nseg));
+  adamw_kernel<<<grid, 256, 0, stream>>>(s, b1, b2, eps, wd, static_cast<float>(bc1),
+                                         static_cast<float>(std::sqrt(bc2)));
   return launch_status();
 }
 

@@ -20,7 +20,7 @@ if not os.path.exists(LIB_PATH):
                       "`python -m post_quantization_lwc_b200.build`")
 _lib = ctypes.CDLL(LIB_PATH)
 
-OMQ_F32, OMQ_BF16 = 0, 1
+OMQ_F32, OMQ_BF16, OMQ_F16 = 0, 1, 2
 STATUS = {0: "OMQ_OK", 1: "OMQ_ERR_NULL", 2: "OMQ_ERR_SHAPE", 3: "OMQ_ERR_DTYPE",
           4: "OMQ_ERR_ALIGN", 5: "OMQ_ERR_BITS", 6: "OMQ_ERR_WORKSPACE", 7: "OMQ_ERR_CUDA",
           8: "OMQ_ERR_UNSUPPORTED", 9: "OMQ_ERR_TIMEOUT"}
@@ -49,7 +49,7 @@ class OmqError(RuntimeError):
 
 class BwdArgs(ctypes.Structure):
     _fields_ = [("M", _i64), ("N", _i64), ("K", _i64), ("group", _i64), ("bits", _i32),
-                ("abits", _i32), ("dt", _i32),
+                ("abits", _i32), ("dt", _i32), ("op_dt", _i32),
                 ("X", _p), ("W", _p), ("s", _p), ("delta", _p), ("gamma_logit", _p),
                 ("beta_logit", _p), ("Xq", _p), ("W_hat", _p), ("h", _p), ("z", _p),
                 ("grp_range", _p), ("h_a", _p), ("z_a", _p), ("tok_range", _p), ("dY", _p),
@@ -59,7 +59,7 @@ class BwdArgs(ctypes.Structure):
 
 class StepArgs(ctypes.Structure):
     _fields_ = [("M", _i64), ("N", _i64), ("K", _i64), ("group", _i64), ("bits", _i32),
-                ("abits", _i32), ("let", _i32), ("dt", _i32),
+                ("abits", _i32), ("let", _i32), ("dt", _i32), ("op_dt", _i32),
                 ("X", _p), ("W", _p), ("B", _p), ("Y_ref", _p),
                 ("gamma_logit", _p), ("beta_logit", _p), ("s", _p), ("delta", _p),
                 ("m_gamma", _p), ("v_gamma", _p), ("m_beta", _p), ("v_beta", _p),
@@ -113,16 +113,20 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _dt(t: torch.Tensor) -> int:
-    if t.dtype == torch.bfloat16:
-        return OMQ_BF16
-    if t.dtype == torch.float32:
-        return OMQ_F32
-    raise TypeError(f"unsupported dtype {t.dtype}")
+_DTYPES = {torch.float32: OMQ_F32, torch.bfloat16: OMQ_BF16, torch.float16: OMQ_F16}
 
 
-def _tdt(code: int):
-    return torch.bfloat16 if code == OMQ_BF16 else torch.float32
+def _dt(t) -> int:
+    dtype = t if isinstance(t, torch.dtype) else t.dtype
+    if dtype not in _DTYPES:
+        raise TypeError(f"unsupported dtype {dtype}")
+    return _DTYPES[dtype]
+
+
+def operand_dtype(storage: torch.dtype) -> torch.dtype:
+    """GEMM operand dtype the step uses for a storage dtype: float16 for 16-bit storage
+    (3 more mantissa bits than bfloat16 at the same tensor-core rate), float32 otherwise."""
+    return torch.float32 if storage == torch.float32 else torch.float16
 
 
 def _stream(stream=None):
@@ -256,7 +260,7 @@ def fq_linear_bwd(*, X, W, gamma_logit, beta_logit, Xq, W_hat, h, z, grp_range, 
     out = dict(d_gamma_logit=f(N, K // group), d_beta_logit=f(N, K // group),
                d_s=f(K) if want_let else None, d_delta=f(K) if want_let else None,
                d_B_tilde=f(N) if want_dBt else None)
-    a = BwdArgs(M=M, N=N, K=K, group=group, bits=bits, abits=abits, dt=_dt(Xq),
+    a = BwdArgs(M=M, N=N, K=K, group=group, bits=bits, abits=abits, dt=_dt(W), op_dt=_dt(Xq),
                 X=_ptr(X), W=_ptr(W), s=_ptr(s), delta=_ptr(delta), gamma_logit=_ptr(gamma_logit),
                 beta_logit=_ptr(beta_logit), Xq=_ptr(Xq), W_hat=_ptr(W_hat), h=_ptr(h), z=_ptr(z),
                 grp_range=_ptr(grp_range), h_a=_ptr(h_a), z_a=_ptr(z_a), tok_range=_ptr(tok_range),
@@ -328,9 +332,10 @@ class LinearCalibration:
         self.s, self.delta = f(K), f(K)
         self.moments = {k: (f(*shape), f(*shape)) for k, shape in
                         (("gamma", (N, ng)), ("beta", (N, ng)), ("s", (K,)), ("delta", (K,)))}
-        need_act = self.let or self.abits < 16
-        self.Xq = torch.empty(M, K, dtype=self.dtype, device=dev) if need_act else None
-        self.W_hat = torch.empty(N, K, dtype=self.dtype, device=dev)
+        self.op_dtype = operand_dtype(self.dtype)
+        need_act = self.let or self.abits < 16 or self.op_dtype != self.dtype
+        self.Xq = torch.empty(M, K, dtype=self.op_dtype, device=dev) if need_act else None
+        self.W_hat = torch.empty(N, K, dtype=self.op_dtype, device=dev)
         self.B_tilde = f(N)
         self.h = f(N, ng)
         self.z = torch.zeros(N, ng, dtype=torch.int32, device=dev)
@@ -339,7 +344,7 @@ class LinearCalibration:
         self.h_a = f(M) if q else None
         self.z_a = torch.zeros(M, dtype=torch.int32, device=dev) if q else None
         self.tok_range = new_range(M, dev) if q else None
-        self.dY = torch.empty(M, N, dtype=self.dtype, device=dev)
+        self.dY = torch.empty(M, N, dtype=self.op_dtype, device=dev)
         self.d_gamma, self.d_beta = f(N, ng), f(N, ng)
         self.d_s, self.d_delta = f(K), f(K)
         self.loss = f(1)
@@ -366,7 +371,8 @@ class LinearCalibration:
         mo = self.moments
         return StepArgs(
             M=self.M, N=self.N, K=self.K, group=self.group, bits=self.bits, abits=self.abits,
-            let=1 if self.let else 0, dt=_dt(self.W), X=_ptr(X), W=_ptr(self.W), B=_ptr(self.B),
+            let=1 if self.let else 0, dt=_dt(self.W), op_dt=_dt(self.op_dtype), X=_ptr(X),
+            W=_ptr(self.W), B=_ptr(self.B),
             Y_ref=_ptr(Y_ref), gamma_logit=_ptr(self.gamma_logit), beta_logit=_ptr(self.beta_logit),
             s=_ptr(self.s), delta=_ptr(self.delta),
             m_gamma=_ptr(mo["gamma"][0]), v_gamma=_ptr(mo["gamma"][1]),

@@ -110,7 +110,7 @@ def test_fwd_validation(omq):
     assert f(FAKE, FAKE, 1, 64, 64, 64, None, FAKE, None, None, None, None, 0, None) == 1
     assert f(FAKE, FAKE, 1, 64, 64, 64, None, FAKE, None, FAKE, FAKE, None, 0, None) == 6
     assert f(FAKE, FAKE, 1, 64, 60, 64, None, FAKE, None, FAKE, FAKE, FAKE, 1 << 20, None) == 2
-    assert f(FAKE, FAKE, 2, 64, 64, 64, None, FAKE, None, FAKE, FAKE, FAKE, 1 << 20, None) == 3
+    assert f(FAKE, FAKE, 7, 64, 64, 64, None, FAKE, None, FAKE, FAKE, FAKE, 1 << 20, None) == 3
 
 
 def test_bwd_validation(omq):

@@ -7,8 +7,8 @@ import torch
 
 from oracle import omniquant as om
 from post_quantization_lwc_b200 import synth
-from tests.gpu_common import (SMALL_CASES, close, dtype_round, frob_rel, max_rel, oracle_step,
-                              prepare)
+from tests.gpu_common import (SMALL_CASES, TORCH, close, dtype_round, frob_rel, max_rel,
+                              operand, oracle_step, prepare)
 
 pytestmark = pytest.mark.gpu
 
@@ -32,11 +32,14 @@ def _dev(p, dev):
 
 
 def _gpu_forward(omq, p, d):
+    """The step's forward with the step's operand type (float16 for 16-bit storage)."""
     c = p.case
     s = d["s"] if c.let else None
-    lw = omq.lwc_quant(d["W"], d["gl"], d["bl"], c.bits, c.group, s=s, codes=True)
+    op = TORCH[operand(c.dtype)]
+    lw = omq.lwc_quant(d["W"], d["gl"], d["bl"], c.bits, c.group, s=s, codes=True,
+                       hat_dtype=op)
     la = omq.let_apply(d["X"], c.abits, s=s, delta=d["d"] if c.let else None, W=d["W"],
-                       B=d["B"], want_bias=True)
+                       B=d["B"], want_bias=True, xq_dtype=op)
     fw = omq.fq_linear_fwd(la["Xq"], lw["W_hat"], B_tilde=la["B_tilde"], Y_ref=d["Yref"])
     return lw, la, fw
 
@@ -100,13 +103,14 @@ def test_forward_loss(omq, cuda_device, case):
     r = oracle_step(p, need_backward=False)
     ok, e = close(_np(fw["Y"]), r.Y, case.dtype)
     assert ok, f"Y rel err {e}"
-    ok, e = close(_np(fw["dY"]), r.dY, case.dtype)
+    # dY holds the residual Y - Y*; the oracle's dL/dY is 2 (Y - Y*) / (M N)
+    ok, e = close(_np(fw["dY"]), r.dY * (case.M * case.N / 2.0), case.dtype)
     assert ok, f"dY rel err {e}"
     assert abs(fw["loss"].item() - r.loss) <= (1e-4 if case.dtype == "f32" else 2e-2) * r.loss
-    # the GEMM itself: fp64 product of the oracle's operands in the storage dtype; only the
+    # the GEMM itself: fp64 product of the oracle's operands in the operand dtype; only the
     # fp32 accumulation order differs
-    Xq = dtype_round(r.Xq, case.dtype).astype(np.float64)
-    Wq = dtype_round(r.wenc.deq, case.dtype).astype(np.float64)
+    Xq = dtype_round(r.Xq, operand(case.dtype)).astype(np.float64)
+    Wq = dtype_round(r.wenc.deq, operand(case.dtype)).astype(np.float64)
     Y_tight = Xq @ Wq.T + r.Bt[None, :]
     assert frob_rel(_np(fw["Y"]), Y_tight) <= 2e-6
 
@@ -211,6 +215,28 @@ def test_fold_pack_bit_exact(omq, cuda_device, case):
     assert np.array_equal(packed.cpu().numpy(), want)
     assert np.array_equal(h.cpu().numpy().view(np.uint32), wh.view(np.uint32))
     assert np.array_equal(z.cpu().numpy(), wz)
+
+
+@pytest.mark.parametrize("M,N,K,dtype", [(1024, 8192, 128, torch.bfloat16),
+                                         (600, 2824, 200, torch.float16),
+                                         (4096, 2048, 64, torch.float16)])
+def test_gemm_many_tiles_per_cta(omq, cuda_device, M, N, K, dtype):
+    """More output tiles than SMs: every CTA cycles through both accumulator buffers."""
+    gen = torch.Generator().manual_seed(M + N + K)
+    Xq = torch.randn(M, K, generator=gen).to(dtype)
+    W = (torch.randn(N, K, generator=gen) * 0.05).to(dtype)
+    B = torch.randn(N, generator=gen) * 0.1
+    Yref = torch.randn(M, N, generator=gen)
+    out = omq.fq_linear_fwd(Xq.to(cuda_device), W.to(cuda_device), B_tilde=B.to(cuda_device),
+                            Y_ref=Yref.to(cuda_device))
+    torch.cuda.synchronize()
+    omq.sync_check()
+    Y64 = Xq.double().numpy() @ W.double().numpy().T + B.double().numpy()[None, :]
+    assert frob_rel(_np(out["Y"]), Y64) <= 2e-6
+    loss64 = float(np.mean((Y64 - Yref.double().numpy()) ** 2))
+    assert abs(out["loss"].item() - loss64) <= 1e-5 * loss64
+    R64 = Y64 - Yref.double().numpy()              # the residual stored as dY
+    assert frob_rel(_np(out["dY"]), R64) <= 1e-2
 
 
 def test_adamw_matches_oracle(omq, cuda_device):
