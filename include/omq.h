@@ -163,8 +163,8 @@ size_t omq_fwd_workspace_bytes(int64_t M, int64_t N, int64_t K);
  * float per output tile) in a fixed array compiled into the library and allocates nothing.
  * Arguments are those of omq_fq_linear_fwd without the workspace; Y_ref, dY and loss are
  * required, Y may be NULL.
- *   - Limit: ceil(M/128)*ceil(N/256) (16-bit operands) or ceil(M/64)*ceil(N/64) (float32) must not
- *     exceed 16384; larger problems return OMQ_ERR_SHAPE and launch nothing.
+ *   - Limit: 2*ceil(M/256)*ceil(N/256) (16-bit operands) or ceil(M/64)*ceil(N/64) (float32)
+ *     must not exceed 16384; larger problems return OMQ_ERR_SHAPE and launch nothing.
  *   - The array (64 KiB) is held on every GPU that loads the library until the process exits.
  *   - All calls on a device share it and it keeps the last call's contents; each call writes
  *     every slot it reads first, so nothing needs clearing. Calls that overlap on the GPU

@@ -1,31 +1,40 @@
-// bf16 x bf16 -> fp32 GEMM on the 5th-generation tensor cores (tcgen05, sm_100a).
+// 16-bit x 16-bit -> fp32 GEMM on the 5th-generation tensor cores (tcgen05, sm_100a).
 //
-// C[i, j] = sum_k A(i, k) B(j, k) over 128 x BN output tiles, persistent: one CTA per SM
-// walks tiles t, t + grid, t + 2 grid, ... Warp roles (192 threads):
-//   warp 0      TMA producer: one elected lane streams A and B k-blocks into a STAGES-deep
-//               shared-memory ring (128-byte swizzle), completing "full" mbarriers.
-//   warp 1      allocates TMEM for two accumulators (2 x BN columns); one lane issues
-//               tcgen05.mma (M=128, N=BN, K=16) per k-slice, tcgen05.commit's each stage back
-//               to its "empty" mbarrier and each finished tile to its accumulator's "full"
-//               mbarrier. It starts a tile as soon as the epilogue has released the other
-//               accumulator, so tile i+1's MMAs run while tile i is being stored.
-//   warps 2..5  epilogue: tcgen05.ld 32 lanes x 32 columns at a time, fused epilogue (bias,
-//               MSE loss, dY) and global stores; then release the accumulator.
+// C[i, j] = sum_k A(i, k) B(j, k) over 256 x 256 output tiles computed by CTA pairs
+// (clusters of 2, tcgen05 cta_group::2), persistent: each pair walks tiles p, p + pairs, ...
+// Each CTA of a pair keeps half of every operand tile in its shared memory (A rows
+// 128 r .. 128 r + 127 and B rows 128 r .. 128 r + 127 of the tile, r = rank in the pair),
+// and the pair's 256 x 256 x 16 MMA reads both halves, so a CTA streams 32 KB per k-block of
+// 64 instead of the 48 KB a single-CTA 128 x 256 tile needs. The accumulator rows of CTA r
+// live in its own TMEM (2 x 256 columns: two tiles in flight).
+// Warp roles (320 threads per CTA):
+//   warp 0      TMA producer (one lane): loads this CTA's halves of each k-block into a
+//               STAGES-deep ring (128-byte swizzle); both CTAs complete the leader's "full"
+//               mbarrier (cta_group::2 copies).
+//   warp 1      allocates TMEM (both CTAs, cta_group::2); in the leader CTA one lane issues
+//               the pair's tcgen05.mma (M=256, N=256, K=16) and commits each consumed stage
+//               to both CTAs' "empty" mbarriers and each finished tile to both CTAs'
+//               accumulator "full" mbarriers (tcgen05.commit multicast to the pair).
+//   warps 2..9  epilogue: warp w reads TMEM lanes 32 (w mod 4) .. + 31 (its accumulator rows)
+//               and one 128-column half of the tile (w < 6: first half), 32 x 32 at a time
+//               (tcgen05.ld), applies the fused epilogue (bias, MSE loss and residual, scaled
+//               store, or the weight-side STE backward), then releases the accumulator.
 // Operands may be K-major (row of the stored matrix runs along k) or MN-major (row runs
 // along i / j), so the three contractions of the step read X, W and dY in their natural
 // layouts without transposed copies:
 //   forward   Y  = Xq  W^^T : A = Xq [M,K] K-major,        B = W^ [N,K] K-major
 //   dW^       dW = dY^T Xq  : A = dY [M,N] MN-major,       B = Xq [M,K] MN-major
 //   dXq       dX = dY W^    : A = dY [M,N] K-major,        B = W^ [N,K] MN-major
-// Every mbarrier wait is bounded in time; on expiry the kernel raises the device error
-// flag, every role stops, outstanding copies and MMAs are drained (bounded), and the TMEM
-// is released.
+// Loads never multicast. Every mbarrier wait is bounded in time; on expiry the kernel raises
+// the device error flag, every role stops, outstanding copies and MMAs are drained
+// (bounded), and both CTAs meet at the final cluster barrier before releasing TMEM.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
 #include <mutex>
 
 #include "gemm_epilogue.cuh"
+#include "ste_common.cuh"
 
 namespace omq {
 
@@ -40,10 +49,13 @@ cudaError_t take_device_error(unsigned* flag) {
 
 namespace tc {
 
-constexpr int BM = 128;
-constexpr int BK = 64;                    // 64 bf16 = 128 bytes = one swizzle row
+constexpr int TILE_M = 256;               // rows of C per CTA pair
+constexpr int TILE_N = 256;               // columns of C per CTA pair
+constexpr int HALF = 128;                 // rows of A and of B held by each CTA
+constexpr int BK = 64;                    // 64 16-bit values = 128 bytes = one swizzle row
 constexpr int UMMA_K = 16;
-constexpr int NUM_THREADS = 192;
+constexpr int EPI_WARPS = 8;
+constexpr int NUM_THREADS = 32 * (2 + EPI_WARPS);
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;   // 2 s per barrier wait
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -53,6 +65,31 @@ __device__ __forceinline__ uint64_t globaltimer() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
+}
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_id() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_count() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+  return r;
+}
+// Address of this shared variable in CTA `rank` of the cluster (shared::cluster window).
+__device__ __forceinline__ uint32_t peer_addr(uint32_t local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+               "barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
@@ -64,17 +101,22 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                : "memory");
 }
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+// Arrive on a barrier of any CTA of the cluster (shared::cluster address).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar)
+               : "memory");
 }
+// One bounded-time probe: the thread may be suspended (not spinning on issue slots) for up
+// to kSuspendNs while the phase is still pending.
+constexpr uint32_t kSuspendNs = 20000;
 __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "n"(kSuspendNs)
       : "memory");
   return ok != 0;
 }
@@ -90,12 +132,14 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigne
   }
   return true;
 }
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                            int x, int y) {
+// Copy of this CTA's part of a pair's stage into its own shared memory, completing the
+// transaction on the leader CTA's barrier (cluster address).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map,
+                                                 uint32_t leader_bar, int x, int y) {
   asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(leader_bar), "r"(x), "r"(y)
       : "memory");
 }
 __device__ __forceinline__ void tc_fence_before() {
@@ -104,17 +148,26 @@ __device__ __forceinline__ void tc_fence_before() {
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+__device__ __forceinline__ void umma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                           uint32_t idesc, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
-__device__ __forceinline__ void umma_commit(uint32_t bar) {
+// Arrive (once each) on the barrier at this shared offset in both CTAs of the pair, when all
+// previously issued tcgen05 operations of this thread have completed.
+__device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
   asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(bar),
+      "h"(static_cast<uint16_t>(0x3))
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit_local(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
       : "memory");
 }
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
@@ -148,12 +201,12 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
   return d;
 }
 
-// Descriptor of the k-slice `kk` (16 elements) of an operand tile at `base`.
-//  K-major tile: `rows` rows of 128 bytes (64 k), 8-row swizzle atoms 1024 bytes apart;
-//                a k-slice starts 32 bytes further along the row.
-//  MN-major tile: chunks of 64 rows(i/j) x 64 k, each BK rows of 128 bytes (one k per row),
-//                 chunks 8192 bytes apart (LBO); 8-k atoms 1024 bytes apart (SBO); a k-slice
-//                 starts 16 k-rows = 2048 bytes further.
+// Descriptor of the k-slice `kk` (16 elements) of a 128-row operand half at `base`.
+//  K-major: 128 rows of 128 bytes (64 k), 8-row swizzle atoms 1024 bytes apart; a k-slice
+//           starts 32 bytes further along the row.
+//  MN-major: 2 chunks of 64 rows(i/j) x 64 k, each BK rows of 128 bytes (one k per row),
+//           chunks 8192 bytes apart (LBO); 8-k atoms 1024 bytes apart (SBO); a k-slice
+//           starts 16 k-rows = 2048 bytes further.
 __device__ __forceinline__ uint64_t operand_desc(uint32_t base, bool mn_major, int kk) {
   if (mn_major) return smem_desc(base + kk * 2048, BK * 128, 1024);
   return smem_desc(base + kk * 32, 16, 1024);
@@ -169,27 +222,143 @@ __host__ __device__ constexpr uint32_t instr_desc(int m, int n, bool a_mn, bool 
          (static_cast<uint32_t>(m >> 4) << 24);
 }
 
-template <int BN, int STAGES>
+// Weight-side straight-through backward fused into the dW^ GEMM: one warp's 32 rows (lane =
+// row n) x 128 columns of the accumulator, whose value times out_scale is dW^[n, k]; dW^ is
+// never stored. Groups of G columns (G = 32, 64 or 128) lie inside the warp's columns, and
+// the group dimension K is a multiple of G, so a group is wholly inside or outside [0, cols).
+//   pass 1: G_h, G_z of the lane's group -> d gamma / d beta logits
+//   pass 2 (LET): dW~ W and dB~[n] W summed over the warp's 32 rows, one partial row per
+//           32-row block of dW^ (fixed order), for d s and d delta.
+// The in-range decisions and dW~ repeat the separate kernels' binary32 arithmetic; only the
+// order of the sums differs.
+template <int G>
+__device__ __forceinline__ void ste_w_epilogue(const GemmEpilogue& epi, uint32_t tcol,
+                                               int64_t wrow0, int64_t col0, int64_t rows,
+                                               int64_t cols, int lane) {
+  const SteWEpi& p = epi.ste;
+  const int64_t row = wrow0 + lane;
+  const bool valid = row < rows;
+  const bool let = p.part_s != nullptr || p.part_d != nullptr;
+#pragma unroll 1
+  for (int g0 = 0; g0 < 128; g0 += G) {
+    const int64_t gcol = col0 + g0;
+    if (gcol >= cols) break;                          // warp-uniform
+    const int64_t gi = row * p.ng + gcol / G;
+    float h = 1.f, z = 0.f, glv = 0.f, blv = 0.f;
+    omq_range rg{0.f, 0.f, 1, 1};
+    if (valid) {
+      h = p.h[gi];
+      z = static_cast<float>(p.z[gi]);
+      rg = p.range[gi];
+      glv = p.gl[gi];
+      blv = p.bl[gi];
+    }
+    float Gh = 0.f, Gz = 0.f;
+#pragma unroll 1
+    for (int c = 0; c < G / 32; ++c) {
+      uint32_t r[32];
+      __syncwarp();
+      tmem_ld32(tcol + g0 + c * 32, r);
+      tmem_ld_wait();
+      if (!valid) continue;
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const int64_t k = gcol + c * 32 + v * 8;
+        float w[8], dq[8];
+        load8(p.W, row * p.K + k, p.wdt, w);
+        if (p.s) {
+          float sv[8];
+          load_f8(p.s, k, sv);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) w[i] = __fmul_rn(w[i], sv[i]);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) dq[i] = epi.out_scale * __uint_as_float(r[v * 8 + i]);
+        bool inr[8];
+        ste8(w, dq, h, z, p.Q, inr, Gh, Gz);
+      }
+    }
+    const float g = strength_value(glv), b = strength_value(blv);
+    const bool active = valid && h_active(h, glv, blv, rg.vmax, rg.vmin, p.Q);
+    const GroupGrad gg = group_grad(Gh, Gz, g, b, h, rg.vmax, rg.vmin, p.Q, active);
+    if (valid) {
+      if (p.d_gl) p.d_gl[gi] = gg.dg * g * (1.f - g);
+      if (p.d_bl) p.d_bl[gi] = gg.db * b * (1.f - b);
+    }
+    if (!let) continue;
+    const float eM = gg.dM / static_cast<float>(rg.nmax);
+    const float em = gg.dm / static_cast<float>(rg.nmin);
+    const float db_n = (valid && p.part_d) ? p.dBt[row] : 0.f;
+#pragma unroll 1
+    for (int c = 0; c < G / 32; ++c) {
+      uint32_t r[32];
+      __syncwarp();
+      tmem_ld32(tcol + g0 + c * 32, r);
+      tmem_ld_wait();
+      float ps[32], pd[32];
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const int64_t k = gcol + c * 32 + v * 8;
+        float w[8], wt[8];
+        bool inr[8];
+        if (valid) {
+          load8(p.W, row * p.K + k, p.wdt, w);
+          if (p.s) {
+            float sv[8];
+            load_f8(p.s, k, sv);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) wt[i] = __fmul_rn(w[i], sv[i]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) wt[i] = w[i];
+          }
+          in_range8(wt, h, z, p.Q, inr);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) { w[i] = 0.f; wt[i] = 0.f; inr[i] = false; }
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          float dwt = inr[i] ? epi.out_scale * __uint_as_float(r[v * 8 + i]) : 0.f;
+          if (valid && wt[i] == rg.vmax) dwt += eM;
+          if (valid && wt[i] == rg.vmin) dwt += em;
+          ps[v * 8 + i] = dwt * w[i];
+          pd[v * 8 + i] = db_n * w[i];
+        }
+      }
+      const float cs = warp_column_sum32(ps, lane);
+      const float cd = warp_column_sum32(pd, lane);
+      if (wrow0 < rows) {
+        const int64_t o = (wrow0 >> 5) * cols + gcol + c * 32 + lane;
+        if (p.part_s) p.part_s[o] = cs;
+        if (p.part_d) p.part_d[o] = cd;
+      }
+    }
+  }
+}
+
+template <int STAGES>
 struct Layout {
-  static constexpr int A_BYTES = BM * BK * 2;
-  static constexpr int B_BYTES = BN * BK * 2;
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int A_BYTES = HALF * BK * 2;          // 16 KB
+  static constexpr int B_BYTES = HALF * BK * 2;          // 16 KB
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // this CTA's part of a stage
   static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
   // barriers: full[S], empty[S], acc_full[2], acc_empty[2], drain; then tmem slot, abort
-  // flag, the epilogue's per-warp loss partials [2][4] and arrival counters [2]
+  // flag, the epilogue's per-warp loss partials [2][EPI_WARPS] and arrival counters [2]
   static constexpr int FULL = 0, EMPTY = 8 * STAGES, ACCF = 16 * STAGES, ACCE = ACCF + 16,
                        DRAIN = ACCE + 16, SLOT = DRAIN + 8, ABORT = SLOT + 4, RED = ABORT + 4,
-                       CNT = RED + 32;
+                       CNT = RED + 8 * EPI_WARPS, CTL_END = CNT + 8;
+  static_assert(CTL_END <= 256, "control block");
   static constexpr int SMEM_BYTES = 1024 /*align slack*/ + BAR_OFF + 256;
-  static constexpr uint32_t TMEM_COLS = 2 * BN;
+  static constexpr uint32_t TMEM_COLS = 2 * TILE_N;
 };
 
-template <int BN, int STAGES>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+template <int STAGES>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    int a_mn, int b_mn, uint32_t fmt, int64_t rows, int64_t cols, int64_t depth,
                    GemmEpilogue epi, int tiles_n, int num_tiles) {
-  using L = Layout<BN, STAGES>;
+  using L = Layout<STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -202,21 +371,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t bar_drain = sbase + L::BAR_OFF + L::DRAIN;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctl + L::SLOT);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(ctl + L::ABORT);
-  volatile float* red = reinterpret_cast<volatile float*>(ctl + L::RED);     // [2][4]
+  volatile float* red = reinterpret_cast<volatile float*>(ctl + L::RED);  // [2][EPI_WARPS]
   int* cnt = reinterpret_cast<int*>(ctl + L::CNT);                           // [2]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();          // 0 = leader of the pair
+  const int pair = static_cast<int>(cluster_id());
+  const int pairs = static_cast<int>(cluster_count());
   const int nk = static_cast<int>((depth + BK - 1) / BK);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(bar_full + 8 * s, 1);
-      mbar_init(bar_empty + 8 * s, 1);
+      mbar_init(bar_full + 8 * s, 1);     // leader's: one expect_tx arrival + both CTAs' bytes
+      mbar_init(bar_empty + 8 * s, 1);    // the leader's commit, multicast to both CTAs
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(bar_accf + 8 * b, 1);
-      mbar_init(bar_acce + 8 * b, 4);   // one arrival per epilogue warp
+      mbar_init(bar_accf + 8 * b, 1);     // the leader's commit, multicast to both CTAs
+      mbar_init(bar_acce + 8 * b, 2 * EPI_WARPS);   // leader's: every epilogue warp of both
       cnt[b] = 0;
     }
     mbar_init(bar_drain, 1);
@@ -224,23 +396,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     fence_mbar_init();
   }
   if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(tmem_slot)),
                  "r"(L::TMEM_COLS));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();            // both CTAs' barriers exist before either touches the other's
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0 && lane == 0) {
-    // ---------------- TMA producer
+    // ---------------- TMA producer (both CTAs)
     int it = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-      const int row0 = (t / tiles_n) * BM;
-      const int col0 = (t % tiles_n) * BN;
+    for (int t = pair; t < num_tiles && ok; t += pairs) {
+      const int row0 = (t / tiles_n) * TILE_M + static_cast<int>(rank) * HALF;
+      const int col0 = (t % tiles_n) * TILE_N + static_cast<int>(rank) * HALF;
       for (int kb = 0; kb < nk; ++kb, ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
@@ -250,69 +422,76 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         const uint32_t a_dst = sbase + s * L::STAGE_BYTES;
         const uint32_t b_dst = a_dst + L::A_BYTES;
-        const uint32_t full = bar_full + 8 * s;
-        mbar_expect_tx(full, L::STAGE_BYTES);
+        const uint32_t full_leader = peer_addr(bar_full + 8 * s, 0);
+        if (rank == 0) mbar_expect_tx(bar_full + 8 * s, 2 * L::STAGE_BYTES);
         const int k0 = kb * BK;
         if (a_mn) {
-          for (int c = 0; c < BM / 64; ++c) tma_load_2d(a_dst + c * 8192, &tmA, full, row0 + 64 * c, k0);
+          for (int c = 0; c < HALF / 64; ++c)
+            tma_load_2d_pair(a_dst + c * 8192, &tmA, full_leader, row0 + 64 * c, k0);
         } else {
-          tma_load_2d(a_dst, &tmA, full, k0, row0);
+          tma_load_2d_pair(a_dst, &tmA, full_leader, k0, row0);
         }
         if (b_mn) {
-          for (int c = 0; c < BN / 64; ++c) tma_load_2d(b_dst + c * 8192, &tmB, full, col0 + 64 * c, k0);
+          for (int c = 0; c < HALF / 64; ++c)
+            tma_load_2d_pair(b_dst + c * 8192, &tmB, full_leader, col0 + 64 * c, k0);
         } else {
-          tma_load_2d(b_dst, &tmB, full, k0, col0);
+          tma_load_2d_pair(b_dst, &tmB, full_leader, k0, col0);
         }
       }
     }
     if (!ok) {
       *abort_flag = 1;
-      // let the copies already in flight land before the CTA can exit
-      for (int j = it - STAGES < 0 ? 0 : it - STAGES; j < it; ++j)
-        mbar_wait(bar_full + 8 * (j % STAGES), (j / STAGES) & 1, DEV_ERR_TMA_WAIT);
+      // the leader waits for the copies already in flight before the pair can exit
+      if (rank == 0)
+        for (int j = it - STAGES < 0 ? 0 : it - STAGES; j < it; ++j)
+          mbar_wait(bar_full + 8 * (j % STAGES), (j / STAGES) & 1, DEV_ERR_TMA_WAIT);
     }
-  } else if (warp == 1 && lane == 0) {
-    // ---------------- MMA issuer
-    const uint32_t idesc = instr_desc(BM, BN, a_mn != 0, b_mn != 0, fmt);
+  } else if (warp == 1 && lane == 0 && rank == 0) {
+    // ---------------- MMA issuer (leader CTA only)
+    const uint32_t idesc = instr_desc(TILE_M, TILE_N, a_mn != 0, b_mn != 0, fmt);
     int it = 0, lt = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++lt) {
+    for (int t = pair; t < num_tiles && ok; t += pairs, ++lt) {
       const int buf = lt & 1;
       if (*abort_flag || !mbar_wait(bar_acce + 8 * buf, ((lt >> 1) & 1) ^ 1, DEV_ERR_MMA_WAIT)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const uint32_t d = tmem + static_cast<uint32_t>(buf * BN);
+      const uint32_t d = tmem + static_cast<uint32_t>(buf * TILE_N);
       for (int kb = 0; kb < nk; ++kb, ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
+        // the stage was written by the copy engine (async proxy) and published through the
+        // barrier: no tcgen05 fence is needed before the MMAs read it
         if (*abort_flag || !mbar_wait(bar_full + 8 * s, ph, DEV_ERR_MMA_WAIT)) {
           ok = false;
           break;
         }
-        tc_fence_after();
         const uint32_t a_base = sbase + s * L::STAGE_BYTES;
         const uint32_t b_base = a_base + L::A_BYTES;
 #pragma unroll
         for (int kk = 0; kk < BK / UMMA_K; ++kk) {
-          umma_bf16(d, operand_desc(a_base, a_mn != 0, kk), operand_desc(b_base, b_mn != 0, kk),
+          umma_pair(d, operand_desc(a_base, a_mn != 0, kk), operand_desc(b_base, b_mn != 0, kk),
                     idesc, (kb | kk) != 0 ? 1u : 0u);
         }
-        umma_commit(bar_empty + 8 * s);
+        umma_commit_pair(bar_empty + 8 * s);
       }
       if (!ok) break;
-      umma_commit(bar_accf + 8 * buf);
+      umma_commit_pair(bar_accf + 8 * buf);
     }
     if (!ok) *abort_flag = 1;
     // every MMA issued above has completed once this commit arrives
-    umma_commit(bar_drain);
+    umma_commit_local(bar_drain);
     mbar_wait(bar_drain, 0, DEV_ERR_MMA_WAIT);
   } else if (warp >= 2) {
-    // ---------------- epilogue
+    // ---------------- epilogue (both CTAs: this CTA's 128 rows of the tile)
+    const int ew = warp - 2;                         // 0 .. EPI_WARPS-1
     const int quad = warp & 3;                       // TMEM lanes 32*quad .. 32*quad+31
+    const int chalf = ew >> 2;                       // columns 128*chalf .. 128*chalf+127
+    const uint32_t acce_leader = peer_addr(bar_acce, 0);
     int lt = 0;
-    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++lt) {
+    for (int t = pair; t < num_tiles; t += pairs, ++lt) {
       const int buf = lt & 1;
       // one lane polls; the decision is broadcast so the warp-wide tcgen05.ld stays uniform
       int go = 0;
@@ -322,61 +501,73 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       go = __shfl_sync(0xffffffffu, go, 0);
       tc_fence_after();
       if (!go) break;
-      const int64_t row0 = static_cast<int64_t>(t / tiles_n) * BM;
-      const int64_t col0 = static_cast<int64_t>(t % tiles_n) * BN;
-      const int64_t row = row0 + quad * 32 + lane;
+      const int64_t wrow0 = static_cast<int64_t>(t / tiles_n) * TILE_M + rank * HALF + quad * 32;
+      const int64_t col0 = static_cast<int64_t>(t % tiles_n) * TILE_N + chalf * 128;
+      const int64_t row = wrow0 + lane;
       float lsum = 0.f;
       const uint32_t tbase = tmem + (static_cast<uint32_t>(quad * 32) << 16) +
-                             static_cast<uint32_t>(buf * BN);
-      for (int ch = 0; ch < BN / 32; ++ch) {
-        uint32_t r[32];
-        tmem_ld32(tbase + ch * 32, r);
-        tmem_ld_wait();
-        const int64_t cbase = col0 + ch * 32;
-        if (row < rows && cbase < cols) {
-          if (cbase + 32 <= cols) {
+                             static_cast<uint32_t>(buf * TILE_N + chalf * 128);
+      if (epi.kind == Epi::SteW) {
+        switch (epi.ste.G) {
+          case 32: ste_w_epilogue<32>(epi, tbase, wrow0, col0, rows, cols, lane); break;
+          case 64: ste_w_epilogue<64>(epi, tbase, wrow0, col0, rows, cols, lane); break;
+          default: ste_w_epilogue<128>(epi, tbase, wrow0, col0, rows, cols, lane); break;
+        }
+      } else {
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t r[32];
+          tmem_ld32(tbase + ch * 32, r);
+          tmem_ld_wait();
+          const int64_t cbase = col0 + ch * 32;
+          if (row < rows && cbase < cols) {
+            if (cbase + 32 <= cols) {
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              float acc[8];
+              for (int v = 0; v < 4; ++v) {
+                float acc[8];
 #pragma unroll
-              for (int q = 0; q < 8; ++q) acc[q] = __uint_as_float(r[v * 8 + q]);
-              epi_vec8(epi, row, cbase + v * 8, cols, acc, lsum);
+                for (int q = 0; q < 8; ++q) acc[q] = __uint_as_float(r[v * 8 + q]);
+                epi_vec8(epi, row, cbase + v * 8, cols, acc, lsum);
+              }
+            } else {
+#pragma unroll
+              for (int q = 0; q < 32; ++q)
+                if (cbase + q < cols)
+                  epi_element(epi, row, cbase + q, cols, __uint_as_float(r[q]), lsum);
             }
-          } else {
-#pragma unroll
-            for (int q = 0; q < 32; ++q)
-              if (cbase + q < cols) epi_element(epi, row, cbase + q, cols, __uint_as_float(r[q]), lsum);
           }
         }
       }
       if (epi.kind == Epi::MseLoss) {
-        // per-tile partial: the last of the four warps adds the warps' sums in a fixed order.
-        // red[buf] / cnt[buf] are next touched two tiles later, which cannot start before all
-        // four warps have released this accumulator below.
+        // per-half-tile partial: the last of this CTA's epilogue warps adds the warps' sums in
+        // a fixed order. red[buf] / cnt[buf] are next touched two tiles later, which cannot
+        // start before every warp has released this accumulator below.
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
         if (lane == 0) {
-          red[buf * 4 + quad] = lsum;
+          red[buf * EPI_WARPS + ew] = lsum;
           __threadfence_block();
-          if (atomicAdd(&cnt[buf], 1) == 3) {
+          if (atomicAdd(&cnt[buf], 1) == EPI_WARPS - 1) {
             __threadfence_block();
-            epi.loss_partials[t] = ((red[buf * 4 + 0] + red[buf * 4 + 1]) + red[buf * 4 + 2]) +
-                                   red[buf * 4 + 3];
+            float sum = 0.f;
+#pragma unroll
+            for (int q = 0; q < EPI_WARPS; ++q) sum += red[buf * EPI_WARPS + q];
+            epi.loss_partials[2 * t + rank] = sum;
             cnt[buf] = 0;
           }
         }
       }
-      // the accumulator has been read: hand it back to the MMA warp
+      // the accumulator has been read: hand it back to the leader's MMA warp
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar_acce + 8 * buf);
+      if (lane == 0) mbar_arrive_cluster(acce_leader + 8 * buf);
     }
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync();            // no CTA leaves while its partner may still signal it
   if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                  "r"(L::TMEM_COLS));
   }
 }
@@ -397,10 +588,11 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// Tensor map of one operand. K-major: stored [n_rows, depth] -> dims {depth, n_rows},
-// box {64, box_rows}. MN-major: stored [depth, n_rows] -> dims {n_rows, depth}, box {64, 64}.
+// Tensor map of one operand, boxes of one CTA's half tile. K-major: stored [n_rows, depth]
+// -> dims {depth, n_rows}, box {64, 128}. MN-major: stored [depth, n_rows] ->
+// dims {n_rows, depth}, box {64, 64}.
 bool make_map(CUtensorMap* map, omq_dtype dt, const GemmOperand& op, int64_t n_rows,
-              int64_t depth, int box_rows) {
+              int64_t depth) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2];
@@ -414,25 +606,25 @@ bool make_map(CUtensorMap* map, omq_dtype dt, const GemmOperand& op, int64_t n_r
     dims[0] = static_cast<cuuint64_t>(depth);
     dims[1] = static_cast<cuuint64_t>(n_rows);
     box[0] = BK;
-    box[1] = static_cast<cuuint32_t>(box_rows);
+    box[1] = HALF;
   }
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(op.ld) * 2};
   cuuint32_t estr[2] = {1, 1};
   const CUtensorMapDataType ty =
       dt == OMQ_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  CUresult r = fn(map, ty, 2, const_cast<void*>(op.ptr), dims,
-                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  CUresult r = fn(map, ty, 2, const_cast<void*>(op.ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
-constexpr int kBN = 256;
-constexpr int kStages = 4;
+constexpr int kStages = 7;   // 7 x 32 KB + control: the 227 KB shared-memory limit
 
 }  // namespace tc
 
+// Loss partial slots: one per 128-row half of each 256 x 256 output tile.
 int64_t gemm_tc_tiles(int64_t rows, int64_t cols) {
-  return ceil_div(rows, tc::BM) * ceil_div(cols, tc::kBN);
+  return 2 * ceil_div(rows, tc::TILE_M) * ceil_div(cols, tc::TILE_N);
 }
 
 omq_status gemm_tc(omq_dtype dt, const GemmOperand& A, const GemmOperand& B, int64_t rows,
@@ -441,15 +633,15 @@ omq_status gemm_tc(omq_dtype dt, const GemmOperand& A, const GemmOperand& B, int
   using namespace tc;
   if (dt != OMQ_BF16 && dt != OMQ_F16) return OMQ_ERR_DTYPE;
   CUtensorMap ma, mb;
-  if (!make_map(&ma, dt, A, rows, depth, BM) || !make_map(&mb, dt, B, cols, depth, kBN)) {
+  if (!make_map(&ma, dt, A, rows, depth) || !make_map(&mb, dt, B, cols, depth)) {
     set_cuda_error(cudaErrorInvalidValue);
     return OMQ_ERR_CUDA;
   }
-  const int64_t tiles_m = ceil_div(rows, BM), tiles_n = ceil_div(cols, kBN);
+  const int64_t tiles_m = ceil_div(rows, TILE_M), tiles_n = ceil_div(cols, TILE_N);
   const int64_t tiles = tiles_m * tiles_n;
-  if (n_tiles) *n_tiles = tiles;
-  auto kern = gemm_tc_kernel<kBN, kStages>;
-  const int smem = Layout<kBN, kStages>::SMEM_BYTES;
+  if (n_tiles) *n_tiles = 2 * tiles;
+  auto kern = gemm_tc_kernel<kStages>;
+  const int smem = Layout<kStages>::SMEM_BYTES;
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once, [&] {
@@ -459,11 +651,11 @@ omq_status gemm_tc(omq_dtype dt, const GemmOperand& A, const GemmOperand& B, int
     set_cuda_error(attr_err);
     return OMQ_ERR_CUDA;
   }
-  const int64_t sms = num_sms();
-  const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);
-  kern<<<grid, NUM_THREADS, smem, stream>>>(ma, mb, A.mn_major ? 1 : 0, B.mn_major ? 1 : 0,
-                                            dt == OMQ_F16 ? 0u : 1u, rows, cols, depth, epi,
-                                            static_cast<int>(tiles_n), static_cast<int>(tiles));
+  const int64_t max_pairs = num_sms() / 2;
+  const int64_t pairs = tiles < max_pairs ? tiles : max_pairs;
+  kern<<<static_cast<unsigned>(2 * pairs), NUM_THREADS, smem, stream>>>(
+      ma, mb, A.mn_major ? 1 : 0, B.mn_major ? 1 : 0, dt == OMQ_F16 ? 0u : 1u, rows, cols, depth,
+      epi, static_cast<int>(tiles_n), static_cast<int>(tiles));
   return launch_status();
 }
 

@@ -18,10 +18,15 @@ constexpr int kRowsSmallW = 128;            // rows per block, weight STE, lane-
 constexpr int kRowsLargeW = 16;             // rows per block, weight STE, larger groups
 constexpr int kRowsX = 64;                  // tokens per block, activation STE column sums
 constexpr int kRowsColsum = 64;             // rows per block of the dY column sums
+constexpr int kRowsFusedW = 32;             // rows per partial, weight STE in the dW^ epilogue
 
 size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
 
 int64_t rows_per_block_w(int64_t group) { return small_group(group) ? kRowsSmallW : kRowsLargeW; }
+
+// The weight-side STE runs inside the dW^ GEMM's epilogue for 16-bit operands and groups of
+// 32, 64 or 128; otherwise it is a separate kernel reading a stored dW^.
+bool fused_ste_w(omq_dtype op_dt, int64_t group) { return op_dt != OMQ_F32 && ste_fusable(group); }
 
 struct BwdLayout {
   size_t dbt_part, dbt, dwhat, dxq, part_ws, part_wd, part_xs, part_xd, rowstat, total;
@@ -31,7 +36,8 @@ struct BwdLayout {
 BwdLayout bwd_layout(int64_t M, int64_t N, int64_t K, int64_t group) {
   BwdLayout L{};
   L.rb_colsum = ceil_div(M, kRowsColsum);
-  L.rb_w = ceil_div(N, rows_per_block_w(group));
+  // enough partial rows for either weight-side STE (the fused one writes one per 32 rows)
+  L.rb_w = ceil_div(N, ste_fusable(group) ? kRowsFusedW : rows_per_block_w(group));
   L.rb_x = ceil_div(M, kRowsX);
   size_t off = 0;
   auto take = [&](size_t bytes) { size_t o = off; off += align256(bytes); return o; };
@@ -331,20 +337,32 @@ static omq_status bwd_impl(const omq_bwd_args* a, void* workspace, size_t ws_byt
     OMQ_TRY(launch_reduce_cols(dbt_part, L.rb_colsum, nullptr, 0, N, gscale, dbt, st));
   }
   // dW^ = G^T Xq   [N, K]
+  const float Q = static_cast<float>((1 << a->bits) - 1);
+  const bool fused = fused_ste_w(a->op_dt, G);
+  const int64_t rb_w = fused ? ceil_div(N, kRowsFusedW) : ceil_div(N, rows_per_block_w(G));
   OMQ_TRY(ph.mark(OMQ_PH_DW_GEMM));
   {
     GemmOperand A{a->dY, N, true}, B{a->Xq, K, true};
     GemmEpilogue epi{};
-    epi.kind = Epi::StoreF32;
-    epi.out = dwhat;
     epi.out_scale = gscale;
+    if (fused) {
+      // weight-side STE in the epilogue: d gamma / d beta logits and the W-side LET column
+      // partials straight from the accumulator
+      epi.kind = Epi::SteW;
+      epi.ste = SteWEpi{a->W, a->dt, K, G, K / G, Q, a->s, a->gamma_logit, a->beta_logit,
+                        a->h, a->z, a->grp_range, a->d_delta ? dbt : nullptr,
+                        a->d_gamma_logit, a->d_beta_logit, a->d_s ? part_ws : nullptr,
+                        a->d_delta ? part_wd : nullptr};
+    } else {
+      epi.kind = Epi::StoreF32;
+      epi.out = dwhat;
+    }
     OMQ_TRY(run_gemm(a->op_dt, A, B, N, K, M, epi, nullptr, st));
   }
   // weight-side STE: d gamma / d beta logits and the W-side LET column partials
   OMQ_TRY(ph.mark(OMQ_PH_STE_W));
-  {
-    SteWParams p{a->W, a->dt, N, K, G, K / G, static_cast<float>((1 << a->bits) - 1),
-                 a->s, a->gamma_logit, a->beta_logit, a->h, a->z,
+  if (!fused) {
+    SteWParams p{a->W, a->dt, N, K, G, K / G, Q, a->s, a->gamma_logit, a->beta_logit, a->h, a->z,
                  a->grp_range, dwhat, a->d_delta ? dbt : nullptr, a->d_gamma_logit,
                  a->d_beta_logit, a->d_s ? part_ws : nullptr, a->d_delta ? part_wd : nullptr,
                  static_cast<int>(rows_per_block_w(G))};
@@ -373,9 +391,9 @@ static omq_status bwd_impl(const omq_bwd_args* a, void* workspace, size_t ws_byt
     OMQ_TRY(launch_ste_x(p, st));
   }
   OMQ_TRY(ph.mark(OMQ_PH_LET_REDUCE));
-  if (a->d_s) OMQ_TRY(launch_reduce_cols(part_ws, L.rb_w, part_xs, L.rb_x, K, 1.f, a->d_s, st));
+  if (a->d_s) OMQ_TRY(launch_reduce_cols(part_ws, rb_w, part_xs, L.rb_x, K, 1.f, a->d_s, st));
   if (a->d_delta)
-    OMQ_TRY(launch_reduce_cols(part_wd, L.rb_w, part_xd, L.rb_x, K, 1.f, a->d_delta, st));
+    OMQ_TRY(launch_reduce_cols(part_wd, rb_w, part_xd, L.rb_x, K, 1.f, a->d_delta, st));
   return OMQ_OK;
 }
 

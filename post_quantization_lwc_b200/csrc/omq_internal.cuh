@@ -159,7 +159,27 @@ struct GemmOperand {
   bool mn_major;
 };
 
-enum class Epi { StoreF32 = 0, MseLoss = 1 };
+enum class Epi { StoreF32 = 0, MseLoss = 1, SteW = 2 };
+
+// Weight-side straight-through backward fused into the dW^ GEMM's epilogue (groups of 32, 64
+// or 128 elements): the tile's accumulator is dW^ / out_scale.
+struct SteWEpi {
+  const void* W;
+  omq_dtype wdt;
+  int64_t K, G, ng;
+  float Q;
+  const float* s;          // [K] or NULL
+  const float* gl;
+  const float* bl;
+  const float* h;
+  const int32_t* z;
+  const omq_range* range;
+  const float* dBt;        // [N] (with part_d)
+  float* d_gl;
+  float* d_bl;
+  float* part_s;           // [ceil(N/32), K] or NULL: per 32-row block, sum dW~ W
+  float* part_d;           // [ceil(N/32), K] or NULL: per 32-row block, sum dB~ W
+};
 
 struct GemmEpilogue {
   Epi kind;
@@ -168,9 +188,14 @@ struct GemmEpilogue {
   const float* y_ref;      // MseLoss: [rows, cols]
   void* dy;                // MseLoss: [rows, cols] residual in dy_dt
   omq_dtype dy_dt;
-  float out_scale;         // StoreF32: out = out_scale * acc (+ bias)
+  float out_scale;         // StoreF32: out = out_scale * acc (+ bias); SteW: dW^ = out_scale * acc
   float* loss_partials;    // MseLoss: one per output tile (fixed order)
+  SteWEpi ste;             // SteW
 };
+
+// Group lengths the dW^ GEMM's epilogue handles (whole groups inside one epilogue warp's
+// 128 columns, at least one 32-column TMEM load each).
+inline bool ste_fusable(int64_t g) { return g == 32 || g == 64 || g == 128; }
 
 // 16-bit operands (BF16 or F16, both the same type) on tcgen05 (sm_100a). Reports the
 // number of output tiles (loss partial slots).

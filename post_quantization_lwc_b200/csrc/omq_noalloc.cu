@@ -10,8 +10,9 @@
 // buffer, and the call allocates nothing.
 //
 // Limits and sharing:
-//   - The array holds kNoAllocTiles partial sums. A problem needs ceil(M/128) * ceil(N/256)
-//     of them on the 16-bit tensor-core path, or ceil(M/64) * ceil(N/64) on the float32 path;
+//   - The array holds kNoAllocTiles partial sums. A problem needs 2 * ceil(M/256) *
+//     ceil(N/256) of them on the 16-bit tensor-core path (one per 128-row half of each
+//     256 x 256 output tile), or ceil(M/64) * ceil(N/64) on the float32 path;
 //     larger problems are rejected with OMQ_ERR_SHAPE before anything is launched.
 //   - Every GPU that loads the library holds the array (64 KiB) until the process exits.
 //   - All calls on a device share the one array, and it keeps the last call's contents.

@@ -56,8 +56,8 @@ def test_noalloc_forward_matches_workspace_forward(omq, cuda_device, calls):
 
 def test_noalloc_rejects_problems_beyond_its_scratch(omq, cuda_device):
     import ctypes
-    # 129 x 128 = 16512 output tiles of 128 x 256 > 16384 slots: rejected on the host before
-    # any buffer is touched, so one small tensor stands in for every pointer
+    # 2 x ceil(16512/256) x 128 = 16640 partial sums > 16384 slots: rejected on the host
+    # before any buffer is touched, so one small tensor stands in for every pointer
     buf = torch.zeros(64, dtype=torch.float32, device=cuda_device)
     p = ctypes.c_void_p(buf.data_ptr())
     st = omq._lib.omq_fq_linear_fwd_noalloc(p, p, omq.OMQ_BF16, 128 * 129, 256 * 128, 64, None,
