@@ -24,9 +24,11 @@ size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
 
 int64_t rows_per_block_w(int64_t group) { return small_group(group) ? kRowsSmallW : kRowsLargeW; }
 
-// The weight-side STE runs inside the dW^ GEMM's epilogue for 16-bit operands and groups of
-// 32, 64 or 128; otherwise it is a separate kernel reading a stored dW^.
-bool fused_ste_w(omq_dtype op_dt, int64_t group) { return op_dt != OMQ_F32 && ste_fusable(group); }
+// The weight-side STE runs inside the dW^ GEMM's epilogue for 16-bit operands and weights
+// and groups of 32, 64 or 128; otherwise it is a separate kernel reading a stored dW^.
+bool fused_ste_w(omq_dtype op_dt, omq_dtype wdt, int64_t group) {
+  return op_dt != OMQ_F32 && wdt != OMQ_F32 && ste_fusable(group);
+}
 
 struct BwdLayout {
   size_t dbt_part, dbt, dwhat, dxq, part_ws, part_wd, part_xs, part_xd, rowstat, total;
@@ -333,13 +335,16 @@ static omq_status bwd_impl(const omq_bwd_args* a, void* workspace, size_t ws_byt
   // dB~ = column sums of dY (needed for d_delta, or when asked for)
   OMQ_TRY(ph.mark(OMQ_PH_DBIAS));
   if (a->d_delta || a->d_B_tilde) {
-    OMQ_TRY(launch_colsum(a->dY, a->op_dt, M, N, kRowsColsum, dbt_part, st));
+    OMQ_TRY(launch_colsum(a->dY, a->op_dt, M, N, kRowsColsum, nullptr, dbt_part, st));
     OMQ_TRY(launch_reduce_cols(dbt_part, L.rb_colsum, nullptr, 0, N, gscale, dbt, st));
   }
   // dW^ = G^T Xq   [N, K]
   const float Q = static_cast<float>((1 << a->bits) - 1);
-  const bool fused = fused_ste_w(a->op_dt, G);
+  const bool fused = fused_ste_w(a->op_dt, a->dt, G);
   const int64_t rb_w = fused ? ceil_div(N, kRowsFusedW) : ceil_div(N, rows_per_block_w(G));
+  // the W side of d delta, sum_n dB~[n] W[n, k], in row blocks of kRowsColsum when the STE
+  // is fused (the separate STE kernel produces it in its own row blocks)
+  const int64_t rb_wd = fused ? ceil_div(N, kRowsColsum) : rb_w;
   OMQ_TRY(ph.mark(OMQ_PH_DW_GEMM));
   {
     GemmOperand A{a->dY, N, true}, B{a->Xq, K, true};
@@ -350,9 +355,8 @@ static omq_status bwd_impl(const omq_bwd_args* a, void* workspace, size_t ws_byt
       // partials straight from the accumulator
       epi.kind = Epi::SteW;
       epi.ste = SteWEpi{a->W, a->dt, K, G, K / G, Q, a->s, a->gamma_logit, a->beta_logit,
-                        a->h, a->z, a->grp_range, a->d_delta ? dbt : nullptr,
-                        a->d_gamma_logit, a->d_beta_logit, a->d_s ? part_ws : nullptr,
-                        a->d_delta ? part_wd : nullptr};
+                        a->h, a->z, a->grp_range, a->d_gamma_logit, a->d_beta_logit,
+                        a->d_s ? part_ws : nullptr};
     } else {
       epi.kind = Epi::StoreF32;
       epi.out = dwhat;
@@ -361,6 +365,8 @@ static omq_status bwd_impl(const omq_bwd_args* a, void* workspace, size_t ws_byt
   }
   // weight-side STE: d gamma / d beta logits and the W-side LET column partials
   OMQ_TRY(ph.mark(OMQ_PH_STE_W));
+  if (fused && a->d_delta)
+    OMQ_TRY(launch_colsum(a->W, a->dt, N, K, kRowsColsum, dbt, part_wd, st));
   if (!fused) {
     SteWParams p{a->W, a->dt, N, K, G, K / G, Q, a->s, a->gamma_logit, a->beta_logit, a->h, a->z,
                  a->grp_range, dwhat, a->d_delta ? dbt : nullptr, a->d_gamma_logit,
@@ -393,7 +399,7 @@ static omq_status bwd_impl(const omq_bwd_args* a, void* workspace, size_t ws_byt
   OMQ_TRY(ph.mark(OMQ_PH_LET_REDUCE));
   if (a->d_s) OMQ_TRY(launch_reduce_cols(part_ws, rb_w, part_xs, L.rb_x, K, 1.f, a->d_s, st));
   if (a->d_delta)
-    OMQ_TRY(launch_reduce_cols(part_wd, rb_w, part_xd, L.rb_x, K, 1.f, a->d_delta, st));
+    OMQ_TRY(launch_reduce_cols(part_wd, rb_wd, part_xd, L.rb_x, K, 1.f, a->d_delta, st));
   return OMQ_OK;
 }
 

@@ -161,10 +161,10 @@ struct GemmOperand {
 
 enum class Epi { StoreF32 = 0, MseLoss = 1, SteW = 2 };
 
-// Weight-side straight-through backward fused into the dW^ GEMM's epilogue (groups of 32, 64
-// or 128 elements): the tile's accumulator is dW^ / out_scale.
+// Weight-side straight-through backward fused into the dW^ GEMM's epilogue (16-bit weights,
+// groups of 32, 64 or 128 elements): the tile's accumulator is dW^ / out_scale.
 struct SteWEpi {
-  const void* W;
+  const void* W;           // [N, K] BF16 or F16
   omq_dtype wdt;
   int64_t K, G, ng;
   float Q;
@@ -174,11 +174,9 @@ struct SteWEpi {
   const float* h;
   const int32_t* z;
   const omq_range* range;
-  const float* dBt;        // [N] (with part_d)
   float* d_gl;
   float* d_bl;
   float* part_s;           // [ceil(N/32), K] or NULL: per 32-row block, sum dW~ W
-  float* part_d;           // [ceil(N/32), K] or NULL: per 32-row block, sum dB~ W
 };
 
 struct GemmEpilogue {
@@ -193,8 +191,8 @@ struct GemmEpilogue {
   SteWEpi ste;             // SteW
 };
 
-// Group lengths the dW^ GEMM's epilogue handles (whole groups inside one epilogue warp's
-// 128 columns, at least one 32-column TMEM load each).
+// Group lengths the dW^ GEMM's epilogue handles (a group covers one or two 32-column chunks
+// of an epilogue warp's 64 columns, or the 128 columns of a warp pair).
 inline bool ste_fusable(int64_t g) { return g == 32 || g == 64 || g == 128; }
 
 // 16-bit operands (BF16 or F16, both the same type) on tcgen05 (sm_100a). Reports the
@@ -298,8 +296,9 @@ omq_status launch_let_bias(const void* W, omq_dtype wdt, int64_t N, int64_t K, c
                            const float* B, float* Bt, cudaStream_t stream);
 omq_status launch_ste_w(const SteWParams& p, cudaStream_t stream);
 omq_status launch_ste_x(const SteXParams& p, cudaStream_t stream);
+// part[rb, j] = sum over rows i of block rb (R rows) of w[i] A[i, j] (w NULL: 1).
 omq_status launch_colsum(const void* A, omq_dtype dt, int64_t rows, int64_t cols, int R,
-                         float* part, cudaStream_t stream);
+                         const float* w, float* part, cudaStream_t stream);
 omq_status launch_reduce_cols(const float* p0, int64_t r0n, const float* p1, int64_t r1n,
                               int64_t cols, float scale, float* out, cudaStream_t stream);
 omq_status launch_loss_finalize(const float* part, int64_t n, double inv_count, float* loss,

@@ -357,11 +357,12 @@ __global__ void __launch_bounds__(256, 2) ste_x_cols_kernel(SteXParams p) {
 }
 
 // ------------------------------------------------------------------ column sums
-// part[rb, j] = sum of A[i, j] over the rows of row block rb (A [rows, cols] in dt, cols % 8
-// == 0). Same launch shape as ste_x_cols_kernel.
+// part[rb, j] = sum of wrow[i] A[i, j] (wrow NULL: A[i, j]) over the rows of row block rb
+// (A [rows, cols] in dt, cols % 8 == 0). Same launch shape as ste_x_cols_kernel.
 template <int U>
 __global__ void __launch_bounds__(256) colsum_kernel(const void* A, omq_dtype dt, int64_t rows,
-                                                     int64_t cols, int R, float* part) {
+                                                     int64_t cols, int R, const float* wrow,
+                                                     float* part) {
   __shared__ float red[8][256];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int64_t c0 = static_cast<int64_t>(blockIdx.x) * 256 + lane * 8;
@@ -382,9 +383,12 @@ __global__ void __launch_bounds__(256) colsum_kernel(const void* A, omq_dtype dt
       }
     }
 #pragma unroll
-    for (int u = 0; u < U; ++u)
+    for (int u = 0; u < U; ++u) {
+      const int64_t m = mb + 8 * u;
+      const float f = wrow ? (m < r1 ? wrow[m] : 0.f) : 1.f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] += v[u][i];
+      for (int i = 0; i < 8; ++i) acc[i] += f * v[u][i];
+    }
   }
 #pragma unroll
   for (int i = 0; i < 8; ++i) red[w][lane * 8 + i] = acc[i];
@@ -503,9 +507,9 @@ omq_status launch_ste_x(const SteXParams& p, cudaStream_t stream) {
 }
 
 omq_status launch_colsum(const void* A, omq_dtype dt, int64_t rows, int64_t cols, int R,
-                         float* part, cudaStream_t stream) {
+                         const float* w, float* part, cudaStream_t stream) {
   dim3 grid(static_cast<unsigned>(ceil_div(cols, 256)), static_cast<unsigned>(ceil_div(rows, R)));
-  colsum_kernel<4><<<grid, 256, 0, stream>>>(A, dt, rows, cols, R, part);
+  colsum_kernel<4><<<grid, 256, 0, stream>>>(A, dt, rows, cols, R, w, part);
   return launch_status();
 }
 
