@@ -19,8 +19,6 @@
 //               and one 64-column quarter of the tile ((w - 2) / 4), 32 x 32 at a time
 //               (tcgen05.ld), applies the fused epilogue (bias, MSE loss and residual, scaled
 //               store, or the weight-side STE backward), then releases the accumulator.
-//               Sixteen warps (four per scheduler) hide the latency of the epilogue's loads
-//               and dependent arithmetic; registers are capped at 112 per thread for it.
 // Operands may be K-major (row of the stored matrix runs along k) or MN-major (row runs
 // along i / j), so the three contractions of the step read X, W and dY in their natural
 // layouts without transposed copies:
@@ -56,18 +54,19 @@ constexpr int TILE_N = 256;               // columns of C per CTA pair
 constexpr int HALF = 128;                 // rows of A and of B held by each CTA
 constexpr int BK = 64;                    // 64 16-bit values = 128 bytes = one swizzle row
 constexpr int UMMA_K = 16;
-// Per epilogue variant: the store / MSE epilogue (STE_G = 0) is light and runs with 8
-// epilogue warps and a 7-deep operand ring; the weight-side STE epilogue (STE_G > 0) is the
-// step's heaviest arithmetic and runs with 16 epilogue warps (four per scheduler, 96
-// registers a thread), a 6-deep ring (its exchange slots take the rest of shared memory),
-// and producer / MMA waits that sleep between probes, leaving issue slots to the epilogue.
-template <int STE_G>
+
+// Epilogue variants: EV = 0 the store / MSE epilogue (epi.kind), light, with 8 epilogue warps
+// of 128 columns; EV = 1 / 2 the weight-side STE epilogue (BF16 / F16 weights), the step's
+// heaviest per-element arithmetic, with 16 epilogue warps of 64 columns (four per scheduler,
+// 96 registers a thread) and producer / MMA waits that sleep between probes, leaving issue
+// slots to the epilogue. One kernel per variant keeps each within its register budget.
+template <int EV>
 struct Cfg {
-  static constexpr int EPI_WARPS = STE_G ? 16 : 8;
+  static constexpr int EPI_WARPS = EV ? 16 : 8;
   static constexpr int EPI_COLS = TILE_N * 4 / EPI_WARPS;   // accumulator columns per warp
   static constexpr int NUM_THREADS = 32 * (2 + EPI_WARPS);
-  static constexpr int STAGES = STE_G ? 6 : 7;
-  static constexpr bool SLEEPY = STE_G != 0;
+  static constexpr int STAGES = 7;
+  static constexpr bool SLEEPY = EV != 0;
 };
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;   // 2 s per barrier wait
 
@@ -219,19 +218,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
-      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(
-          taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
-      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
-      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
-      "r"(r[29]), "r"(r[30]), "r"(r[31])
-      : "memory");
-}
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
@@ -241,19 +227,6 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
         "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
 }
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
-      "r"(r[15])
-      : "memory");
-}
-__device__ __forceinline__ void tmem_st_wait() {
-  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-
 // Shared-memory matrix descriptor, 128-byte swizzle (sm_100 layout: start address,
 // leading / stride byte offsets in 16-byte units, version 1 at bit 46, layout type 2 at
 // bits 61-63).
@@ -288,35 +261,6 @@ __host__ __device__ constexpr uint32_t instr_desc(int m, int n, bool a_mn, bool 
          (static_cast<uint32_t>(m >> 4) << 24);
 }
 
-// Two partner epilogue warps (same accumulator rows, adjacent 64-column quarters) add their
-// partial group sums: each writes its pair to shared memory, both arrive on the pair's
-// mbarrier (one phase per exchange), then each reads the other's. Slots alternate with the
-// phase parity, so a slot is rewritten only after the partner has read it. The wait is
-// bounded; on expiry the error flag is raised and the partner's values are not used.
-struct PairX {
-  float2* mine;          // [2][32]
-  const float2* theirs;  // [2][32]
-  uint32_t bar;
-  uint32_t k;            // exchanges so far
-};
-__device__ __forceinline__ void pair_add(PairX& px, int lane, float& a, float& b) {
-  const uint32_t slot = px.k & 1;
-  px.mine[slot * 32 + lane] = make_float2(a, b);
-  __syncwarp();
-  int ok = 1;
-  if (lane == 0) {
-    mbar_arrive_local(px.bar);
-    ok = mbar_wait(px.bar, slot, DEV_ERR_EPI_WAIT) ? 1 : 0;
-  }
-  ok = __shfl_sync(0xffffffffu, ok, 0);
-  __syncwarp();
-  ++px.k;
-  if (!ok) return;
-  const float2 o = px.theirs[slot * 32 + lane];
-  a += o.x;              // a + b == b + a: both partners obtain the same sums
-  b += o.y;
-}
-
 // 8 weights of one row from their 16-bit storage.
 template <bool F16>
 __device__ __forceinline__ void unpack8(const uint4& q, float (&w)[8]) {
@@ -336,159 +280,104 @@ __device__ __forceinline__ void unpack8(const uint4& q, float (&w)[8]) {
 
 // Weight-side straight-through backward fused into the dW^ GEMM: one warp's 32 rows (lane =
 // row n) x 64 columns of the accumulator, whose value times out_scale is dW^[n, k]; dW^ is
-// never stored. Each 32-column chunk's weights are loaded before its accumulator columns are
-// read from TMEM, so the two latencies overlap.
-// Groups of G columns: G = 32 or 64 lie inside the warp's columns; a group of 128 spans the
-// warp and its partner (pair_add). K is a multiple of G, so a group is wholly inside or
-// outside [0, cols).
-//   pass 1: G_h, G_z of the lane's group -> d gamma / d beta logits; with LET, the
-//           in-range part of dW~ (dq where the level is not clipped, else 0) is written back
-//           over the accumulator.
-//   pass 2 (LET): dW~ = that + dM/n_max at the group's max elements + dm/n_min at its min
-//           elements; dW~ W summed over the warp's 32 rows gives one partial row per 32-row
-//           block (fixed order) for d s.
-// The in-range decisions and dW~ repeat the separate kernel's binary32 arithmetic; only the
-// order of the sums differs.
-template <int G, bool F16>
+// never stored. The group length is a multiple of 32, so each 32-column chunk lies in one
+// group (h, z of row n). Per chunk and row the epilogue writes
+//   gh_part[chunk, n] = sum dq (round(u) - u) over in-range elements + dq (code - z) over
+//                       clipped ones                                   (G_h's share)
+//   gc_part[chunk, n] = sum dq over clipped elements                   (G_z = -h * that)
+// and, with LET, the chunk's column sums over the warp's 32 rows of (in range ? dq : 0) W,
+// one partial row per 32-row block for d s. The group's own terms (its G_h, G_z, the logit
+// gradients and the max / min elements' shares) are finished by ste_w_finish_kernel and
+// ste_w_corr_kernel after the GEMM. Rows past the end read as zero weights and zero
+// accumulators (the operand loads fill zeros) and store nothing.
+template <bool F16>
 __device__ __forceinline__ void ste_w_epilogue(const GemmEpilogue& epi, uint32_t tcol,
                                                int64_t wrow0, int64_t col0, int64_t rows,
-                                               int64_t cols, int lane, bool writer,
-                                               PairX& px) {
+                                               int64_t cols, int lane) {
   const SteWEpi& p = epi.ste;
   const int64_t row = wrow0 + lane;
   const bool valid = row < rows;
   const bool let = p.part_s != nullptr;
   const uint4* wrow = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.W) +
-                                                     (valid ? row : 0) * p.K + col0);  // 8 per uint4
-  constexpr int CPG = G >= 64 ? 2 : 1;       // this warp's 32-column chunks per group
-#pragma unroll
-  for (int c0 = 0; c0 < 2; c0 += CPG) {
-    const int64_t kw = col0 + 32 * c0;       // first column of this warp's part of the group
-    if (kw >= cols) break;                   // warp-uniform
-    const int64_t gi = row * p.ng + kw / G;
-    float h = 1.f, z = 0.f, glv = 0.f, blv = 0.f;
-    omq_range rg{0.f, 0.f, 1, 1};
+                                                     (valid ? row : 0) * p.K + col0);
+#pragma unroll 1
+  for (int c = 0; c < 2; ++c) {
+    const int64_t k0 = col0 + 32 * c;
+    if (k0 >= cols) break;                           // warp-uniform
+    const int64_t gi = row * p.ng + static_cast<int>(k0) / static_cast<int>(p.G);
+    float h = 1.f, z = 0.f;
     if (valid) {
       h = p.h[gi];
       z = static_cast<float>(p.z[gi]);
-      rg = p.range[gi];
-      glv = p.gl[gi];
-      blv = p.bl[gi];
     }
     const float hinv = __frcp_rn(h);
-    float Gh = 0.f, Gc = 0.f;                // Gc: sum of dq over clipped elements
-    // 16 columns at a time (keeps the live registers within the 576-thread budget)
+    float Gh = 0.f, Gc = 0.f;
+    float ps[32];
 #pragma unroll
-    for (int q = 2 * c0; q < 2 * (c0 + CPG); ++q) {
+    for (int hh = 0; hh < 2; ++hh) {
+      const int q = 2 * c + hh;
       uint4 wq[2];
-      if (valid) {
-        wq[0] = __ldg(wrow + 2 * q);
-        wq[1] = __ldg(wrow + 2 * q + 1);
-      }
+      wq[0] = valid ? __ldg(wrow + 2 * q) : make_uint4(0, 0, 0, 0);
+      wq[1] = valid ? __ldg(wrow + 2 * q + 1) : make_uint4(0, 0, 0, 0);
       uint32_t r[16];
       __syncwarp();
       tmem_ld16(tcol + 16 * q, r);
       tmem_ld_wait();
-      if (valid) {
 #pragma unroll
-        for (int v = 0; v < 2; ++v) {
-          float w[8], sv[8];
-          unpack8<F16>(wq[v], w);
-          if (p.s) load_f8(p.s, col0 + 16 * q + 8 * v, sv);
+      for (int v = 0; v < 2; ++v) {
+        float w[8], sv[8];
+        unpack8<F16>(wq[v], w);
+        if (p.s) load_f8(p.s, col0 + 16 * q + 8 * v, sv);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float wt = p.s ? __fmul_rn(w[i], sv[i]) : w[i];
-            const float dq = epi.out_scale * __uint_as_float(r[8 * v + i]);
-            const float rq = round_quotient(wt, h, hinv);
-            const float lvl = __fadd_rn(rq, z);
-            const bool inr = lvl >= 0.f && lvl <= p.Q;
-            const float cl = fminf(fmaxf(lvl, 0.f), p.Q);
-            Gh += dq * (inr ? (rq - wt * hinv) : (cl - z));
-            Gc += inr ? 0.f : dq;
-            r[8 * v + i] = __float_as_uint(inr ? dq : 0.f);
-          }
+        for (int i = 0; i < 8; ++i) {
+          const float wt = p.s ? __fmul_rn(w[i], sv[i]) : w[i];
+          const float dq = epi.out_scale * __uint_as_float(r[8 * v + i]);
+          const float rq = round_quotient(wt, h, hinv);
+          const float lvl = __fadd_rn(rq, z);
+          const bool inr = lvl >= 0.f && lvl <= p.Q;
+          const float cl = fminf(fmaxf(lvl, 0.f), p.Q);
+          Gh += dq * (inr ? (rq - wt * hinv) : (cl - z));
+          Gc += inr ? 0.f : dq;
+          ps[16 * hh + 8 * v + i] = inr ? dq * w[i] : 0.f;
         }
       }
-      if (let) tmem_st16(tcol + 16 * q, r);
     }
-    if (let) tmem_st_wait();
-    float Gz = -h * Gc;
-    if (G == 128) pair_add(px, lane, Gh, Gz);
-    const float g = strength_value(glv), b = strength_value(blv);
-    const bool active = valid && h_active(h, glv, blv, rg.vmax, rg.vmin, p.Q);
-    const GroupGrad gg = group_grad(Gh, Gz, g, b, h, rg.vmax, rg.vmin, p.Q, active);
-    if (valid && writer) {
-      if (p.d_gl) p.d_gl[gi] = gg.dg * g * (1.f - g);
-      if (p.d_bl) p.d_bl[gi] = gg.db * b * (1.f - b);
+    if (valid) {
+      p.gh_part[(k0 >> 5) * rows + row] = Gh;
+      p.gc_part[(k0 >> 5) * rows + row] = Gc;
     }
-    if (!let) continue;
-    const float eM = gg.dM / static_cast<float>(rg.nmax);
-    const float em = gg.dm / static_cast<float>(rg.nmin);
-#pragma unroll
-    for (int c = c0; c < c0 + CPG; ++c) {
-      float ps[32];
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const int q = 2 * c + hh;
-        uint4 wq[2];
-        wq[0] = valid ? __ldg(wrow + 2 * q) : make_uint4(0, 0, 0, 0);
-        wq[1] = valid ? __ldg(wrow + 2 * q + 1) : make_uint4(0, 0, 0, 0);
-        uint32_t r[16];
-        __syncwarp();
-        tmem_ld16(tcol + 16 * q, r);
-        tmem_ld_wait();
-#pragma unroll
-        for (int v = 0; v < 2; ++v) {
-          float w[8], sv[8];
-          unpack8<F16>(wq[v], w);
-          if (p.s) load_f8(p.s, col0 + 16 * q + 8 * v, sv);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float wt = p.s ? __fmul_rn(w[i], sv[i]) : w[i];
-            float dwt = __uint_as_float(r[8 * v + i]);
-            if (wt == rg.vmax) dwt += eM;
-            if (wt == rg.vmin) dwt += em;
-            ps[16 * hh + 8 * v + i] = valid ? dwt * w[i] : 0.f;
-          }
-        }
-      }
+    if (let) {
       const float cs = warp_column_sum32(ps, lane);
-      if (wrow0 < rows) p.part_s[(wrow0 >> 5) * cols + col0 + 32 * c + lane] = cs;
+      if (wrow0 < rows) p.part_s[(wrow0 >> 5) * cols + k0 + lane] = cs;
     }
   }
 }
 
-template <int STAGES, int EPI_WARPS, bool PAIRS>
+template <int STAGES, int EPI_WARPS>
 struct Layout {
   static constexpr int A_BYTES = HALF * BK * 2;          // 16 KB
   static constexpr int B_BYTES = HALF * BK * 2;          // 16 KB
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // this CTA's part of a stage
   static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
-  // control block: barriers full[S], empty[S], acc_full[2], acc_empty[2], drain, the
-  // epilogue pairs' exchange barriers [8]; tmem slot, abort flag, the epilogue's per-warp
-  // loss partials [2][EPI_WARPS] and arrival counters [2]. Then the pairs' exchange slots.
+  // control block: barriers full[S], empty[S], acc_full[2], acc_empty[2], drain; tmem slot,
+  // abort flag, the epilogue's per-warp loss partials [2][EPI_WARPS] and arrival counters [2]
   static constexpr int CTL_BYTES = 512;
   static constexpr int FULL = 0, EMPTY = 8 * STAGES, ACCF = 16 * STAGES, ACCE = ACCF + 16,
-                       DRAIN = ACCE + 16, PAIRB = DRAIN + 8, SLOT = PAIRB + 64, ABORT = SLOT + 4,
-                       RED = ABORT + 4, CNT = RED + 8 * EPI_WARPS, CTL_END = CNT + 8;
+                       DRAIN = ACCE + 16, SLOT = DRAIN + 8, ABORT = SLOT + 4, RED = ABORT + 4,
+                       CNT = RED + 8 * EPI_WARPS, CTL_END = CNT + 8;
   static_assert(CTL_END <= CTL_BYTES, "control block");
-  static constexpr int XCHG = BAR_OFF + CTL_BYTES;
-  static constexpr int XCHG_BYTES = PAIRS ? EPI_WARPS * 2 * 32 * 8 : 0;
-  static constexpr int SMEM_BYTES = 1024 /*align slack*/ + XCHG + XCHG_BYTES;
+  static constexpr int SMEM_BYTES = 1024 /*align slack*/ + BAR_OFF + CTL_BYTES;
   static constexpr uint32_t TMEM_COLS = 2 * TILE_N;
 };
 
-// STE_G = 0: the store / MSE epilogue (epi.kind); STE_G = 32, 64, 128: the weight-side STE
-// epilogue for that group length, weights in F16 (STE_F16) or BF16. One kernel per variant
-// keeps each epilogue's registers within the 96 a thread has here.
-template <int STE_G, bool STE_F16>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<STE_G>::NUM_THREADS, 1)
+template <int EV>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV>::NUM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    int a_mn, int b_mn, uint32_t fmt, int64_t rows, int64_t cols, int64_t depth,
                    GemmEpilogue epi, int tiles_n, int num_tiles) {
-  using C = Cfg<STE_G>;
+  using C = Cfg<EV>;
   constexpr int STAGES = C::STAGES, EPI_WARPS = C::EPI_WARPS, EPI_COLS = C::EPI_COLS;
-  using L = Layout<STAGES, EPI_WARPS, STE_G == 128>;
+  using L = Layout<STAGES, EPI_WARPS>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -499,8 +388,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<STE_G>::NUM_THRE
   const uint32_t bar_accf = sbase + L::BAR_OFF + L::ACCF;
   const uint32_t bar_acce = sbase + L::BAR_OFF + L::ACCE;
   const uint32_t bar_drain = sbase + L::BAR_OFF + L::DRAIN;
-  const uint32_t bar_pair = sbase + L::BAR_OFF + L::PAIRB;
-  float2* xchg = reinterpret_cast<float2*>(smem + L::XCHG);   // [EPI_WARPS][2][32] (G = 128)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctl + L::SLOT);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(ctl + L::ABORT);
   volatile float* red = reinterpret_cast<volatile float*>(ctl + L::RED);  // [2][EPI_WARPS]
@@ -524,7 +411,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<STE_G>::NUM_THRE
       cnt[b] = 0;
     }
     mbar_init(bar_drain, 1);
-    for (int q = 0; q < 8; ++q) mbar_init(bar_pair + 8 * q, 2);   // lane 0 of both partners
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -628,9 +514,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<STE_G>::NUM_THRE
     const int quad = warp & 3;                       // TMEM lanes 32*quad .. 32*quad+31
     const int cq = ew >> 2;                          // columns 64*cq .. 64*cq+63 of the tile
     const uint32_t acce_leader = peer_addr(bar_acce, 0);
-    // partner for groups of 128: the same rows, the adjacent quarter (cq ^ 1)
-    PairX px{xchg + ew * 64, xchg + (ew ^ 4) * 64,
-             bar_pair + 8 * static_cast<uint32_t>(quad + 4 * (cq >> 1)), 0};
     int lt = 0;
     for (int t = pair; t < num_tiles; t += pairs, ++lt) {
       const int buf = lt & 1;
@@ -649,9 +532,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<STE_G>::NUM_THRE
       float lsum = 0.f;
       const uint32_t tbase = tmem + (static_cast<uint32_t>(quad * 32) << 16) +
                              static_cast<uint32_t>(buf * TILE_N + cq * EPI_COLS);
-      if constexpr (STE_G != 0) {
-        const bool writer = STE_G < 128 || (cq & 1) == 0;
-        ste_w_epilogue<STE_G, STE_F16>(epi, tbase, wrow0, col0, rows, cols, lane, writer, px);
+      if constexpr (EV != 0) {
+        ste_w_epilogue<EV == 2>(epi, tbase, wrow0, col0, rows, cols, lane);
       } else {
         for (int ch = 0; ch < EPI_COLS / 32; ++ch) {
           uint32_t r[32];
@@ -757,8 +639,8 @@ bool make_map(CUtensorMap* map, omq_dtype dt, const GemmOperand& op, int64_t n_r
   return r == CUDA_SUCCESS;
 }
 
-static_assert(Layout<Cfg<0>::STAGES, Cfg<0>::EPI_WARPS, false>::SMEM_BYTES <= 232448, "smem");
-static_assert(Layout<Cfg<128>::STAGES, Cfg<128>::EPI_WARPS, true>::SMEM_BYTES <= 232448, "smem");
+static_assert(Layout<Cfg<0>::STAGES, Cfg<0>::EPI_WARPS>::SMEM_BYTES <= 232448, "smem");
+static_assert(Layout<Cfg<1>::STAGES, Cfg<1>::EPI_WARPS>::SMEM_BYTES <= 232448, "smem");
 
 using GemmKernel = void (*)(CUtensorMap, CUtensorMap, int, int, uint32_t, int64_t, int64_t,
                             int64_t, GemmEpilogue, int, int);
@@ -768,19 +650,10 @@ struct KernelChoice {
   int threads, smem;
 };
 
-template <int G, bool F16>
+template <int EV>
 KernelChoice choice() {
-  return {gemm_tc_kernel<G, F16>, Cfg<G>::NUM_THREADS,
-          Layout<Cfg<G>::STAGES, Cfg<G>::EPI_WARPS, G == 128>::SMEM_BYTES};
-}
-
-KernelChoice pick_kernel(int ste_g, bool f16w) {
-  switch (ste_g) {
-    case 32: return f16w ? choice<32, true>() : choice<32, false>();
-    case 64: return f16w ? choice<64, true>() : choice<64, false>();
-    case 128: return f16w ? choice<128, true>() : choice<128, false>();
-    default: return choice<0, false>();
-  }
+  return {gemm_tc_kernel<EV>, Cfg<EV>::NUM_THREADS,
+          Layout<Cfg<EV>::STAGES, Cfg<EV>::EPI_WARPS>::SMEM_BYTES};
 }
 
 // Opt each kernel variant into the large dynamic shared memory once.
@@ -817,14 +690,12 @@ omq_status gemm_tc(omq_dtype dt, const GemmOperand& A, const GemmOperand& B, int
   const int64_t tiles_m = ceil_div(rows, TILE_M), tiles_n = ceil_div(cols, TILE_N);
   const int64_t tiles = tiles_m * tiles_n;
   if (n_tiles) *n_tiles = 2 * tiles;
-  int ste_g = 0;
+  KernelChoice kc = choice<0>();
   if (epi.kind == Epi::SteW) {
     if (!ste_fusable(epi.ste.G) || (epi.ste.wdt != OMQ_BF16 && epi.ste.wdt != OMQ_F16))
       return OMQ_ERR_SHAPE;
-    ste_g = static_cast<int>(epi.ste.G);
+    kc = epi.ste.wdt == OMQ_F16 ? choice<2>() : choice<1>();
   }
-  const bool f16w = epi.kind == Epi::SteW && epi.ste.wdt == OMQ_F16;
-  const KernelChoice kc = pick_kernel(ste_g, f16w);
   const cudaError_t attr_err = kernel_attr(kc.fn, kc.smem);
   if (attr_err != cudaSuccess) {
     set_cuda_error(attr_err);

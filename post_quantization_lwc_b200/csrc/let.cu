@@ -33,23 +33,39 @@ __device__ __forceinline__ void let8(const LetParams& p, int64_t off, int64_t co
   for (int i = 0; i < 8; ++i) v[i] = __fdiv_rn(__fsub_rn(v[i], dv[i]), sv[i]);
 }
 
-// U chunks of 8 per thread per iteration, all loaded before any is converted.
-template <int U>
+// Unquantized activations (16-bit): X~ = (X - delta) / s stored in the operand type, or a
+// plain conversion when there is no LET (AFFINE false). Grid (256-column segments, row
+// blocks of kLetRows); a lane keeps 8 fixed columns (and their s, delta in registers), the 8
+// warps take every 8th row, U rows loaded before any is converted.
+constexpr int kLetRows = 64;
+
+template <int U, bool AFFINE>
 __global__ void __launch_bounds__(256) let_elem_kernel(LetParams p) {
-  const int64_t chunks = p.M * p.K / 8;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t c0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; c0 < chunks;
-       c0 += stride * U) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * 256 + lane * 8;
+  if (c0 >= p.K) return;
+  float sv[8], dv[8];
+  if (AFFINE) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) { sv[i] = 1.f; dv[i] = 0.f; }
+    if (p.s) load_f8(p.s, c0, sv);
+    if (p.d) load_f8(p.d, c0, dv);
+  }
+  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * kLetRows;
+  const int64_t r1 = min(p.M, r0 + kLetRows);
+  for (int64_t mb = r0 + w; mb < r1; mb += 8 * U) {
     float v[U][8];
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int64_t c = c0 + u * stride;
-      if (c < chunks) let8(p, c * 8, (c * 8) % p.K, v[u]);
-    }
+    for (int u = 0; u < U; ++u)
+      if (mb + 8 * u < r1) load8(p.X, (mb + 8 * u) * p.K + c0, p.xdt, v[u]);
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const int64_t c = c0 + u * stride;
-      if (c < chunks) store8(p.Xq, c * 8, p.xq_dt, v[u]);
+      if (mb + 8 * u >= r1) continue;
+      if (AFFINE) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[u][i] = __fdiv_rn(__fsub_rn(v[u][i], dv[i]), sv[i]);
+      }
+      store8(p.Xq, (mb + 8 * u) * p.K + c0, p.xq_dt, v[u]);
     }
   }
 }
@@ -149,10 +165,10 @@ __global__ void __launch_bounds__(256) let_bias_kernel(const void* W, omq_dtype 
 omq_status launch_let(const LetParams& p, int abits, cudaStream_t stream) {
   const int sms = num_sms();
   if (abits >= 16) {
-    const int64_t chunks = p.M * p.K / 8;
-    const int64_t want = ceil_div(chunks, 256 * 4);
-    const unsigned grid = static_cast<unsigned>(want < int64_t(sms) * 8 ? want : int64_t(sms) * 8);
-    let_elem_kernel<4><<<grid, 256, 0, stream>>>(p);
+    const dim3 grid(static_cast<unsigned>(ceil_div(p.K, 256)),
+                    static_cast<unsigned>(ceil_div(p.M, kLetRows)));
+    if (p.s || p.d) let_elem_kernel<4, true><<<grid, 256, 0, stream>>>(p);
+    else let_elem_kernel<4, false><<<grid, 256, 0, stream>>>(p);
     return launch_status();
   }
   const size_t smem = static_cast<size_t>(p.K) * sizeof(float);

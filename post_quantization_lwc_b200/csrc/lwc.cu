@@ -81,14 +81,18 @@ constexpr int kLwcRows = 64;
 template <int LPG, int U>
 __global__ void __launch_bounds__(256) lwc_small_kernel(LwcParams p) {
   constexpr int GPW = 32 / LPG;   // groups per segment
+  // The clipping strengths (binary64 sigmoids) of the U rows' groups are spread over the
+  // warp's lanes: SPR strengths a row (gamma, beta of each group), RPP rows a pass of 32
+  // lanes, NP passes. Lane t of pass q evaluates row q*RPP + t/SPR, group t%SPR / 2, beta
+  // for odd t.
+  constexpr int SPR = 2 * GPW, RPP = 32 / SPR, NP = (U + RPP - 1) / RPP;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int sub = lane / LPG, lig = lane % LPG;
   const int64_t c0 = static_cast<int64_t>(blockIdx.x) * 256 + lane * 8;
   const bool cvalid = c0 < p.K;
   const int64_t j = c0 / (LPG * 8);                        // this lane's group in the row
-  // lane t evaluates the strength of group (segment's first + t/2), gamma for even t
-  const int64_t jt = static_cast<int64_t>(blockIdx.x) * GPW + (lane >> 1);
-  const bool tvalid = lane < 2 * GPW && jt < p.ng;
+  const int64_t jt = static_cast<int64_t>(blockIdx.x) * GPW + (lane % SPR) / 2;
+  const bool tvalid = jt < p.ng;
   const float* logit = (lane & 1) ? p.bl : p.gl;
   float sv[8];
   if (p.s && cvalid) {
@@ -100,7 +104,13 @@ __global__ void __launch_bounds__(256) lwc_small_kernel(LwcParams p) {
   const int64_t r0 = static_cast<int64_t>(blockIdx.y) * kLwcRows;
   const int64_t r1 = min(p.N, r0 + kLwcRows);
   for (int64_t nb = r0 + w; nb < r1; nb += 8 * U) {
-    float v[U][8], st[U];
+    float v[U][8], st[NP];
+#pragma unroll
+    for (int q = 0; q < NP; ++q) {
+      const int u = q * RPP + lane / SPR;
+      const int64_t n = nb + 8 * u;
+      st[q] = (u < U && n < r1 && tvalid) ? strength(logit[n * p.ng + jt]) : 1.f;
+    }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int64_t n = nb + 8 * u;
@@ -114,7 +124,6 @@ __global__ void __launch_bounds__(256) lwc_small_kernel(LwcParams p) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) v[u][i] = 0.f;
       }
-      st[u] = (n < r1 && tvalid) ? strength(logit[n * p.ng + jt]) : 1.f;
     }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
@@ -135,8 +144,9 @@ __global__ void __launch_bounds__(256) lwc_small_kernel(LwcParams p) {
         nmax += __shfl_xor_sync(0xffffffffu, nmax, o);
         nmin += __shfl_xor_sync(0xffffffffu, nmin, o);
       }
-      const float g = __shfl_sync(0xffffffffu, st[u], 2 * sub);
-      const float b = __shfl_sync(0xffffffffu, st[u], 2 * sub + 1);
+      const int src = (u % RPP) * SPR + 2 * sub;
+      const float g = __shfl_sync(0xffffffffu, st[u / RPP], src);
+      const float b = __shfl_sync(0xffffffffu, st[u / RPP], src + 1);
       if (n >= r1 || !cvalid) continue;
       const GroupQ q = group_params(g, b, vmax, vmin, p.Q);
       encode8(p, n * p.K + c0, v[u], q);

@@ -25,13 +25,16 @@ size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
 int64_t rows_per_block_w(int64_t group) { return small_group(group) ? kRowsSmallW : kRowsLargeW; }
 
 // The weight-side STE runs inside the dW^ GEMM's epilogue for 16-bit operands and weights
-// and groups of 32, 64 or 128; otherwise it is a separate kernel reading a stored dW^.
+// and group lengths that are multiples of 32 (per-channel groups included); otherwise it is
+// a separate kernel reading a stored dW^.
 bool fused_ste_w(omq_dtype op_dt, omq_dtype wdt, int64_t group) {
   return op_dt != OMQ_F32 && wdt != OMQ_F32 && ste_fusable(group);
 }
 
 struct BwdLayout {
-  size_t dbt_part, dbt, dwhat, dxq, part_ws, part_wd, part_xs, part_xd, rowstat, total;
+  size_t dbt_part, dbt, dwhat, dxq, part_ws, part_wd, part_xs, part_xd, rowstat, red;
+  size_t gh_part, gc_part, emax, emin;   // fused weight-side STE (group a multiple of 32)
+  size_t total;
   int64_t rb_colsum, rb_w, rb_x;
 };
 
@@ -39,7 +42,8 @@ BwdLayout bwd_layout(int64_t M, int64_t N, int64_t K, int64_t group) {
   BwdLayout L{};
   L.rb_colsum = ceil_div(M, kRowsColsum);
   // enough partial rows for either weight-side STE (the fused one writes one per 32 rows)
-  L.rb_w = ceil_div(N, ste_fusable(group) ? kRowsFusedW : rows_per_block_w(group));
+  L.rb_w = ceil_div(N, rows_per_block_w(group));
+  if (ste_fusable(group) && ceil_div(N, kRowsFusedW) > L.rb_w) L.rb_w = ceil_div(N, kRowsFusedW);
   L.rb_x = ceil_div(M, kRowsX);
   size_t off = 0;
   auto take = [&](size_t bytes) { size_t o = off; off += align256(bytes); return o; };
@@ -52,6 +56,12 @@ BwdLayout bwd_layout(int64_t M, int64_t N, int64_t K, int64_t group) {
   L.part_xs = take(sizeof(float) * L.rb_x * K);
   L.part_xd = take(sizeof(float) * L.rb_x * K);
   L.rowstat = take(sizeof(float) * 2 * M);
+  L.red = take(sizeof(double) * 2 * kReduceChunks * (N > K ? N : K));
+  const bool fusable = ste_fusable(group);
+  L.gh_part = take(fusable ? sizeof(float) * (K / 32) * N : 0);
+  L.gc_part = take(fusable ? sizeof(float) * (K / 32) * N : 0);
+  L.emax = take(fusable ? sizeof(float) * N * (K / group) : 0);
+  L.emin = take(fusable ? sizeof(float) * N * (K / group) : 0);
   L.total = off;
   return L;
 }
@@ -331,31 +341,30 @@ static omq_status bwd_impl(const omq_bwd_args* a, void* workspace, size_t ws_byt
   float* part_wd = at<float>(workspace, L.part_wd);
   float* part_xs = at<float>(workspace, L.part_xs);
   float* part_xd = at<float>(workspace, L.part_xd);
+  double* red = at<double>(workspace, L.red);
 
   // dB~ = column sums of dY (needed for d_delta, or when asked for)
   OMQ_TRY(ph.mark(OMQ_PH_DBIAS));
   if (a->d_delta || a->d_B_tilde) {
     OMQ_TRY(launch_colsum(a->dY, a->op_dt, M, N, kRowsColsum, nullptr, dbt_part, st));
-    OMQ_TRY(launch_reduce_cols(dbt_part, L.rb_colsum, nullptr, 0, N, gscale, dbt, st));
+    const ColReduce r{dbt_part, L.rb_colsum, nullptr, 0, gscale, dbt};
+    OMQ_TRY(launch_reduce_cols(&r, 1, N, red, st));
   }
   // dW^ = G^T Xq   [N, K]
   const float Q = static_cast<float>((1 << a->bits) - 1);
   const bool fused = fused_ste_w(a->op_dt, a->dt, G);
   const int64_t rb_w = fused ? ceil_div(N, kRowsFusedW) : ceil_div(N, rows_per_block_w(G));
-  // the W side of d delta, sum_n dB~[n] W[n, k], in row blocks of kRowsColsum when the STE
-  // is fused (the separate STE kernel produces it in its own row blocks)
-  const int64_t rb_wd = fused ? ceil_div(N, kRowsColsum) : rb_w;
   OMQ_TRY(ph.mark(OMQ_PH_DW_GEMM));
   {
     GemmOperand A{a->dY, N, true}, B{a->Xq, K, true};
     GemmEpilogue epi{};
     epi.out_scale = gscale;
     if (fused) {
-      // weight-side STE in the epilogue: d gamma / d beta logits and the W-side LET column
+      // weight-side STE in the epilogue: per-chunk partial sums and the W-side LET column
       // partials straight from the accumulator
       epi.kind = Epi::SteW;
-      epi.ste = SteWEpi{a->W, a->dt, K, G, K / G, Q, a->s, a->gamma_logit, a->beta_logit,
-                        a->h, a->z, a->grp_range, a->d_gamma_logit, a->d_beta_logit,
+      epi.ste = SteWEpi{a->W, a->dt, K, G, K / G, Q, a->s, a->h, a->z,
+                        at<float>(workspace, L.gh_part), at<float>(workspace, L.gc_part),
                         a->d_s ? part_ws : nullptr};
     } else {
       epi.kind = Epi::StoreF32;
@@ -365,9 +374,19 @@ static omq_status bwd_impl(const omq_bwd_args* a, void* workspace, size_t ws_byt
   }
   // weight-side STE: d gamma / d beta logits and the W-side LET column partials
   OMQ_TRY(ph.mark(OMQ_PH_STE_W));
-  if (fused && a->d_delta)
-    OMQ_TRY(launch_colsum(a->W, a->dt, N, K, kRowsColsum, dbt, part_wd, st));
-  if (!fused) {
+  if (fused) {
+    float* emax = a->d_s ? at<float>(workspace, L.emax) : nullptr;
+    float* emin = a->d_s ? at<float>(workspace, L.emin) : nullptr;
+    const SteWFinish f{N, G, K / G, Q, at<float>(workspace, L.gh_part),
+                       at<float>(workspace, L.gc_part), a->h, a->grp_range, a->gamma_logit,
+                       a->beta_logit, a->d_gamma_logit, a->d_beta_logit, emax, emin};
+    OMQ_TRY(launch_ste_w_finish(f, st));
+    if (a->d_s || a->d_delta) {
+      const SteWCorr c{a->W, a->dt, N, K, G, a->s, a->grp_range, emax, emin, dbt,
+                       a->d_s ? part_ws : nullptr, a->d_delta ? part_wd : nullptr};
+      OMQ_TRY(launch_ste_w_corr(c, st));
+    }
+  } else {
     SteWParams p{a->W, a->dt, N, K, G, K / G, Q, a->s, a->gamma_logit, a->beta_logit, a->h, a->z,
                  a->grp_range, dwhat, a->d_delta ? dbt : nullptr, a->d_gamma_logit,
                  a->d_beta_logit, a->d_s ? part_ws : nullptr, a->d_delta ? part_wd : nullptr,
@@ -397,9 +416,11 @@ static omq_status bwd_impl(const omq_bwd_args* a, void* workspace, size_t ws_byt
     OMQ_TRY(launch_ste_x(p, st));
   }
   OMQ_TRY(ph.mark(OMQ_PH_LET_REDUCE));
-  if (a->d_s) OMQ_TRY(launch_reduce_cols(part_ws, rb_w, part_xs, L.rb_x, K, 1.f, a->d_s, st));
-  if (a->d_delta)
-    OMQ_TRY(launch_reduce_cols(part_wd, rb_wd, part_xd, L.rb_x, K, 1.f, a->d_delta, st));
+  ColReduce r[2];
+  int nr = 0;
+  if (a->d_s) r[nr++] = ColReduce{part_ws, rb_w, part_xs, L.rb_x, 1.f, a->d_s};
+  if (a->d_delta) r[nr++] = ColReduce{part_wd, rb_w, part_xd, L.rb_x, 1.f, a->d_delta};
+  if (nr) OMQ_TRY(launch_reduce_cols(r, nr, K, red, st));
   return OMQ_OK;
 }
 

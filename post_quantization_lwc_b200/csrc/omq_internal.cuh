@@ -61,6 +61,12 @@ __device__ __forceinline__ void load8(const void* p, int64_t i, omq_dtype dt, fl
     v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
   }
 }
+// 8 consecutive floats starting at a multiple of 4 (two 16-byte loads).
+__device__ __forceinline__ void load_f8(const float* p, int64_t off, float (&v)[8]) {
+  const float4* q = reinterpret_cast<const float4*>(p + off);
+  const float4 a = q[0], b = q[1];
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
 __device__ __forceinline__ void store8(void* p, int64_t i, omq_dtype dt, const float (&v)[8]) {
   if (dt == OMQ_BF16) {
     uint4 raw;
@@ -162,21 +168,19 @@ struct GemmOperand {
 enum class Epi { StoreF32 = 0, MseLoss = 1, SteW = 2 };
 
 // Weight-side straight-through backward fused into the dW^ GEMM's epilogue (16-bit weights,
-// groups of 32, 64 or 128 elements): the tile's accumulator is dW^ / out_scale.
+// group length a multiple of 32): the tile's accumulator is dW^ / out_scale. The epilogue
+// writes per-(32-column chunk, row) partial sums; ste_w_finish / ste_w_corr complete them.
 struct SteWEpi {
   const void* W;           // [N, K] BF16 or F16
   omq_dtype wdt;
   int64_t K, G, ng;
   float Q;
   const float* s;          // [K] or NULL
-  const float* gl;
-  const float* bl;
   const float* h;
   const int32_t* z;
-  const omq_range* range;
-  float* d_gl;
-  float* d_bl;
-  float* part_s;           // [ceil(N/32), K] or NULL: per 32-row block, sum dW~ W
+  float* gh_part;          // [K/32, N]
+  float* gc_part;          // [K/32, N]
+  float* part_s;           // [ceil(N/32), K] or NULL: per 32-row block, sum (in range) dW~ W
 };
 
 struct GemmEpilogue {
@@ -191,9 +195,9 @@ struct GemmEpilogue {
   SteWEpi ste;             // SteW
 };
 
-// Group lengths the dW^ GEMM's epilogue handles (a group covers one or two 32-column chunks
-// of an epilogue warp's 64 columns, or the 128 columns of a warp pair).
-inline bool ste_fusable(int64_t g) { return g == 32 || g == 64 || g == 128; }
+// Group lengths whose weight-side STE runs in the dW^ GEMM's epilogue: whole 32-column
+// chunks (per-channel groups included).
+inline bool ste_fusable(int64_t g) { return g >= 32 && g % 32 == 0; }
 
 // 16-bit operands (BF16 or F16, both the same type) on tcgen05 (sm_100a). Reports the
 // number of output tiles (loss partial slots).
@@ -295,12 +299,60 @@ omq_status launch_let(const LetParams& p, int abits, cudaStream_t stream);
 omq_status launch_let_bias(const void* W, omq_dtype wdt, int64_t N, int64_t K, const float* delta,
                            const float* B, float* Bt, cudaStream_t stream);
 omq_status launch_ste_w(const SteWParams& p, cudaStream_t stream);
+
+// Completes the fused weight-side STE from the epilogue's partial sums: per group, G_h and
+// G_z, the logit gradients and (emax / emin not NULL) the gradient share of each max / min
+// element, dM / n_max and dm / n_min.
+struct SteWFinish {
+  int64_t N, G, ng;
+  float Q;
+  const float* gh_part;    // [K/32, N]
+  const float* gc_part;
+  const float* h;
+  const omq_range* range;
+  const float* gl;
+  const float* bl;
+  float* d_gl;
+  float* d_bl;
+  float* emax;             // [N, ng] or NULL
+  float* emin;
+};
+omq_status launch_ste_w_finish(const SteWFinish& p, cudaStream_t stream);
+// The W-side LET terms the fused epilogue leaves out, per 32-row block rb (one pass over W):
+//   part_s[rb, k] += sum_n emax W[n,k] where W~[n,k] is its group's max, emin W[n,k] where it
+//                    is the min (part_s NULL: skipped)
+//   part_d[rb, k]  = sum_n dBt[n] W[n,k]  (part_d NULL: skipped)
+struct SteWCorr {
+  const void* W;
+  omq_dtype wdt;
+  int64_t N, K, G;
+  const float* s;
+  const omq_range* range;
+  const float* emax;
+  const float* emin;
+  const float* dBt;
+  float* part_s;
+  float* part_d;
+};
+omq_status launch_ste_w_corr(const SteWCorr& p, cudaStream_t stream);
 omq_status launch_ste_x(const SteXParams& p, cudaStream_t stream);
 // part[rb, j] = sum over rows i of block rb (R rows) of w[i] A[i, j] (w NULL: 1).
 omq_status launch_colsum(const void* A, omq_dtype dt, int64_t rows, int64_t cols, int R,
                          const float* w, float* part, cudaStream_t stream);
-omq_status launch_reduce_cols(const float* p0, int64_t r0n, const float* p1, int64_t r1n,
-                              int64_t cols, float scale, float* out, cudaStream_t stream);
+// out[j] = scale * sum over the rows of p0 [r0n, cols] and p1 [r1n, cols] (p1 may be NULL),
+// binary64 in a fixed order, for one or two problems with the same cols in one launch pair;
+// scratch holds 2 * kReduceChunks * cols doubles.
+constexpr int kReduceChunks = 16;
+struct ColReduce {
+  const float* p0;
+  int64_t r0n;
+  const float* p1;
+  int64_t r1n;
+  float scale;
+  float* out;
+};
+omq_status launch_reduce_cols(const ColReduce* probs, int nprob, int64_t cols, double* scratch,
+                              cudaStream_t stream);
 omq_status launch_loss_finalize(const float* part, int64_t n, double inv_count, float* loss,
                                 cudaStream_t stream);
 omq_status launch_adamw(const AdamSeg* segs, int nseg, float b1, float b2, float eps, float wd,

@@ -8,6 +8,8 @@
 // over rows: kernels write per-(row block, column) partial sums that reduce_cols_kernel adds
 // in a fixed order, so results are bitwise reproducible (no floating-point atomics). The
 // memory-bound kernels issue the loads of several rows before computing on any of them.
+#include <algorithm>
+
 #include "ste_common.cuh"
 
 namespace omq {
@@ -219,6 +221,156 @@ __global__ void __launch_bounds__(256) ste_w_large_kernel(SteWParams p) {
     }
 }
 
+// ------------------------------------------------------------------ fused weight side
+// Completion of the STE that the dW^ GEMM's epilogue started. Grid (32-row tiles, 32-group
+// tile strides), 256 threads; a tile of 32 rows x 32 groups is read in two mappings so both
+// layouts stay coalesced: the chunk partials ([K/32, N]) with the row fastest, staged in
+// shared memory, then the per-group arrays ([N, ng]) with the group fastest. A group's
+// chunk partials are added in chunk order (groups of up to 8 chunks) or as 8 interleaved
+// partial sums added in a fixed order (longer groups).
+__global__ void __launch_bounds__(256) ste_w_finish_kernel(SteWFinish p) {
+  __shared__ float sgh[32][33], sgc[32][33];   // [group in tile][row in tile]
+  __shared__ float wred[2][8][32];
+  const int64_t n0 = static_cast<int64_t>(blockIdx.x) * 32;
+  const int64_t cpg = p.G / 32;
+  for (int64_t j0 = static_cast<int64_t>(blockIdx.y) * 32; j0 < p.ng; j0 += 32 * gridDim.y) {
+    if (cpg <= 8) {
+      for (int e = threadIdx.x; e < 1024; e += blockDim.x) {
+        const int nl = e & 31, jl = e >> 5;
+        const int64_t n = n0 + nl, j = j0 + jl;
+        float Gh = 0.f, Gc = 0.f;
+        if (n < p.N && j < p.ng)
+#pragma unroll 8
+          for (int64_t c = j * cpg; c < (j + 1) * cpg; ++c) {
+            Gh += p.gh_part[c * p.N + n];
+            Gc += p.gc_part[c * p.N + n];
+          }
+        sgh[jl][nl] = Gh;
+        sgc[jl][nl] = Gc;
+      }
+    } else {
+      // long groups (per-channel ones included): the 8 warps take every 8th chunk of a group
+      // (lane = row), then warp 0 adds the 8 partial sums in warp order
+      const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+      const int64_t n = n0 + lane;
+      for (int jl = 0; jl < 32; ++jl) {
+        const int64_t j = j0 + jl;
+        float Gh = 0.f, Gc = 0.f;
+        if (n < p.N && j < p.ng)
+#pragma unroll 4
+          for (int64_t c = j * cpg + w; c < (j + 1) * cpg; c += 8) {
+            Gh += p.gh_part[c * p.N + n];
+            Gc += p.gc_part[c * p.N + n];
+          }
+        wred[0][w][lane] = Gh;
+        wred[1][w][lane] = Gc;
+        __syncthreads();
+        if (w == 0) {
+          float a = 0.f, b = 0.f;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            a += wred[0][q][lane];
+            b += wred[1][q][lane];
+          }
+          sgh[jl][lane] = a;
+          sgc[jl][lane] = b;
+        }
+        __syncthreads();
+        if (j0 + jl + 1 >= p.ng) break;   // uniform
+      }
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < 1024; e += blockDim.x) {
+      const int jl = e & 31, nl = e >> 5;
+      const int64_t n = n0 + nl, j = j0 + jl;
+      if (n >= p.N || j >= p.ng) continue;
+      const int64_t gi = n * p.ng + j;
+      const float h = p.h[gi];
+      const float Gh = sgh[jl][nl];
+      const float Gz = -h * sgc[jl][nl];
+      const omq_range rg = p.range[gi];
+      const float glv = p.gl[gi], blv = p.bl[gi];
+      const float g = strength_value(glv), b = strength_value(blv);
+      const bool active = h_active(h, glv, blv, rg.vmax, rg.vmin, p.Q);
+      const GroupGrad gg = group_grad(Gh, Gz, g, b, h, rg.vmax, rg.vmin, p.Q, active);
+      if (p.d_gl) p.d_gl[gi] = gg.dg * g * (1.f - g);
+      if (p.d_bl) p.d_bl[gi] = gg.db * b * (1.f - b);
+      if (p.emax) {
+        p.emax[gi] = gg.dM / static_cast<float>(rg.nmax);
+        p.emin[gi] = gg.dm / static_cast<float>(rg.nmin);
+      }
+    }
+    __syncthreads();   // the tiles are rewritten for the next group stride
+  }
+}
+
+// The W-side LET terms that the epilogue leaves out, in one pass over W. Grid (256-column
+// segments, 32-row block strides); lane = 8 columns of one group, the 8 warps take rows w,
+// w + 8, w + 16, w + 24 of a block; the warps' sums are added in warp order.
+//   part_s[rb, k] += sum_n (emax W[n,k] where W~[n,k] is its group's max, emin W[n,k] where
+//                    it is the min)                       (the clipping-range terms of d s)
+//   part_d[rb, k]  = sum_n dBt[n] W[n,k]                  (the bias term of d delta)
+__global__ void __launch_bounds__(256) ste_w_corr_kernel(SteWCorr p) {
+  __shared__ float red_s[8][256];
+  __shared__ float red_d[8][256];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * 256 + lane * 8;
+  const bool cvalid = c0 < p.K;
+  const int64_t ng = p.K / p.G, j = c0 / p.G;
+  float sv[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) sv[i] = 1.f;
+  if (p.s && cvalid) load_f8(p.s, c0, sv);
+  for (int64_t rb = blockIdx.y; rb * 32 < p.N; rb += gridDim.y) {
+    float acc_s[8] = {}, acc_d[8] = {};
+    float v[4][8];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t n = rb * 32 + w + 8 * u;
+      if (n < p.N && cvalid) load8(p.W, n * p.K + c0, p.wdt, v[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t n = rb * 32 + w + 8 * u;
+      if (n >= p.N || !cvalid) continue;
+      if (p.part_s) {
+        const int64_t gi = n * ng + j;
+        const omq_range rg = p.range[gi];
+        const float eM = p.emax[gi], em = p.emin[gi];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float wt = p.s ? __fmul_rn(v[u][i], sv[i]) : v[u][i];
+          if (wt == rg.vmax) acc_s[i] += eM * v[u][i];
+          if (wt == rg.vmin) acc_s[i] += em * v[u][i];
+        }
+      }
+      if (p.part_d) {
+        const float db = p.dBt[n];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc_d[i] += db * v[u][i];
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      red_s[w][lane * 8 + i] = acc_s[i];
+      red_d[w][lane * 8 + i] = acc_d[i];
+    }
+    __syncthreads();
+    const int64_t col = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
+    if (col < p.K) {
+      float a = 0.f, d = 0.f;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        a += red_s[q][threadIdx.x];
+        d += red_d[q][threadIdx.x];
+      }
+      if (p.part_s) p.part_s[rb * p.K + col] += a;
+      if (p.part_d) p.part_d[rb * p.K + col] = d;
+    }
+    __syncthreads();   // red is rewritten by the next row block
+  }
+}
+
 // ------------------------------------------------------------------ activation side
 __device__ __forceinline__ void xtilde8(const SteXParams& p, int64_t off, const float (&sv)[8],
                                         const float (&dv)[8], float (&v)[8]) {
@@ -402,31 +554,55 @@ __global__ void __launch_bounds__(256) colsum_kernel(const void* A, omq_dtype dt
   }
 }
 
-// out[j] = scale * (sum_r p0[r, j] (+ sum_r p1[r, j])), binary64 accumulation in a fixed
-// order: 8 warps take every 8th row of 32 consecutive columns, then combine in warp order.
-__global__ void __launch_bounds__(256) reduce_cols_kernel(const float* p0, int64_t r0n,
-                                                          const float* p1, int64_t r1n,
-                                                          int64_t cols, float scale, float* out) {
+// out[j] = scale * (sum_r p0[r, j] + sum_r p1[r, j]) for up to two such problems (blockIdx.z)
+// in two levels, binary64, fixed order. Level 1, grid (32-column blocks, row chunks,
+// problems): chunk c takes rows [c rpc, (c + 1) rpc) of p0 followed by p1; its 8 warps take
+// every 8th row (lane = column) and are combined in warp order into scratch[problem, c, j],
+// or, with a single chunk, straight into out.
+struct ColReduceSet {
+  ColReduce pr[2];
+  int64_t cols, rpc;
+  int chunks;
+};
+
+__global__ void __launch_bounds__(256) reduce_cols_partial_kernel(ColReduceSet rs,
+                                                                  double* scratch) {
   __shared__ double red[8][32];
+  const ColReduce& q = rs.pr[blockIdx.z];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int64_t j = static_cast<int64_t>(blockIdx.x) * 32 + lane;
+  const int64_t r0n = q.r0n, total = q.r0n + (q.p1 ? q.r1n : 0);
+  const int64_t ra = static_cast<int64_t>(blockIdx.y) * rs.rpc;
+  const int64_t rb = min(total, ra + rs.rpc);
   double a = 0.0;
-  if (j < cols) {
+  if (j < rs.cols) {
 #pragma unroll 4
-    for (int64_t r = w; r < r0n; r += 8) a += p0[r * cols + j];
-    if (p1) {
-#pragma unroll 4
-      for (int64_t r = w; r < r1n; r += 8) a += p1[r * cols + j];
-    }
+    for (int64_t r = ra + w; r < rb; r += 8)
+      a += r < r0n ? q.p0[r * rs.cols + j] : q.p1[(r - r0n) * rs.cols + j];
   }
   red[w][lane] = a;
   __syncthreads();
-  if (w == 0 && j < cols) {
+  if (w == 0 && j < rs.cols) {
     double t = 0.0;
 #pragma unroll
-    for (int q = 0; q < 8; ++q) t += red[q][lane];
-    out[j] = static_cast<float>(t * static_cast<double>(scale));
+    for (int k = 0; k < 8; ++k) t += red[k][lane];
+    if (rs.chunks == 1)
+      q.out[j] = static_cast<float>(t * static_cast<double>(q.scale));
+    else
+      scratch[(static_cast<int64_t>(blockIdx.z) * rs.chunks + blockIdx.y) * rs.cols + j] = t;
   }
+}
+
+// Level 2, grid (column blocks, problems): out[j] = scale * sum over chunks c (in order).
+__global__ void __launch_bounds__(256) reduce_cols_final_kernel(ColReduceSet rs,
+                                                                const double* scratch) {
+  const ColReduce& q = rs.pr[blockIdx.y];
+  const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (j >= rs.cols) return;
+  const double* sc = scratch + static_cast<int64_t>(blockIdx.y) * rs.chunks * rs.cols;
+  double t = 0.0;
+  for (int c = 0; c < rs.chunks; ++c) t += sc[c * rs.cols + j];
+  q.out[j] = static_cast<float>(t * static_cast<double>(q.scale));
 }
 
 // loss = (sum of per-tile partials) / count, binary64, fixed order.
@@ -492,6 +668,20 @@ omq_status launch_ste_w(const SteWParams& p, cudaStream_t stream) {
   return launch_status();
 }
 
+omq_status launch_ste_w_finish(const SteWFinish& p, cudaStream_t stream) {
+  const dim3 grid(static_cast<unsigned>(ceil_div(p.N, 32)),
+                  static_cast<unsigned>(std::min<int64_t>(ceil_div(p.ng, 32), 65535)));
+  ste_w_finish_kernel<<<grid, 256, 0, stream>>>(p);
+  return launch_status();
+}
+
+omq_status launch_ste_w_corr(const SteWCorr& p, cudaStream_t stream) {
+  const dim3 grid(static_cast<unsigned>(ceil_div(p.K, 256)),
+                  static_cast<unsigned>(std::min<int64_t>(ceil_div(p.N, 32), 65535)));
+  ste_w_corr_kernel<<<grid, 256, 0, stream>>>(p);
+  return launch_status();
+}
+
 omq_status launch_ste_x(const SteXParams& p, cudaStream_t stream) {
   if (p.quantized) {
     const int sms = num_sms();
@@ -513,10 +703,27 @@ omq_status launch_colsum(const void* A, omq_dtype dt, int64_t rows, int64_t cols
   return launch_status();
 }
 
-omq_status launch_reduce_cols(const float* p0, int64_t r0n, const float* p1, int64_t r1n,
-                              int64_t cols, float scale, float* out, cudaStream_t stream) {
-  reduce_cols_kernel<<<static_cast<unsigned>(ceil_div(cols, 32)), 256, 0, stream>>>(
-      p0, r0n, p1, r1n, cols, scale, out);
+omq_status launch_reduce_cols(const ColReduce* probs, int nprob, int64_t cols, double* scratch,
+                              cudaStream_t stream) {
+  if (nprob < 1 || nprob > 2) return OMQ_ERR_SHAPE;
+  ColReduceSet rs{};
+  int64_t total = 0;
+  for (int i = 0; i < nprob; ++i) {
+    rs.pr[i] = probs[i];
+    const int64_t t = probs[i].r0n + (probs[i].p1 ? probs[i].r1n : 0);
+    total = t > total ? t : total;
+  }
+  rs.cols = cols;
+  rs.chunks = static_cast<int>(
+      std::min<int64_t>(kReduceChunks, std::max<int64_t>(1, ceil_div(total, 32))));
+  rs.rpc = ceil_div(std::max<int64_t>(total, 1), rs.chunks);
+  const dim3 grid(static_cast<unsigned>(ceil_div(cols, 32)), static_cast<unsigned>(rs.chunks),
+                  static_cast<unsigned>(nprob));
+  reduce_cols_partial_kernel<<<grid, 256, 0, stream>>>(rs, scratch);
+  const omq_status st = launch_status();
+  if (st != OMQ_OK || rs.chunks == 1) return st;
+  const dim3 g2(static_cast<unsigned>(ceil_div(cols, 256)), static_cast<unsigned>(nprob));
+  reduce_cols_final_kernel<<<g2, 256, 0, stream>>>(rs, scratch);
   return launch_status();
 }
 

@@ -75,12 +75,6 @@ __device__ __forceinline__ void in_range8(const float (&v)[8], float h, float z,
   }
 }
 
-__device__ __forceinline__ void load_f8(const float* p, int64_t off, float (&v)[8]) {
-  const float4* q = reinterpret_cast<const float4*>(p + off);
-  const float4 a = q[0], b = q[1];
-  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-}
-
 // Column sums over a warp's 32 rows: lane l holds 32 values (its row, 32 columns); on return
 // lane l holds the sum of column l over the 32 lanes. Five butterfly rounds (31 shuffles),
 // a fixed combination order.

@@ -64,8 +64,8 @@ class Case:
 # Small cases: several 256 x 256 output tiles with ragged tails in every GEMM dimension
 # (M, N, K not multiples of 256 / 64 / 32), both LWC launch shapes (group <= 256 power of
 # two, and larger or irregular groups), the weight-side STE both inside the dW^ GEMM's
-# epilogue (16-bit operands, groups 32 / 64 / 128) and as its own kernel, every weight /
-# activation bit width the configs use.
+# epilogue (16-bit operands, groups a multiple of 32, per-channel included) and as its own
+# kernels (fp32 operands, groups of 16), every weight / activation bit width the configs use.
 SMALL_CASES = [
     Case("f32_w4a16_perchannel", 64, 256, 256, 256, 4, 16, False, "f32", "tiny_w4a16", 0),
     Case("f32_w4a8_g32_let", 72, 320, 136, 32, 4, 8, True, "f32", "llama7b_gateup_w4a4", 1),
@@ -78,6 +78,10 @@ SMALL_CASES = [
     Case("bf16_w8a16_g256", 128, 768, 512, 256, 8, 16, False, "bf16", "llama7b_qproj_w4a16g128",
          6),
     Case("bf16_w4a8_g32_let", 96, 416, 264, 32, 4, 8, True, "bf16", "llama7b_gateup_w4a4", 7),
+    Case("bf16_w4a16_g16_let", 80, 272, 200, 16, 4, 16, True, "bf16", "llama7b_qproj_w4a16g128",
+         8),
+    Case("f32_w4a4_perchannel_let", 72, 320, 136, 320, 4, 4, True, "f32", "llama7b_gateup_w4a4",
+         9),
 ]
 
 
