@@ -300,6 +300,131 @@ omq_status omq_calib_step(const omq_step_args* args, void* workspace, size_t ws_
                           omq_stream_t stream);
 size_t omq_step_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t group);
 
+/* ====================================================================================
+ * One transformer block ([ICLR] section 框架: calibration runs block by block, the loss is
+ * the block output's error against the full-precision block; section LET: the transforms
+ * of every linear's input except the FFN's second linear, the attention-affinity scaling
+ * Q / s_a, s_a K, Q, K and V quantized, V transformed by the output projection's inverse
+ * LET, softmax kept in full precision). The block, LLaMA-shaped:
+ *
+ *   a  = RMSNorm(x)  (weight 1, eps 1e-6);       qa = Q_a((a - δ1) / s1)        per token
+ *   [q | k | v] = qa Ŵ_qkv^T + W_qkv δ1           (W~_qkv = W_qkv s1)
+ *   q~ = RoPE(q) / s_a;  k~ = RoPE(k) s_a;  v~ = (v - δ_o) / s_o
+ *   Qq, Qk, Qv = Q_a(q~), Q_a(k~), Q_a(v~)        per (token, head) row of 128
+ *   P_h = softmax(causal(Qq_h Qk_h^T / sqrt(128)))   binary32;   O = [P_h Qv_h]_h
+ *   x2 = x + Q_a(O) Ŵ_o^T + W_o δ_o               (W~_o = W_o s_o; Q_a per token)
+ *   b  = RMSNorm(x2);  qb = Q_a((b - δ2) / s2);   [gate | up] = qb Ŵ_gu^T + W_gu δ2
+ *   m  = SiLU(gate) up;  y = x2 + Q_a(m) Ŵ_d^T   (no LET on the down projection)
+ *   loss = mean over M*D of (y - y_ref)^2
+ * RoPE: rotate-half pairs (i, i + 64) of each head, angle = position * 10000^(-i/64),
+ * positions 0..M-1. Each Ŵ is the LWC fake-quant of its W~ (omq_lwc_quant's rule).
+ * The backward is the straight-through chain of every quantizer (omq_fq_linear_bwd's rule)
+ * through the whole block; it fills d_theta for every learnable tensor.
+ *
+ * Storage: x, the weights and every GEMM operand BF16; y_ref, theta, gradients float32.
+ * Weights: W_qkv [3D, D] (rows of q_proj, then k_proj, then v_proj), W_o [D, D],
+ * W_gu [2I, D] (rows of gate_proj, then up_proj), W_d [D, I].
+ * ==================================================================================== */
+typedef struct {
+  int64_t M;       /* tokens, a multiple of 8 */
+  int64_t D;       /* hidden size = 128 H */
+  int64_t H;       /* heads (head size 128) */
+  int64_t I;       /* FFN size, a multiple of 32 */
+  int64_t group;   /* LWC group length, a multiple of 32 dividing D and I; 0 = per channel */
+  int wbits;       /* 2, 3, 4 or 8 */
+  int abits;       /* 2, 3, 4, 6, 8, or 16 (activations not quantized) */
+} omq_block_dims;
+
+/* The parameter vector theta: float32, these tensors back to back in this order. LWC
+ * logits have one entry per (row, group) of their weight; LET vectors one per channel. */
+enum {
+  OMQ_TH_GAMMA_QKV = 0, OMQ_TH_BETA_QKV, OMQ_TH_GAMMA_O, OMQ_TH_BETA_O,
+  OMQ_TH_GAMMA_GU, OMQ_TH_BETA_GU, OMQ_TH_GAMMA_D, OMQ_TH_BETA_D,
+  OMQ_TH_S1, OMQ_TH_DELTA1, OMQ_TH_S_A, OMQ_TH_S_O, OMQ_TH_DELTA_O, OMQ_TH_S2, OMQ_TH_DELTA2,
+  OMQ_TH_COUNT
+};
+/* Offset and length (in floats) of tensor `id` of theta; total length for id = OMQ_TH_COUNT. */
+omq_status omq_block_theta_range(const omq_block_dims* dims, int id, int64_t* offset,
+                                 int64_t* count);
+
+/* Tensors the step keeps in its workspace (forward activations and the gradients that flow
+ * between stages), at fixed offsets: omq_block_buffer reports offset and size in bytes. */
+enum {
+  OMQ_BB_ROPE = 0,   /* float32 [2, M, 64]: cos, then sin, of the rotation angles */
+  OMQ_BB_A,          /* float32 [M, D]  RMSNorm(x) */
+  OMQ_BB_QA,         /* BF16 [M, D]     qa */
+  OMQ_BB_WHAT_QKV,   /* BF16 [3D, D]    Ŵ_qkv (then _O, _GU, _D) */
+  OMQ_BB_WHAT_O, OMQ_BB_WHAT_GU, OMQ_BB_WHAT_D,
+  OMQ_BB_QKV,        /* float32 [M, 3D] q | k | v */
+  OMQ_BB_QQKV,       /* BF16 [M, 3D]    Qq | Qk | Qv */
+  OMQ_BB_P,          /* float32 [H, M, M] softmax (zero above the diagonal) */
+  OMQ_BB_P16,        /* BF16 [H, M, M]  the same, GEMM operand */
+  OMQ_BB_O,          /* float32 [M, D]  attention output */
+  OMQ_BB_QO,         /* BF16 [M, D]     Q_a(O) */
+  OMQ_BB_X2,         /* float32 [M, D]  x2 */
+  OMQ_BB_B,          /* float32 [M, D]  RMSNorm(x2) */
+  OMQ_BB_QB,         /* BF16 [M, D]     qb */
+  OMQ_BB_GU,         /* float32 [M, 2I] gate | up */
+  OMQ_BB_MID,        /* float32 [M, I]  m = SiLU(gate) up */
+  OMQ_BB_QM,         /* BF16 [M, I]     Q_a(m) */
+  OMQ_BB_RES,        /* BF16 [M, D]     y - y_ref (the loss gradient is 2 res / (M D)) */
+  OMQ_BB_DMID,       /* float32 [M, I]  dL/dm */
+  OMQ_BB_DGU,        /* BF16 [M, 2I]    dL/d[gate | up] */
+  OMQ_BB_DB,         /* float32 [M, D]  dL/db */
+  OMQ_BB_DX2,        /* BF16 [M, D]     dL/dx2 */
+  OMQ_BB_DO,         /* BF16 [M, D]     dL/dO */
+  OMQ_BB_DQQKV,      /* float32 [M, 3D] dL/d[Qq | Qk | Qv] */
+  OMQ_BB_DQKV,       /* BF16 [M, 3D]    dL/d[q | k | v] */
+  OMQ_BB_COUNT
+};
+omq_status omq_block_buffer(const omq_block_dims* dims, int id, size_t* offset, size_t* bytes);
+size_t omq_block_workspace_bytes(const omq_block_dims* dims);
+
+/* Phases of omq_block_step for per-phase event timing (events: NULL or OMQ_BPH_COUNT + 1). */
+enum {
+  OMQ_BPH_WEIGHTS = 0,  /* LWC of the four weights, B~ */
+  OMQ_BPH_ATTN_IN,      /* RMSNorm, LET, act quant, qkv GEMM, RoPE / affinity / head quant */
+  OMQ_BPH_ATTN,         /* scores, softmax, P V */
+  OMQ_BPH_FFN,          /* o_proj, RMSNorm, gate/up, SwiGLU, down + loss */
+  OMQ_BPH_BWD_FFN,      /* down, SwiGLU, gate/up backward, RMSNorm backward */
+  OMQ_BPH_BWD_ATTN,     /* o_proj backward, attention backward, head / RoPE STE */
+  OMQ_BPH_BWD_QKV,      /* qkv backward */
+  OMQ_BPH_REDUCE,       /* LET gradient reductions, loss */
+  OMQ_BPH_ADAMW,
+  OMQ_BPH_COUNT
+};
+
+typedef struct {
+  omq_block_dims dims;
+  const void* x;          /* [M, D] BF16 */
+  const float* y_ref;     /* [M, D] the full-precision block output (omq_block_reference) */
+  const void* W_qkv;      /* BF16 weights, shapes above */
+  const void* W_o;
+  const void* W_gu;
+  const void* W_d;
+  float* theta;           /* [P] parameters (omq_block_theta_range) */
+  float* d_theta;         /* [P] gradient, written */
+  float* loss;            /* device scalar, written */
+  float* adam_m;          /* [P] AdamW moments, or both NULL: no update */
+  float* adam_v;
+  int64_t step;           /* AdamW step, from 1 */
+  float lr_lwc, lr_let;   /* AdamW rates of the LWC logits and of the LET vectors */
+  void* const* events;    /* NULL, or OMQ_BPH_COUNT + 1 cudaEvent_t */
+} omq_block_args;
+
+/* One calibration step of the block: forward, loss, straight-through backward, and (when
+ * adam_m / adam_v are given) AdamW (beta 0.9 / 0.999, eps 1e-8, no weight decay) on theta.
+ * Workspace: omq_block_workspace_bytes. The block's tensors stay in the workspace
+ * (omq_block_buffer) until the next call. */
+omq_status omq_block_step(const omq_block_args* args, void* workspace, size_t ws_bytes,
+                          omq_stream_t stream);
+
+/* The full-precision block (no quantizer, no transform): y [M, D] float32. Uses the same
+ * workspace layout (omq_block_workspace_bytes of the same dims). */
+omq_status omq_block_reference(const omq_block_dims* dims, const void* x, const void* W_qkv,
+                               const void* W_o, const void* W_gu, const void* W_d, float* y,
+                               void* workspace, size_t ws_bytes, omq_stream_t stream);
+
 /* Number of kernels this library has launched in this process (all threads, all devices),
  * counted on the host at each launch. */
 uint64_t omq_launch_count(void);

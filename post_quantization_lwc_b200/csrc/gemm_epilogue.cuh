@@ -1,6 +1,7 @@
 // Per-element GEMM epilogues shared by the tcgen05 and CUDA-core GEMMs.
 //
 // StoreF32: out[i, j] = out_scale * acc (+ bias[j]).
+// Row i of out, y_ref and dy starts at i * ldo (ldo = 0: i * cols).
 // MseLoss : the fake-quant forward's tail ("Y = Q_a(X~) Q_w(W~) + B~", then the squared
 //           reconstruction error against the full-precision output):
 //           Y = acc + bias[j]; optionally stored; R = Y - Y_ref written as the residual
@@ -14,7 +15,7 @@ namespace omq {
 
 __device__ __forceinline__ void epi_element(const GemmEpilogue& e, int64_t i, int64_t j,
                                             int64_t cols, float acc, float& lsum) {
-  const int64_t o = i * cols + j;
+  const int64_t o = i * (e.ldo ? e.ldo : cols) + j;
   if (e.kind == Epi::StoreF32) {
     e.out[o] = e.out_scale * acc + (e.bias ? e.bias[j] : 0.f);
     return;
@@ -26,10 +27,11 @@ __device__ __forceinline__ void epi_element(const GemmEpilogue& e, int64_t i, in
   store_elem(e.dy, o, d, e.dy_dt);
 }
 
-// 8 consecutive columns j0..j0+7 of row i, all in range, j0 % 8 == 0, cols % 8 == 0.
+// 8 consecutive columns j0..j0+7 of row i, all in range, j0 % 8 == 0, cols % 8 == 0 and the
+// row stride a multiple of 8.
 __device__ __forceinline__ void epi_vec8(const GemmEpilogue& e, int64_t i, int64_t j0,
                                          int64_t cols, const float (&acc)[8], float& lsum) {
-  const int64_t o = i * cols + j0;
+  const int64_t o = i * (e.ldo ? e.ldo : cols) + j0;
   const float sc = e.kind == Epi::StoreF32 ? e.out_scale : 1.f;
   float y[8];
   if (e.bias) {

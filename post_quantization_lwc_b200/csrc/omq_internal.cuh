@@ -193,6 +193,7 @@ struct GemmEpilogue {
   float out_scale;         // StoreF32: out = out_scale * acc (+ bias); SteW: dW^ = out_scale * acc
   float* loss_partials;    // MseLoss: one per output tile (fixed order)
   SteWEpi ste;             // SteW
+  int64_t ldo;             // row stride of out / y_ref / dy in elements (0: cols)
 };
 
 // Group lengths whose weight-side STE runs in the dW^ GEMM's epilogue: whole 32-column
@@ -278,9 +279,11 @@ struct SteXParams {
   const omq_range* range;
   const float* dXq;     // [M,K] fp32
   float* rowstat;       // [M, 2] scratch: gradient share of each token's max / min element
-  float* part_s;        // [row blocks, K]: -sum_m dX~ X~ / s
-  float* part_d;        // [row blocks, K]: -sum_m dX~ / s
+  float* part_s;        // [row blocks, K]: -sum_m dX~ X~ / s (NULL: skipped)
+  float* part_d;        // [row blocks, K]: -sum_m dX~ / s (NULL: skipped)
   int rows_per_block;
+  void* dX;             // [M, K] in dx_dt or NULL: the gradient of the LET's input, dX~ / s
+  omq_dtype dx_dt;
 };
 
 // One parameter tensor of a fused AdamW launch.

@@ -481,14 +481,18 @@ __global__ void __launch_bounds__(256, 2) ste_x_cols_kernel(SteXParams p) {
           dxt[i] = dq[u][i];
         }
       }
+      float dxs[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const float q = dxt[i] * rs[i];
+        dxs[i] = q;
         acc_s[i] += q * v[u][i];
         acc_d[i] += q;
       }
+      if (p.dX) store8(p.dX, m * p.K + c0, p.dx_dt, dxs);
     }
   }
+  if (!p.part_s && !p.part_d) return;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     red_s[w][lane * 8 + i] = acc_s[i];
@@ -503,8 +507,8 @@ __global__ void __launch_bounds__(256, 2) ste_x_cols_kernel(SteXParams p) {
       a += red_s[q][threadIdx.x];
       d += red_d[q][threadIdx.x];
     }
-    p.part_s[rb * p.K + col] = -a;
-    p.part_d[rb * p.K + col] = -d;
+    if (p.part_s) p.part_s[rb * p.K + col] = -a;
+    if (p.part_d) p.part_d[rb * p.K + col] = -d;
   }
 }
 

@@ -30,7 +30,8 @@ EXPORTS = ("omq_status_str", "omq_last_cuda_error", "omq_version", "omq_sync_che
            "omq_lwc_quant", "omq_let_apply", "omq_fq_linear_fwd", "omq_fwd_workspace_bytes",
            "omq_fq_linear_bwd", "omq_bwd_workspace_bytes", "omq_adamw_step", "omq_fold_pack",
            "omq_calib_step", "omq_step_workspace_bytes", "omq_launch_count",
-           "omq_fq_linear_fwd_noalloc")
+           "omq_fq_linear_fwd_noalloc", "omq_block_theta_range", "omq_block_buffer",
+           "omq_block_workspace_bytes", "omq_block_step", "omq_block_reference")
 
 _p = ctypes.c_void_p
 _i64 = ctypes.c_int64
@@ -73,6 +74,18 @@ class StepArgs(ctypes.Structure):
                 ("events", _p)]
 
 
+class BlockDims(ctypes.Structure):
+    _fields_ = [("M", _i64), ("D", _i64), ("H", _i64), ("I", _i64), ("group", _i64),
+                ("wbits", _i32), ("abits", _i32)]
+
+
+class BlockArgs(ctypes.Structure):
+    _fields_ = [("dims", BlockDims), ("x", _p), ("y_ref", _p), ("W_qkv", _p), ("W_o", _p),
+                ("W_gu", _p), ("W_d", _p), ("theta", _p), ("d_theta", _p), ("loss", _p),
+                ("adam_m", _p), ("adam_v", _p), ("step", _i64), ("lr_lwc", _f32),
+                ("lr_let", _f32), ("events", _p)]
+
+
 # phases of omq_calib_step (OMQ_PH_* in include/omq.h), in order
 PHASES = ("let", "lwc", "fwd_gemm", "loss", "dbias", "dw_gemm", "ste_w", "dx_gemm", "ste_x",
           "let_reduce", "adamw")
@@ -102,6 +115,14 @@ _sig("omq_calib_step", _i32, [ctypes.POINTER(StepArgs), _p, _sz, _p])
 _sig("omq_step_workspace_bytes", _sz, [_i64, _i64, _i64, _i64])
 _sig("omq_launch_count", ctypes.c_uint64, [])
 _sig("omq_fq_linear_fwd_noalloc", _i32, [_p, _p, _i32, _i64, _i64, _i64, _p, _p, _p, _p, _p, _p])
+_sig("omq_block_theta_range", _i32, [ctypes.POINTER(BlockDims), _i32, ctypes.POINTER(_i64),
+                                     ctypes.POINTER(_i64)])
+_sig("omq_block_buffer", _i32, [ctypes.POINTER(BlockDims), _i32, ctypes.POINTER(_sz),
+                                ctypes.POINTER(_sz)])
+_sig("omq_block_workspace_bytes", _sz, [ctypes.POINTER(BlockDims)])
+_sig("omq_block_step", _i32, [ctypes.POINTER(BlockArgs), _p, _sz, _p])
+_sig("omq_block_reference", _i32, [ctypes.POINTER(BlockDims), _p, _p, _p, _p, _p, _p, _p, _sz,
+                                   _p])
 
 
 def _check(status: int, where: str):
@@ -422,3 +443,108 @@ class PhaseTimer:
             for i in range(len(PHASES)):
                 tot[i] += evs[i].elapsed_time(evs[i + 1])
         return {p: t / len(self.sets) for p, t in zip(PHASES, tot)}
+
+
+# ---------------------------------------------------------------------------- transformer block
+
+# theta tensors (OMQ_TH_* in include/omq.h) and workspace tensors (OMQ_BB_*), in order
+THETA = ("gamma_qkv", "beta_qkv", "gamma_o", "beta_o", "gamma_gu", "beta_gu", "gamma_d",
+         "beta_d", "s1", "delta1", "s_a", "s_o", "delta_o", "s2", "delta2")
+BLOCK_BUFFERS = (
+    ("rope", torch.float32), ("a", torch.float32), ("qa", torch.bfloat16),
+    ("what_qkv", torch.bfloat16), ("what_o", torch.bfloat16), ("what_gu", torch.bfloat16),
+    ("what_d", torch.bfloat16), ("qkv", torch.float32), ("qqkv", torch.bfloat16),
+    ("p", torch.float32), ("p16", torch.bfloat16), ("o", torch.float32), ("qo", torch.bfloat16),
+    ("x2", torch.float32), ("b", torch.float32), ("qb", torch.bfloat16), ("gu", torch.float32),
+    ("mid", torch.float32), ("qm", torch.bfloat16), ("res", torch.bfloat16),
+    ("dmid", torch.float32), ("dgu", torch.bfloat16), ("db", torch.float32),
+    ("dx2", torch.bfloat16), ("do", torch.bfloat16), ("dqqkv", torch.float32),
+    ("dqkv", torch.bfloat16))
+BLOCK_PHASES = ("weights", "attn_in", "attn", "ffn", "bwd_ffn", "bwd_attn", "bwd_qkv", "reduce",
+                "adamw")
+
+
+class Block:
+    """Device buffers of one transformer block's calibration, driven by omq_block_step.
+
+    ``dims``: M tokens, D hidden (128 per head), H heads, I FFN size, LWC group (0 = per
+    channel), wbits, abits. Holds the BF16 weights (W_qkv [3D, D], W_o [D, D], W_gu [2I, D],
+    W_d [D, I]), the parameter vector theta with its gradient and AdamW moments, and the
+    workspace whose tensors ``buffer(name)`` views.
+    """
+
+    def __init__(self, M, D, H, I, group=0, wbits=4, abits=4, device="cuda", lr_lwc=5e-3,
+                 lr_let=1e-2):
+        self.dims = BlockDims(M=M, D=D, H=H, I=I, group=group, wbits=wbits, abits=abits)
+        self.device = torch.device(device)
+        self.lr_lwc, self.lr_let = lr_lwc, lr_let
+        nbytes = _lib.omq_block_workspace_bytes(ctypes.byref(self.dims))
+        if nbytes == 0:
+            raise ValueError("invalid block dimensions")
+        off, cnt = _i64(), _i64()
+        self.theta_slices = {}
+        for i, name in enumerate(THETA):
+            _check(_lib.omq_block_theta_range(ctypes.byref(self.dims), i, ctypes.byref(off),
+                                              ctypes.byref(cnt)), "omq_block_theta_range")
+            self.theta_slices[name] = (off.value, cnt.value)
+        _check(_lib.omq_block_theta_range(ctypes.byref(self.dims), len(THETA), ctypes.byref(off),
+                                          ctypes.byref(cnt)), "omq_block_theta_range")
+        self.P = cnt.value
+        f = lambda n: torch.zeros(n, dtype=torch.float32, device=self.device)  # noqa: E731
+        self.theta, self.d_theta = f(self.P), f(self.P)
+        self.adam_m, self.adam_v = f(self.P), f(self.P)
+        self.loss = f(1)
+        self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+        b = lambda *shape: torch.zeros(*shape, dtype=torch.bfloat16, device=self.device)  # noqa
+        self.W = {"qkv": b(3 * D, D), "o": b(D, D), "gu": b(2 * I, D), "d": b(D, I)}
+        self.t = 0
+
+    def theta_part(self, name, t=None):
+        o, n = self.theta_slices[name]
+        return (self.theta if t is None else t)[o:o + n]
+
+    def buffer(self, name):
+        """The workspace tensor `name` (BLOCK_BUFFERS) as a flat tensor view."""
+        idx = [n for n, _ in BLOCK_BUFFERS].index(name)
+        dtype = BLOCK_BUFFERS[idx][1]
+        off, nb = _sz(), _sz()
+        _check(_lib.omq_block_buffer(ctypes.byref(self.dims), idx, ctypes.byref(off),
+                                     ctypes.byref(nb)), "omq_block_buffer")
+        esz = torch.empty(0, dtype=dtype).element_size()
+        return self.workspace[off.value:off.value + nb.value].view(dtype)[: nb.value // esz]
+
+    def load(self, W, theta):
+        for k in self.W:
+            self.W[k].copy_(W[k])
+        self.theta.copy_(theta)
+        self.adam_m.zero_()
+        self.adam_v.zero_()
+        self.t = 0
+
+    def reference(self, x, stream=None):
+        """omq_block_reference: the full-precision block output y* [M, D] float32."""
+        _dev(x)
+        y = torch.empty(self.dims.M, self.dims.D, dtype=torch.float32, device=self.device)
+        _check(_lib.omq_block_reference(ctypes.byref(self.dims), _ptr(x), _ptr(self.W["qkv"]),
+                                        _ptr(self.W["o"]), _ptr(self.W["gu"]), _ptr(self.W["d"]),
+                                        _ptr(y), _ptr(self.workspace), self.workspace.numel(),
+                                        _stream(stream)), "omq_block_reference")
+        return y
+
+    def step(self, x, y_ref, update=True, stream=None, events=None):
+        """omq_block_step: forward, loss, backward (d_theta) and, with update, AdamW."""
+        _dev(x, y_ref)
+        if update:
+            self.t += 1
+        a = BlockArgs(dims=self.dims, x=_ptr(x), y_ref=_ptr(y_ref), W_qkv=_ptr(self.W["qkv"]),
+                      W_o=_ptr(self.W["o"]), W_gu=_ptr(self.W["gu"]), W_d=_ptr(self.W["d"]),
+                      theta=_ptr(self.theta), d_theta=_ptr(self.d_theta), loss=_ptr(self.loss),
+                      adam_m=_ptr(self.adam_m) if update else None,
+                      adam_v=_ptr(self.adam_v) if update else None, step=max(self.t, 1),
+                      lr_lwc=self.lr_lwc, lr_let=self.lr_let)
+        if events is not None:
+            arr = (ctypes.c_void_p * (len(BLOCK_PHASES) + 1))(*[e.cuda_event for e in events])
+            a.events = ctypes.cast(arr, ctypes.c_void_p)
+        _check(_lib.omq_block_step(ctypes.byref(a), _ptr(self.workspace), self.workspace.numel(),
+                                   _stream(stream)), "omq_block_step")
+        return self.loss

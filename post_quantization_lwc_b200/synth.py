@@ -186,3 +186,95 @@ def random_let(gen_seed: int, k_in: int):
 def as_f32_numpy(t: torch.Tensor):
     """Exact float32 numpy copy of a CPU tensor (bf16 widens exactly)."""
     return t.detach().to(torch.float32).cpu().numpy()
+
+
+# ------------------------------------------------------------------ one transformer block
+
+@dataclasses.dataclass(frozen=True)
+class BlockConfig:
+    """One block-calibration workload: a LLaMA-shaped block (M tokens, hidden D = 128 H,
+    H heads, FFN size I), LWC group (0 = per output channel), weight / activation bits."""
+    name: str
+    M: int
+    D: int
+    H: int
+    I: int
+    group: int
+    wbits: int
+    abits: int
+    seed: int
+    x_outlier_frac: float = 0.01
+    x_outlier_scale: float = 50.0
+    w_std: float = 0.02
+    logit_init: float = 4.0
+
+
+BLOCK_CONFIGS = {
+    # LLaMA-7B block: q/k/v/o 4096 x 4096, gate/up 4096 -> 11008, down 11008 -> 4096,
+    # 32 heads of 128, 2048 tokens, per-channel W4A4
+    "llama7b_block_w4a4": BlockConfig(name="llama7b_block_w4a4", M=2048, D=4096, H=32,
+                                      I=11008, group=0, wbits=4, abits=4, seed=4),
+}
+
+
+def scaled_block(cfg: BlockConfig, M: int, H: int, I: int, seed: int | None = None,
+                 name: str | None = None, **kw) -> BlockConfig:
+    """The same recipe at another size."""
+    return dataclasses.replace(cfg, M=M, D=128 * H, H=H, I=I,
+                               seed=cfg.seed if seed is None else seed,
+                               name=name or f"{cfg.name}@{M}x{128 * H}x{I}", **kw)
+
+
+@dataclasses.dataclass
+class BlockInputs:
+    cfg: BlockConfig
+    x: torch.Tensor            # [M, D] bf16
+    W: dict                    # qkv [3D, D], o [D, D], gu [2I, D], d [D, I], bf16
+
+
+def make_block_inputs(cfg: BlockConfig) -> BlockInputs:
+    """Weights ~ N(0, w_std) (rows of q, k, v, o, gate, up, down in that order), then the
+    block input x ~ N(0, 1) with a fixed 1% of channels (first of a seeded permutation)
+    scaled by x_outlier_scale."""
+    gen = torch.Generator().manual_seed(cfg.seed)
+    D, I, M = cfg.D, cfg.I, cfg.M
+
+    def w(n, k):
+        return (torch.randn(n, k, generator=gen, dtype=torch.float64) * cfg.w_std).to(
+            torch.bfloat16)
+    W = {"qkv": w(3 * D, D), "o": w(D, D), "gu": w(2 * I, D), "d": w(D, I)}
+    x = torch.randn(M, D, generator=gen, dtype=torch.float64)
+    n_out = max(1, int(math.floor(cfg.x_outlier_frac * D)))
+    chans = torch.randperm(D, generator=gen)[:n_out]
+    x[:, chans] *= cfg.x_outlier_scale
+    return BlockInputs(cfg=cfg, x=x.to(torch.bfloat16), W=W)
+
+
+def random_block_theta(gen_seed: int, names_counts, spread: float = 0.3,
+                       logit_range=(1.0, 5.0)):
+    """A non-trivial parameter vector for tests: logits uniform in logit_range, s in
+    1 +- spread/2, delta ~ N(0, spread / 3). names_counts: ordered (name, length) pairs."""
+    gen = torch.Generator().manual_seed(gen_seed)
+    parts = []
+    for name, n in names_counts:
+        if name.startswith(("gamma", "beta")):
+            lo, hi = logit_range
+            parts.append(lo + (hi - lo) * torch.rand(n, generator=gen))
+        elif name.startswith("delta"):
+            parts.append(spread / 3 * torch.randn(n, generator=gen))
+        else:
+            parts.append(1.0 + spread * (torch.rand(n, generator=gen) - 0.5))
+    return torch.cat(parts).to(torch.float32)
+
+
+def init_block_theta(cfg: BlockConfig, names_counts):
+    """The starting point of calibration: logits logit_init, s = 1, delta = 0, s_a = 1."""
+    parts = []
+    for name, n in names_counts:
+        if name.startswith(("gamma", "beta")):
+            parts.append(torch.full((n,), cfg.logit_init))
+        elif name.startswith("delta"):
+            parts.append(torch.zeros(n))
+        else:
+            parts.append(torch.ones(n))
+    return torch.cat(parts).to(torch.float32)
