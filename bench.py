@@ -383,9 +383,231 @@ def run_omq(args, cfg, rank: int, world: int, local_rank: int):
     return 0
 
 
+# ----------------------------------------------------------------------------- block workload
+
+def block_flops(bc) -> dict:
+    """Dense contractions of one block step: the seven linears (forward, dW^, dXq each; the
+    q/k/v and gate/up linears as one [3D, D] and one [2I, D] weight), and the six attention
+    products with only the causal lower triangle counted (half of each M x M product)."""
+    M, D, H, I = bc.M, bc.D, bc.H, bc.I
+    lin = 3 * 2 * M * (3 * D * D + D * D + 2 * I * D + D * I)
+    attn = 6 * 2 * M * M * 128 * H // 2
+    return {"linears": lin, "attention": attn, "total": lin + attn}
+
+
+def block_oracle_sample(bc, tokens: int):
+    """The oracle's block step on the first `tokens` tokens of the workload (full weights)."""
+    import numpy as np
+
+    from oracle import block as ob
+    from post_quantization_lwc_b200 import synth
+    inp = synth.make_block_inputs(bc)
+    sh = ob.BlockShape(M=tokens, D=bc.D, H=bc.H, I=bc.I, wbits=bc.wbits, abits=bc.abits,
+                       group=bc.group)
+    x = synth.as_f32_numpy(inp.x[:tokens])
+    W = {k: synth.as_f32_numpy(v) for k, v in inp.W.items()}
+    theta = synth.init_block_theta(bc, ob.theta_layout(sh)).numpy()
+    y_ref = ob.block_reference(sh, x, W)
+    return sh, x, W, theta, y_ref
+
+
+def block_cpu_time(bc, tokens: int, steps: int):
+    from oracle import block as ob
+    sh, x, W, theta, y_ref = block_oracle_sample(bc, tokens)
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        ob.block_step(sh, x, W, theta, y_ref)
+    return time.perf_counter() - t0
+
+
+def block_cpu_baseline(bc, tokens: int = 128, steps: int = 1):
+    """The oracle (as it stands) on a bounded sample: whole block steps on the first `tokens`
+    tokens with the full weights, throughput scaled to the workload by the step's flops."""
+    dt = block_cpu_time(bc, tokens, steps)
+    import dataclasses
+    small = dataclasses.replace(bc, M=tokens)
+    scale = block_flops(small)["total"] / block_flops(bc)["total"]
+    return {"value": steps * scale / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{steps} block step(s) of the numpy binary64 oracle on the first {tokens} "
+                      f"of {bc.M} tokens with the full {bc.name} weights ({dt:.1f} s), "
+                      f"throughput scaled by the flop ratio {scale:.4f}"}
+
+
+def run_block_reference(args, bc, rank: int, world: int):
+    if rank != 0:
+        return 0
+    tokens = 128
+    t1 = block_cpu_time(bc, tokens, 1)
+    if args.warmup > 1:
+        block_cpu_time(bc, tokens, min(args.warmup - 1, 2))
+    steps = max(1, min(args.steps, int(120.0 / max(t1, 1e-3))))
+    dt = block_cpu_time(bc, tokens, steps)
+    import dataclasses
+    scale = block_flops(dataclasses.replace(bc, M=tokens))["total"] / block_flops(bc)["total"]
+    value = steps * scale / dt
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / value,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {**block_config(bc), "parallelism": "host cores"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(),
+                             "kind": "oracle",
+                             "sample": f"{steps} oracle block step(s) on the first {tokens} "
+                                       f"tokens, scaled by the flop ratio {scale:.4f}"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def block_config(bc):
+    return {"workload": bc.name, "M_tokens": bc.M, "hidden": bc.D, "heads": bc.H,
+            "ffn": bc.I, "group": bc.group or "per-channel", "bits": bc.wbits,
+            "abits": bc.abits, "let": "all linears but down; Q/K affinity", "storage": "bf16"}
+
+
+def run_block(args, bc, rank: int, world: int, local_rank: int):
+    import dataclasses
+
+    import torch
+    import torch.distributed as dist
+
+    from post_quantization_lwc_b200 import omq, synth
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    my = dataclasses.replace(bc, seed=bc.seed + 1000 * rank) if rank else bc
+    inp = synth.make_block_inputs(my)
+    blk = omq.Block(bc.M, bc.D, bc.H, bc.I, group=bc.group, wbits=bc.wbits, abits=bc.abits,
+                    device=dev)
+    names = [(n, blk.theta_slices[n][1]) for n in omq.THETA]
+    blk.load({k: v.to(dev) for k, v in inp.W.items()}, synth.init_block_theta(bc, names).to(dev))
+    x = inp.x.to(dev).contiguous()
+    y_ref = blk.reference(x).contiguous()
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        blk.step(x, y_ref)
+    torch.cuda.synchronize()
+    omq.sync_check()
+    nph = len(omq.BLOCK_PHASES)
+    sets = [[torch.cuda.Event(enable_timing=True) for _ in range(nph + 1)]
+            for _ in range(args.steps)]
+    for es in sets:
+        for e in es:
+            e.record()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev.index)
+    barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    n0 = omq.launch_count()
+    ev0.record()
+    for i in range(args.steps):
+        blk.step(x, y_ref, events=sets[i])
+    ev1.record()
+    torch.cuda.synchronize()
+    n1 = omq.launch_count()
+    sampler.stop()
+    barrier()
+    omq.sync_check()
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    phases = {p: sum(es[j].elapsed_time(es[j + 1]) for es in sets) / args.steps
+              for j, p in enumerate(omq.BLOCK_PHASES)}
+
+    e2e = None
+    if not args.no_e2e:
+        xh = inp.x.pin_memory()
+        yh = y_ref.cpu().pin_memory()
+        lh = torch.empty(1, dtype=torch.float32).pin_memory()
+        xd, yd = torch.empty_like(x), torch.empty_like(y_ref)
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            xd.copy_(xh, non_blocking=True)
+            yd.copy_(yh, non_blocking=True)
+            blk.step(xd, yd)
+            lh.copy_(blk.loss, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        barrier()
+        ems = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([ems], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        e2e = {"value": world * args.steps / (ems / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": xh.numel() * xh.element_size() + yh.numel() * yh.element_size(),
+               "d2h_bytes_per_step": 4}
+    if rank != 0:
+        return 0
+    peaks, peak_src = load_peaks()
+    value = world * args.steps / (ms / 1e3)
+    fl = block_flops(bc)
+    step_s = ms / 1e3 / args.steps
+    peak_key = "bf16_tflops" if ms / 1e3 < 1.0 else "bf16_tflops_sustained"
+    peak = float(peaks.get(peak_key, FALLBACK_PEAKS[peak_key]))
+    achieved = fl["total"] / step_s / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded LLaMA-7B-shaped block weights, outlier-channel inputs)",
+        "config": {**block_config(bc),
+                   "l2": "no flush: the step's working set (weights, scores, probabilities) "
+                         "exceeds the 126 MB L2",
+                   "parallelism": f"replicas x{world} (one independent block per GPU)"},
+        "tflops": fl["total"] * value / 1e12,
+        "roofline": {"bound": "tensor", "kernel": "whole step (tcgen05 GEMMs dominate)",
+                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "peak_source": f"{peak_key} of {peak_src}",
+                     "per_launch": f"{fl['total'] / 1e9:.0f} GFLOP per step (linears "
+                                   f"{fl['linears'] / 1e9:.0f}, causal attention "
+                                   f"{fl['attention'] / 1e9:.0f}) over the step time"},
+        "phases_ms": {k: round(v, 4) for k, v in phases.items()},
+        "loss": float(blk.loss.item()),
+        "gpu_launches": int(n1 - n0),
+        "clocks": sampler.summary(),
+    }
+    if e2e is not None:
+        line["e2e"] = e2e
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = block_cpu_baseline(bc)
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     from post_quantization_lwc_b200 import synth
+    if args.config in synth.BLOCK_CONFIGS:
+        bc = synth.BLOCK_CONFIGS[args.config]
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+        if args.impl == "reference":
+            return run_block_reference(args, bc, rank, world)
+        if world > 1:
+            import torch
+            import torch.distributed as dist
+            torch.cuda.set_device(local_rank)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", local_rank))
+        try:
+            return run_block(args, bc, rank, world, local_rank)
+        finally:
+            if world > 1:
+                import torch.distributed as dist
+                dist.destroy_process_group()
     cfg = synth.CONFIGS[args.config]
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

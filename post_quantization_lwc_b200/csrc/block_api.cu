@@ -5,8 +5,9 @@
 //
 // The four linears are fake-quant linears of the single-layer step (LWC with the LET
 // weight scale folded into the load, per-token activation quantizer, tcgen05 GEMMs, the
-// weight-side STE fused into the dW GEMM). Attention runs one head at a time on the same
-// GEMM with the scores and probabilities materialised in float32.
+// weight-side STE fused into the dW GEMM). Attention runs on the same GEMM, all heads of a
+// product in one launch, the causal structure skipping the tiles and contraction blocks the
+// mask zeroes; scores and probabilities are materialised in float32.
 #include <cmath>
 #include <vector>
 
@@ -210,6 +211,20 @@ omq_status gemm_store(const GemmOperand& A, const GemmOperand& B, int64_t rows, 
   return gemm_tc(OMQ_BF16, A, B, rows, cols, depth, e, nullptr, st);
 }
 
+// The attention products, all heads in one launch each (heads are the batch).
+omq_status gemm_heads(const GemmOperand& A, int64_t a_stride, const GemmOperand& B,
+                      int64_t b_stride, int64_t rows, int64_t cols, int64_t depth, float* out,
+                      int64_t ldo, int64_t out_stride, float scale, int64_t heads, int causal,
+                      cudaStream_t st) {
+  GemmEpilogue e{};
+  e.kind = Epi::StoreF32;
+  e.out = out;
+  e.ldo = ldo;
+  e.out_scale = scale;
+  const GemmBatch b{heads, a_stride, b_stride, out_stride, causal};
+  return gemm_tc(OMQ_BF16, A, B, rows, cols, depth, e, nullptr, st, &b);
+}
+
 omq_status act_quant(const void* X, omq_dtype xdt, int64_t M, int64_t K, const float* s,
                      const float* d, int abits, void* Xq, float* h_a, int32_t* z_a,
                      omq_range* range, cudaStream_t st) {
@@ -313,15 +328,11 @@ omq_status block_forward(const View& v, const Inputs& in, const Marks& mk, cudaS
     float* P = v.bb<float>(OMQ_BB_P);
     __nv_bfloat16* P16 = v.bb<__nv_bfloat16>(OMQ_BB_P16);
     const float scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(kHead)));
-    for (int64_t h = 0; h < H; ++h)
-      BLK_TRY(gemm_store(GemmOperand{qqkv + h * kHead, 3 * D, false},
-                         GemmOperand{qqkv + D + h * kHead, 3 * D, false}, M, M, kHead,
-                         P + h * M * M, 0, scale, nullptr, st));
+    BLK_TRY(gemm_heads(GemmOperand{qqkv, 3 * D, false}, kHead, GemmOperand{qqkv + D, 3 * D, false},
+                       kHead, M, M, kHead, P, 0, M * M, scale, H, 1, st));
     BLK_TRY(launch_softmax(P, P16, H * M, M, st));
-    for (int64_t h = 0; h < H; ++h)
-      BLK_TRY(gemm_store(GemmOperand{P16 + h * M * M, M, false},
-                         GemmOperand{qqkv + 2 * D + h * kHead, 3 * D, true}, M, kHead, M,
-                         v.bb<float>(OMQ_BB_O) + h * kHead, D, 1.f, nullptr, st));
+    BLK_TRY(gemm_heads(GemmOperand{P16, M, false}, M * M, GemmOperand{qqkv + 2 * D, 3 * D, true},
+                       kHead, M, kHead, M, v.bb<float>(OMQ_BB_O), D, kHead, 1.f, H, 2, st));
   }
   // o_proj, residual, RMSNorm, gate / up, SwiGLU, down (+ loss)
   BLK_TRY(mk.mark(OMQ_BPH_FFN));
@@ -516,24 +527,18 @@ omq_status block_backward(const View& v, const Inputs& in, float* d_theta, const
     float* dP = v.in<float>(L.dP);
     __nv_bfloat16* dS = v.in<__nv_bfloat16>(L.dS);
     float* dq = v.bb<float>(OMQ_BB_DQQKV);
-    for (int64_t h = 0; h < H; ++h) {
-      // dQv_h = P_h^T dO_h;  dP_h = dO_h Qv_h^T
-      BLK_TRY(gemm_store(GemmOperand{P16 + h * M * M, M, true}, GemmOperand{dO + h * kHead, D, true},
-                         M, kHead, M, dq + 2 * D + h * kHead, 3 * D, 1.f, nullptr, st));
-      BLK_TRY(gemm_store(GemmOperand{dO + h * kHead, D, false},
-                         GemmOperand{qqkv + 2 * D + h * kHead, 3 * D, false}, M, M, kHead,
-                         dP + h * M * M, 0, 1.f, nullptr, st));
-    }
+    // dQv_h = P_h^T dO_h;  dP_h = dO_h Qv_h^T
+    BLK_TRY(gemm_heads(GemmOperand{P16, M, true}, M * M, GemmOperand{dO, D, true}, kHead, M, kHead,
+                       M, dq + 2 * D, 3 * D, kHead, 1.f, H, 3, st));
+    BLK_TRY(gemm_heads(GemmOperand{dO, D, false}, kHead, GemmOperand{qqkv + 2 * D, 3 * D, false},
+                       kHead, M, M, kHead, dP, 0, M * M, 1.f, H, 1, st));
     const float scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(kHead)));
     BLK_TRY(launch_softmax_bwd(v.bb<float>(OMQ_BB_P), dP, dS, H * M, M, scale, st));
-    for (int64_t h = 0; h < H; ++h) {
-      // dQq_h = dS_h Qk_h;  dQk_h = dS_h^T Qq_h
-      BLK_TRY(gemm_store(GemmOperand{dS + h * M * M, M, false},
-                         GemmOperand{qqkv + D + h * kHead, 3 * D, true}, M, kHead, M,
-                         dq + h * kHead, 3 * D, 1.f, nullptr, st));
-      BLK_TRY(gemm_store(GemmOperand{dS + h * M * M, M, true}, GemmOperand{qqkv + h * kHead, 3 * D, true},
-                         M, kHead, M, dq + D + h * kHead, 3 * D, 1.f, nullptr, st));
-    }
+    // dQq_h = dS_h Qk_h;  dQk_h = dS_h^T Qq_h
+    BLK_TRY(gemm_heads(GemmOperand{dS, M, false}, M * M, GemmOperand{qqkv + D, 3 * D, true}, kHead,
+                       M, kHead, M, dq, 3 * D, kHead, 1.f, H, 2, st));
+    BLK_TRY(gemm_heads(GemmOperand{dS, M, true}, M * M, GemmOperand{qqkv, 3 * D, true}, kHead, M,
+                       kHead, M, dq + D, 3 * D, kHead, 1.f, H, 3, st));
     AttnPrepParams p{};
     p.qkv = v.bb<float>(OMQ_BB_QKV);
     p.cos_t = v.bb<float>(OMQ_BB_ROPE);

@@ -6,6 +6,7 @@
 namespace omq {
 
 constexpr int kAttnRows = 64;   // tokens per block of attn_prep_bwd_kernel (column partials)
+constexpr int64_t kCausalTile = 256;   // output tile of the tcgen05 GEMM (rows = columns)
 
 struct RmsParams {
   const void* x;        // [M, D] in xdt

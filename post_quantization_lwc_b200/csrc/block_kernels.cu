@@ -356,9 +356,17 @@ __global__ void __launch_bounds__(256) attn_prep_bwd_kernel(AttnPrepParams p) {
 }
 
 // ------------------------------------------------------------------ causal softmax
-// Rows r of [H, M, M] (query i = r mod M): P[r, j] = exp(S - max) / sum over j <= i, zero for
-// j > i, in place (float32) and as BF16 (the P V operand). One warp per row, 4 columns a lane
-// per step; the row is read twice (the second read is served by L2).
+// Rows r of [H, M, M] (query i = r mod M): P[r, j] = exp(S - max) / sum over j <= i, in place
+// (float32, written for the 4-column chunks holding j <= i) and as BF16 (the operand of the
+// causal P V and P^T dO products, written up to the end of the row's 256-column GEMM tile,
+// zero past the diagonal: the products read no further). S is read only at j <= i: the score
+// GEMM skips tiles above the diagonal. One warp per row, 4 columns a lane per step; the row
+// is read twice (the second read is served by L2).
+__device__ __forceinline__ int64_t causal_span(int64_t i, int64_t M) {
+  const int64_t e = (i / kCausalTile + 1) * kCausalTile;
+  return e < M ? e : M;
+}
+
 __global__ void __launch_bounds__(256) softmax_kernel(float* S, __nv_bfloat16* P16, int64_t rows,
                                                       int64_t M) {
   const int lane = threadIdx.x & 31;
@@ -368,7 +376,6 @@ __global__ void __launch_bounds__(256) softmax_kernel(float* S, __nv_bfloat16* P
   float* row = S + r * M;
   __nv_bfloat16* row16 = P16 + r * M;
   const int64_t nvalid = i + 1;
-  const int64_t nq = M / 4;
   float mx = -FLT_MAX;
   for (int64_t q = lane; q * 4 < nvalid; q += 32) {
     const float4 v = *reinterpret_cast<const float4*>(row + q * 4);
@@ -390,6 +397,7 @@ __global__ void __launch_bounds__(256) softmax_kernel(float* S, __nv_bfloat16* P
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
   const float inv = 1.f / sum;
+  const int64_t nq = causal_span(i, M) / 4;
   for (int64_t q = lane; q < nq; q += 32) {
     float e[4] = {0.f, 0.f, 0.f, 0.f};
     if (q * 4 < nvalid) {
@@ -397,8 +405,8 @@ __global__ void __launch_bounds__(256) softmax_kernel(float* S, __nv_bfloat16* P
       const float x[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int t = 0; t < 4; ++t) e[t] = q * 4 + t < nvalid ? expf(x[t] - mx) * inv : 0.f;
+      *reinterpret_cast<float4*>(row + q * 4) = make_float4(e[0], e[1], e[2], e[3]);
     }
-    *reinterpret_cast<float4*>(row + q * 4) = make_float4(e[0], e[1], e[2], e[3]);
     __nv_bfloat162 a = __floats2bfloat162_rn(e[0], e[1]), b = __floats2bfloat162_rn(e[2], e[3]);
     uint2 pk;
     pk.x = *reinterpret_cast<uint32_t*>(&a);
@@ -407,7 +415,9 @@ __global__ void __launch_bounds__(256) softmax_kernel(float* S, __nv_bfloat16* P
   }
 }
 
-// dS[r, j] = scale P (dP - sum_j' P dP) for j <= i, zero above the diagonal (BF16).
+// dS[r, j] = scale P (dP - sum_j' P dP) for j <= i, zero above the diagonal up to the end of
+// the row's 256-column tile (BF16; the causal dS Qk and dS^T Qq products read no further).
+// P and dP are read only at j <= i.
 __global__ void __launch_bounds__(256) softmax_bwd_kernel(const float* P, const float* dP,
                                                           __nv_bfloat16* dS, int64_t rows,
                                                           int64_t M, float scale) {
@@ -419,7 +429,7 @@ __global__ void __launch_bounds__(256) softmax_bwd_kernel(const float* P, const 
   const float* drow = dP + r * M;
   __nv_bfloat16* orow = dS + r * M;
   const int64_t nvalid = i + 1;
-  const int64_t nq = M / 4;
+  const int64_t nq = causal_span(i, M) / 4;
   float dot = 0.f;
   for (int64_t q = lane; q * 4 < nvalid; q += 32) {
     const float4 a = *reinterpret_cast<const float4*>(prow + q * 4);

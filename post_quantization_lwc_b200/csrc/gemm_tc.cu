@@ -173,6 +173,56 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap
       "l"(reinterpret_cast<uint64_t>(map)), "r"(leader_bar), "r"(x), "r"(y)
       : "memory");
 }
+__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* map,
+                                                 uint32_t leader_bar, int x, int y, int w) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(leader_bar), "r"(x), "r"(y), "r"(w)
+      : "memory");
+}
+// One operand box: 2D (bmode 0) or 3D with the batch as the middle (1) or outer (2)
+// coordinate; (x, y) are the 2D coordinates (inner, outer) of the unbatched operand.
+__device__ __forceinline__ void tma_load_op(uint32_t dst, const CUtensorMap* map,
+                                            uint32_t leader_bar, int x, int y, int bmode,
+                                            int b) {
+  if (bmode == 0) tma_load_2d_pair(dst, map, leader_bar, x, y);
+  else if (bmode == 1) tma_load_3d_pair(dst, map, leader_bar, x, b, y);
+  else tma_load_3d_pair(dst, map, leader_bar, x, y, b);
+}
+
+// The pair's tile t: batch, origin, and the k-blocks it contracts. Causal modes (square
+// batches of attention, rows and columns both token positions):
+//   1 skip tiles wholly above the diagonal (columns > rows): the lower-triangle tiles are
+//     enumerated row by row, tn <= tm
+//   2 the contraction index is a column position: k < row0 + TILE_M
+//   3 the contraction index is a row position: k >= row0
+struct TileWork {
+  int b, row0, col0, kb0, kb1;
+};
+__device__ __forceinline__ TileWork tile_of(const TileSched& sc, int t, int nk) {
+  TileWork w;
+  w.b = t / sc.per_batch;
+  const int u = t - w.b * sc.per_batch;
+  int tm, tn;
+  if (sc.causal == 1) {
+    tm = static_cast<int>((sqrtf(8.f * static_cast<float>(u) + 1.f) - 1.f) * 0.5f);
+    while ((tm + 1) * (tm + 2) / 2 <= u) ++tm;
+    while (tm * (tm + 1) / 2 > u) --tm;
+    tn = u - tm * (tm + 1) / 2;
+  } else {
+    tm = u / sc.tiles_n;
+    tn = u - tm * sc.tiles_n;
+  }
+  w.row0 = tm * TILE_M;
+  w.col0 = tn * TILE_N;
+  w.kb0 = 0;
+  w.kb1 = nk;
+  if (sc.causal == 2) w.kb1 = min(nk, (w.row0 + TILE_M + BK - 1) / BK);
+  if (sc.causal == 3) w.kb0 = w.row0 / BK;
+  return w;
+}
+
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -374,7 +424,7 @@ template <int EV>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV>::NUM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    int a_mn, int b_mn, uint32_t fmt, int64_t rows, int64_t cols, int64_t depth,
-                   GemmEpilogue epi, int tiles_n, int num_tiles) {
+                   GemmEpilogue epi, TileSched sc) {
   using C = Cfg<EV>;
   constexpr int STAGES = C::STAGES, EPI_WARPS = C::EPI_WARPS, EPI_COLS = C::EPI_COLS;
   using L = Layout<STAGES, EPI_WARPS>;
@@ -399,6 +449,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV>::NUM_THREADS
   const int pair = static_cast<int>(cluster_id());
   const int pairs = static_cast<int>(cluster_count());
   const int nk = static_cast<int>((depth + BK - 1) / BK);
+  const int num_tiles = sc.num_tiles;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -430,9 +481,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV>::NUM_THREADS
     int it = 0;
     bool ok = true;
     for (int t = pair; t < num_tiles && ok; t += pairs) {
-      const int row0 = (t / tiles_n) * TILE_M + static_cast<int>(rank) * HALF;
-      const int col0 = (t % tiles_n) * TILE_N + static_cast<int>(rank) * HALF;
-      for (int kb = 0; kb < nk; ++kb, ++it) {
+      const TileWork tw = tile_of(sc, t, nk);
+      const int row0 = tw.row0 + static_cast<int>(rank) * HALF;
+      const int col0 = tw.col0 + static_cast<int>(rank) * HALF;
+      for (int kb = tw.kb0; kb < tw.kb1; ++kb, ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
         const bool got = C::SLEEPY ? mbar_wait_sleep(bar_empty + 8 * s, ph ^ 1, DEV_ERR_TMA_WAIT, 64)
@@ -448,15 +500,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV>::NUM_THREADS
         const int k0 = kb * BK;
         if (a_mn) {
           for (int c = 0; c < HALF / 64; ++c)
-            tma_load_2d_pair(a_dst + c * 8192, &tmA, full_leader, row0 + 64 * c, k0);
+            tma_load_op(a_dst + c * 8192, &tmA, full_leader, row0 + 64 * c, k0, sc.a_bmode, tw.b);
         } else {
-          tma_load_2d_pair(a_dst, &tmA, full_leader, k0, row0);
+          tma_load_op(a_dst, &tmA, full_leader, k0, row0, sc.a_bmode, tw.b);
         }
         if (b_mn) {
           for (int c = 0; c < HALF / 64; ++c)
-            tma_load_2d_pair(b_dst + c * 8192, &tmB, full_leader, col0 + 64 * c, k0);
+            tma_load_op(b_dst + c * 8192, &tmB, full_leader, col0 + 64 * c, k0, sc.b_bmode, tw.b);
         } else {
-          tma_load_2d_pair(b_dst, &tmB, full_leader, k0, col0);
+          tma_load_op(b_dst, &tmB, full_leader, k0, col0, sc.b_bmode, tw.b);
         }
       }
     }
@@ -483,7 +535,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV>::NUM_THREADS
       }
       tc_fence_after();
       const uint32_t d = tmem + static_cast<uint32_t>(buf * TILE_N);
-      for (int kb = 0; kb < nk; ++kb, ++it) {
+      const TileWork tw = tile_of(sc, t, nk);
+      for (int kb = tw.kb0; kb < tw.kb1; ++kb, ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
         // the stage was written by the copy engine (async proxy) and published through the
@@ -497,7 +550,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV>::NUM_THREADS
 #pragma unroll
         for (int kk = 0; kk < BK / UMMA_K; ++kk) {
           umma_pair(d, operand_desc(a_base, a_mn != 0, kk), operand_desc(b_base, b_mn != 0, kk),
-                    idesc, (kb | kk) != 0 ? 1u : 0u);
+                    idesc, (kb != tw.kb0 || kk != 0) ? 1u : 0u);
         }
         umma_commit_pair(bar_empty + 8 * s);
       }
@@ -517,8 +570,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV>::NUM_THREADS
     int lt = 0;
     for (int t = pair; t < num_tiles; t += pairs, ++lt) {
       const int buf = lt & 1;
-      const int64_t wrow0 = static_cast<int64_t>(t / tiles_n) * TILE_M + rank * HALF + quad * 32;
-      const int64_t col0 = static_cast<int64_t>(t % tiles_n) * TILE_N + cq * EPI_COLS;
+      const TileWork tw = tile_of(sc, t, nk);
+      const int64_t wrow0 = static_cast<int64_t>(tw.row0) + rank * HALF + quad * 32;
+      const int64_t col0 = static_cast<int64_t>(tw.col0) + cq * EPI_COLS;
       const int64_t row = wrow0 + lane;
       // one lane polls; the decision is broadcast so the warp-wide tcgen05.ld stays uniform
       int go = 0;
@@ -535,6 +589,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV>::NUM_THREADS
       if constexpr (EV != 0) {
         ste_w_epilogue<EV == 2>(epi, tbase, wrow0, col0, rows, cols, lane);
       } else {
+        GemmEpilogue eb = epi;                     // this tile's batch of the output
+        if (tw.b) eb.out += static_cast<int64_t>(tw.b) * sc.out_bstride;
         for (int ch = 0; ch < EPI_COLS / 32; ++ch) {
           uint32_t r[32];
           tmem_ld32(tbase + ch * 32, r);
@@ -547,13 +603,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV>::NUM_THREADS
                 float acc[8];
 #pragma unroll
                 for (int q = 0; q < 8; ++q) acc[q] = __uint_as_float(r[v * 8 + q]);
-                epi_vec8(epi, row, cbase + v * 8, cols, acc, lsum);
+                epi_vec8(eb, row, cbase + v * 8, cols, acc, lsum);
               }
             } else {
 #pragma unroll
               for (int q = 0; q < 32; ++q)
                 if (cbase + q < cols)
-                  epi_element(epi, row, cbase + q, cols, __uint_as_float(r[q]), lsum);
+                  epi_element(eb, row, cbase + q, cols, __uint_as_float(r[q]), lsum);
             }
           }
         }
@@ -611,31 +667,57 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // Tensor map of one operand, boxes of one CTA's half tile. K-major: stored [n_rows, depth]
 // -> dims {depth, n_rows}, box {64, 128}. MN-major: stored [depth, n_rows] ->
-// dims {n_rows, depth}, box {64, 64}.
+// dims {n_rows, depth}, box {64, 64}. A batch of `count` operands `bstride` elements apart
+// adds a third dimension of extent `count`, placed by stride: in the middle when the batch
+// stride is below the row stride (heads side by side in a row), else outermost; the box is
+// one problem deep. *bmode reports the placement (0: 2D).
 bool make_map(CUtensorMap* map, omq_dtype dt, const GemmOperand& op, int64_t n_rows,
-              int64_t depth) {
+              int64_t depth, int64_t count, int64_t bstride, int* bmode) {
   auto fn = encode_fn();
   if (!fn) return false;
-  cuuint64_t dims[2];
-  cuuint32_t box[2];
+  cuuint64_t d2[2];
+  cuuint32_t b2[2];
   if (op.mn_major) {
-    dims[0] = static_cast<cuuint64_t>(n_rows);
-    dims[1] = static_cast<cuuint64_t>(depth);
-    box[0] = 64;
-    box[1] = BK;
+    d2[0] = static_cast<cuuint64_t>(n_rows);
+    d2[1] = static_cast<cuuint64_t>(depth);
+    b2[0] = 64;
+    b2[1] = BK;
   } else {
-    dims[0] = static_cast<cuuint64_t>(depth);
-    dims[1] = static_cast<cuuint64_t>(n_rows);
-    box[0] = BK;
-    box[1] = HALF;
+    d2[0] = static_cast<cuuint64_t>(depth);
+    d2[1] = static_cast<cuuint64_t>(n_rows);
+    b2[0] = BK;
+    b2[1] = HALF;
   }
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(op.ld) * 2};
-  cuuint32_t estr[2] = {1, 1};
+  const cuuint64_t row_bytes = static_cast<cuuint64_t>(op.ld) * 2;
   const CUtensorMapDataType ty =
       dt == OMQ_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  CUresult r = fn(map, ty, 2, const_cast<void*>(op.ptr), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r;
+  if (count <= 1) {
+    *bmode = 0;
+    cuuint64_t strides[1] = {row_bytes};
+    r = fn(map, ty, 2, const_cast<void*>(op.ptr), d2, strides, b2, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  } else {
+    const cuuint64_t batch_bytes = static_cast<cuuint64_t>(bstride) * 2;
+    cuuint64_t d3[3], st3[2];
+    cuuint32_t b3[3];
+    if (batch_bytes < row_bytes) {
+      *bmode = 1;
+      d3[0] = d2[0]; d3[1] = static_cast<cuuint64_t>(count); d3[2] = d2[1];
+      st3[0] = batch_bytes; st3[1] = row_bytes;
+      b3[0] = b2[0]; b3[1] = 1; b3[2] = b2[1];
+    } else {
+      *bmode = 2;
+      d3[0] = d2[0]; d3[1] = d2[1]; d3[2] = static_cast<cuuint64_t>(count);
+      st3[0] = row_bytes; st3[1] = batch_bytes;
+      b3[0] = b2[0]; b3[1] = b2[1]; b3[2] = 1;
+    }
+    r = fn(map, ty, 3, const_cast<void*>(op.ptr), d3, st3, b3, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  }
   return r == CUDA_SUCCESS;
 }
 
@@ -643,7 +725,7 @@ static_assert(Layout<Cfg<0>::STAGES, Cfg<0>::EPI_WARPS>::SMEM_BYTES <= 232448, "
 static_assert(Layout<Cfg<1>::STAGES, Cfg<1>::EPI_WARPS>::SMEM_BYTES <= 232448, "smem");
 
 using GemmKernel = void (*)(CUtensorMap, CUtensorMap, int, int, uint32_t, int64_t, int64_t,
-                            int64_t, GemmEpilogue, int, int);
+                            int64_t, GemmEpilogue, TileSched);
 
 struct KernelChoice {
   GemmKernel fn;
@@ -679,16 +761,25 @@ int64_t gemm_tc_tiles(int64_t rows, int64_t cols) {
 
 omq_status gemm_tc(omq_dtype dt, const GemmOperand& A, const GemmOperand& B, int64_t rows,
                    int64_t cols, int64_t depth, const GemmEpilogue& epi, int64_t* n_tiles,
-                   cudaStream_t stream) {
+                   cudaStream_t stream, const GemmBatch* batch) {
   using namespace tc;
   if (dt != OMQ_BF16 && dt != OMQ_F16) return OMQ_ERR_DTYPE;
+  const int64_t count = batch ? batch->count : 1;
+  const int causal = batch ? batch->causal : 0;
+  if (count < 1 || causal < 0 || causal > 3) return OMQ_ERR_SHAPE;
+  if ((count > 1 || causal) && epi.kind != Epi::StoreF32) return OMQ_ERR_UNSUPPORTED;
+  if (causal && rows != (causal == 1 ? cols : depth)) return OMQ_ERR_SHAPE;
   CUtensorMap ma, mb;
-  if (!make_map(&ma, dt, A, rows, depth) || !make_map(&mb, dt, B, cols, depth)) {
+  int amode = 0, bmode = 0;
+  if (!make_map(&ma, dt, A, rows, depth, count, batch ? batch->a_stride : 0, &amode) ||
+      !make_map(&mb, dt, B, cols, depth, count, batch ? batch->b_stride : 0, &bmode)) {
     set_cuda_error(cudaErrorInvalidValue);
     return OMQ_ERR_CUDA;
   }
   const int64_t tiles_m = ceil_div(rows, TILE_M), tiles_n = ceil_div(cols, TILE_N);
-  const int64_t tiles = tiles_m * tiles_n;
+  const int64_t per = causal == 1 ? tiles_m * (tiles_m + 1) / 2 : tiles_m * tiles_n;
+  const int64_t tiles = per * count;
+  if (tiles > (int64_t(1) << 30)) return OMQ_ERR_SHAPE;
   if (n_tiles) *n_tiles = 2 * tiles;
   KernelChoice kc = choice<0>();
   if (epi.kind == Epi::SteW) {
@@ -701,11 +792,14 @@ omq_status gemm_tc(omq_dtype dt, const GemmOperand& A, const GemmOperand& B, int
     set_cuda_error(attr_err);
     return OMQ_ERR_CUDA;
   }
+  const TileSched sc{static_cast<int>(tiles_m), static_cast<int>(tiles_n), static_cast<int>(per),
+                     static_cast<int>(tiles), causal, amode, bmode,
+                     batch ? batch->out_stride : 0};
   const int64_t max_pairs = num_sms() / 2;
   const int64_t pairs = tiles < max_pairs ? tiles : max_pairs;
   kc.fn<<<static_cast<unsigned>(2 * pairs), kc.threads, kc.smem, stream>>>(
       ma, mb, A.mn_major ? 1 : 0, B.mn_major ? 1 : 0, dt == OMQ_F16 ? 0u : 1u, rows, cols, depth,
-      epi, static_cast<int>(tiles_n), static_cast<int>(tiles));
+      epi, sc);
   return launch_status();
 }
 

@@ -200,11 +200,32 @@ struct GemmEpilogue {
 // chunks (per-channel groups included).
 inline bool ste_fusable(int64_t g) { return g >= 32 && g % 32 == 0; }
 
+// A batch of `count` GEMMs of one shape whose A, B and output origins are a_stride,
+// b_stride and out_stride elements apart (attention: one problem per head), with an
+// optional causal schedule for square problems over token positions:
+//   causal 1: C[i, j] is needed only for j <= i: tiles wholly above the diagonal are skipped
+//   causal 2: A(i, k) vanishes for k > i: the contraction stops at the tile's last row
+//   causal 3: A(i, k) vanishes for k < i: the contraction starts at the tile's first row
+struct GemmBatch {
+  int64_t count;
+  int64_t a_stride, b_stride, out_stride;
+  int causal;
+};
+// The kernel's view of the schedule.
+struct TileSched {
+  int tiles_m, tiles_n;   // per problem
+  int per_batch;          // tiles per problem (causal 1: the lower triangle)
+  int num_tiles;          // all problems
+  int causal;
+  int a_bmode, b_bmode;   // operand maps: 0 2D; 1 / 2 3D, the problem index the middle / outer
+  int64_t out_bstride;
+};
+
 // 16-bit operands (BF16 or F16, both the same type) on tcgen05 (sm_100a). Reports the
-// number of output tiles (loss partial slots).
+// number of output tiles (loss partial slots). `batch` (StoreF32 epilogue only) may be NULL.
 omq_status gemm_tc(omq_dtype dt, const GemmOperand& A, const GemmOperand& B, int64_t rows,
                    int64_t cols, int64_t depth, const GemmEpilogue& epi, int64_t* n_tiles,
-                   cudaStream_t stream);
+                   cudaStream_t stream, const GemmBatch* batch = nullptr);
 int64_t gemm_tc_tiles(int64_t rows, int64_t cols);
 // f32 operands on CUDA cores.
 omq_status gemm_f32_simt(const GemmOperand& A, const GemmOperand& B, int64_t rows, int64_t cols,
