@@ -285,10 +285,12 @@ omq_status block_forward(const View& v, const Inputs& in, const Marks& mk, cudaS
                 th(OMQ_TH_BETA_QKV + 2 * l), s_w[l], v.bb<void>(what_id[l]), OMQ_BF16,
                 v.in<float>(c.h), v.in<int32_t>(c.z), nullptr, v.in<omq_range>(c.range), nullptr,
                 d.wbits};
+    if (dl_w[l]) {   // B~ = W delta out of the same pass over W
+      p.delta = dl_w[l];
+      p.Bt = v.in<float>(c.bt);
+    }
     BLK_TRY(launch_lwc(p, st));
     Wop[l] = v.bb<void>(what_id[l]);
-    if (dl_w[l])
-      BLK_TRY(launch_let_bias(in.W[l], OMQ_BF16, s.N, s.K, dl_w[l], nullptr, v.in<float>(c.bt), st));
   }
   auto bias = [&](int l) -> const float* { return fp || !dl_w[l] ? nullptr : v.in<float>(L.lin[l].bt); };
 

@@ -13,15 +13,16 @@
 
 namespace omq {
 
-__device__ __forceinline__ void epi_element(const GemmEpilogue& e, int64_t i, int64_t j,
-                                            int64_t cols, float acc, float& lsum) {
+// `out` is e.out, or the output of this tile's problem in a batch.
+__device__ __forceinline__ void epi_element(const GemmEpilogue& e, float* out, int64_t i,
+                                            int64_t j, int64_t cols, float acc, float& lsum) {
   const int64_t o = i * (e.ldo ? e.ldo : cols) + j;
   if (e.kind == Epi::StoreF32) {
-    e.out[o] = e.out_scale * acc + (e.bias ? e.bias[j] : 0.f);
+    out[o] = e.out_scale * acc + (e.bias ? e.bias[j] : 0.f);
     return;
   }
   const float y = acc + (e.bias ? e.bias[j] : 0.f);
-  if (e.out) e.out[o] = y;
+  if (out) out[o] = y;
   const float d = y - e.y_ref[o];
   lsum += d * d;
   store_elem(e.dy, o, d, e.dy_dt);
@@ -29,8 +30,9 @@ __device__ __forceinline__ void epi_element(const GemmEpilogue& e, int64_t i, in
 
 // 8 consecutive columns j0..j0+7 of row i, all in range, j0 % 8 == 0, cols % 8 == 0 and the
 // row stride a multiple of 8.
-__device__ __forceinline__ void epi_vec8(const GemmEpilogue& e, int64_t i, int64_t j0,
-                                         int64_t cols, const float (&acc)[8], float& lsum) {
+__device__ __forceinline__ void epi_vec8(const GemmEpilogue& e, float* out, int64_t i,
+                                         int64_t j0, int64_t cols, const float (&acc)[8],
+                                         float& lsum) {
   const int64_t o = i * (e.ldo ? e.ldo : cols) + j0;
   const float sc = e.kind == Epi::StoreF32 ? e.out_scale : 1.f;
   float y[8];
@@ -45,10 +47,10 @@ __device__ __forceinline__ void epi_vec8(const GemmEpilogue& e, int64_t i, int64
     for (int t = 0; t < 8; ++t) y[t] = sc * acc[t];
   }
   if (e.kind == Epi::StoreF32) {
-    store8(e.out, o, OMQ_F32, y);
+    store8(out, o, OMQ_F32, y);
     return;
   }
-  if (e.out) store8(e.out, o, OMQ_F32, y);
+  if (out) store8(out, o, OMQ_F32, y);
   float r[8];
   load8(e.y_ref, o, OMQ_F32, r);
   float d[8];

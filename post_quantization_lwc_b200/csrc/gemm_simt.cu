@@ -59,7 +59,7 @@ __global__ void __launch_bounds__(256) gemm_f32_kernel(GemmOperand A, GemmOperan
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
       const int64_t i = i0 + ty * 4 + u, j = j0 + tx * 4 + w;
-      if (i < rows && j < cols) epi_element(epi, i, j, cols, acc[u][w], lsum);
+      if (i < rows && j < cols) epi_element(epi, epi.out, i, j, cols, acc[u][w], lsum);
     }
   if (epi.kind == Epi::MseLoss) {
 #pragma unroll

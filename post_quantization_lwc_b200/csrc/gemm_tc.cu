@@ -183,10 +183,11 @@ __device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap
 }
 // One operand box: 2D (bmode 0) or 3D with the batch as the middle (1) or outer (2)
 // coordinate; (x, y) are the 2D coordinates (inner, outer) of the unbatched operand.
+template <bool BATCH>
 __device__ __forceinline__ void tma_load_op(uint32_t dst, const CUtensorMap* map,
                                             uint32_t leader_bar, int x, int y, int bmode,
                                             int b) {
-  if (bmode == 0) tma_load_2d_pair(dst, map, leader_bar, x, y);
+  if (!BATCH || bmode == 0) tma_load_2d_pair(dst, map, leader_bar, x, y);
   else if (bmode == 1) tma_load_3d_pair(dst, map, leader_bar, x, b, y);
   else tma_load_3d_pair(dst, map, leader_bar, x, y, b);
 }
@@ -200,8 +201,18 @@ __device__ __forceinline__ void tma_load_op(uint32_t dst, const CUtensorMap* map
 struct TileWork {
   int b, row0, col0, kb0, kb1;
 };
+template <bool BATCH>
 __device__ __forceinline__ TileWork tile_of(const TileSched& sc, int t, int nk) {
   TileWork w;
+  if (!BATCH) {   // one problem, no causal structure
+    const int tm = t / sc.tiles_n;
+    w.b = 0;
+    w.row0 = tm * TILE_M;
+    w.col0 = (t - tm * sc.tiles_n) * TILE_N;
+    w.kb0 = 0;
+    w.kb1 = nk;
+    return w;
+  }
   w.b = t / sc.per_batch;
   const int u = t - w.b * sc.per_batch;
   int tm, tn;
@@ -420,7 +431,8 @@ struct Layout {
   static constexpr uint32_t TMEM_COLS = 2 * TILE_N;
 };
 
-template <int EV>
+// BATCH: a batched and / or causal schedule (attention); false compiles the plain tile loop.
+template <int EV, bool BATCH>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV>::NUM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    int a_mn, int b_mn, uint32_t fmt, int64_t rows, int64_t cols, int64_t depth,
@@ -481,7 +493,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV>::NUM_THREADS
     int it = 0;
     bool ok = true;
     for (int t = pair; t < num_tiles && ok; t += pairs) {
-      const TileWork tw = tile_of(sc, t, nk);
+      const TileWork tw = tile_of<BATCH>(sc, t, nk);
       const int row0 = tw.row0 + static_cast<int>(rank) * HALF;
       const int col0 = tw.col0 + static_cast<int>(rank) * HALF;
       for (int kb = tw.kb0; kb < tw.kb1; ++kb, ++it) {
@@ -500,15 +512,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV>::NUM_THREADS
         const int k0 = kb * BK;
         if (a_mn) {
           for (int c = 0; c < HALF / 64; ++c)
-            tma_load_op(a_dst + c * 8192, &tmA, full_leader, row0 + 64 * c, k0, sc.a_bmode, tw.b);
+            tma_load_op<BATCH>(a_dst + c * 8192, &tmA, full_leader, row0 + 64 * c, k0, sc.a_bmode, tw.b);
         } else {
-          tma_load_op(a_dst, &tmA, full_leader, k0, row0, sc.a_bmode, tw.b);
+          tma_load_op<BATCH>(a_dst, &tmA, full_leader, k0, row0, sc.a_bmode, tw.b);
         }
         if (b_mn) {
           for (int c = 0; c < HALF / 64; ++c)
-            tma_load_op(b_dst + c * 8192, &tmB, full_leader, col0 + 64 * c, k0, sc.b_bmode, tw.b);
+            tma_load_op<BATCH>(b_dst + c * 8192, &tmB, full_leader, col0 + 64 * c, k0, sc.b_bmode, tw.b);
         } else {
-          tma_load_op(b_dst, &tmB, full_leader, k0, col0, sc.b_bmode, tw.b);
+          tma_load_op<BATCH>(b_dst, &tmB, full_leader, k0, col0, sc.b_bmode, tw.b);
         }
       }
     }
@@ -535,7 +547,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV>::NUM_THREADS
       }
       tc_fence_after();
       const uint32_t d = tmem + static_cast<uint32_t>(buf * TILE_N);
-      const TileWork tw = tile_of(sc, t, nk);
+      const TileWork tw = tile_of<BATCH>(sc, t, nk);
       for (int kb = tw.kb0; kb < tw.kb1; ++kb, ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
@@ -570,7 +582,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV>::NUM_THREADS
     int lt = 0;
     for (int t = pair; t < num_tiles; t += pairs, ++lt) {
       const int buf = lt & 1;
-      const TileWork tw = tile_of(sc, t, nk);
+      const TileWork tw = tile_of<BATCH>(sc, t, nk);
       const int64_t wrow0 = static_cast<int64_t>(tw.row0) + rank * HALF + quad * 32;
       const int64_t col0 = static_cast<int64_t>(tw.col0) + cq * EPI_COLS;
       const int64_t row = wrow0 + lane;
@@ -589,8 +601,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV>::NUM_THREADS
       if constexpr (EV != 0) {
         ste_w_epilogue<EV == 2>(epi, tbase, wrow0, col0, rows, cols, lane);
       } else {
-        GemmEpilogue eb = epi;                     // this tile's batch of the output
-        if (tw.b) eb.out += static_cast<int64_t>(tw.b) * sc.out_bstride;
+        float* const out_b = BATCH ? epi.out + static_cast<int64_t>(tw.b) * sc.out_bstride : epi.out;
         for (int ch = 0; ch < EPI_COLS / 32; ++ch) {
           uint32_t r[32];
           tmem_ld32(tbase + ch * 32, r);
@@ -603,13 +614,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV>::NUM_THREADS
                 float acc[8];
 #pragma unroll
                 for (int q = 0; q < 8; ++q) acc[q] = __uint_as_float(r[v * 8 + q]);
-                epi_vec8(eb, row, cbase + v * 8, cols, acc, lsum);
+                epi_vec8(epi, out_b, row, cbase + v * 8, cols, acc, lsum);
               }
             } else {
 #pragma unroll
               for (int q = 0; q < 32; ++q)
                 if (cbase + q < cols)
-                  epi_element(eb, row, cbase + q, cols, __uint_as_float(r[q]), lsum);
+                  epi_element(epi, out_b, row, cbase + q, cols, __uint_as_float(r[q]), lsum);
             }
           }
         }
@@ -732,9 +743,9 @@ struct KernelChoice {
   int threads, smem;
 };
 
-template <int EV>
+template <int EV, bool BATCH = false>
 KernelChoice choice() {
-  return {gemm_tc_kernel<EV>, Cfg<EV>::NUM_THREADS,
+  return {gemm_tc_kernel<EV, BATCH>, Cfg<EV>::NUM_THREADS,
           Layout<Cfg<EV>::STAGES, Cfg<EV>::EPI_WARPS>::SMEM_BYTES};
 }
 
@@ -781,7 +792,7 @@ omq_status gemm_tc(omq_dtype dt, const GemmOperand& A, const GemmOperand& B, int
   const int64_t tiles = per * count;
   if (tiles > (int64_t(1) << 30)) return OMQ_ERR_SHAPE;
   if (n_tiles) *n_tiles = 2 * tiles;
-  KernelChoice kc = choice<0>();
+  KernelChoice kc = (count > 1 || causal) ? choice<0, true>() : choice<0>();
   if (epi.kind == Epi::SteW) {
     if (!ste_fusable(epi.ste.G) || (epi.ste.wdt != OMQ_BF16 && epi.ste.wdt != OMQ_F16))
       return OMQ_ERR_SHAPE;

@@ -136,24 +136,32 @@ __global__ void __launch_bounds__(256) act_quant_kernel(LetParams p) {
   }
 }
 
-// B~[n] = B[n] + sum_k W[n,k] delta[k]  (one warp per row; lanes stride 8-element chunks)
+// B~[n] = B[n] + sum_k W[n,k] delta[k]  (one warp per row; lanes stride 8-element chunks,
+// eight 16-byte loads in flight a lane before any is used)
 __global__ void __launch_bounds__(256) let_bias_kernel(const void* W, omq_dtype wdt, int64_t N,
                                                        int64_t K, const float* delta,
                                                        const float* B, float* Bt) {
+  constexpr int U = 8;
   const int lane = threadIdx.x & 31;
   const int64_t warp_g = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t n_warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  const int64_t nc = K / 8;
   for (int64_t n = warp_g; n < N; n += n_warps) {
     float acc = 0.f;
     if (delta) {
-#pragma unroll 4
-      for (int64_t c = lane; c < K / 8; c += 32) {
-        float v[8];
-        load8(W, n * K + c * 8, wdt, v);
-        const float4* q = reinterpret_cast<const float4*>(delta + c * 8);
-        const float4 a = q[0], b = q[1];
-        acc += v[0] * a.x + v[1] * a.y + v[2] * a.z + v[3] * a.w + v[4] * b.x + v[5] * b.y +
-               v[6] * b.z + v[7] * b.w;
+      for (int64_t c0 = lane; c0 < nc; c0 += 32 * U) {
+        float v[U][8];
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+          if (c0 + 32 * u < nc) load8(W, n * K + (c0 + 32 * u) * 8, wdt, v[u]);
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          if (c0 + 32 * u >= nc) continue;
+          float d[8];
+          load_f8(delta, (c0 + 32 * u) * 8, d);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc += v[u][i] * d[i];
+        }
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);

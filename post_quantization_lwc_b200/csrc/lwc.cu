@@ -20,15 +20,35 @@
 namespace omq {
 
 // Encode 8 values of one group; write W^, codes and packed codes of element `off`.
+// round(v/h) of the correctly rounded quotient equals the rounding of the product v*hinv
+// (hinv = 1/h correctly rounded) wherever the product is below 256 in magnitude and at most
+// 0.49995 from its nearest integer: the product is within 2^-23 |v/h| of v/h (two roundings)
+// and the quotient within 2^-24 |v/h|, so the two differ by less than 4.6e-5 and the
+// quotient lies strictly inside the same rounding interval. The other elements (about 1e-4
+// of them) take the IEEE quotient, in a branch the active lanes enter together only when one
+// of them needs it.
 __device__ __forceinline__ void encode8(const LwcParams& p, int64_t off, const float (&v)[8],
                                         const GroupQ& q) {
   const float hinv = __frcp_rn(q.h);
+  float r[8];
+  unsigned slow = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float ua = __fmul_rn(v[i], hinv);
+    r[i] = rne_small(ua);
+    const bool ok = fabsf(ua) < 256.f && fabsf(__fsub_rn(ua, r[i])) <= 0.49995f;
+    slow |= ok ? 0u : (1u << i);
+  }
+  if (__any_sync(__activemask(), slow != 0)) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if (slow & (1u << i)) r[i] = rintf(__fdiv_rn(v[i], q.h));
+  }
   float deq[8];
   uint32_t c[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const float lvl = __fadd_rn(round_quotient(v[i], q.h, hinv), q.z);
-    const float cc = fminf(fmaxf(lvl, 0.f), p.Q);
+    const float cc = fminf(fmaxf(__fadd_rn(r[i], q.z), 0.f), p.Q);
     deq[i] = __fmul_rn(__fsub_rn(cc, q.z), q.h);
     c[i] = small_uint(cc);
   }
@@ -79,7 +99,7 @@ __device__ __forceinline__ void load_scaled8(const LwcParams& p, int64_t off, in
 constexpr int kLwcRows = 64;
 
 template <int LPG, int U>
-__global__ void __launch_bounds__(256) lwc_small_kernel(LwcParams p) {
+__global__ void __launch_bounds__(256, 3) lwc_small_kernel(LwcParams p) {
   constexpr int GPW = 32 / LPG;   // groups per segment
   // The clipping strengths (binary64 sigmoids) of the U rows' groups are spread over the
   // warp's lanes: SPR strengths a row (gamma, beta of each group), RPP rows a pass of 32
@@ -238,6 +258,11 @@ __global__ void __launch_bounds__(256) lwc_large_kernel(LwcParams p) {
 omq_status launch_lwc(const LwcParams& p, cudaStream_t stream) {
   const int64_t total = p.N * p.ng;
   const int sms = num_sms();
+  if (p.Bt) {
+    // B~ = B + W delta: its own pass over W
+    const omq_status st = launch_let_bias(p.W, p.wdt, p.N, p.K, p.delta, p.B, p.Bt, stream);
+    if (st != OMQ_OK) return st;
+  }
   if (small_group(p.G)) {
     constexpr int U = 4;
     dim3 grid(static_cast<unsigned>(ceil_div(p.K, 256)),

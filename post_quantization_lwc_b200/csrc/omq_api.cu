@@ -473,13 +473,24 @@ omq_status omq_calib_step(const omq_step_args* a, void* workspace, size_t ws_byt
   OMQ_TRY(ph.mark(OMQ_PH_LET));
   if (need_act) {
     OMQ_TRY(omq_let_apply(a->X, a->dt, M, K, let ? a->s : nullptr, let ? a->delta : nullptr,
-                          a->abits, a->Xq, a->op_dt, a->h_a, a->z_a, a->tok_range, a->W, a->dt,
-                          N, a->B, let ? a->B_tilde : nullptr, stream));
+                          a->abits, a->Xq, a->op_dt, a->h_a, a->z_a, a->tok_range, nullptr, a->dt,
+                          N, nullptr, nullptr, stream));
   }
   OMQ_TRY(ph.mark(OMQ_PH_LWC));
-  OMQ_TRY(omq_lwc_quant(a->W, a->dt, N, K, G, a->bits, a->gamma_logit, a->beta_logit,
-                        let ? a->s : nullptr, a->W_hat, a->op_dt, a->h, a->z, nullptr,
-                        a->grp_range, stream));
+  {
+    // LWC, with B~ = B + W delta out of the same pass over W
+    OMQ_TRY(check_lwc(a->W, a->dt, N, K, G, a->bits, a->gamma_logit, a->beta_logit,
+                      let ? a->s : nullptr, a->op_dt, a->W_hat, nullptr, a->h, a->z));
+    LwcParams p{a->W, a->dt, N, K, G, K / G, static_cast<float>((1 << a->bits) - 1),
+                a->gamma_logit, a->beta_logit, let ? a->s : nullptr, a->W_hat, a->op_dt, a->h,
+                a->z, nullptr, a->grp_range, nullptr, a->bits};
+    if (let) {
+      p.delta = a->delta;
+      p.B = a->B;
+      p.Bt = a->B_tilde;
+    }
+    OMQ_TRY(launch_lwc(p, reinterpret_cast<cudaStream_t>(stream)));
+  }
   OMQ_TRY(fwd_impl(Xq, a->W_hat, a->op_dt, M, N, K, Bt, a->Y_ref, nullptr, a->dY, a->loss,
                    workspace, fwd_ws, stream, ph));
   omq_bwd_args b{};

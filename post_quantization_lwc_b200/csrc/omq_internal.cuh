@@ -251,6 +251,11 @@ struct LwcParams {
   omq_range* range;
   uint8_t* packed;
   int bits;
+  // optional, fused into the same pass over W when the row-tile kernel runs (else a
+  // separate launch): Bt[n] = B[n] + sum_k W[n,k] delta[k] with the original W
+  const float* delta;
+  const float* B;
+  float* Bt;
 };
 
 struct LetParams {
