@@ -40,7 +40,7 @@ __device__ __forceinline__ void let8(const LetParams& p, int64_t off, int64_t co
 constexpr int kLetRows = 64;
 
 template <int U, bool AFFINE>
-__global__ void __launch_bounds__(256) let_elem_kernel(LetParams p) {
+__global__ void __launch_bounds__(256, 2) let_elem_kernel(LetParams p) {
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int64_t c0 = static_cast<int64_t>(blockIdx.x) * 256 + lane * 8;
   if (c0 >= p.K) return;

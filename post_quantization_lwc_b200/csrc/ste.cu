@@ -222,20 +222,23 @@ __global__ void __launch_bounds__(256) ste_w_large_kernel(SteWParams p) {
 }
 
 // ------------------------------------------------------------------ fused weight side
-// Completion of the STE that the dW^ GEMM's epilogue started. Grid (32-row tiles, 32-group
-// tile strides), 256 threads; a tile of 32 rows x 32 groups is read in two mappings so both
-// layouts stay coalesced: the chunk partials ([K/32, N]) with the row fastest, staged in
-// shared memory, then the per-group arrays ([N, ng]) with the group fastest. A group's
+constexpr int kFinishJ = 8;   // groups per tile of ste_w_finish_kernel (32 rows a tile)
+// Completion of the STE that the dW^ GEMM's epilogue started. Grid (32-row tiles, kFinishJ-
+// group tile strides), 256 threads; a tile of 32 rows x kFinishJ groups is read in two
+// mappings so both layouts stay coalesced: the chunk partials ([K/32, N]) with the row
+// fastest, staged in shared memory, then the per-group arrays ([N, ng]) with the group
+// fastest. A group's
 // chunk partials are added in chunk order (groups of up to 8 chunks) or as 8 interleaved
 // partial sums added in a fixed order (longer groups).
 __global__ void __launch_bounds__(256) ste_w_finish_kernel(SteWFinish p) {
-  __shared__ float sgh[32][33], sgc[32][33];   // [group in tile][row in tile]
+  __shared__ float sgh[kFinishJ][33], sgc[kFinishJ][33];   // [group in tile][row in tile]
   __shared__ float wred[2][8][32];
   const int64_t n0 = static_cast<int64_t>(blockIdx.x) * 32;
   const int64_t cpg = p.G / 32;
-  for (int64_t j0 = static_cast<int64_t>(blockIdx.y) * 32; j0 < p.ng; j0 += 32 * gridDim.y) {
+  for (int64_t j0 = static_cast<int64_t>(blockIdx.y) * kFinishJ; j0 < p.ng;
+       j0 += kFinishJ * gridDim.y) {
     if (cpg <= 8) {
-      for (int e = threadIdx.x; e < 1024; e += blockDim.x) {
+      for (int e = threadIdx.x; e < 32 * kFinishJ; e += blockDim.x) {
         const int nl = e & 31, jl = e >> 5;
         const int64_t n = n0 + nl, j = j0 + jl;
         float Gh = 0.f, Gc = 0.f;
@@ -253,7 +256,7 @@ __global__ void __launch_bounds__(256) ste_w_finish_kernel(SteWFinish p) {
       // (lane = row), then warp 0 adds the 8 partial sums in warp order
       const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
       const int64_t n = n0 + lane;
-      for (int jl = 0; jl < 32; ++jl) {
+      for (int jl = 0; jl < kFinishJ; ++jl) {
         const int64_t j = j0 + jl;
         float Gh = 0.f, Gc = 0.f;
         if (n < p.N && j < p.ng)
@@ -280,8 +283,8 @@ __global__ void __launch_bounds__(256) ste_w_finish_kernel(SteWFinish p) {
       }
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < 1024; e += blockDim.x) {
-      const int jl = e & 31, nl = e >> 5;
+    for (int e = threadIdx.x; e < 32 * kFinishJ; e += blockDim.x) {
+      const int jl = e % kFinishJ, nl = e / kFinishJ;
       const int64_t n = n0 + nl, j = j0 + jl;
       if (n >= p.N || j >= p.ng) continue;
       const int64_t gi = n * p.ng + j;
@@ -304,70 +307,95 @@ __global__ void __launch_bounds__(256) ste_w_finish_kernel(SteWFinish p) {
   }
 }
 
-// The W-side LET terms that the epilogue leaves out, in one pass over W. Grid (256-column
-// segments, 32-row block strides); lane = 8 columns of one group, the 8 warps take rows w,
-// w + 8, w + 16, w + 24 of a block; the warps' sums are added in warp order.
+// The W-side LET terms that the epilogue leaves out, in one pass over W. One warp per task
+// (32-row block, 256-column segment), persistent warps; lane = 8 columns (one group), the
+// block's 32 rows walked in order, eight row loads in flight before any is used:
 //   part_s[rb, k] += sum_n (emax W[n,k] where W~[n,k] is its group's max, emin W[n,k] where
 //                    it is the min)                       (the clipping-range terms of d s)
 //   part_d[rb, k]  = sum_n dBt[n] W[n,k]                  (the bias term of d delta)
-__global__ void __launch_bounds__(256) ste_w_corr_kernel(SteWCorr p) {
-  __shared__ float red_s[8][256];
-  __shared__ float red_d[8][256];
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * 256 + lane * 8;
-  const bool cvalid = c0 < p.K;
-  const int64_t ng = p.K / p.G, j = c0 / p.G;
-  float sv[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) sv[i] = 1.f;
-  if (p.s && cvalid) load_f8(p.s, c0, sv);
-  for (int64_t rb = blockIdx.y; rb * 32 < p.N; rb += gridDim.y) {
+__global__ void __launch_bounds__(256, 2) ste_w_corr_kernel(SteWCorr p) {
+  constexpr int U = 8;
+  const int lane = threadIdx.x & 31;
+  const int64_t warp_g = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t n_warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  const int64_t segs = (p.K + 255) / 256, rbs = (p.N + 31) / 32;
+  const int64_t ng = p.K / p.G;
+  const bool f16 = p.wdt == OMQ_F16;
+  for (int64_t task = warp_g; task < segs * rbs; task += n_warps) {
+    const int64_t rb = task / segs, seg = task - rb * segs;
+    const int64_t c0 = seg * 256 + lane * 8;
+    const bool cvalid = c0 < p.K;
+    const int64_t j = cvalid ? c0 / p.G : 0;
+    const uint4* wcol = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.W) + c0);
+    const int64_t wstride = p.K / 8;                 // uint4 per row
     float acc_s[8] = {}, acc_d[8] = {};
-    float v[4][8];
+    for (int r = 0; r < 32; r += U) {
+      // every load of the U rows (weights as packed 16-bit, the groups' records) before use
+      uint4 raw[U];
+      float2 mm[U];
+      float eM[U], em[U], db[U];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int64_t n = rb * 32 + w + 8 * u;
-      if (n < p.N && cvalid) load8(p.W, n * p.K + c0, p.wdt, v[u]);
-    }
+      for (int u = 0; u < U; ++u) {
+        const int64_t n = rb * 32 + r + u;
+        const bool ok = n < p.N && cvalid;
+        raw[u] = ok ? __ldg(wcol + n * wstride) : make_uint4(0, 0, 0, 0);
+        const int64_t gi = ok ? n * ng + j : 0;
+        mm[u] = make_float2(0.f, 0.f);
+        eM[u] = em[u] = db[u] = 0.f;
+        if (ok && p.part_s) {
+          mm[u] = *reinterpret_cast<const float2*>(p.range + gi);   // vmax, vmin
+          eM[u] = p.emax[gi];
+          em[u] = p.emin[gi];
+        }
+        if (ok && p.part_d) db[u] = p.dBt[n];
+      }
+      float sv[8];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int64_t n = rb * 32 + w + 8 * u;
-      if (n >= p.N || !cvalid) continue;
-      if (p.part_s) {
-        const int64_t gi = n * ng + j;
-        const omq_range rg = p.range[gi];
-        const float eM = p.emax[gi], em = p.emin[gi];
+      for (int i = 0; i < 8; ++i) sv[i] = 1.f;
+      if (p.s && cvalid) load_f8(p.s, c0, sv);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float wt = p.s ? __fmul_rn(v[u][i], sv[i]) : v[u][i];
-          if (wt == rg.vmax) acc_s[i] += eM * v[u][i];
-          if (wt == rg.vmin) acc_s[i] += em * v[u][i];
+      for (int u = 0; u < U; ++u) {
+        float v[8];
+        if (f16) {
+          const __half2* h2 = reinterpret_cast<const __half2*>(&raw[u]);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float2 f = __half22float2(h2[q]);
+            v[2 * q] = f.x;
+            v[2 * q + 1] = f.y;
+          }
+        } else {
+          const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&raw[u]);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float2 f = __bfloat1622float2(b2[q]);
+            v[2 * q] = f.x;
+            v[2 * q + 1] = f.y;
+          }
+        }
+        if (p.part_s) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float wt = p.s ? __fmul_rn(v[i], sv[i]) : v[i];
+            if (wt == mm[u].x) acc_s[i] += eM[u] * v[i];
+            if (wt == mm[u].y) acc_s[i] += em[u] * v[i];
+          }
+        }
+        if (p.part_d) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc_d[i] += db[u] * v[i];
         }
       }
-      if (p.part_d) {
-        const float db = p.dBt[n];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc_d[i] += db * v[u][i];
-      }
     }
+    if (!cvalid) continue;
+    if (p.part_s) {
+      float cur[8];
+      load_f8(p.part_s, rb * p.K + c0, cur);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      red_s[w][lane * 8 + i] = acc_s[i];
-      red_d[w][lane * 8 + i] = acc_d[i];
+      for (int i = 0; i < 8; ++i) cur[i] += acc_s[i];
+      store8(p.part_s, rb * p.K + c0, OMQ_F32, cur);
     }
-    __syncthreads();
-    const int64_t col = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
-    if (col < p.K) {
-      float a = 0.f, d = 0.f;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        a += red_s[q][threadIdx.x];
-        d += red_d[q][threadIdx.x];
-      }
-      if (p.part_s) p.part_s[rb * p.K + col] += a;
-      if (p.part_d) p.part_d[rb * p.K + col] = d;
-    }
-    __syncthreads();   // red is rewritten by the next row block
+    if (p.part_d) store8(p.part_d, rb * p.K + c0, OMQ_F32, acc_d);
   }
 }
 
@@ -674,15 +702,16 @@ omq_status launch_ste_w(const SteWParams& p, cudaStream_t stream) {
 
 omq_status launch_ste_w_finish(const SteWFinish& p, cudaStream_t stream) {
   const dim3 grid(static_cast<unsigned>(ceil_div(p.N, 32)),
-                  static_cast<unsigned>(std::min<int64_t>(ceil_div(p.ng, 32), 65535)));
+                  static_cast<unsigned>(std::min<int64_t>(ceil_div(p.ng, kFinishJ), 65535)));
   ste_w_finish_kernel<<<grid, 256, 0, stream>>>(p);
   return launch_status();
 }
 
 omq_status launch_ste_w_corr(const SteWCorr& p, cudaStream_t stream) {
-  const dim3 grid(static_cast<unsigned>(ceil_div(p.K, 256)),
-                  static_cast<unsigned>(std::min<int64_t>(ceil_div(p.N, 32), 65535)));
-  ste_w_corr_kernel<<<grid, 256, 0, stream>>>(p);
+  const int64_t tasks = ceil_div(p.K, 256) * ceil_div(p.N, 32);
+  const int64_t cap = static_cast<int64_t>(num_sms()) * 16;    // resident warps
+  const int64_t warps = tasks < cap ? tasks : cap;
+  ste_w_corr_kernel<<<static_cast<unsigned>(ceil_div(warps, 8)), 256, 0, stream>>>(p);
   return launch_status();
 }
 
