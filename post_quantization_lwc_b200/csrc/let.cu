@@ -136,32 +136,71 @@ __global__ void __launch_bounds__(256) act_quant_kernel(LetParams p) {
   }
 }
 
-// B~[n] = B[n] + sum_k W[n,k] delta[k]  (one warp per row; lanes stride 8-element chunks,
-// eight 16-byte loads in flight a lane before any is used)
-__global__ void __launch_bounds__(256) let_bias_kernel(const void* W, omq_dtype wdt, int64_t N,
-                                                       int64_t K, const float* delta,
-                                                       const float* B, float* Bt) {
-  constexpr int U = 8;
+// B~[n] = B[n] + sum_k W[n,k] delta[k]. One warp per row, persistent warps taking rows in
+// equal shares; the row is read in passes of 16 segments of 256 columns (lane = 8 columns of
+// each), the 16 loads of a pass issued before any is used and kept packed.
+constexpr int kBiasSegs = 16;
+
+__global__ void __launch_bounds__(256, 2) let_bias_kernel(const void* W, omq_dtype wdt, int64_t N,
+                                                          int64_t K, const float* delta,
+                                                          const float* B, float* Bt,
+                                                          int64_t rows_per_warp) {
   const int lane = threadIdx.x & 31;
   const int64_t warp_g = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t n_warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-  const int64_t nc = K / 8;
+  const int64_t nseg = (K + 255) / 256;
+  for (int64_t it = 0; it < rows_per_warp; ++it) {
+    const int64_t n = warp_g + it * n_warps;
+    if (n >= N) break;                                     // warp-uniform
+    float acc = 0.f;
+    if (delta) {
+      for (int64_t s0 = 0; s0 < nseg; s0 += kBiasSegs) {
+        uint4 raw[kBiasSegs];
+#pragma unroll
+        for (int i = 0; i < kBiasSegs; ++i) {
+          const int64_t col = (s0 + i) * 256 + lane * 8;
+          raw[i] = col < K ? *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(W) +
+                                                              n * K + col)
+                           : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int i = 0; i < kBiasSegs; ++i) {
+          const int64_t col = (s0 + i) * 256 + lane * 8;
+          if (col >= K) break;
+          float v[8], d[8];
+          const uint16_t* h = reinterpret_cast<const uint16_t*>(&raw[i]);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            v[e] = wdt == OMQ_F16 ? __half2float(__ushort_as_half(h[e]))
+                                  : __bfloat162float(__ushort_as_bfloat16(h[e]));
+          load_f8(delta, col, d);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc += v[e] * d[e];
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    }
+    if (lane == 0) Bt[n] = (B ? B[n] : 0.f) + acc;
+  }
+}
+
+// float32 W (the CUDA-core path): one warp per row, lanes stride 8-element chunks.
+__global__ void __launch_bounds__(256) let_bias_f32_kernel(const float* W, int64_t N, int64_t K,
+                                                           const float* delta, const float* B,
+                                                           float* Bt) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp_g = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t n_warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   for (int64_t n = warp_g; n < N; n += n_warps) {
     float acc = 0.f;
     if (delta) {
-      for (int64_t c0 = lane; c0 < nc; c0 += 32 * U) {
-        float v[U][8];
+      for (int64_t c = lane; c < K / 8; c += 32) {
+        float v[8], d[8];
+        load_f8(W, n * K + c * 8, v);
+        load_f8(delta, c * 8, d);
 #pragma unroll
-        for (int u = 0; u < U; ++u)
-          if (c0 + 32 * u < nc) load8(W, n * K + (c0 + 32 * u) * 8, wdt, v[u]);
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-          if (c0 + 32 * u >= nc) continue;
-          float d[8];
-          load_f8(delta, (c0 + 32 * u) * 8, d);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) acc += v[u][i] * d[i];
-        }
+        for (int e = 0; e < 8; ++e) acc += v[e] * d[e];
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
@@ -193,9 +232,18 @@ omq_status launch_let(const LetParams& p, int abits, cudaStream_t stream) {
 omq_status launch_let_bias(const void* W, omq_dtype wdt, int64_t N, int64_t K, const float* delta,
                            const float* B, float* Bt, cudaStream_t stream) {
   const int sms = num_sms();
-  const int64_t want = ceil_div(N, 8);
-  const unsigned grid = static_cast<unsigned>(want < int64_t(sms) * 16 ? want : int64_t(sms) * 16);
-  let_bias_kernel<<<grid, 256, 0, stream>>>(W, wdt, N, K, delta, B, Bt);
+  if (wdt == OMQ_F32) {
+    const int64_t want = ceil_div(N, 8);
+    const unsigned grid = static_cast<unsigned>(want < int64_t(sms) * 16 ? want : int64_t(sms) * 16);
+    let_bias_f32_kernel<<<grid, 256, 0, stream>>>(static_cast<const float*>(W), N, K, delta, B,
+                                                  Bt);
+    return launch_status();
+  }
+  const int64_t max_warps = static_cast<int64_t>(sms) * 16;
+  const int64_t per = (N + max_warps - 1) / max_warps;
+  const int64_t warps = (N + per - 1) / per;
+  let_bias_kernel<<<static_cast<unsigned>((warps + 7) / 8), 256, 0, stream>>>(W, wdt, N, K, delta,
+                                                                            B, Bt, per);
   return launch_status();
 }
 

@@ -255,9 +255,118 @@ __global__ void __launch_bounds__(256) lwc_large_kernel(LwcParams p) {
   }
 }
 
+// 8 values of a 16-bit vector load.
+__device__ __forceinline__ void unpack16x8(const uint4& q, bool f16, float (&v)[8]) {
+  if (f16) {
+    const __half2* h2 = reinterpret_cast<const __half2*>(&q);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __half22float2(h2[j]);
+      v[2 * j] = f.x;
+      v[2 * j + 1] = f.y;
+    }
+  } else {
+    const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&q);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __bfloat1622float2(b2[j]);
+      v[2 * j] = f.x;
+      v[2 * j + 1] = f.y;
+    }
+  }
+}
+// W~ = W s for 8 columns starting at col (binary32, one rounding).
+__device__ __forceinline__ void scale8(const float* s, int64_t col, float (&v)[8]) {
+  float sv[8];
+  load_f8(s, col, sv);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(v[i], sv[i]);
+}
+
+// One group per row (per-channel), 16-bit W, K a multiple of 256 up to 4096: one warp per
+// row, persistent warps taking rows in equal shares. Lane l holds columns 256 i + 8 l .. + 7
+// of every 256-column segment i (coalesced 16-byte loads, all issued before any is used, the
+// row kept packed in registers), so the max / min, the tie counts and the codes come from
+// one read of W; B~[n] = B[n] + sum_k W[n,k] delta[k] (when requested) from the same data.
+constexpr int kRowSegs = 16;
+
+__global__ void __launch_bounds__(256, 2) lwc_row_kernel(LwcParams p, int64_t rows_per_warp) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp_g = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t n_warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  const int S = static_cast<int>(p.K / 256);
+  const bool f16 = p.wdt == OMQ_F16;
+  for (int64_t it = 0; it < rows_per_warp; ++it) {
+    const int64_t n = warp_g + it * n_warps;
+    if (n >= p.N) break;                                  // warp-uniform
+    const uint4* wrow = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.W) + n * p.K) + lane;
+    uint4 raw[kRowSegs];
+#pragma unroll
+    for (int i = 0; i < kRowSegs; ++i)
+      if (i < S) raw[i] = __ldg(wrow + 32 * i);
+    float vmax = -FLT_MAX, vmin = FLT_MAX;
+#pragma unroll
+    for (int i = 0; i < kRowSegs; ++i) {
+      if (i >= S) break;
+      float v[8];
+      unpack16x8(raw[i], f16, v);
+      if (p.s) scale8(p.s, 256 * i + 8 * lane, v);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) { vmax = fmaxf(vmax, v[e]); vmin = fminf(vmin, v[e]); }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+      vmin = fminf(vmin, __shfl_xor_sync(0xffffffffu, vmin, o));
+    }
+    float st = 1.f;
+    if (lane < 2) st = strength((lane ? p.bl : p.gl)[n]);
+    const float g = __shfl_sync(0xffffffffu, st, 0), b = __shfl_sync(0xffffffffu, st, 1);
+    const GroupQ q = group_params(g, b, vmax, vmin, p.Q);
+    int cnt = 0;                                          // nmax | nmin << 16
+    float bias = 0.f;
+#pragma unroll
+    for (int i = 0; i < kRowSegs; ++i) {
+      if (i >= S) break;
+      const int64_t col = 256 * i + 8 * lane;
+      float v[8];
+      unpack16x8(raw[i], f16, v);
+      if (p.Bt && p.delta) {
+        float d[8];
+        load_f8(p.delta, col, d);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) bias += v[e] * d[e];
+      }
+      if (p.s) scale8(p.s, col, v);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) cnt += (v[e] == vmax ? 1 : 0) + (v[e] == vmin ? 0x10000 : 0);
+      encode8(p, n * p.K + col, v, q);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+      bias += __shfl_xor_sync(0xffffffffu, bias, o);
+    }
+    if (lane == 0) {
+      if (p.h) p.h[n] = q.h;
+      if (p.z) p.z[n] = z_to_i32(q.z);
+      if (p.range) p.range[n] = omq_range{vmax, vmin, cnt & 0xffff, cnt >> 16};
+      if (p.Bt) p.Bt[n] = (p.B ? p.B[n] : 0.f) + bias;
+    }
+  }
+}
+
 omq_status launch_lwc(const LwcParams& p, cudaStream_t stream) {
   const int64_t total = p.N * p.ng;
   const int sms = num_sms();
+  if ((p.wdt == OMQ_BF16 || p.wdt == OMQ_F16) && p.G == p.K && p.K % 256 == 0 &&
+      p.K <= 256 * kRowSegs) {
+    const int64_t max_warps = static_cast<int64_t>(sms) * 16;   // 2 blocks of 8 warps an SM
+    const int64_t per = (p.N + max_warps - 1) / max_warps;
+    const int64_t warps = (p.N + per - 1) / per;
+    lwc_row_kernel<<<static_cast<unsigned>((warps + 7) / 8), 256, 0, stream>>>(p, per);
+    return launch_status();
+  }
   if (p.Bt) {
     // B~ = B + W delta: its own pass over W
     const omq_status st = launch_let_bias(p.W, p.wdt, p.N, p.K, p.delta, p.B, p.Bt, stream);
