@@ -240,9 +240,10 @@ omq_status omq_adamw_step(float* param, const float* grad, float* m, float* v, i
 /* ------------------------------------------------------------------------------------
  * omq_fold_pack — fold the learned parameters into deployable integer weights
  * ([ICLR] section 框架: the learned transforms fold back into the weights).
- * codes as in omq_lwc_quant, packed row-major: element k of a row goes to byte
- * k*bits/8 at bit offset (k*bits) mod 8, least-significant bits first.
- * packed [N, K*bits/8] uint8; h, z [N, K/group]. bits in {2,4,8} (3: OMQ_ERR_UNSUPPORTED).
+ * codes as in omq_lwc_quant, packed row-major: element k of a row occupies bits
+ * k*bits .. k*bits + bits - 1 of the row's little-endian bit string (it starts in byte
+ * k*bits/8 at bit offset (k*bits) mod 8, least-significant bits first; a 3-bit code may
+ * straddle two bytes). packed [N, K*bits/8] uint8; h, z [N, K/group]. bits in {2,3,4,8}.
  * ------------------------------------------------------------------------------------ */
 omq_status omq_fold_pack(const void* W, omq_dtype wdt, int64_t N, int64_t K, int64_t group,
                          int bits, const float* gamma_logit, const float* beta_logit,

@@ -365,26 +365,36 @@ LR_LET = 1e-2
 # ----------------------------------------------------------------------------- fold / pack
 
 def pack_codes(codes, bits: int) -> np.ndarray:
-    """Row-major bit packing: element k of a row lands in byte (k*bits)//8 at bit offset
-    (k*bits) % 8, least-significant bits first. Supports bits in {2, 4, 8}."""
-    c = np.asarray(codes).astype(np.uint32)
+    """Row-major bit packing: element k of a row occupies bits k*bits .. k*bits + bits - 1 of
+    the row's little-endian bit string, i.e. it starts in byte (k*bits)//8 at bit offset
+    (k*bits) % 8, least-significant bits first; a 3-bit code may straddle two bytes.
+    Supports bits in {2, 3, 4, 8} with a row length whose bits fill whole bytes."""
+    c = np.asarray(codes).astype(np.uint64)
     R, C = c.shape
-    if bits not in (2, 4, 8) or (C * bits) % 8:
+    if bits not in (2, 3, 4, 8) or (C * bits) % 8:
         raise ValueError("unsupported packing")
-    per = 8 // bits
-    out = np.zeros((R, C // per), dtype=np.uint32)
-    for j in range(per):
-        out |= c[:, j::per] << (j * bits)
+    out = np.zeros((R, C * bits // 8), dtype=np.uint64)
+    for k in range(C):
+        pos = k * bits
+        byte, off = pos // 8, pos % 8
+        v = c[:, k] << np.uint64(off)                     # at most 10 bits
+        out[:, byte] |= v & np.uint64(0xFF)
+        if off + bits > 8:
+            out[:, byte + 1] |= v >> np.uint64(8)
     return out.astype(np.uint8)
 
 
 def unpack_codes(packed, bits: int, C: int) -> np.ndarray:
-    p = np.asarray(packed, dtype=np.uint8).astype(np.uint32)
-    per = 8 // bits
-    mask = (1 << bits) - 1
-    out = np.zeros((p.shape[0], C), dtype=np.uint32)
-    for j in range(per):
-        out[:, j::per] = (p >> (j * bits)) & mask
+    p = np.asarray(packed, dtype=np.uint8).astype(np.uint64)
+    mask = np.uint64((1 << bits) - 1)
+    out = np.zeros((p.shape[0], C), dtype=np.uint64)
+    for k in range(C):
+        pos = k * bits
+        byte, off = pos // 8, pos % 8
+        v = p[:, byte] >> np.uint64(off)
+        if off + bits > 8:
+            v |= p[:, byte + 1] << np.uint64(8 - off)
+        out[:, k] = v & mask
     return out.astype(np.uint8)
 
 

@@ -206,7 +206,6 @@ omq_status omq_fold_pack(const void* W, omq_dtype wdt, int64_t N, int64_t K, int
   if (!packed) return OMQ_ERR_NULL;
   OMQ_TRY(check_lwc(W, wdt, N, K, group, bits, gamma_logit, beta_logit, s, OMQ_F32, nullptr,
                     packed, h, z));
-  if (bits == 3) return OMQ_ERR_UNSUPPORTED;
   LwcParams p{W, wdt, N, K, group, K / group, static_cast<float>((1 << bits) - 1), gamma_logit,
               beta_logit, s, nullptr, OMQ_F32, h, z, nullptr, nullptr, packed, bits};
   return launch_lwc(p, reinterpret_cast<cudaStream_t>(stream));

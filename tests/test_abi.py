@@ -84,9 +84,9 @@ def test_lwc_validation(omq):
     assert call(s=MISALIGNED) == 4
 
 
-def test_fold_pack_rejects_three_bits(omq):
+def test_fold_pack_validation(omq):
     lib = omq._lib
-    assert lib.omq_fold_pack(FAKE, 1, 16, 256, 128, 3, FAKE, FAKE, None, FAKE, FAKE, FAKE, None) == 8
+    assert lib.omq_fold_pack(FAKE, 1, 16, 256, 128, 5, FAKE, FAKE, None, FAKE, FAKE, FAKE, None) == 5
     assert lib.omq_fold_pack(FAKE, 1, 16, 256, 128, 4, FAKE, FAKE, None, None, FAKE, FAKE, None) == 1
 
 

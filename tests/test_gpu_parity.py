@@ -202,8 +202,7 @@ def test_calib_step_through_one_call(omq, cuda_device, case):
         check_update(lc.delta, p.delta.numpy(), r.d_delta, om.LR_LET)
 
 
-@pytest.mark.parametrize("case", [c for c in SMALL_CASES if c.bits in (2, 4, 8)],
-                         ids=lambda c: c.name)
+@pytest.mark.parametrize("case", SMALL_CASES, ids=lambda c: c.name)
 def test_fold_pack_bit_exact(omq, cuda_device, case):
     p = prepare(case)
     d = _dev(p, cuda_device)

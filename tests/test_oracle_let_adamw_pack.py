@@ -74,11 +74,15 @@ def test_pack_hand_examples():
     c2 = np.array([[1, 2, 3, 0, 3, 3, 3, 3]], np.uint8)
     assert om.pack_codes(c2, 2).tolist() == [[1 | 2 << 2 | 3 << 4, 0xFF]]
     assert om.pack_codes(np.array([[7, 200]], np.uint8), 8).tolist() == [[7, 200]]
+    # 3 bits: codes 1..7, 0 are the bit string 001 010 011 100 101 110 111 000 written from
+    # the least-significant end: byte 0 = 11|010|001, byte 1 = 0|101|100|0, byte 2 = 000|111|11
+    c3 = np.array([[1, 2, 3, 4, 5, 6, 7, 0]], np.uint8)
+    assert om.pack_codes(c3, 3).tolist() == [[0xD1, 0x58, 0x1F]]
     with pytest.raises(ValueError):
         om.pack_codes(np.zeros((1, 3), np.uint8), 4)
 
 
-@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
 def test_pack_roundtrip(bits):
     gen = np.random.default_rng(bits)
     c = gen.integers(0, 2 ** bits, size=(7, 64)).astype(np.uint8)
