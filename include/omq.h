@@ -103,7 +103,7 @@ omq_status omq_sync_check(omq_stream_t stream);
  * Outputs: W_hat [N,K] in `hat_dt` (bf16 holds the binary32 value rounded to nearest
  * even); h [N, K/group] float32; z [N, K/group] int32; codes [N,K] uint8 or NULL;
  * grp_range [N, K/group] or NULL (needed by omq_fq_linear_bwd).
- * Requires K % group == 0, group % 8 == 0, bits in {2,3,4,8}.
+ * Requires K % group == 0, group % 8 == 0, bits in 2..8.
  * ------------------------------------------------------------------------------------ */
 omq_status omq_lwc_quant(const void* W, omq_dtype wdt, int64_t N, int64_t K, int64_t group,
                          int bits, const float* gamma_logit, const float* beta_logit,
@@ -242,8 +242,8 @@ omq_status omq_adamw_step(float* param, const float* grad, float* m, float* v, i
  * ([ICLR] section 框架: the learned transforms fold back into the weights).
  * codes as in omq_lwc_quant, packed row-major: element k of a row occupies bits
  * k*bits .. k*bits + bits - 1 of the row's little-endian bit string (it starts in byte
- * k*bits/8 at bit offset (k*bits) mod 8, least-significant bits first; a 3-bit code may
- * straddle two bytes). packed [N, K*bits/8] uint8; h, z [N, K/group]. bits in {2,3,4,8}.
+ * k*bits/8 at bit offset (k*bits) mod 8, least-significant bits first; 3-, 5-, 6- and 7-bit
+ * codes may straddle two bytes). packed [N, K*bits/8] uint8; h, z [N, K/group]. bits 2..8.
  * ------------------------------------------------------------------------------------ */
 omq_status omq_fold_pack(const void* W, omq_dtype wdt, int64_t N, int64_t K, int64_t group,
                          int bits, const float* gamma_logit, const float* beta_logit,
@@ -332,7 +332,7 @@ typedef struct {
   int64_t H;       /* heads (head size 128) */
   int64_t I;       /* FFN size, a multiple of 32 */
   int64_t group;   /* LWC group length, a multiple of 32 dividing D and I; 0 = per channel */
-  int wbits;       /* 2, 3, 4 or 8 */
+  int wbits;       /* 2 .. 8 */
   int abits;       /* 2, 3, 4, 6, 8, or 16 (activations not quantized) */
 } omq_block_dims;
 
@@ -425,6 +425,44 @@ omq_status omq_block_step(const omq_block_args* args, void* workspace, size_t ws
 omq_status omq_block_reference(const omq_block_dims* dims, const void* x, const void* W_qkv,
                                const void* W_o, const void* W_gu, const void* W_d, float* y,
                                void* workspace, size_t ws_bytes, omq_stream_t stream);
+
+/* The block's output with the quantizers and transforms of theta (the fake-quantized block
+ * the calibration optimises): y [M, D] in y_dt (OMQ_F32 or OMQ_BF16, rounded once from
+ * binary32). This is what block-sequential calibration feeds to the next block ([ICLR]
+ * section 框架: a block is calibrated, then its quantized weights compute the next block's
+ * input). Same workspace as omq_block_step. */
+omq_status omq_block_quant_forward(const omq_block_dims* dims, const void* x, const void* W_qkv,
+                                   const void* W_o, const void* W_gu, const void* W_d,
+                                   const float* theta, void* y, omq_dtype y_dt, void* workspace,
+                                   size_t ws_bytes, omq_stream_t stream);
+
+/* One block's calibration ([ICLR] sections 框架 and 实验证据: AdamW over the calibration
+ * samples for a number of epochs, batch size 1): for epoch e < epochs, for sample i <
+ * n_samples in order, omq_block_step on (x_i, y_ref_i) followed by AdamW with step counter
+ * first_step + e * n_samples + i. Samples are stored back to back: xs [n_samples, M, D] BF16,
+ * y_refs [n_samples, M, D] float32. losses [epochs * n_samples] float32 receives each step's
+ * loss (device memory, written in step order). theta, adam_m, adam_v are updated in place;
+ * d_theta holds the last step's gradient. All on `stream`, one step after another. */
+typedef struct {
+  omq_block_dims dims;
+  const void* xs;
+  const float* y_refs;
+  int64_t n_samples;
+  int64_t epochs;
+  const void* W_qkv;
+  const void* W_o;
+  const void* W_gu;
+  const void* W_d;
+  float* theta;
+  float* d_theta;
+  float* adam_m;
+  float* adam_v;
+  int64_t first_step;     /* AdamW step counter of the first step, from 1 */
+  float lr_lwc, lr_let;
+  float* losses;
+} omq_block_calib_args;
+omq_status omq_block_calibrate(const omq_block_calib_args* args, void* workspace,
+                               size_t ws_bytes, omq_stream_t stream);
 
 /* Number of kernels this library has launched in this process (all threads, all devices),
  * counted on the host at each launch. */

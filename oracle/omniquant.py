@@ -367,11 +367,12 @@ LR_LET = 1e-2
 def pack_codes(codes, bits: int) -> np.ndarray:
     """Row-major bit packing: element k of a row occupies bits k*bits .. k*bits + bits - 1 of
     the row's little-endian bit string, i.e. it starts in byte (k*bits)//8 at bit offset
-    (k*bits) % 8, least-significant bits first; a 3-bit code may straddle two bytes.
-    Supports bits in {2, 3, 4, 8} with a row length whose bits fill whole bytes."""
+    (k*bits) % 8, least-significant bits first; a 3-, 5-, 6- or 7-bit code may straddle two
+    bytes.
+    Supports bits 2 to 8 with a row length whose bits fill whole bytes."""
     c = np.asarray(codes).astype(np.uint64)
     R, C = c.shape
-    if bits not in (2, 3, 4, 8) or (C * bits) % 8:
+    if not 2 <= bits <= 8 or (C * bits) % 8:
         raise ValueError("unsupported packing")
     out = np.zeros((R, C * bits // 8), dtype=np.uint64)
     for k in range(C):

@@ -70,15 +70,13 @@ __device__ __forceinline__ void encode8(const LwcParams& p, int64_t off, const f
 #pragma unroll
       for (int i = 0; i < 8; ++i) w |= c[i] << (2 * i);
       *reinterpret_cast<uint16_t*>(p.packed + off / 4) = static_cast<uint16_t>(w);
-    } else if (p.bits == 3) {
-      // 8 codes = 24 bits = 3 bytes, starting at byte 3 off / 8
-      uint32_t w = 0;
+    } else if (p.bits != 8) {
+      // 3, 5, 6 or 7 bits: 8 codes fill `bits` bytes starting at byte bits * off / 8
+      uint64_t w = 0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) w |= c[i] << (3 * i);
-      uint8_t* b = p.packed + off / 8 * 3;
-      b[0] = static_cast<uint8_t>(w);
-      b[1] = static_cast<uint8_t>(w >> 8);
-      b[2] = static_cast<uint8_t>(w >> 16);
+      for (int i = 0; i < 8; ++i) w |= static_cast<uint64_t>(c[i]) << (p.bits * i);
+      uint8_t* b = p.packed + off / 8 * p.bits;
+      for (int k = 0; k < p.bits; ++k) b[k] = static_cast<uint8_t>(w >> (8 * k));
     } else {  // 8 bits
       uint2 w;
       w.x = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);

@@ -78,7 +78,7 @@ T* at(void* base, size_t off) {
 }
 
 bool dtype_ok(omq_dtype d) { return d == OMQ_F32 || d == OMQ_BF16 || d == OMQ_F16; }
-bool wbits_ok(int b) { return b == 2 || b == 3 || b == 4 || b == 8; }
+bool wbits_ok(int b) { return b >= 2 && b <= 8; }
 bool abits_ok(int b) { return b == 2 || b == 3 || b == 4 || b == 6 || b == 8 || b == 16; }
 bool a16(const void* p) { return p == nullptr || aligned16(p); }
 

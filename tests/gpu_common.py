@@ -82,6 +82,7 @@ SMALL_CASES = [
          8),
     Case("f32_w4a4_perchannel_let", 72, 320, 136, 320, 4, 4, True, "f32", "llama7b_gateup_w4a4",
          9),
+    Case("bf16_w6a6_g64_let", 96, 320, 136, 64, 6, 6, True, "bf16", "llama7b_gateup_w4a4", 10),
 ]
 
 

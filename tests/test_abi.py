@@ -74,7 +74,7 @@ def test_lwc_validation(omq):
     assert call(W=None) == 1
     assert call(h=None) == 1
     assert call(wdt=7) == 3
-    assert call(bits=5) == 5
+    assert call(bits=9) == 5
     assert call(bits=1) == 5
     assert call(K=250) == 2            # not a multiple of the group
     assert call(group=12) == 2         # group not a multiple of 8
@@ -86,7 +86,7 @@ def test_lwc_validation(omq):
 
 def test_fold_pack_validation(omq):
     lib = omq._lib
-    assert lib.omq_fold_pack(FAKE, 1, 16, 256, 128, 5, FAKE, FAKE, None, FAKE, FAKE, FAKE, None) == 5
+    assert lib.omq_fold_pack(FAKE, 1, 16, 256, 128, 9, FAKE, FAKE, None, FAKE, FAKE, FAKE, None) == 5
     assert lib.omq_fold_pack(FAKE, 1, 16, 256, 128, 4, FAKE, FAKE, None, None, FAKE, FAKE, None) == 1
 
 

@@ -78,11 +78,15 @@ def test_pack_hand_examples():
     # the least-significant end: byte 0 = 11|010|001, byte 1 = 0|101|100|0, byte 2 = 000|111|11
     c3 = np.array([[1, 2, 3, 4, 5, 6, 7, 0]], np.uint8)
     assert om.pack_codes(c3, 3).tolist() == [[0xD1, 0x58, 0x1F]]
+    # 6 bits: 0x3F, 0x01, 0x20, 0x15 -> 111111 | 000001 | 100000 | 010101 from the low end:
+    # byte 0 = 01|111111, byte 1 = 0000|0000, byte 2 = 010101|10
+    c6 = np.array([[0x3F, 0x01, 0x20, 0x15]], np.uint8)
+    assert om.pack_codes(c6, 6).tolist() == [[0x7F, 0x00, 0x56]]
     with pytest.raises(ValueError):
         om.pack_codes(np.zeros((1, 3), np.uint8), 4)
 
 
-@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+@pytest.mark.parametrize("bits", [2, 3, 4, 5, 6, 7, 8])
 def test_pack_roundtrip(bits):
     gen = np.random.default_rng(bits)
     c = gen.integers(0, 2 ** bits, size=(7, 64)).astype(np.uint8)
