@@ -474,3 +474,34 @@ def block_step(sh: BlockShape, x, W, theta, y_ref):
             g["gamma_" + name] = np.zeros(n)
             g["beta_" + name] = np.zeros(n)
     return st["loss"], theta_join(sh, g), st, inter
+
+
+def block_calibrate(sh: BlockShape, xs, W, theta0, epochs: int, lr_lwc: float = om.LR_LWC,
+                    lr_let: float = om.LR_LET):
+    """One block's calibration ([ICLR] sections 框架, 实验证据): targets y*_i = the
+    full-precision block on each sample's input, then `epochs` passes over the samples in
+    order, each a block_step followed by AdamW (LWC logits at lr_lwc, LET vectors at lr_let;
+    the parameters kept in binary32 between steps, as a device vector holds them). Returns
+    (per-step losses, final theta float32, the samples' quantized block outputs float32)."""
+    theta = np.asarray(theta0, F32).copy()
+    n_lwc = dict(theta_layout(sh))
+    split = sum(n for name, n in theta_layout(sh) if name.startswith(("gamma", "beta")))
+    assert split == sum(n_lwc[k] for k in n_lwc if k.startswith(("gamma", "beta")))
+    m = np.zeros(theta.size)
+    v = np.zeros(theta.size)
+    y_refs = [block_reference(sh, x, W) for x in xs]
+    losses = []
+    t = 0
+    for _ in range(epochs):
+        for x, y_ref in zip(xs, y_refs):
+            t += 1
+            loss, g, _, _ = block_step(sh, x, W, theta, y_ref)
+            losses.append(loss)
+            p1, m[:split], v[:split] = om.adamw_step(theta[:split], g[:split], m[:split],
+                                                     v[:split], t, lr_lwc)
+            p2, m[split:], v[split:] = om.adamw_step(theta[split:], g[split:], m[split:],
+                                                     v[split:], t, lr_let)
+            theta = np.concatenate([p1, p2]).astype(F32)
+    th = theta_split(sh, theta)
+    outs = [block_forward(sh, x, W, th)["y"].astype(F32) for x in xs]
+    return np.array(losses), theta, outs

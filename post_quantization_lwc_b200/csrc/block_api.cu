@@ -38,7 +38,7 @@ bool dims_ok(const omq_block_dims& d) {
   return true;
 }
 bool bits_ok(const omq_block_dims& d) {
-  const bool w = d.wbits == 2 || d.wbits == 3 || d.wbits == 4 || d.wbits == 8;
+  const bool w = d.wbits >= 2 && d.wbits <= 8;
   const bool a = d.abits == 2 || d.abits == 3 || d.abits == 4 || d.abits == 6 || d.abits == 8 ||
                  d.abits == 16;
   return w && a;
@@ -248,8 +248,9 @@ struct Inputs {
   const void* x;
   const void* W[L_COUNT];
   const float* y_ref;   // NULL: forward only, y written to y_out
-  float* y_out;
+  void* y_out;
   const float* theta;   // NULL: the full-precision block
+  omq_dtype y_dt;       // of y_out
 };
 
 // Forward of the block (the formulas of omq.h). With theta NULL every quantizer and transform
@@ -363,8 +364,8 @@ omq_status block_forward(const View& v, const Inputs& in, const Marks& mk, cudaS
     GemmEpilogue e{};
     e.kind = Epi::MseLoss;
     e.y_ref = v.in<float>(L.tgt);
-    e.dy = in.y_ref ? v.bb<void>(OMQ_BB_RES) : static_cast<void*>(in.y_out);
-    e.dy_dt = in.y_ref ? OMQ_BF16 : OMQ_F32;
+    e.dy = in.y_ref ? v.bb<void>(OMQ_BB_RES) : in.y_out;
+    e.dy_dt = in.y_ref ? OMQ_BF16 : in.y_dt;
     e.loss_partials = v.in<float>(L.loss_part);
     BLK_TRY(gemm_tc(OMQ_BF16, GemmOperand{v.bb<void>(OMQ_BB_QM), I, false},
                     GemmOperand{Wop[L_D], I, false}, M, D, I, e, nullptr, st));
@@ -651,7 +652,7 @@ omq_status omq_block_step(const omq_block_args* a, void* workspace, size_t ws_by
   const BlockLayout L = block_layout(d);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const View v{d, L, workspace};
-  const Inputs in{a->x, {W[0], W[1], W[2], W[3]}, a->y_ref, nullptr, a->theta};
+  const Inputs in{a->x, {W[0], W[1], W[2], W[3]}, a->y_ref, nullptr, a->theta, OMQ_F32};
   const Marks mk{a->events, st};
   BLK_TRY(block_forward(v, in, mk, st));
   BLK_TRY(block_backward(v, in, a->d_theta, mk, st));
@@ -682,8 +683,60 @@ omq_status omq_block_reference(const omq_block_dims* dims, const void* x, const 
   const BlockLayout L = block_layout(*dims);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const View v{*dims, L, workspace};
-  const Inputs in{x, {W[0], W[1], W[2], W[3]}, nullptr, y, nullptr};
+  const Inputs in{x, {W[0], W[1], W[2], W[3]}, nullptr, y, nullptr, OMQ_F32};
   return block_forward(v, in, Marks{}, st);
+}
+
+omq_status omq_block_quant_forward(const omq_block_dims* dims, const void* x, const void* W_qkv,
+                                   const void* W_o, const void* W_gu, const void* W_d,
+                                   const float* theta, void* y, omq_dtype y_dt, void* workspace,
+                                   size_t ws_bytes, omq_stream_t stream) {
+  if (!dims || !y || !theta) return OMQ_ERR_NULL;
+  if (y_dt != OMQ_F32 && y_dt != OMQ_BF16) return OMQ_ERR_DTYPE;
+  const void* W[L_COUNT] = {W_qkv, W_o, W_gu, W_d};
+  BLK_TRY(check_common(*dims, x, W, workspace, ws_bytes));
+  if (!aligned16(y) || !aligned16(theta)) return OMQ_ERR_ALIGN;
+  const BlockLayout L = block_layout(*dims);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const View v{*dims, L, workspace};
+  // with theta and no target: every quantizer on, the down GEMM's epilogue writes y itself
+  const Inputs in{x, {W[0], W[1], W[2], W[3]}, nullptr, y, theta, y_dt};
+  return block_forward(v, in, Marks{}, st);
+}
+
+omq_status omq_block_calibrate(const omq_block_calib_args* c, void* workspace, size_t ws_bytes,
+                               omq_stream_t stream) {
+  if (!c) return OMQ_ERR_NULL;
+  if (!c->xs || !c->y_refs || !c->theta || !c->d_theta || !c->adam_m || !c->adam_v ||
+      !c->losses)
+    return OMQ_ERR_NULL;
+  if (c->n_samples < 1 || c->epochs < 1 || c->first_step < 1) return OMQ_ERR_SHAPE;
+  const omq_block_dims& d = c->dims;
+  if (!dims_ok(d)) return OMQ_ERR_SHAPE;
+  const int64_t xs_stride = d.M * d.D;                 // elements per sample
+  for (int64_t e = 0; e < c->epochs; ++e) {
+    for (int64_t i = 0; i < c->n_samples; ++i) {
+      const int64_t k = e * c->n_samples + i;
+      omq_block_args a{};
+      a.dims = d;
+      a.x = static_cast<const uint16_t*>(c->xs) + i * xs_stride;
+      a.y_ref = c->y_refs + i * xs_stride;
+      a.W_qkv = c->W_qkv;
+      a.W_o = c->W_o;
+      a.W_gu = c->W_gu;
+      a.W_d = c->W_d;
+      a.theta = c->theta;
+      a.d_theta = c->d_theta;
+      a.loss = c->losses + k;
+      a.adam_m = c->adam_m;
+      a.adam_v = c->adam_v;
+      a.step = c->first_step + k;
+      a.lr_lwc = c->lr_lwc;
+      a.lr_let = c->lr_let;
+      BLK_TRY(omq_block_step(&a, workspace, ws_bytes, stream));
+    }
+  }
+  return OMQ_OK;
 }
 
 }  // extern "C"

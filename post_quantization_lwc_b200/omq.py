@@ -31,7 +31,8 @@ EXPORTS = ("omq_status_str", "omq_last_cuda_error", "omq_version", "omq_sync_che
            "omq_fq_linear_bwd", "omq_bwd_workspace_bytes", "omq_adamw_step", "omq_fold_pack",
            "omq_calib_step", "omq_step_workspace_bytes", "omq_launch_count",
            "omq_fq_linear_fwd_noalloc", "omq_block_theta_range", "omq_block_buffer",
-           "omq_block_workspace_bytes", "omq_block_step", "omq_block_reference")
+           "omq_block_workspace_bytes", "omq_block_step", "omq_block_reference",
+           "omq_block_quant_forward", "omq_block_calibrate")
 
 _p = ctypes.c_void_p
 _i64 = ctypes.c_int64
@@ -86,6 +87,13 @@ class BlockArgs(ctypes.Structure):
                 ("lr_let", _f32), ("events", _p)]
 
 
+class BlockCalibArgs(ctypes.Structure):
+    _fields_ = [("dims", BlockDims), ("xs", _p), ("y_refs", _p), ("n_samples", _i64),
+                ("epochs", _i64), ("W_qkv", _p), ("W_o", _p), ("W_gu", _p), ("W_d", _p),
+                ("theta", _p), ("d_theta", _p), ("adam_m", _p), ("adam_v", _p),
+                ("first_step", _i64), ("lr_lwc", _f32), ("lr_let", _f32), ("losses", _p)]
+
+
 # phases of omq_calib_step (OMQ_PH_* in include/omq.h), in order
 PHASES = ("let", "lwc", "fwd_gemm", "loss", "dbias", "dw_gemm", "ste_w", "dx_gemm", "ste_x",
           "let_reduce", "adamw")
@@ -123,6 +131,9 @@ _sig("omq_block_workspace_bytes", _sz, [ctypes.POINTER(BlockDims)])
 _sig("omq_block_step", _i32, [ctypes.POINTER(BlockArgs), _p, _sz, _p])
 _sig("omq_block_reference", _i32, [ctypes.POINTER(BlockDims), _p, _p, _p, _p, _p, _p, _p, _sz,
                                    _p])
+_sig("omq_block_quant_forward", _i32, [ctypes.POINTER(BlockDims), _p, _p, _p, _p, _p, _p, _p,
+                                       _i32, _p, _sz, _p])
+_sig("omq_block_calibrate", _i32, [ctypes.POINTER(BlockCalibArgs), _p, _sz, _p])
 
 
 def _check(status: int, where: str):
@@ -521,10 +532,12 @@ class Block:
         self.adam_v.zero_()
         self.t = 0
 
-    def reference(self, x, stream=None):
-        """omq_block_reference: the full-precision block output y* [M, D] float32."""
-        _dev(x)
-        y = torch.empty(self.dims.M, self.dims.D, dtype=torch.float32, device=self.device)
+    def reference(self, x, out=None, stream=None):
+        """omq_block_reference: the full-precision block output y* [M, D] float32 (written
+        into `out` when given)."""
+        _dev(x, out)
+        y = out if out is not None else torch.empty(self.dims.M, self.dims.D,
+                                                    dtype=torch.float32, device=self.device)
         _check(_lib.omq_block_reference(ctypes.byref(self.dims), _ptr(x), _ptr(self.W["qkv"]),
                                         _ptr(self.W["o"]), _ptr(self.W["gu"]), _ptr(self.W["d"]),
                                         _ptr(y), _ptr(self.workspace), self.workspace.numel(),
@@ -548,3 +561,51 @@ class Block:
         _check(_lib.omq_block_step(ctypes.byref(a), _ptr(self.workspace), self.workspace.numel(),
                                    _stream(stream)), "omq_block_step")
         return self.loss
+
+    def quant_forward(self, x, dtype=torch.float32, out=None, stream=None):
+        """omq_block_quant_forward: the fake-quantized block's output at the current theta
+        (written into `out`, float32 or bfloat16, when given)."""
+        _dev(x, out)
+        y = out if out is not None else torch.empty(self.dims.M, self.dims.D, dtype=dtype,
+                                                    device=self.device)
+        _check(_lib.omq_block_quant_forward(ctypes.byref(self.dims), _ptr(x), _ptr(self.W["qkv"]),
+                                            _ptr(self.W["o"]), _ptr(self.W["gu"]),
+                                            _ptr(self.W["d"]), _ptr(self.theta), _ptr(y), _dt(y),
+                                            _ptr(self.workspace), self.workspace.numel(),
+                                            _stream(stream)), "omq_block_quant_forward")
+        return y
+
+    def calibrate(self, xs, y_refs, epochs, stream=None):
+        """omq_block_calibrate: `epochs` passes over the samples xs [S, M, D] (BF16) with
+        targets y_refs [S, M, D] (float32), one step and AdamW update per sample. Returns the
+        per-step losses [epochs * S] (device tensor)."""
+        _dev(xs, y_refs)
+        S = xs.shape[0]
+        losses = torch.empty(epochs * S, dtype=torch.float32, device=self.device)
+        a = BlockCalibArgs(dims=self.dims, xs=_ptr(xs), y_refs=_ptr(y_refs), n_samples=S,
+                           epochs=epochs, W_qkv=_ptr(self.W["qkv"]), W_o=_ptr(self.W["o"]),
+                           W_gu=_ptr(self.W["gu"]), W_d=_ptr(self.W["d"]), theta=_ptr(self.theta),
+                           d_theta=_ptr(self.d_theta), adam_m=_ptr(self.adam_m),
+                           adam_v=_ptr(self.adam_v), first_step=self.t + 1, lr_lwc=self.lr_lwc,
+                           lr_let=self.lr_let, losses=_ptr(losses))
+        _check(_lib.omq_block_calibrate(ctypes.byref(a), _ptr(self.workspace),
+                                        self.workspace.numel(), _stream(stream)),
+               "omq_block_calibrate")
+        self.t += epochs * S
+        return losses
+
+    def fold(self, stream=None):
+        """omq_fold_pack of the four weights at the current theta (each with its linear's LET
+        scale): dict name -> (packed codes, h, z)."""
+        d = self.dims
+        s_of = {"qkv": "s1", "o": "s_o", "gu": "s2", "d": None}
+        out = {}
+        for name, W in self.W.items():
+            K = W.shape[1]
+            G = K if d.group == 0 else d.group
+            rows = W.shape[0]
+            s = self.theta_part(s_of[name]) if s_of[name] else None
+            gl = self.theta_part("gamma_" + name).view(rows, K // G)
+            bl = self.theta_part("beta_" + name).view(rows, K // G)
+            out[name] = fold_pack(W, gl, bl, d.wbits, G, s=s, stream=stream)
+        return out

@@ -304,3 +304,17 @@ def test_stage_functions_compose():
     P, O = ob.stage_attention(ap["Qq"], ap["Qk"], ap["Qv"], sh.H)
     np.testing.assert_array_equal(O.astype(np.float32), st["O32"])
     assert om.F32 is np.float32
+
+
+def test_block_calibrate_is_steps_then_adamw():
+    """One epoch over one sample: the loss of block_step, then AdamW from zero moments (whose
+    first step moves every parameter by -lr sign(g) up to eps: the bias corrections cancel)."""
+    sh = SHAPES[1]
+    x, W, theta = make_case(sh, 77)
+    losses, theta1, _ = ob.block_calibrate(sh, [x], W, theta, 1)
+    loss, g, _, _ = ob.block_step(sh, x, W, theta, ob.block_reference(sh, x, W))
+    assert losses[0] == loss
+    split = sum(n for name, n in ob.theta_layout(sh) if name.startswith(("gamma", "beta")))
+    lr = np.where(np.arange(theta.size) < split, om.LR_LWC, om.LR_LET)
+    step = lr * g / (np.abs(g) + 1e-8)
+    np.testing.assert_allclose(theta1, (theta - step).astype(np.float32), rtol=0, atol=1e-6)
