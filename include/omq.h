@@ -251,6 +251,19 @@ omq_status omq_fold_pack(const void* W, omq_dtype wdt, int64_t N, int64_t K, int
                          omq_stream_t stream);
 
 /* ------------------------------------------------------------------------------------
+ * omq_qgemv — inference with the folded weights for a few tokens ([ICLR] section 框架: the
+ * learned transforms fold into the weights; the quantized model runs as an ordinary low-bit
+ * model):  y[m, n] = sum_k x[m, k] (c[n, k] - z[n, k/group]) h[n, k/group]
+ * x [M, K] in xdt (the linear's input after its folded LET, i.e. (X - delta)/s), packed /
+ * h / z as written by omq_fold_pack, y [M, N] float32 (add B~ for the bias). bits in {2, 4, 8},
+ * 1 <= M <= 8, group a multiple of 128/bits, K a multiple of group, M (K + K bits/128) floats
+ * of shared memory at most 200 KiB. Decode-shaped: memory-bound on the codes.
+ * ------------------------------------------------------------------------------------ */
+omq_status omq_qgemv(const void* x, omq_dtype xdt, int64_t M, int64_t K, const uint8_t* packed,
+                     const float* h, const int32_t* z, int64_t N, int64_t group, int bits,
+                     float* y, omq_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
  * omq_calib_step — one whole calibration step on one stream: omq_let_apply (when LET is
  * on or abits < 16), omq_lwc_quant, omq_fq_linear_fwd, omq_fq_linear_bwd, then AdamW on
  * the logits (lr_lwc) and, with LET, on s and delta (lr_let). `step` counts from 1.

@@ -32,7 +32,7 @@ EXPORTS = ("omq_status_str", "omq_last_cuda_error", "omq_version", "omq_sync_che
            "omq_calib_step", "omq_step_workspace_bytes", "omq_launch_count",
            "omq_fq_linear_fwd_noalloc", "omq_block_theta_range", "omq_block_buffer",
            "omq_block_workspace_bytes", "omq_block_step", "omq_block_reference",
-           "omq_block_quant_forward", "omq_block_calibrate")
+           "omq_block_quant_forward", "omq_block_calibrate", "omq_qgemv")
 
 _p = ctypes.c_void_p
 _i64 = ctypes.c_int64
@@ -134,6 +134,7 @@ _sig("omq_block_reference", _i32, [ctypes.POINTER(BlockDims), _p, _p, _p, _p, _p
 _sig("omq_block_quant_forward", _i32, [ctypes.POINTER(BlockDims), _p, _p, _p, _p, _p, _p, _p,
                                        _i32, _p, _sz, _p])
 _sig("omq_block_calibrate", _i32, [ctypes.POINTER(BlockCalibArgs), _p, _sz, _p])
+_sig("omq_qgemv", _i32, [_p, _i32, _i64, _i64, _p, _p, _p, _i64, _i64, _i32, _p, _p])
 
 
 def _check(status: int, where: str):
@@ -326,6 +327,17 @@ def fold_pack(W, gamma_logit, beta_logit, bits, group, s=None, stream=None):
                               _ptr(beta_logit), _ptr(s), _ptr(packed), _ptr(h), _ptr(z),
                               _stream(stream)), "omq_fold_pack")
     return packed, h, z
+
+
+def qgemv(x, packed, h, z, group, bits, stream=None):
+    """omq_qgemv: y [M, N] float32 = x dequant(packed, h, z)^T for 1..8 tokens."""
+    _dev(x, packed, h, z)
+    M, K = x.shape
+    N = packed.shape[0]
+    y = torch.empty(M, N, dtype=torch.float32, device=x.device)
+    _check(_lib.omq_qgemv(_ptr(x), _dt(x), M, K, _ptr(packed), _ptr(h), _ptr(z), N, group, bits,
+                          _ptr(y), _stream(stream)), "omq_qgemv")
+    return y
 
 
 def step_workspace_bytes(M, N, K, group) -> int:
