@@ -15,6 +15,9 @@
 //     group staged in shared memory as fp32, block reductions.
 #include <float.h>
 
+#include <algorithm>
+#include <mutex>
+
 #include "omq_internal.cuh"
 
 namespace omq {
@@ -290,90 +293,474 @@ __device__ __forceinline__ void scale8(const float* s, int64_t col, float (&v)[8
   for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(v[i], sv[i]);
 }
 
-// One group per row (per-channel), 16-bit W, K a multiple of 256 up to 4096: one warp per
-// row, persistent warps taking rows in equal shares. Lane l holds columns 256 i + 8 l .. + 7
-// of every 256-column segment i (coalesced 16-byte loads, all issued before any is used, the
-// row kept packed in registers), so the max / min, the tie counts and the codes come from
-// one read of W; B~[n] = B[n] + sum_k W[n,k] delta[k] (when requested) from the same data.
-constexpr int kRowSegs = 16;
+// ---- row-staged launch shape -----------------------------------------------------------
+// 16-bit W and W^, groups of 32, 64, 128 or 256 columns or one group per row. One warp per
+// row, persistent warps: the row is copied into the warp's shared-memory buffer by 16-byte
+// cp.async copies (the next row's copies in flight while this one is encoded, when two
+// buffers fit), then walked in 256-column segments by a rolled loop, lane l holding columns
+// 256 i + 8 l .. + 7 of segment i. A group of G = 8 LPG columns is a sub-warp of LPG lanes;
+// one group per row (LPG = 0) takes two passes over the staged row (max / min, then the
+// encoder). B~[n] = B[n] + sum_k W[n,k] delta[k] comes out of the same pass over the row.
 
-__global__ void __launch_bounds__(256, 2) lwc_row_kernel(LwcParams p, int64_t rows_per_warp) {
-  const int lane = threadIdx.x & 31;
-  const int64_t warp_g = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t n_warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-  const int S = static_cast<int>(p.K / 256);
-  const bool f16 = p.wdt == OMQ_F16;
-  for (int64_t it = 0; it < rows_per_warp; ++it) {
-    const int64_t n = warp_g + it * n_warps;
-    if (n >= p.N) break;                                  // warp-uniform
-    const uint4* wrow = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.W) + n * p.K) + lane;
-    uint4 raw[kRowSegs];
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(a), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* smem, const void* gmem) {
+  const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(a), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;\n" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
+// three-input maximum / minimum (one instruction on sm_100)
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float min3f(float a, float b, float c) {
+  float d;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Packed binary32 pairs (the sm_100 f32x2 operations: two IEEE round-to-nearest results
+// per instruction, each exactly the scalar operation's).
+__device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
+__device__ __forceinline__ void unpack16x8_x2(const uint4& q, bool f16, float2 (&V)[4]) {
+  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-    for (int i = 0; i < kRowSegs; ++i)
-      if (i < S) raw[i] = __ldg(wrow + 32 * i);
-    float vmax = -FLT_MAX, vmin = FLT_MAX;
+  for (int j = 0; j < 4; ++j)
+    V[j] = f16 ? __half22float2(*reinterpret_cast<const __half2*>(&w[j]))
+               : __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[j]));
+}
+__device__ __forceinline__ void load_f8_x2(const float* p, int64_t off, float2 (&S)[4]) {
+  const float4* q = reinterpret_cast<const float4*>(p + off);
+  const float4 a = q[0], b = q[1];
+  S[0] = make_float2(a.x, a.y); S[1] = make_float2(a.z, a.w);
+  S[2] = make_float2(b.x, b.y); S[3] = make_float2(b.z, b.w);
+}
+__device__ __forceinline__ float max8(const float2 (&V)[4], float init) {
+  return max3f(max3f(V[0].x, V[0].y, V[1].x), max3f(V[1].y, V[2].x, V[2].y),
+               max3f(V[3].x, V[3].y, init));
+}
+__device__ __forceinline__ float min8(const float2 (&V)[4], float init) {
+  return min3f(min3f(V[0].x, V[0].y, V[1].x), min3f(V[1].y, V[2].x, V[2].y),
+               min3f(V[3].x, V[3].y, init));
+}
+// 1.0f where a == b, else 0.0f (one compare-and-set)
+__device__ __forceinline__ float eqf(float a, float b) {
+  float d;
+  asm("set.eq.f32.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
+}
+// ties at the extremes of 8 values: count(v == vmax) + 512 count(v == vmin), exact in
+// binary32 while the counts stay below 512
+__device__ __forceinline__ float ties8(const float2 (&V)[4], float vmax, float vmin) {
+  float2 t[4];
 #pragma unroll
-    for (int i = 0; i < kRowSegs; ++i) {
-      if (i >= S) break;
-      float v[8];
-      unpack16x8(raw[i], f16, v);
-      if (p.s) scale8(p.s, 256 * i + 8 * lane, v);
+  for (int j = 0; j < 4; ++j)
+    t[j] = __ffma2_rn(make_float2(eqf(V[j].x, vmin), eqf(V[j].y, vmin)), f2(512.f),
+                      make_float2(eqf(V[j].x, vmax), eqf(V[j].y, vmax)));
+  const float2 u = __fadd2_rn(__fadd2_rn(t[0], t[1]), __fadd2_rn(t[2], t[3]));
+  return __fadd_rn(u.x, u.y);
+}
+
+// A group's encoder constants. thr: the largest |ua - r| the fast path accepts (see
+// encode8_x2), 0.49999 - A 2^-22 with A = max(|vmax|, |vmin|) / h bounding |ua| over the
+// group; -1 (no element fast) unless A < 2^20 and |z| < 2^21.
+struct StageQ {
+  float h, hinv, z, thr;
+};
+__device__ __forceinline__ StageQ stage_q(const GroupQ& q, float vmax, float vmin) {
+  StageQ r{q.h, __frcp_rn(q.h), q.z, -1.f};
+  const float A = __fmul_rn(fmaxf(fabsf(vmax), fabsf(vmin)), r.hinv);
+  if (fabsf(q.z) < 2097152.f && A < 1048576.f)
+    r.thr = __fsub_rn(0.49999f, __fmul_rn(A, 2.384185791015625e-07f));
+  return r;
+}
+
+// The encoder of encode8 for 8 values of one group, W^ packed as 16-bit values.
+//
+// Fast path: ua = v*hinv (hinv = 1/h correctly rounded) is within 3.0001*2^-24 |ua| <
+// 2^-22 A of the correctly rounded quotient v/h (A bounds |ua| over the group, A < 2^20).
+// t = ua + (B + z), B = 1.5*2^23, |z| < 2^21, lies in [2^23, 2^24) where binary32 integers
+// are spaced 1 apart, so t - (B + z) = r is an integer next to ua and d = ua - r is exact;
+// |d| <= thr = 0.49999 - 2^-22 A (thr itself within 2^-25 of that) then puts v/h strictly
+// inside r's rounding interval, so r = rint(v/h) (a tie of ua, or of the addition, has
+// |d| = 1/2 and fails the check). The code stays biased: clamp(t, B, B + Q) = B + clamp(r
+// + z, 0, Q), and W^ = (clamp - (B + z)) h, every sum exact, so the result is bitwise that
+// of the plain order (round, add z, clamp, subtract z, multiply by h). A lane with an
+// element outside the check (about 2e-5 + 5e-7 A of them), or of a group outside the
+// bounds, redoes its 8 values in the plain order with the IEEE quotient where needed.
+__device__ __forceinline__ uint4 encode8_x2(const float2 (&V)[4], const StageQ& q, float Q,
+                                            bool hat_f16) {
+  constexpr float kBias = 12582912.f;                  // 1.5 * 2^23
+  const float cz = __fadd_rn(kBias, q.z), top = __fadd_rn(kBias, Q);
+  bool slow = false;
+  float2 deq[4];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) { vmax = fmaxf(vmax, v[e]); vmin = fminf(vmin, v[e]); }
-    }
+  for (int j = 0; j < 4; ++j) {
+    const float2 ua = __fmul2_rn(V[j], f2(q.hinv));
+    const float2 t = __fadd2_rn(ua, f2(cz));
+    const float2 r = __fadd2_rn(t, f2(-cz));
+    const float2 d = __ffma2_rn(r, f2(-1.f), ua);
+    slow |= !(fabsf(d.x) <= q.thr) || !(fabsf(d.y) <= q.thr);
+    const float2 cb = make_float2(fminf(fmaxf(t.x, kBias), top), fminf(fmaxf(t.y, kBias), top));
+    deq[j] = __fmul2_rn(__fadd2_rn(cb, f2(-cz)), f2(q.h));
+  }
+  if (__any_sync(0xffffffffu, slow)) {
+    if (slow) {
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
-      vmin = fminf(vmin, __shfl_xor_sync(0xffffffffu, vmin, o));
-    }
-    float st = 1.f;
-    if (lane < 2) st = strength((lane ? p.bl : p.gl)[n]);
-    const float g = __shfl_sync(0xffffffffu, st, 0), b = __shfl_sync(0xffffffffu, st, 1);
-    const GroupQ q = group_params(g, b, vmax, vmin, p.Q);
-    int cnt = 0;                                          // nmax | nmin << 16
-    float bias = 0.f;
+      for (int j = 0; j < 4; ++j) {
+        float* dj = reinterpret_cast<float*>(&deq[j]);
+        const float vj[2] = {V[j].x, V[j].y};
 #pragma unroll
-    for (int i = 0; i < kRowSegs; ++i) {
-      if (i >= S) break;
-      const int64_t col = 256 * i + 8 * lane;
-      float v[8];
-      unpack16x8(raw[i], f16, v);
-      if (p.Bt && p.delta) {
-        float d[8];
-        load_f8(p.delta, col, d);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) bias += v[e] * d[e];
+        for (int e = 0; e < 2; ++e) {
+          const float r = round_quotient(vj[e], q.h, q.hinv);
+          const float cc = fminf(fmaxf(__fadd_rn(r, q.z), 0.f), Q);
+          dj[e] = __fmul_rn(__fsub_rn(cc, q.z), q.h);
+        }
       }
-      if (p.s) scale8(p.s, col, v);
+    }
+  }
+  uint4 out;
+  uint32_t* w = reinterpret_cast<uint32_t*>(&out);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) cnt += (v[e] == vmax ? 1 : 0) + (v[e] == vmin ? 0x10000 : 0);
-      encode8(p, n * p.K + col, v, q);
+  for (int j = 0; j < 4; ++j) {
+    if (hat_f16) {
+      const __half2 x = __float22half2_rn(deq[j]);
+      w[j] = *reinterpret_cast<const uint32_t*>(&x);
+    } else {
+      const __nv_bfloat162 x = __float22bfloat162_rn(deq[j]);
+      w[j] = *reinterpret_cast<const uint32_t*>(&x);
     }
+  }
+  return out;
+}
+
+constexpr int kStageSegs = 4;   // 256-column segments a grouped batch holds in registers
+
+// Warps a block may hold: one group per row keeps few registers and takes more warps.
+constexpr int stage_max_warps(int lpg) { return lpg == 0 ? 24 : 16; }
+
+template <int LPG, bool F16>
+__global__ void __launch_bounds__(32 * stage_max_warps(LPG))
+    lwc_stage_kernel(LwcParams p, int nbuf, int64_t rows_per_warp) {
+  extern __shared__ __align__(16) unsigned char lsm[];
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5, wpb = blockDim.x >> 5;
+  const int64_t K = p.K, ng = p.ng, chunks = K / 8;
+  uint16_t* rows = reinterpret_cast<uint16_t*>(lsm) + static_cast<int64_t>(wib) * nbuf * K;
+  // grouped: per warp, nbuf staged copies of the row's logits (gamma then beta), then the
+  // row's strengths (gamma, beta of each group interleaved)
+  float* lgb = reinterpret_cast<float*>(lsm + static_cast<size_t>(wpb) * nbuf * K * 2) +
+               static_cast<int64_t>(wib) * (nbuf + 1) * 2 * ng;
+  float* sst = lgb + nbuf * 2 * ng;
+  // warp w of block b is warp w * gridDim.x + b, so a partial last round of rows spreads
+  // over all blocks
+  const int64_t n_warps = static_cast<int64_t>(gridDim.x) * wpb;
+  const int64_t wg = static_cast<int64_t>(wib) * gridDim.x + blockIdx.x;
+  const bool hat_f16 = p.hat_dt == OMQ_F16;
+  const bool let = p.s != nullptr, bias_on = p.Bt != nullptr && p.delta != nullptr;
+  auto issue = [&](int64_t it) {
+    const int64_t n = wg + it * n_warps;
+    if (it < rows_per_warp && n < p.N) {
+      const unsigned char* src = static_cast<const unsigned char*>(p.W) + n * K * 2;
+      uint16_t* dst = rows + (it % nbuf) * K;
+      for (int64_t c = lane; c < chunks; c += 32) cp_async16(dst + c * 8, src + c * 16);
+      if constexpr (LPG != 0) {
+        float* lg = lgb + (it % nbuf) * 2 * ng;
+        for (int64_t i = lane; i < 2 * ng; i += 32)
+          cp_async4(lg + i, i < ng ? p.gl + n * ng + i : p.bl + n * ng + (i - ng));
+      }
+    }
+    cp_async_commit();
+  };
+  issue(0);
+  for (int64_t it = 0; it < rows_per_warp; ++it) {
+    const int64_t n = wg + it * n_warps;
+    if (n >= p.N) break;                                       // warp-uniform
+    if (nbuf == 2) {
+      issue(it + 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncwarp();
+    const uint16_t* row = rows + (it % nbuf) * K;
+    uint16_t* hat = static_cast<uint16_t*>(p.W_hat) + n * K;
+    float2 bias2 = make_float2(0.f, 0.f);
+    if constexpr (LPG == 0) {
+      // one group per row: max / min over the staged row, then the encoder
+      float st = 1.f;
+      if (lane < 2) st = strength((lane ? p.bl : p.gl)[n]);
+      float vmax = -FLT_MAX, vmin = FLT_MAX;
+#pragma unroll 2
+      for (int64_t c0 = 0; c0 < chunks; c0 += 32) {
+        const int64_t c = c0 + lane;
+        if (c < chunks) {
+          float2 V[4];
+          unpack16x8_x2(*reinterpret_cast<const uint4*>(row + c * 8), F16, V);
+          if (let) {
+            float2 S[4];
+            load_f8_x2(p.s, c * 8, S);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-      bias += __shfl_xor_sync(0xffffffffu, bias, o);
+            for (int j = 0; j < 4; ++j) V[j] = __fmul2_rn(V[j], S[j]);
+          }
+          vmax = max8(V, vmax);
+          vmin = min8(V, vmin);
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+        vmin = fminf(vmin, __shfl_xor_sync(0xffffffffu, vmin, o));
+      }
+      const float g = __shfl_sync(0xffffffffu, st, 0), b = __shfl_sync(0xffffffffu, st, 1);
+      const GroupQ gq = group_params(g, b, vmax, vmin, p.Q);
+      const StageQ q = stage_q(gq, vmax, vmin);
+      int nmax = 0, nmin = 0;
+      // the next round's row chunk, scale and shift are loaded before this round's store
+      uint4 nraw = make_uint4(0u, 0u, 0u, 0u);
+      float2 nS[4], nD[4];
+      auto fetch = [&](int64_t c) {
+        nraw = *reinterpret_cast<const uint4*>(row + c * 8);
+        if (let) load_f8_x2(p.s, c * 8, nS);
+        if (bias_on) load_f8_x2(p.delta, c * 8, nD);
+      };
+      if (lane < chunks) fetch(lane);
+      for (int64_t c0 = 0; c0 < chunks; c0 += 32) {
+        const int64_t c = c0 + lane;
+        const bool ok = c < chunks;
+        const uint4 raw = nraw;
+        float2 S[4], D[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) { S[j] = nS[j]; D[j] = nD[j]; }
+        if (c + 32 < chunks) fetch(c + 32);
+        float2 V[4];
+        if (ok) {
+          unpack16x8_x2(raw, F16, V);
+          if (bias_on) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) bias2 = __ffma2_rn(V[j], D[j], bias2);
+          }
+          if (let) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) V[j] = __fmul2_rn(V[j], S[j]);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) V[j] = make_float2(0.f, 0.f);
+        }
+        // ties are counted only in the rare rounds where some lane's 8 values reach an
+        // extreme of the row
+        const bool ext = ok && (max8(V, V[0].x) == vmax || min8(V, V[0].x) == vmin);
+        if (__any_sync(0xffffffffu, ext)) {
+          if (ext) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              nmax += (V[j].x == vmax) + (V[j].y == vmax);
+              nmin += (V[j].x == vmin) + (V[j].y == vmin);
+            }
+          }
+        }
+        const uint4 out = encode8_x2(V, q, p.Q, hat_f16);
+        if (ok) *reinterpret_cast<uint4*>(hat + c * 8) = out;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        nmax += __shfl_xor_sync(0xffffffffu, nmax, o);
+        nmin += __shfl_xor_sync(0xffffffffu, nmin, o);
+      }
+      if (lane == 0) {
+        if (p.h) p.h[n] = q.h;
+        if (p.z) p.z[n] = z_to_i32(q.z);
+        if (p.range) p.range[n] = omq_range{vmax, vmin, nmax, nmin};
+      }
+    } else {
+      // groups of 8 LPG columns: kStageSegs segments at a time; the batch's GPB groups get
+      // their parameters from one lane each (lane t serves group t % GPB) and hand them back
+      // by shuffles
+      constexpr int GPS = 32 / LPG, GPB = kStageSegs * GPS;
+      static_assert(GPB <= 32, "one lane per group of a batch");
+      const float* lg = lgb + (it % nbuf) * 2 * ng;
+      for (int64_t i = lane; i < 2 * ng; i += 32)
+        sst[i] = strength(lg[(i & 1) * ng + (i >> 1)]);
+      __syncwarp();
+      const int64_t nseg = (K + 255) / 256;
+      for (int64_t s0 = 0; s0 < nseg; s0 += kStageSegs) {
+        float2 V[kStageSegs][4];
+        float vmx[kStageSegs], vmn[kStageSegs], cnt[kStageSegs];
+#pragma unroll
+        for (int u = 0; u < kStageSegs; ++u) {
+          const int64_t col = (s0 + u) * 256 + lane * 8;
+          if (col < K) {     // whole groups: a group's lanes are all in or all out
+            unpack16x8_x2(*reinterpret_cast<const uint4*>(row + col), F16, V[u]);
+            if (bias_on) {
+              float2 D[4];
+              load_f8_x2(p.delta, col, D);
+#pragma unroll
+              for (int j = 0; j < 4; ++j) bias2 = __ffma2_rn(V[u][j], D[j], bias2);
+            }
+            if (let) {
+              float2 S[4];
+              load_f8_x2(p.s, col, S);
+#pragma unroll
+              for (int j = 0; j < 4; ++j) V[u][j] = __fmul2_rn(V[u][j], S[j]);
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) V[u][j] = make_float2(0.f, 0.f);
+          }
+          vmx[u] = max8(V[u], V[u][0].x);
+          vmn[u] = min8(V[u], V[u][0].x);
+#pragma unroll
+          for (int o = LPG / 2; o > 0; o >>= 1) {
+            vmx[u] = fmaxf(vmx[u], __shfl_xor_sync(0xffffffffu, vmx[u], o));
+            vmn[u] = fminf(vmn[u], __shfl_xor_sync(0xffffffffu, vmn[u], o));
+          }
+          cnt[u] = ties8(V[u], vmx[u], vmn[u]);
+#pragma unroll
+          for (int o = LPG / 2; o > 0; o >>= 1)
+            cnt[u] = __fadd_rn(cnt[u], __shfl_xor_sync(0xffffffffu, cnt[u], o));
+        }
+        // this lane's group of the batch: segment ut, sub-warp sg
+        const int gb = lane % GPB, ut = gb / GPS, sg = gb % GPS, src = sg * LPG;
+        float gmx = 0.f, gmn = 0.f, gc = 0.f;
+#pragma unroll
+        for (int u = 0; u < kStageSegs; ++u) {
+          const float x = __shfl_sync(0xffffffffu, vmx[u], src);
+          const float y = __shfl_sync(0xffffffffu, vmn[u], src);
+          const float c = __shfl_sync(0xffffffffu, cnt[u], src);
+          if (u == ut) { gmx = x; gmn = y; gc = c; }
+        }
+        const int64_t j = (s0 + ut) * GPS + sg;                  // group within the row
+        StageQ gq{H_FLOOR, 0.f, 0.f, 0.4f};
+        if (j < ng) {
+          const GroupQ q = group_params(sst[2 * j], sst[2 * j + 1], gmx, gmn, p.Q);
+          gq = stage_q(q, gmx, gmn);
+          if (lane < GPB) {
+            const int64_t gi = n * ng + j;
+            const int ic = static_cast<int>(gc);
+            if (p.h) p.h[gi] = q.h;
+            if (p.z) p.z[gi] = z_to_i32(q.z);
+            if (p.range) p.range[gi] = omq_range{gmx, gmn, ic & 511, ic >> 9};
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < kStageSegs; ++u) {
+          const int holder = u * GPS + lane / LPG;
+          StageQ q;
+          q.h = __shfl_sync(0xffffffffu, gq.h, holder);
+          q.hinv = __shfl_sync(0xffffffffu, gq.hinv, holder);
+          q.z = __shfl_sync(0xffffffffu, gq.z, holder);
+          q.thr = __shfl_sync(0xffffffffu, gq.thr, holder);
+          const uint4 out = encode8_x2(V[u], q, p.Q, hat_f16);
+          const int64_t col = (s0 + u) * 256 + lane * 8;
+          if (col < K) *reinterpret_cast<uint4*>(hat + col) = out;
+        }
+      }
     }
-    if (lane == 0) {
-      if (p.h) p.h[n] = q.h;
-      if (p.z) p.z[n] = z_to_i32(q.z);
-      if (p.range) p.range[n] = omq_range{vmax, vmin, cnt & 0xffff, cnt >> 16};
-      if (p.Bt) p.Bt[n] = (p.B ? p.B[n] : 0.f) + bias;
+    if (p.Bt) {
+      float bias = __fadd_rn(bias2.x, bias2.y);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) bias += __shfl_xor_sync(0xffffffffu, bias, o);
+      if (lane == 0) p.Bt[n] = (p.B ? p.B[n] : 0.f) + bias;
     }
+    __syncwarp();                      // every lane is done with the buffer before it refills
+    if (nbuf == 1) issue(it + 1);
+  }
+  cp_async_wait<0>();
+}
+
+// Shared memory of the row-staged shape: buffers per warp and warps per block.
+struct StageShape {
+  int lpg = -1;          // lanes per group (0: one group per row); -1: shape not applicable
+  int nbuf = 0, wpb = 0;
+  size_t smem = 0;
+};
+constexpr size_t kStageSmem = 200 * 1024;
+
+StageShape stage_shape(const LwcParams& p) {
+  StageShape s;
+  const bool w16 = p.wdt == OMQ_BF16 || p.wdt == OMQ_F16;
+  const bool h16 = p.hat_dt == OMQ_BF16 || p.hat_dt == OMQ_F16;
+  if (!w16 || !h16 || !p.W_hat || p.codes || p.packed || p.K % 8 || p.N < 1) return s;
+  if (p.G == p.K) {
+    if (p.K > 16384) return s;               // tie counts are packed in 16 bits
+    s.lpg = 0;
+  } else if (p.K % p.G == 0 && (p.G == 32 || p.G == 64 || p.G == 128 || p.G == 256)) {
+    s.lpg = static_cast<int>(p.G / 8);
+  } else {
+    return s;
+  }
+  const size_t row = static_cast<size_t>(p.K) * 2;
+  const size_t lg = s.lpg ? static_cast<size_t>(p.ng) * 8 : 0;   // logits or strengths, a row
+  const size_t cap = static_cast<size_t>(s.lpg == 0 ? stage_max_warps(0) : stage_max_warps(8));
+  // two staged rows a warp only when that still leaves room for the most warps
+  s.nbuf = cap * (2 * row + 3 * lg) <= kStageSmem ? 2 : 1;
+  const size_t per_warp = s.nbuf * (row + lg) + lg;
+  s.wpb = static_cast<int>(std::min<size_t>(cap, kStageSmem / per_warp));
+  if (s.wpb < 1) { s.lpg = -1; return s; }
+  s.smem = per_warp * s.wpb;
+  return s;
+}
+
+template <int LPG, bool F16>
+omq_status launch_stage(const LwcParams& p, const StageShape& s, cudaStream_t stream) {
+  auto kernel = lwc_stage_kernel<LPG, F16>;
+  static std::mutex mu;
+  static uint64_t done = 0;                  // devices opted into the large shared memory
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) {
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev >= 64 || !(done >> dev & 1)) {
+      e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(kStageSmem));
+      if (e == cudaSuccess && dev < 64) done |= uint64_t(1) << dev;
+    }
+  }
+  if (e != cudaSuccess) {
+    set_cuda_error(e);
+    return OMQ_ERR_CUDA;
+  }
+  // rows per warp from the most warps that fit, then those warps spread over every SM
+  const int64_t sms = num_sms();
+  const int64_t per = (p.N + sms * s.wpb - 1) / (sms * s.wpb);
+  const int64_t warps = (p.N + per - 1) / per;
+  const int64_t wpb = std::min<int64_t>(s.wpb, (warps + sms - 1) / sms);
+  const int64_t blocks = (warps + wpb - 1) / wpb;
+  const size_t smem = s.smem / s.wpb * wpb;
+  kernel<<<static_cast<unsigned>(blocks), static_cast<unsigned>(32 * wpb), smem, stream>>>(
+      p, s.nbuf, per);
+  return launch_status();
+}
+
+omq_status launch_stage_any(const LwcParams& p, const StageShape& s, cudaStream_t stream) {
+  const bool f16 = p.wdt == OMQ_F16;
+  switch (s.lpg) {
+    case 0: return f16 ? launch_stage<0, true>(p, s, stream) : launch_stage<0, false>(p, s, stream);
+    case 4: return f16 ? launch_stage<4, true>(p, s, stream) : launch_stage<4, false>(p, s, stream);
+    case 8: return f16 ? launch_stage<8, true>(p, s, stream) : launch_stage<8, false>(p, s, stream);
+    case 16:
+      return f16 ? launch_stage<16, true>(p, s, stream) : launch_stage<16, false>(p, s, stream);
+    default:
+      return f16 ? launch_stage<32, true>(p, s, stream) : launch_stage<32, false>(p, s, stream);
   }
 }
 
 omq_status launch_lwc(const LwcParams& p, cudaStream_t stream) {
   const int64_t total = p.N * p.ng;
   const int sms = num_sms();
-  if ((p.wdt == OMQ_BF16 || p.wdt == OMQ_F16) && p.G == p.K && p.K % 256 == 0 &&
-      p.K <= 256 * kRowSegs) {
-    const int64_t max_warps = static_cast<int64_t>(sms) * 16;   // 2 blocks of 8 warps an SM
-    const int64_t per = (p.N + max_warps - 1) / max_warps;
-    const int64_t warps = (p.N + per - 1) / per;
-    lwc_row_kernel<<<static_cast<unsigned>((warps + 7) / 8), 256, 0, stream>>>(p, per);
-    return launch_status();
-  }
+  const StageShape shape = stage_shape(p);
+  if (shape.lpg >= 0) return launch_stage_any(p, shape, stream);
   if (p.Bt) {
     // B~ = B + W delta: its own pass over W
     const omq_status st = launch_let_bias(p.W, p.wdt, p.N, p.K, p.delta, p.B, p.Bt, stream);
