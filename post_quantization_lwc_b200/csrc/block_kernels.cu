@@ -16,6 +16,8 @@ namespace omq {
 // ------------------------------------------------------------------ rotary table
 // cos / sin of pos * base^(-2i/Dh) in binary64, rounded once: [M, Dh/2] each.
 __global__ void rope_table_kernel(int64_t M, int half, double base, float* cos_t, float* sin_t) {
+  pdl_wait();
+  pdl_launch();
   const int64_t total = M * half;
   for (int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < total;
        t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -45,6 +47,8 @@ __device__ __forceinline__ float block_sum(float v, float* sm) {
 }
 
 __global__ void __launch_bounds__(256) rms_kernel(RmsParams p) {
+  pdl_wait();
+  pdl_launch();
   __shared__ float sm[32];
   const int chunks = static_cast<int>(p.D / 8);
   for (int64_t m = blockIdx.x; m < p.M; m += gridDim.x) {
@@ -91,6 +95,8 @@ __global__ void __launch_bounds__(256) rms_kernel(RmsParams p) {
 
 // RMSNorm backward with the residual path: dx2 = res_scale res + rstd (dn - n mean(dn n)).
 __global__ void __launch_bounds__(256) rms_bwd_kernel(RmsBwdParams p) {
+  pdl_wait();
+  pdl_launch();
   __shared__ float sm[32];
   const int chunks = static_cast<int>(p.D / 8);
   for (int64_t m = blockIdx.x; m < p.M; m += gridDim.x) {
@@ -254,6 +260,8 @@ __device__ __forceinline__ void head_forward(const AttnPrepParams& p, int which,
 // grid (H, ceil(M / 8)), 8 warps: warp w takes token blockIdx.y * 8 + w of head blockIdx.x,
 // for q, k and v in turn; stats index (which * M + m) * H + h.
 __global__ void __launch_bounds__(256) attn_prep_kernel(AttnPrepParams p) {
+  pdl_wait();
+  pdl_launch();
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int h = blockIdx.x;
   const int64_t m = static_cast<int64_t>(blockIdx.y) * 8 + w;
@@ -284,6 +292,8 @@ __global__ void __launch_bounds__(256) attn_prep_kernel(AttnPrepParams p) {
 // grid (H, ceil(M / kAttnRows)); warp w takes tokens w, w + 8, ... of the block; the 8 warps'
 // sums are added in warp order.
 __global__ void __launch_bounds__(256) attn_prep_bwd_kernel(AttnPrepParams p) {
+  pdl_wait();
+  pdl_launch();
   __shared__ float red[3][8][128];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int h = blockIdx.x;
@@ -369,6 +379,8 @@ __device__ __forceinline__ int64_t causal_span(int64_t i, int64_t M) {
 
 __global__ void __launch_bounds__(256) softmax_kernel(float* S, __nv_bfloat16* P16, int64_t rows,
                                                       int64_t M) {
+  pdl_wait();
+  pdl_launch();
   const int lane = threadIdx.x & 31;
   const int64_t r = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   if (r >= rows) return;
@@ -421,6 +433,8 @@ __global__ void __launch_bounds__(256) softmax_kernel(float* S, __nv_bfloat16* P
 __global__ void __launch_bounds__(256) softmax_bwd_kernel(const float* P, const float* dP,
                                                           __nv_bfloat16* dS, int64_t rows,
                                                           int64_t M, float scale) {
+  pdl_wait();
+  pdl_launch();
   const int lane = threadIdx.x & 31;
   const int64_t r = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   if (r >= rows) return;
@@ -462,6 +476,8 @@ __global__ void __launch_bounds__(256) softmax_bwd_kernel(const float* P, const 
 // m[t, j] = SiLU(gu[t, j]) gu[t, I + j] (float32), 8 columns a thread.
 __global__ void __launch_bounds__(256) swiglu_kernel(const float* gu, float* mid, int64_t M,
                                                      int64_t I) {
+  pdl_wait();
+  pdl_launch();
   const int64_t per_row = I / 8, total = M * per_row;
   for (int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < total;
        t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -479,6 +495,8 @@ __global__ void __launch_bounds__(256) swiglu_kernel(const float* gu, float* mid
 __global__ void __launch_bounds__(256) swiglu_bwd_kernel(const float* gu, const float* dmid,
                                                          __nv_bfloat16* dgu, int64_t M,
                                                          int64_t I) {
+  pdl_wait();
+  pdl_launch();
   const int64_t per_row = I / 8, total = M * per_row;
   for (int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < total;
        t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -507,52 +525,52 @@ static unsigned grid_for(int64_t work, int64_t per_block, int cap_per_sm) {
 
 omq_status launch_rope_table(int64_t M, double base, float* cos_t, float* sin_t,
                              cudaStream_t st) {
-  rope_table_kernel<<<grid_for(M * 64, 256, 8), 256, 0, st>>>(M, 64, base, cos_t, sin_t);
+  launch_k(rope_table_kernel, grid_for(M * 64, 256, 8), 256, 0, st, M, 64, base, cos_t, sin_t);
   return launch_status();
 }
 
 omq_status launch_rms(const RmsParams& p, cudaStream_t st) {
-  rms_kernel<<<grid_for(p.M, 1, 16), 256, 0, st>>>(p);
+  launch_k(rms_kernel, grid_for(p.M, 1, 16), 256, 0, st, p);
   return launch_status();
 }
 
 omq_status launch_rms_bwd(const RmsBwdParams& p, cudaStream_t st) {
-  rms_bwd_kernel<<<grid_for(p.M, 1, 16), 256, 0, st>>>(p);
+  launch_k(rms_bwd_kernel, grid_for(p.M, 1, 16), 256, 0, st, p);
   return launch_status();
 }
 
 omq_status launch_attn_prep(const AttnPrepParams& p, bool backward, cudaStream_t st) {
   if (backward) {
     const dim3 grid(static_cast<unsigned>(p.H), static_cast<unsigned>(ceil_div(p.M, kAttnRows)));
-    attn_prep_bwd_kernel<<<grid, 256, 0, st>>>(p);
+    launch_k(attn_prep_bwd_kernel, grid, 256, 0, st, p);
   } else {
     const dim3 grid(static_cast<unsigned>(p.H), static_cast<unsigned>(ceil_div(p.M, 8)));
-    attn_prep_kernel<<<grid, 256, 0, st>>>(p);
+    launch_k(attn_prep_kernel, grid, 256, 0, st, p);
   }
   return launch_status();
 }
 
 omq_status launch_softmax(float* S, __nv_bfloat16* P16, int64_t rows, int64_t M,
                           cudaStream_t st) {
-  softmax_kernel<<<static_cast<unsigned>(ceil_div(rows, 8)), 256, 0, st>>>(S, P16, rows, M);
+  launch_k(softmax_kernel, static_cast<unsigned>(ceil_div(rows, 8)), 256, 0, st, S, P16, rows, M);
   return launch_status();
 }
 
 omq_status launch_softmax_bwd(const float* P, const float* dP, __nv_bfloat16* dS, int64_t rows,
                               int64_t M, float scale, cudaStream_t st) {
-  softmax_bwd_kernel<<<static_cast<unsigned>(ceil_div(rows, 8)), 256, 0, st>>>(P, dP, dS, rows,
-                                                                               M, scale);
+  launch_k(softmax_bwd_kernel, static_cast<unsigned>(ceil_div(rows, 8)), 256, 0, st,
+      P, dP, dS, rows, M, scale);
   return launch_status();
 }
 
 omq_status launch_swiglu(const float* gu, float* mid, int64_t M, int64_t I, cudaStream_t st) {
-  swiglu_kernel<<<grid_for(M * I / 8, 256, 8), 256, 0, st>>>(gu, mid, M, I);
+  launch_k(swiglu_kernel, grid_for(M * I / 8, 256, 8), 256, 0, st, gu, mid, M, I);
   return launch_status();
 }
 
 omq_status launch_swiglu_bwd(const float* gu, const float* dmid, __nv_bfloat16* dgu, int64_t M,
                              int64_t I, cudaStream_t st) {
-  swiglu_bwd_kernel<<<grid_for(M * I / 8, 256, 8), 256, 0, st>>>(gu, dmid, dgu, M, I);
+  launch_k(swiglu_bwd_kernel, grid_for(M * I / 8, 256, 8), 256, 0, st, gu, dmid, dgu, M, I);
   return launch_status();
 }
 

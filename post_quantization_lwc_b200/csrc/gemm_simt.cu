@@ -18,6 +18,8 @@ __device__ __forceinline__ float op_at(const GemmOperand& o, int64_t i, int64_t 
 __global__ void __launch_bounds__(256) gemm_f32_kernel(GemmOperand A, GemmOperand B, int64_t rows,
                                                        int64_t cols, int64_t depth,
                                                        GemmEpilogue epi, int tiles_n) {
+  pdl_wait();
+  pdl_launch();
   __shared__ float As[TK][T + 1];
   __shared__ float Bs[TK][T + 1];
   __shared__ float red[8];
@@ -86,7 +88,7 @@ omq_status gemm_f32_simt(const GemmOperand& A, const GemmOperand& B, int64_t row
   const int64_t tn = ceil_div(cols, simt::T);
   const int64_t tiles = ceil_div(rows, simt::T) * tn;
   if (n_tiles) *n_tiles = tiles;
-  simt::gemm_f32_kernel<<<static_cast<unsigned>(tiles), 256, 0, stream>>>(
+  launch_k(simt::gemm_f32_kernel, static_cast<unsigned>(tiles), 256, 0, stream,
       A, B, rows, cols, depth, epi, static_cast<int>(tn));
   return launch_status();
 }

@@ -487,6 +487,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV>::NUM_THREADS
   cluster_sync();            // both CTAs' barriers exist before either touches the other's
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // the prologue above touches only shared memory and TMEM: it may overlap the previous
+  // kernel of the stream; operands and outputs wait for that kernel's completion
+  pdl_wait();
+  pdl_launch();
 
   if (warp == 0 && lane == 0) {
     // ---------------- TMA producer (both CTAs)
@@ -808,7 +812,7 @@ omq_status gemm_tc(omq_dtype dt, const GemmOperand& A, const GemmOperand& B, int
                      batch ? batch->out_stride : 0};
   const int64_t max_pairs = num_sms() / 2;
   const int64_t pairs = tiles < max_pairs ? tiles : max_pairs;
-  kc.fn<<<static_cast<unsigned>(2 * pairs), kc.threads, kc.smem, stream>>>(
+  launch_k(kc.fn, static_cast<unsigned>(2 * pairs), kc.threads, kc.smem, stream,
       ma, mb, A.mn_major ? 1 : 0, B.mn_major ? 1 : 0, dt == OMQ_F16 ? 0u : 1u, rows, cols, depth,
       epi, sc);
   return launch_status();

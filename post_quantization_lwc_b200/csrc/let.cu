@@ -41,6 +41,8 @@ constexpr int kLetRows = 64;
 
 template <int U, bool AFFINE>
 __global__ void __launch_bounds__(256, 2) let_elem_kernel(LetParams p) {
+  pdl_wait();
+  pdl_launch();
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int64_t c0 = static_cast<int64_t>(blockIdx.x) * 256 + lane * 8;
   if (c0 >= p.K) return;
@@ -71,6 +73,8 @@ __global__ void __launch_bounds__(256, 2) let_elem_kernel(LetParams p) {
 }
 
 __global__ void __launch_bounds__(256) act_quant_kernel(LetParams p) {
+  pdl_wait();
+  pdl_launch();
   extern __shared__ float row[];   // K floats: X~[m, :]
   __shared__ float smf[64];
   __shared__ int smi[64];
@@ -145,6 +149,8 @@ __global__ void __launch_bounds__(256, 2) let_bias_kernel(const void* W, omq_dty
                                                           int64_t K, const float* delta,
                                                           const float* B, float* Bt,
                                                           int64_t rows_per_warp) {
+  pdl_wait();
+  pdl_launch();
   const int lane = threadIdx.x & 31;
   const int64_t warp_g = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t n_warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
@@ -189,6 +195,8 @@ __global__ void __launch_bounds__(256, 2) let_bias_kernel(const void* W, omq_dty
 __global__ void __launch_bounds__(256) let_bias_f32_kernel(const float* W, int64_t N, int64_t K,
                                                            const float* delta, const float* B,
                                                            float* Bt) {
+  pdl_wait();
+  pdl_launch();
   const int lane = threadIdx.x & 31;
   const int64_t warp_g = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t n_warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
@@ -214,8 +222,8 @@ omq_status launch_let(const LetParams& p, int abits, cudaStream_t stream) {
   if (abits >= 16) {
     const dim3 grid(static_cast<unsigned>(ceil_div(p.K, 256)),
                     static_cast<unsigned>(ceil_div(p.M, kLetRows)));
-    if (p.s || p.d) let_elem_kernel<4, true><<<grid, 256, 0, stream>>>(p);
-    else let_elem_kernel<4, false><<<grid, 256, 0, stream>>>(p);
+    if (p.s || p.d) launch_k(let_elem_kernel<4, true>, grid, 256, 0, stream, p);
+    else launch_k(let_elem_kernel<4, false>, grid, 256, 0, stream, p);
     return launch_status();
   }
   const size_t smem = static_cast<size_t>(p.K) * sizeof(float);
@@ -225,7 +233,7 @@ omq_status launch_let(const LetParams& p, int abits, cudaStream_t stream) {
     if (e != cudaSuccess) { set_cuda_error(e); return OMQ_ERR_CUDA; }
   }
   const unsigned grid = static_cast<unsigned>(p.M < int64_t(sms) * 8 ? p.M : int64_t(sms) * 8);
-  act_quant_kernel<<<grid, 256, smem, stream>>>(p);
+  launch_k(act_quant_kernel, grid, 256, smem, stream, p);
   return launch_status();
 }
 
@@ -235,15 +243,15 @@ omq_status launch_let_bias(const void* W, omq_dtype wdt, int64_t N, int64_t K, c
   if (wdt == OMQ_F32) {
     const int64_t want = ceil_div(N, 8);
     const unsigned grid = static_cast<unsigned>(want < int64_t(sms) * 16 ? want : int64_t(sms) * 16);
-    let_bias_f32_kernel<<<grid, 256, 0, stream>>>(static_cast<const float*>(W), N, K, delta, B,
-                                                  Bt);
+    launch_k(let_bias_f32_kernel, grid, 256, 0, stream,
+        static_cast<const float*>(W), N, K, delta, B, Bt);
     return launch_status();
   }
   const int64_t max_warps = static_cast<int64_t>(sms) * 16;
   const int64_t per = (N + max_warps - 1) / max_warps;
   const int64_t warps = (N + per - 1) / per;
-  let_bias_kernel<<<static_cast<unsigned>((warps + 7) / 8), 256, 0, stream>>>(W, wdt, N, K, delta,
-                                                                            B, Bt, per);
+  launch_k(let_bias_kernel, static_cast<unsigned>((warps + 7) / 8), 256, 0, stream,
+      W, wdt, N, K, delta, B, Bt, per);
   return launch_status();
 }
 

@@ -110,6 +110,8 @@ constexpr int kLwcRows = 64;
 
 template <int LPG, int U>
 __global__ void __launch_bounds__(256, 3) lwc_small_kernel(LwcParams p) {
+  pdl_wait();
+  pdl_launch();
   constexpr int GPW = 32 / LPG;   // groups per segment
   // The clipping strengths (binary64 sigmoids) of the U rows' groups are spread over the
   // warp's lanes: SPR strengths a row (gamma, beta of each group), RPP rows a pass of 32
@@ -222,6 +224,8 @@ __device__ __forceinline__ void block_sum2i(int& a, int& b, int* sm) {
 }
 
 __global__ void __launch_bounds__(256) lwc_large_kernel(LwcParams p) {
+  pdl_wait();
+  pdl_launch();
   extern __shared__ float buf[];   // G floats: the scaled group
   __shared__ float smf[64];
   __shared__ int smi[64];
@@ -453,6 +457,8 @@ constexpr int stage_max_warps(int lpg) { return lpg == 0 ? 24 : 16; }
 template <int LPG, bool F16>
 __global__ void __launch_bounds__(32 * stage_max_warps(LPG))
     lwc_stage_kernel(LwcParams p, int nbuf, int64_t rows_per_warp) {
+  pdl_wait();
+  pdl_launch();
   extern __shared__ __align__(16) unsigned char lsm[];
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5, wpb = blockDim.x >> 5;
   const int64_t K = p.K, ng = p.ng, chunks = K / 8;
@@ -738,7 +744,7 @@ omq_status launch_stage(const LwcParams& p, const StageShape& s, cudaStream_t st
   const int64_t wpb = std::min<int64_t>(s.wpb, (warps + sms - 1) / sms);
   const int64_t blocks = (warps + wpb - 1) / wpb;
   const size_t smem = s.smem / s.wpb * wpb;
-  kernel<<<static_cast<unsigned>(blocks), static_cast<unsigned>(32 * wpb), smem, stream>>>(
+  launch_k(kernel, static_cast<unsigned>(blocks), static_cast<unsigned>(32 * wpb), smem, stream,
       p, s.nbuf, per);
   return launch_status();
 }
@@ -771,11 +777,11 @@ omq_status launch_lwc(const LwcParams& p, cudaStream_t stream) {
     dim3 grid(static_cast<unsigned>(ceil_div(p.K, 256)),
               static_cast<unsigned>(ceil_div(p.N, kLwcRows)));
     switch (p.G / 8) {
-      case 2: lwc_small_kernel<2, U><<<grid, 256, 0, stream>>>(p); break;
-      case 4: lwc_small_kernel<4, U><<<grid, 256, 0, stream>>>(p); break;
-      case 8: lwc_small_kernel<8, U><<<grid, 256, 0, stream>>>(p); break;
-      case 16: lwc_small_kernel<16, U><<<grid, 256, 0, stream>>>(p); break;
-      default: lwc_small_kernel<32, U><<<grid, 256, 0, stream>>>(p); break;
+      case 2: launch_k(lwc_small_kernel<2, U>, grid, 256, 0, stream, p); break;
+      case 4: launch_k(lwc_small_kernel<4, U>, grid, 256, 0, stream, p); break;
+      case 8: launch_k(lwc_small_kernel<8, U>, grid, 256, 0, stream, p); break;
+      case 16: launch_k(lwc_small_kernel<16, U>, grid, 256, 0, stream, p); break;
+      default: launch_k(lwc_small_kernel<32, U>, grid, 256, 0, stream, p); break;
     }
     return launch_status();
   }
@@ -786,7 +792,7 @@ omq_status launch_lwc(const LwcParams& p, cudaStream_t stream) {
     if (e != cudaSuccess) { set_cuda_error(e); return OMQ_ERR_CUDA; }
   }
   const unsigned grid = static_cast<unsigned>(total < int64_t(sms) * 8 ? total : int64_t(sms) * 8);
-  lwc_large_kernel<<<grid, 256, smem, stream>>>(p);
+  launch_k(lwc_large_kernel, grid, 256, smem, stream, p);
   return launch_status();
 }
 

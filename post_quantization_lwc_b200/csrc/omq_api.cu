@@ -120,6 +120,50 @@ omq_status check_lwc(const void* W, omq_dtype wdt, int64_t N, int64_t K, int64_t
 
 void set_cuda_error(cudaError_t e) { t_last_cuda_error = static_cast<int>(e); }
 
+omq_status SideStream::fork(cudaStream_t main) const {
+  cudaError_t e = cudaEventRecord(fork_ev, main);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s, fork_ev, 0);
+  if (e != cudaSuccess) {
+    set_cuda_error(e);
+    return OMQ_ERR_CUDA;
+  }
+  return OMQ_OK;
+}
+
+omq_status SideStream::join(cudaStream_t main) const {
+  cudaError_t e = cudaEventRecord(join_ev, s);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(main, join_ev, 0);
+  if (e != cudaSuccess) {
+    set_cuda_error(e);
+    return OMQ_ERR_CUDA;
+  }
+  return OMQ_OK;
+}
+
+const SideStream* side_stream() {
+  thread_local std::vector<SideStream> per_device;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    set_cuda_error(e);
+    return nullptr;
+  }
+  if (static_cast<int>(per_device.size()) <= dev) per_device.resize(dev + 1);
+  SideStream& ss = per_device[dev];
+  if (!ss.s) {
+    SideStream n;
+    e = cudaStreamCreateWithFlags(&n.s, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&n.fork_ev, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&n.join_ev, cudaEventDisableTiming);
+    if (e != cudaSuccess) {
+      set_cuda_error(e);
+      return nullptr;
+    }
+    ss = n;
+  }
+  return &ss;
+}
+
 static std::atomic<uint64_t> g_launches{0};
 
 omq_status launch_status() {
@@ -342,77 +386,101 @@ static omq_status bwd_impl(const omq_bwd_args* a, void* workspace, size_t ws_byt
   float* part_xd = at<float>(workspace, L.part_xd);
   double* red = at<double>(workspace, L.red);
 
-  // dB~ = column sums of dY (needed for d_delta, or when asked for)
-  OMQ_TRY(ph.mark(OMQ_PH_DBIAS));
-  if (a->d_delta || a->d_B_tilde) {
-    OMQ_TRY(launch_colsum(a->dY, a->op_dt, M, N, kRowsColsum, nullptr, dbt_part, st));
-    const ColReduce r{dbt_part, L.rb_colsum, nullptr, 0, gscale, dbt};
-    OMQ_TRY(launch_reduce_cols(&r, 1, N, red, st));
-  }
-  // dW^ = G^T Xq   [N, K]
   const float Q = static_cast<float>((1 << a->bits) - 1);
   const bool fused = fused_ste_w(a->op_dt, a->dt, G);
   const int64_t rb_w = fused ? ceil_div(N, kRowsFusedW) : ceil_div(N, rows_per_block_w(G));
-  OMQ_TRY(ph.mark(OMQ_PH_DW_GEMM));
-  {
-    GemmOperand A{a->dY, N, true}, B{a->Xq, K, true};
-    GemmEpilogue epi{};
-    epi.out_scale = gscale;
+
+  // Weight side: dB~, the dW^ GEMM and the weight-side STE.
+  auto weight_side = [&](cudaStream_t s) -> omq_status {
+    // dB~ = column sums of dY (needed for d_delta, or when asked for)
+    OMQ_TRY(ph.mark(OMQ_PH_DBIAS));
+    if (a->d_delta || a->d_B_tilde) {
+      OMQ_TRY(launch_colsum(a->dY, a->op_dt, M, N, kRowsColsum, nullptr, dbt_part, s));
+      const ColReduce r{dbt_part, L.rb_colsum, nullptr, 0, gscale, dbt};
+      OMQ_TRY(launch_reduce_cols(&r, 1, N, red, s));
+    }
+    // dW^ = G^T Xq   [N, K]
+    OMQ_TRY(ph.mark(OMQ_PH_DW_GEMM));
+    {
+      GemmOperand A{a->dY, N, true}, B{a->Xq, K, true};
+      GemmEpilogue epi{};
+      epi.out_scale = gscale;
+      if (fused) {
+        // weight-side STE in the epilogue: per-chunk partial sums and the W-side LET column
+        // partials straight from the accumulator
+        epi.kind = Epi::SteW;
+        epi.ste = SteWEpi{a->W, a->dt, K, G, K / G, Q, a->s, a->h, a->z,
+                          at<float>(workspace, L.gh_part), at<float>(workspace, L.gc_part),
+                          a->d_s ? part_ws : nullptr};
+      } else {
+        epi.kind = Epi::StoreF32;
+        epi.out = dwhat;
+      }
+      OMQ_TRY(run_gemm(a->op_dt, A, B, N, K, M, epi, nullptr, s));
+    }
+    // weight-side STE: d gamma / d beta logits and the W-side LET column partials
+    OMQ_TRY(ph.mark(OMQ_PH_STE_W));
     if (fused) {
-      // weight-side STE in the epilogue: per-chunk partial sums and the W-side LET column
-      // partials straight from the accumulator
-      epi.kind = Epi::SteW;
-      epi.ste = SteWEpi{a->W, a->dt, K, G, K / G, Q, a->s, a->h, a->z,
-                        at<float>(workspace, L.gh_part), at<float>(workspace, L.gc_part),
-                        a->d_s ? part_ws : nullptr};
+      float* emax = a->d_s ? at<float>(workspace, L.emax) : nullptr;
+      float* emin = a->d_s ? at<float>(workspace, L.emin) : nullptr;
+      const SteWFinish f{N, G, K / G, Q, at<float>(workspace, L.gh_part),
+                         at<float>(workspace, L.gc_part), a->h, a->grp_range, a->gamma_logit,
+                         a->beta_logit, a->d_gamma_logit, a->d_beta_logit, emax, emin};
+      OMQ_TRY(launch_ste_w_finish(f, s));
+      if (a->d_s || a->d_delta) {
+        const SteWCorr c{a->W, a->dt, N, K, G, a->s, a->grp_range, emax, emin, dbt,
+                         a->d_s ? part_ws : nullptr, a->d_delta ? part_wd : nullptr};
+        OMQ_TRY(launch_ste_w_corr(c, s));
+      }
     } else {
+      SteWParams p{a->W, a->dt, N, K, G, K / G, Q, a->s, a->gamma_logit, a->beta_logit, a->h,
+                   a->z, a->grp_range, dwhat, a->d_delta ? dbt : nullptr, a->d_gamma_logit,
+                   a->d_beta_logit, a->d_s ? part_ws : nullptr, a->d_delta ? part_wd : nullptr,
+                   static_cast<int>(rows_per_block_w(G))};
+      OMQ_TRY(launch_ste_w(p, s));
+    }
+    return OMQ_OK;
+  };
+  // Activation side (LET only): the dXq GEMM and the activation-side STE.
+  auto act_side = [&](cudaStream_t s) -> omq_status {
+    OMQ_TRY(ph.mark(OMQ_PH_DX_GEMM));
+    // dXq = G W^   [M, K]
+    {
+      GemmOperand A{a->dY, N, false}, B{a->W_hat, K, true};
+      GemmEpilogue epi{};
       epi.kind = Epi::StoreF32;
-      epi.out = dwhat;
+      epi.out = dxq;
+      epi.out_scale = gscale;
+      OMQ_TRY(run_gemm(a->op_dt, A, B, M, K, N, epi, nullptr, s));
     }
-    OMQ_TRY(run_gemm(a->op_dt, A, B, N, K, M, epi, nullptr, st));
-  }
-  // weight-side STE: d gamma / d beta logits and the W-side LET column partials
-  OMQ_TRY(ph.mark(OMQ_PH_STE_W));
-  if (fused) {
-    float* emax = a->d_s ? at<float>(workspace, L.emax) : nullptr;
-    float* emin = a->d_s ? at<float>(workspace, L.emin) : nullptr;
-    const SteWFinish f{N, G, K / G, Q, at<float>(workspace, L.gh_part),
-                       at<float>(workspace, L.gc_part), a->h, a->grp_range, a->gamma_logit,
-                       a->beta_logit, a->d_gamma_logit, a->d_beta_logit, emax, emin};
-    OMQ_TRY(launch_ste_w_finish(f, st));
-    if (a->d_s || a->d_delta) {
-      const SteWCorr c{a->W, a->dt, N, K, G, a->s, a->grp_range, emax, emin, dbt,
-                       a->d_s ? part_ws : nullptr, a->d_delta ? part_wd : nullptr};
-      OMQ_TRY(launch_ste_w_corr(c, st));
-    }
-  } else {
-    SteWParams p{a->W, a->dt, N, K, G, K / G, Q, a->s, a->gamma_logit, a->beta_logit, a->h, a->z,
-                 a->grp_range, dwhat, a->d_delta ? dbt : nullptr, a->d_gamma_logit,
-                 a->d_beta_logit, a->d_s ? part_ws : nullptr, a->d_delta ? part_wd : nullptr,
-                 static_cast<int>(rows_per_block_w(G))};
-    OMQ_TRY(launch_ste_w(p, st));
-  }
-  OMQ_TRY(ph.mark(OMQ_PH_DX_GEMM));
-  if (!need_let) {
     OMQ_TRY(ph.mark(OMQ_PH_STE_X));
-    return ph.mark(OMQ_PH_LET_REDUCE);
-  }
-  // dXq = G W^   [M, K]
-  {
-    GemmOperand A{a->dY, N, false}, B{a->W_hat, K, true};
-    GemmEpilogue epi{};
-    epi.kind = Epi::StoreF32;
-    epi.out = dxq;
-    epi.out_scale = gscale;
-    OMQ_TRY(run_gemm(a->op_dt, A, B, M, K, N, epi, nullptr, st));
-  }
-  OMQ_TRY(ph.mark(OMQ_PH_STE_X));
-  {
     SteXParams p{a->X, a->dt, M, K,
                  static_cast<float>((1 << (a->abits < 16 ? a->abits : 1)) - 1),
                  a->abits < 16 ? 1 : 0, a->s, a->delta, a->h_a, a->z_a, a->tok_range, dxq,
                  at<float>(workspace, L.rowstat), part_xs, part_xd, kRowsX};
-    OMQ_TRY(launch_ste_x(p, st));
+    return launch_ste_x(p, s);
+  };
+
+  // The two sides share only dY (read) and write disjoint buffers: without phase events
+  // the activation side runs on a second stream, so each side's kernels fill the other's
+  // pipeline fill, epilogue tails and launch gaps.
+  const SideStream* ss = (!ph.ev && need_let) ? side_stream() : nullptr;
+  if (ss) {
+    OMQ_TRY(ss->fork(st));
+    const omq_status sa = act_side(ss->s);
+    const omq_status sw = weight_side(st);
+    const omq_status sj = ss->join(st);
+    OMQ_TRY(sa);
+    OMQ_TRY(sw);
+    OMQ_TRY(sj);
+  } else {
+    OMQ_TRY(weight_side(st));
+    if (!need_let) {
+      OMQ_TRY(ph.mark(OMQ_PH_DX_GEMM));
+      OMQ_TRY(ph.mark(OMQ_PH_STE_X));
+      return ph.mark(OMQ_PH_LET_REDUCE);
+    }
+    OMQ_TRY(act_side(st));
   }
   OMQ_TRY(ph.mark(OMQ_PH_LET_REDUCE));
   ColReduce r[2];
@@ -469,17 +537,17 @@ omq_status omq_calib_step(const omq_step_args* a, void* workspace, size_t ws_byt
   const void* Xq = need_act ? a->Xq : a->X;
   const float* Bt = let ? a->B_tilde : a->B;
   Phases ph{a->events, reinterpret_cast<cudaStream_t>(stream)};
-  OMQ_TRY(ph.mark(OMQ_PH_LET));
-  if (need_act) {
-    OMQ_TRY(omq_let_apply(a->X, a->dt, M, K, let ? a->s : nullptr, let ? a->delta : nullptr,
-                          a->abits, a->Xq, a->op_dt, a->h_a, a->z_a, a->tok_range, nullptr, a->dt,
-                          N, nullptr, nullptr, stream));
-  }
-  OMQ_TRY(ph.mark(OMQ_PH_LWC));
-  {
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  OMQ_TRY(check_lwc(a->W, a->dt, N, K, G, a->bits, a->gamma_logit, a->beta_logit,
+                    let ? a->s : nullptr, a->op_dt, a->W_hat, nullptr, a->h, a->z));
+  auto act = [&](cudaStream_t s) -> omq_status {
+    if (!need_act) return OMQ_OK;
+    return omq_let_apply(a->X, a->dt, M, K, let ? a->s : nullptr, let ? a->delta : nullptr,
+                         a->abits, a->Xq, a->op_dt, a->h_a, a->z_a, a->tok_range, nullptr, a->dt,
+                         N, nullptr, nullptr, s);
+  };
+  auto lwc = [&](cudaStream_t s) -> omq_status {
     // LWC, with B~ = B + W delta out of the same pass over W
-    OMQ_TRY(check_lwc(a->W, a->dt, N, K, G, a->bits, a->gamma_logit, a->beta_logit,
-                      let ? a->s : nullptr, a->op_dt, a->W_hat, nullptr, a->h, a->z));
     LwcParams p{a->W, a->dt, N, K, G, K / G, static_cast<float>((1 << a->bits) - 1),
                 a->gamma_logit, a->beta_logit, let ? a->s : nullptr, a->W_hat, a->op_dt, a->h,
                 a->z, nullptr, a->grp_range, nullptr, a->bits};
@@ -488,7 +556,24 @@ omq_status omq_calib_step(const omq_step_args* a, void* workspace, size_t ws_byt
       p.B = a->B;
       p.Bt = a->B_tilde;
     }
-    OMQ_TRY(launch_lwc(p, reinterpret_cast<cudaStream_t>(stream)));
+    return launch_lwc(p, s);
+  };
+  // The activation and weight sides of the forward are independent: without phase events
+  // the weight side runs on a second stream.
+  const SideStream* ss = (!ph.ev && need_act) ? side_stream() : nullptr;
+  if (ss) {
+    OMQ_TRY(ss->fork(st));
+    const omq_status sl = lwc(ss->s);
+    const omq_status sa = act(st);
+    const omq_status sj = ss->join(st);
+    OMQ_TRY(sl);
+    OMQ_TRY(sa);
+    OMQ_TRY(sj);
+  } else {
+    OMQ_TRY(ph.mark(OMQ_PH_LET));
+    OMQ_TRY(act(st));
+    OMQ_TRY(ph.mark(OMQ_PH_LWC));
+    OMQ_TRY(lwc(st));
   }
   OMQ_TRY(fwd_impl(Xq, a->W_hat, a->op_dt, M, N, K, Bt, a->Y_ref, nullptr, a->dY, a->loss,
                    workspace, fwd_ws, stream, ph));

@@ -9,6 +9,7 @@
 #include <stdint.h>
 
 #include <cmath>
+#include <utility>
 
 #include "../../include/omq.h"
 
@@ -145,10 +146,53 @@ __device__ __forceinline__ int32_t z_to_i32(float z) {
   return static_cast<int32_t>(c);
 }
 
+// ---- programmatic dependent launch -----------------------------------------------------
+// Every kernel of the library is launched with programmatic stream serialization (launch_k)
+// and opens with pdl_wait(): the grid may be scheduled while the previous kernel of the
+// stream is still running (its launch and any prologue before the wait overlap that
+// kernel's tail), but nothing it does to global memory precedes the previous grid's
+// completion and memory flush. pdl_launch() then lets the next kernel be scheduled in turn.
+// Both are no-ops for a grid launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---- host-side helpers ------------------------------------------------------------------
 void set_cuda_error(cudaError_t e);
 omq_status launch_status();          // checks cudaGetLastError after a launch
 int num_sms();
+
+// kernel<<<grid, block, smem, stream>>>(args...) with programmatic stream serialization. A
+// failed launch leaves its error for the launch_status() that follows every launch.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                     cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// A second stream of the calling host thread on the current device, for independent work
+// inside one library call: fork() makes it wait for what the caller's stream has queued so
+// far, join() makes the caller's stream wait for what it has queued. Created on first use
+// (non-blocking, never destroyed); the event pair is reused from call to call, which stream
+// order and graph capture both allow.
+struct SideStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork_ev = nullptr, join_ev = nullptr;
+  omq_status fork(cudaStream_t main) const;
+  omq_status join(cudaStream_t main) const;
+};
+const SideStream* side_stream();   // nullptr (and the CUDA error recorded) if it cannot be made
 
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 // Groups handled lane-parallel inside a warp (16 to 256 elements, power of two); other group

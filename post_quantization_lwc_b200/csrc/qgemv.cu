@@ -26,6 +26,8 @@ __global__ void __launch_bounds__(256) qgemv_kernel(const void* x, omq_dtype xdt
                                                     const float* h, const int32_t* z, int64_t N,
                                                     int64_t group, float* y,
                                                     int64_t rows_per_warp) {
+  pdl_wait();
+  pdl_launch();
   constexpr int CPC = 128 / BITS;     // codes per 16-byte chunk
   extern __shared__ float gsm[];      // xf [M][CPC][K / CPC], then xsum [M][K / CPC]
   const int64_t nch = K / CPC;
@@ -168,7 +170,7 @@ extern "C" omq_status omq_qgemv(const void* x, omq_dtype xdt, int64_t M, int64_t
     const int64_t max_warps = static_cast<int64_t>(num_sms()) * 8 * per_sm;
     const int64_t per = (N + max_warps - 1) / max_warps;
     const int64_t warps = (N + per - 1) / per;
-    kernel<<<static_cast<unsigned>((warps + 7) / 8), 256, smem, st>>>(
+    launch_k(kernel, static_cast<unsigned>((warps + 7) / 8), 256, smem, st,
         x, xdt, static_cast<int>(M), K, packed, h, z, N, group, y, per);
     return launch_status();
   };

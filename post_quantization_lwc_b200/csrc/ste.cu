@@ -21,6 +21,8 @@ namespace omq {
 // in shared memory in warp order at the end.
 template <int LPG, int U>
 __global__ void __launch_bounds__(256, 2) ste_w_small_kernel(SteWParams p) {
+  pdl_wait();
+  pdl_launch();
   __shared__ float red_s[8][256];
   __shared__ float red_d[8][256];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
@@ -145,6 +147,8 @@ __device__ __forceinline__ void block_sum2(float& a, float& b, float* sm) {
 // grid (n_groups, row blocks); the block's 256 threads cover the group's columns in chunks
 // of 8; column partial sums live in shared memory (each column owned by one thread).
 __global__ void __launch_bounds__(256) ste_w_large_kernel(SteWParams p) {
+  pdl_wait();
+  pdl_launch();
   extern __shared__ float acc[];   // 2 * G floats
   __shared__ float sm[64];
   float* acc_s = acc;
@@ -231,6 +235,8 @@ constexpr int kFinishJ = 8;   // groups per tile of ste_w_finish_kernel (32 rows
 // chunk partials are added in chunk order (groups of up to 8 chunks) or as 8 interleaved
 // partial sums added in a fixed order (longer groups).
 __global__ void __launch_bounds__(256) ste_w_finish_kernel(SteWFinish p) {
+  pdl_wait();
+  pdl_launch();
   __shared__ float sgh[kFinishJ][33], sgc[kFinishJ][33];   // [group in tile][row in tile]
   __shared__ float wred[2][8][32];
   const int64_t n0 = static_cast<int64_t>(blockIdx.x) * 32;
@@ -314,6 +320,8 @@ __global__ void __launch_bounds__(256) ste_w_finish_kernel(SteWFinish p) {
 //                    it is the min)                       (the clipping-range terms of d s)
 //   part_d[rb, k]  = sum_n dBt[n] W[n,k]                  (the bias term of d delta)
 __global__ void __launch_bounds__(256, 2) ste_w_corr_kernel(SteWCorr p) {
+  pdl_wait();
+  pdl_launch();
   constexpr int U = 8;
   const int lane = threadIdx.x & 31;
   const int64_t warp_g = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
@@ -426,6 +434,8 @@ __device__ __forceinline__ void let_vectors(const SteXParams& p, int64_t col, fl
 // Per token (quantized activations): the gradient share of the token's max and min elements,
 // from the token's G_h and G_z sums (g = b = 1).
 __global__ void __launch_bounds__(256) ste_x_rowstat_kernel(SteXParams p) {
+  pdl_wait();
+  pdl_launch();
   __shared__ float sm[64];
   const int chunks = static_cast<int>(p.K / 8);
   for (int64_t m = blockIdx.x; m < p.M; m += gridDim.x) {
@@ -457,6 +467,8 @@ __global__ void __launch_bounds__(256) ste_x_rowstat_kernel(SteXParams p) {
 // for every 8th row (lane = 8 columns), U rows per iteration.
 template <int U>
 __global__ void __launch_bounds__(256, 2) ste_x_cols_kernel(SteXParams p) {
+  pdl_wait();
+  pdl_launch();
   __shared__ float red_s[8][256];
   __shared__ float red_d[8][256];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
@@ -547,6 +559,8 @@ template <int U>
 __global__ void __launch_bounds__(256) colsum_kernel(const void* A, omq_dtype dt, int64_t rows,
                                                      int64_t cols, int R, const float* wrow,
                                                      float* part) {
+  pdl_wait();
+  pdl_launch();
   __shared__ float red[8][256];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int64_t c0 = static_cast<int64_t>(blockIdx.x) * 256 + lane * 8;
@@ -599,6 +613,8 @@ struct ColReduceSet {
 
 __global__ void __launch_bounds__(256) reduce_cols_partial_kernel(ColReduceSet rs,
                                                                   double* scratch) {
+  pdl_wait();
+  pdl_launch();
   __shared__ double red[8][32];
   const ColReduce& q = rs.pr[blockIdx.z];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
@@ -628,6 +644,8 @@ __global__ void __launch_bounds__(256) reduce_cols_partial_kernel(ColReduceSet r
 // Level 2, grid (column blocks, problems): out[j] = scale * sum over chunks c (in order).
 __global__ void __launch_bounds__(256) reduce_cols_final_kernel(ColReduceSet rs,
                                                                 const double* scratch) {
+  pdl_wait();
+  pdl_launch();
   const ColReduce& q = rs.pr[blockIdx.y];
   const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (j >= rs.cols) return;
@@ -640,6 +658,8 @@ __global__ void __launch_bounds__(256) reduce_cols_final_kernel(ColReduceSet rs,
 // loss = (sum of per-tile partials) / count, binary64, fixed order.
 __global__ void __launch_bounds__(256) loss_finalize_kernel(const float* part, int64_t n,
                                                             double inv_count, float* loss) {
+  pdl_wait();
+  pdl_launch();
   __shared__ double sm[256];
   double a = 0.0;
   for (int64_t i = threadIdx.x; i < n; i += blockDim.x) a += part[i];
@@ -659,6 +679,8 @@ struct AdamSegs {
 // AdamW over up to four parameter tensors in one launch (blockIdx.y selects the tensor).
 __global__ void __launch_bounds__(256) adamw_kernel(AdamSegs segs, float b1, float b2, float eps,
                                                     float wd, float bc1, float bc2_sqrt) {
+  pdl_wait();
+  pdl_launch();
   const AdamSeg sg = segs.s[blockIdx.y];
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < sg.n;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -680,11 +702,11 @@ omq_status launch_ste_w(const SteWParams& p, cudaStream_t stream) {
   if (small_group(p.G)) {
     dim3 grid(static_cast<unsigned>(ceil_div(p.K, 256)), static_cast<unsigned>(rbs));
     switch (p.G / 8) {
-      case 2: ste_w_small_kernel<2, 2><<<grid, 256, 0, stream>>>(p); break;
-      case 4: ste_w_small_kernel<4, 2><<<grid, 256, 0, stream>>>(p); break;
-      case 8: ste_w_small_kernel<8, 2><<<grid, 256, 0, stream>>>(p); break;
-      case 16: ste_w_small_kernel<16, 2><<<grid, 256, 0, stream>>>(p); break;
-      default: ste_w_small_kernel<32, 2><<<grid, 256, 0, stream>>>(p); break;
+      case 2: launch_k(ste_w_small_kernel<2, 2>, grid, 256, 0, stream, p); break;
+      case 4: launch_k(ste_w_small_kernel<4, 2>, grid, 256, 0, stream, p); break;
+      case 8: launch_k(ste_w_small_kernel<8, 2>, grid, 256, 0, stream, p); break;
+      case 16: launch_k(ste_w_small_kernel<16, 2>, grid, 256, 0, stream, p); break;
+      default: launch_k(ste_w_small_kernel<32, 2>, grid, 256, 0, stream, p); break;
     }
     return launch_status();
   }
@@ -696,14 +718,14 @@ omq_status launch_ste_w(const SteWParams& p, cudaStream_t stream) {
                                          static_cast<int>(smem));
     if (e != cudaSuccess) { set_cuda_error(e); return OMQ_ERR_CUDA; }
   }
-  ste_w_large_kernel<<<grid, 256, smem, stream>>>(p);
+  launch_k(ste_w_large_kernel, grid, 256, smem, stream, p);
   return launch_status();
 }
 
 omq_status launch_ste_w_finish(const SteWFinish& p, cudaStream_t stream) {
   const dim3 grid(static_cast<unsigned>(ceil_div(p.N, 32)),
                   static_cast<unsigned>(std::min<int64_t>(ceil_div(p.ng, kFinishJ), 65535)));
-  ste_w_finish_kernel<<<grid, 256, 0, stream>>>(p);
+  launch_k(ste_w_finish_kernel, grid, 256, 0, stream, p);
   return launch_status();
 }
 
@@ -711,7 +733,7 @@ omq_status launch_ste_w_corr(const SteWCorr& p, cudaStream_t stream) {
   const int64_t tasks = ceil_div(p.K, 256) * ceil_div(p.N, 32);
   const int64_t cap = static_cast<int64_t>(num_sms()) * 16;    // resident warps
   const int64_t warps = tasks < cap ? tasks : cap;
-  ste_w_corr_kernel<<<static_cast<unsigned>(ceil_div(warps, 8)), 256, 0, stream>>>(p);
+  launch_k(ste_w_corr_kernel, static_cast<unsigned>(ceil_div(warps, 8)), 256, 0, stream, p);
   return launch_status();
 }
 
@@ -719,20 +741,20 @@ omq_status launch_ste_x(const SteXParams& p, cudaStream_t stream) {
   if (p.quantized) {
     const int sms = num_sms();
     const unsigned grid = static_cast<unsigned>(p.M < int64_t(sms) * 8 ? p.M : int64_t(sms) * 8);
-    ste_x_rowstat_kernel<<<grid, 256, 0, stream>>>(p);
+    launch_k(ste_x_rowstat_kernel, grid, 256, 0, stream, p);
     const omq_status st = launch_status();
     if (st != OMQ_OK) return st;
   }
   dim3 grid(static_cast<unsigned>(ceil_div(p.K, 256)),
             static_cast<unsigned>(ceil_div(p.M, p.rows_per_block)));
-  ste_x_cols_kernel<2><<<grid, 256, 0, stream>>>(p);
+  launch_k(ste_x_cols_kernel<2>, grid, 256, 0, stream, p);
   return launch_status();
 }
 
 omq_status launch_colsum(const void* A, omq_dtype dt, int64_t rows, int64_t cols, int R,
                          const float* w, float* part, cudaStream_t stream) {
   dim3 grid(static_cast<unsigned>(ceil_div(cols, 256)), static_cast<unsigned>(ceil_div(rows, R)));
-  colsum_kernel<4><<<grid, 256, 0, stream>>>(A, dt, rows, cols, R, w, part);
+  launch_k(colsum_kernel<4>, grid, 256, 0, stream, A, dt, rows, cols, R, w, part);
   return launch_status();
 }
 
@@ -752,17 +774,17 @@ omq_status launch_reduce_cols(const ColReduce* probs, int nprob, int64_t cols, d
   rs.rpc = ceil_div(std::max<int64_t>(total, 1), rs.chunks);
   const dim3 grid(static_cast<unsigned>(ceil_div(cols, 32)), static_cast<unsigned>(rs.chunks),
                   static_cast<unsigned>(nprob));
-  reduce_cols_partial_kernel<<<grid, 256, 0, stream>>>(rs, scratch);
+  launch_k(reduce_cols_partial_kernel, grid, 256, 0, stream, rs, scratch);
   const omq_status st = launch_status();
   if (st != OMQ_OK || rs.chunks == 1) return st;
   const dim3 g2(static_cast<unsigned>(ceil_div(cols, 256)), static_cast<unsigned>(nprob));
-  reduce_cols_final_kernel<<<g2, 256, 0, stream>>>(rs, scratch);
+  launch_k(reduce_cols_final_kernel, g2, 256, 0, stream, rs, scratch);
   return launch_status();
 }
 
 omq_status launch_loss_finalize(const float* part, int64_t n, double inv_count, float* loss,
                                 cudaStream_t stream) {
-  loss_finalize_kernel<<<1, 256, 0, stream>>>(part, n, inv_count, loss);
+  launch_k(loss_finalize_kernel, 1, 256, 0, stream, part, n, inv_count, loss);
   return launch_status();
 }
 
@@ -781,8 +803,8 @@ omq_status launch_adamw(const AdamSeg* segs, int nseg, float b1, float b2, float
   const int64_t want = ceil_div(nmax, 256);
   const unsigned gx = static_cast<unsigned>(want < int64_t(sms) * 4 ? want : int64_t(sms) * 4);
   dim3 grid(gx > 0 ? gx : 1, static_cast<unsigned>(nseg));
-  adamw_kernel<<<grid, 256, 0, stream>>>(s, b1, b2, eps, wd, static_cast<float>(bc1),
-                                         static_cast<float>(std::sqrt(bc2)));
+  launch_k(adamw_kernel, grid, 256, 0, stream,
+      s, b1, b2, eps, wd, static_cast<float>(bc1), static_cast<float>(std::sqrt(bc2)));
   return launch_status();
 }
 
