@@ -65,7 +65,10 @@ struct Cfg {
   static constexpr int EPI_WARPS = EV ? 16 : 8;
   static constexpr int EPI_COLS = TILE_N * 4 / EPI_WARPS;   // accumulator columns per warp
   static constexpr int NUM_THREADS = 32 * (2 + EPI_WARPS);
-  static constexpr int STAGES = 7;
+  // the STE variants give two stages of the ring to a 4 KB shared slice per epilogue warp
+  // (its 32 x 64 block of W, staged by coalesced copies)
+  static constexpr int STAGES = EV ? 5 : 7;
+  static constexpr int WST = EV ? 32 * 64 * 2 : 0;
   static constexpr bool SLEEPY = EV != 0;
 };
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;   // 2 s per barrier wait
@@ -322,6 +325,13 @@ __host__ __device__ constexpr uint32_t instr_desc(int m, int n, bool a_mn, bool 
          (static_cast<uint32_t>(m >> 4) << 24);
 }
 
+// 16-byte asynchronous copy global -> shared (no multicast), its group commit and wait.
+__device__ __forceinline__ void cp16_async(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
 // 8 weights of one row from their 16-bit storage.
 template <bool F16>
 __device__ __forceinline__ void unpack8(const uint4& q, float (&w)[8]) {
@@ -354,13 +364,15 @@ __device__ __forceinline__ void unpack8(const uint4& q, float (&w)[8]) {
 template <bool F16>
 __device__ __forceinline__ void ste_w_epilogue(const GemmEpilogue& epi, uint32_t tcol,
                                                int64_t wrow0, int64_t col0, int64_t rows,
-                                               int64_t cols, int lane) {
+                                               int64_t cols, int lane, const uint8_t* wst) {
   const SteWEpi& p = epi.ste;
   const int64_t row = wrow0 + lane;
   const bool valid = row < rows;
   const bool let = p.part_s != nullptr;
-  const uint4* wrow = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.W) +
-                                                     (valid ? row : 0) * p.K + col0);
+  // this warp's weight block was staged in wst (chunk j of row r at (j ^ (r & 7)) * 16 bytes)
+  cp_wait_all();
+  __syncwarp();
+  const uint8_t* wrow = wst + lane * 128;
 #pragma unroll 1
   for (int c = 0; c < 2; ++c) {
     const int64_t k0 = col0 + 32 * c;
@@ -378,8 +390,10 @@ __device__ __forceinline__ void ste_w_epilogue(const GemmEpilogue& epi, uint32_t
     for (int hh = 0; hh < 2; ++hh) {
       const int q = 2 * c + hh;
       uint4 wq[2];
-      wq[0] = valid ? __ldg(wrow + 2 * q) : make_uint4(0, 0, 0, 0);
-      wq[1] = valid ? __ldg(wrow + 2 * q + 1) : make_uint4(0, 0, 0, 0);
+      wq[0] = valid ? *reinterpret_cast<const uint4*>(wrow + (((2 * q) ^ (lane & 7)) << 4))
+                    : make_uint4(0, 0, 0, 0);
+      wq[1] = valid ? *reinterpret_cast<const uint4*>(wrow + (((2 * q + 1) ^ (lane & 7)) << 4))
+                    : make_uint4(0, 0, 0, 0);
       uint32_t r[16];
       __syncwarp();
       tmem_ld16(tcol + 16 * q, r);
@@ -414,12 +428,13 @@ __device__ __forceinline__ void ste_w_epilogue(const GemmEpilogue& epi, uint32_t
   }
 }
 
-template <int STAGES, int EPI_WARPS>
+template <int STAGES, int EPI_WARPS, int WST>
 struct Layout {
   static constexpr int A_BYTES = HALF * BK * 2;          // 16 KB
   static constexpr int B_BYTES = HALF * BK * 2;          // 16 KB
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // this CTA's part of a stage
-  static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
+  static constexpr int WST_OFF = STAGES * STAGE_BYTES;   // epilogue warps' weight slices
+  static constexpr int BAR_OFF = WST_OFF + EPI_WARPS * WST;
   // control block: barriers full[S], empty[S], acc_full[2], acc_empty[2], drain; tmem slot,
   // abort flag, the epilogue's per-warp loss partials [2][EPI_WARPS] and arrival counters [2]
   static constexpr int CTL_BYTES = 512;
@@ -439,7 +454,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV>::NUM_THREADS
                    GemmEpilogue epi, TileSched sc) {
   using C = Cfg<EV>;
   constexpr int STAGES = C::STAGES, EPI_WARPS = C::EPI_WARPS, EPI_COLS = C::EPI_COLS;
-  using L = Layout<STAGES, EPI_WARPS>;
+  using L = Layout<STAGES, EPI_WARPS, C::WST>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -590,6 +605,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV>::NUM_THREADS
       const int64_t wrow0 = static_cast<int64_t>(tw.row0) + rank * HALF + quad * 32;
       const int64_t col0 = static_cast<int64_t>(tw.col0) + cq * EPI_COLS;
       const int64_t row = wrow0 + lane;
+      if constexpr (EV != 0) {
+        // this warp's 32 x 64 block of W into its shared slice by 16-byte copies, 4 rows of
+        // 128 bytes a warp instruction (the epilogue reads a row per lane, which straight
+        // from global memory touches 32 lines an instruction); chunk j of row r goes to
+        // (j ^ (r & 7)) * 16, so those row-per-lane reads are free of bank conflicts. Issued
+        // before the accumulator wait: the copies overlap the tile's MMAs.
+        const SteWEpi& sp = epi.ste;
+        const uint32_t slice = sbase + L::WST_OFF + ew * C::WST;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int m = lane + 32 * k, r = m >> 3, j = m & 7;
+          const int64_t grow = wrow0 + r, gcol = col0 + 8 * j;
+          if (grow < rows && gcol < cols)
+            cp16_async(slice + r * 128 + ((j ^ (r & 7)) << 4),
+                       static_cast<const uint16_t*>(sp.W) + grow * sp.K + gcol);
+        }
+        cp_commit();
+      }
       // one lane polls; the decision is broadcast so the warp-wide tcgen05.ld stays uniform
       int go = 0;
       if (lane == 0)
@@ -603,7 +636,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV>::NUM_THREADS
       const uint32_t tbase = tmem + (static_cast<uint32_t>(quad * 32) << 16) +
                              static_cast<uint32_t>(buf * TILE_N + cq * EPI_COLS);
       if constexpr (EV != 0) {
-        ste_w_epilogue<EV == 2>(epi, tbase, wrow0, col0, rows, cols, lane);
+        ste_w_epilogue<EV == 2>(epi, tbase, wrow0, col0, rows, cols, lane,
+                                smem + L::WST_OFF + ew * C::WST);
       } else {
         float* const out_b = BATCH ? epi.out + static_cast<int64_t>(tw.b) * sc.out_bstride : epi.out;
         for (int ch = 0; ch < EPI_COLS / 32; ++ch) {
@@ -653,6 +687,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV>::NUM_THREADS
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acce_leader + 8 * buf);
     }
+    if constexpr (EV != 0) cp_wait_all();    // no copy in flight when the CTA leaves
   }
   tc_fence_before();
   __syncthreads();
@@ -736,8 +771,8 @@ bool make_map(CUtensorMap* map, omq_dtype dt, const GemmOperand& op, int64_t n_r
   return r == CUDA_SUCCESS;
 }
 
-static_assert(Layout<Cfg<0>::STAGES, Cfg<0>::EPI_WARPS>::SMEM_BYTES <= 232448, "smem");
-static_assert(Layout<Cfg<1>::STAGES, Cfg<1>::EPI_WARPS>::SMEM_BYTES <= 232448, "smem");
+static_assert(Layout<Cfg<0>::STAGES, Cfg<0>::EPI_WARPS, Cfg<0>::WST>::SMEM_BYTES <= 232448, "smem");
+static_assert(Layout<Cfg<1>::STAGES, Cfg<1>::EPI_WARPS, Cfg<1>::WST>::SMEM_BYTES <= 232448, "smem");
 
 using GemmKernel = void (*)(CUtensorMap, CUtensorMap, int, int, uint32_t, int64_t, int64_t,
                             int64_t, GemmEpilogue, TileSched);
@@ -750,7 +785,7 @@ struct KernelChoice {
 template <int EV, bool BATCH = false>
 KernelChoice choice() {
   return {gemm_tc_kernel<EV, BATCH>, Cfg<EV>::NUM_THREADS,
-          Layout<Cfg<EV>::STAGES, Cfg<EV>::EPI_WARPS>::SMEM_BYTES};
+          Layout<Cfg<EV>::STAGES, Cfg<EV>::EPI_WARPS, Cfg<EV>::WST>::SMEM_BYTES};
 }
 
 // Opt each kernel variant into the large dynamic shared memory once.
