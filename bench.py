@@ -6,8 +6,10 @@ weight side), LWC fake-quant of the weight, per-token activation fake-quant (whe
 configured), the tcgen05 forward GEMM with the fused bias / MSE / dY epilogue, the
 straight-through backward (dW^ and dXq GEMMs, STE reductions, LET gradients) and the AdamW
 update, all through one omq_calib_step call on one stream. Inputs are synthetic and
-resident in HBM when the timed region starts (they follow the LLaMA-7B q_proj shape by
-default: 2048 tokens x 4096 -> 4096, W4A16, group 128, LET learnable).
+resident in HBM when the timed region starts. The default workload is the largest
+single-layer case, the LLaMA-13B down_proj shape (2048 tokens x 13824 -> 5120, W2A16, group
+64, no LET: the layer's input follows the FFN nonlinearity); the q_proj (W4A16 g128, LET),
+gate/up (W4A4 per-channel, LET) and whole-block workloads run with --config.
 
 One process per GPU (torchrun for N > 1): each rank calibrates its own independent layer
 (different seed), with no collective on the data path; the timed region is bracketed by a
@@ -46,7 +48,7 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", default="llama7b_qproj_w4a16g128")
+    ap.add_argument("--config", default="llama13b_down_w2a16g64")
     ap.add_argument("--impl", default="omq", choices=["omq", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -160,19 +162,36 @@ def step_flops(cfg) -> int:
 
 
 def phase_bytes(cfg) -> dict:
-    """Compulsory DRAM bytes of the HBM-bound phases (inputs read once, outputs written once)."""
-    es = 4 if cfg.dtype == "f32" else 2
+    """Algorithmic DRAM bytes of the memory-bound phases of omq_calib_step as the step runs them
+    (16-bit storage, float16 GEMM operands, the weight-side STE fused into the dW^ GEMM, B~
+    fused into the LWC pass): every tensor a phase must read or write, once. The GEMM phases
+    are counted in flops instead."""
+    es = 4 if cfg.dtype == "f32" else 2          # storage of W and X
+    op = 4 if cfg.dtype == "f32" else 2          # GEMM operands Xq, W^, dY
     M, N, K, ng = cfg.m_tokens, cfg.n_out, cfg.k_in, cfg.n_groups
-    act = cfg.let or cfg.abits < 16
-    out = {
-        "lwc": 2 * es * N * K + N * ng * (4 + 4 + 4 + 4 + 16) + 4 * K,
-        "ste_w": es * N * K + 4 * N * K + N * ng * (4 + 4 + 4 + 4 + 16 + 4 + 4),
-        "dbias": es * M * N if cfg.let else 0,
-    }
-    if act:
-        out["let"] = 2 * es * M * K + (es * N * K if cfg.let else 0)
+    grp = N * ng
+    rec = 4 + 4 + 16                             # h, z, range record
+    out = {}
+    # activation side of the forward: X~ (LET), per-token act quant, or the operand conversion
+    if cfg.let or cfg.abits < 16 or cfg.dtype == "bf16":   # bf16 X -> f16 operand at least
+        out["let"] = es * M * K + op * M * K + (M * rec if cfg.abits < 16 else 0)
+    # W, logits (and s, delta) in; W^, h, z, ranges (and B~) out
+    out["lwc"] = es * N * K + 8 * grp + op * N * K + rec * grp + (8 * K + 4 * N if cfg.let else 0)
     if cfg.let:
-        out["ste_x"] = es * M * K + 4 * M * K
+        # dB~: column sums of dY, then the 64-row partials reduced
+        out["dbias"] = op * M * N + 2 * 4 * -(-M // 64) * N
+    if op == 2 and cfg.group % 32 == 0:
+        # fused path: finish reads the per-32-column partials and the group records, writes the
+        # logit gradients and the extremes' shares; with LET the correction pass reads W again
+        fin = 2 * 4 * N * (K // 32) + grp * (4 + 16 + 8) + grp * 8 + (grp * 8 if cfg.let else 0)
+        corr = (es * N * K + grp * (16 + 8) + 4 * N + 2 * 4 * -(-N // 32) * K) if cfg.let else 0
+        out["ste_w"] = fin + corr
+    else:
+        out["ste_w"] = 4 * N * K + es * N * K + grp * (rec + 8 + 8)
+    if cfg.let:
+        # X and the float32 dXq in, per-64-token column partials of d s and d delta out
+        out["ste_x"] = es * M * K + 4 * M * K + 2 * 4 * -(-M // 64) * K + \
+            (M * rec if cfg.abits < 16 else 0)
     return out
 
 
@@ -190,12 +209,18 @@ class ClockSampler(threading.Thread):
         self.samples = []
         self.reasons = 0
         self.ok = False
+        self.uuid = None
         self._halt = threading.Event()
         try:
             import pynvml
+            import torch
+            # NVML numbers the node's GPUs without regard to CUDA_VISIBLE_DEVICES: resolve
+            # the CUDA device by its UUID so the samples come from the GPU this process uses
+            uuid = str(torch.cuda.get_device_properties(index).uuid)
+            self.uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
             pynvml.nvmlInit()
             self.nv = pynvml
-            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(self.uuid)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
             self.ok = True
         except Exception:
@@ -219,10 +244,10 @@ class ClockSampler(threading.Thread):
     def summary(self):
         if not self.ok or not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": getattr(self, "max_mhz", None), "reasons": [],
-                    "samples": 0}
+                    "samples": 0, "gpu_uuid": self.uuid}
         return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
                 "reasons": [n for b, n in self.REASONS.items() if self.reasons & b and b != 0x1],
-                "samples": len(self.samples)}
+                "samples": len(self.samples), "gpu_uuid": self.uuid}
 
 
 def workload_config(cfg):
@@ -439,7 +464,10 @@ def run_omq(args, cfg, rank: int, world: int, local_rank: int):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if cfg.dtype == "bf16" else "f32",
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16" if cfg.dtype == "bf16" else "f32",
+        "dtype_detail": ("bf16 storage of W and X; float16 GEMM operands (Xq, W^, dY) with "
+                         "float32 accumulation; float32 quantizer, STE and AdamW arithmetic"
+                         if cfg.dtype == "bf16" else "float32 throughout"),
         "data": "synthetic (seeded LLaMA-shaped weights and outlier-channel activations)",
         "config": {**workload_config(cfg),
                    "l2": "no flush: the step's working set (W, W^, X, Xq, Y*, dY, dW^, dXq) "

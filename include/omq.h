@@ -88,6 +88,20 @@ int omq_version(void);
  * whose bounded wait expired: OMQ_ERR_TIMEOUT if it was set, OMQ_ERR_CUDA if the
  * synchronization failed, OMQ_OK otherwise. */
 omq_status omq_sync_check(omq_stream_t stream);
+/* Longest time, in nanoseconds, that one barrier wait inside a kernel of this library may
+ * take before the kernel gives up, raises the device error flag and returns (default 2 s).
+ * Per device: applies to the current device. 1 ms <= ns <= 60 s, else OMQ_ERR_SHAPE.
+ * Synchronous with respect to the device (a copy to a device variable); set it between
+ * calls, not while kernels of the library run. */
+omq_status omq_set_wait_limit_ns(uint64_t ns);
+/* The current device's limit (0 if it cannot be read). */
+uint64_t omq_wait_limit_ns(void);
+/* Check of the bounded-wait path: one thread waits on a shared-memory barrier with the wait
+ * the GEMM kernels use. arrive != 0: the thread completes the barrier itself and the wait
+ * returns at once. arrive == 0: nothing completes it, so the wait gives up after the limit
+ * and raises the device error flag; the kernel returns normally and omq_sync_check then
+ * reports OMQ_ERR_TIMEOUT (and clears the flag). The context stays usable either way. */
+omq_status omq_wait_probe(int arrive, omq_stream_t stream);
 
 /* ------------------------------------------------------------------------------------
  * omq_lwc_quant — weight side of the step: LET weight scaling, then Learnable Weight
@@ -169,8 +183,10 @@ size_t omq_fwd_workspace_bytes(int64_t M, int64_t N, int64_t K);
  *   - All calls on a device share it and it keeps the last call's contents; each call writes
  *     every slot it reads first, so nothing needs clearing. Calls that overlap on the GPU
  *     (unordered streams) race on it: order them on one stream.
- *   - The first call on a device looks up the array's address with that device current; make
- *     that first call before any stream capture begins.
+ *   - Each call looks up the array's address in the calling thread's current context (a
+ *     host-side lookup, no cached per-device pointer), so the call stays valid after
+ *     cudaDeviceReset or under another context on the same device. The first call in a
+ *     context also loads the library's module there: make it before any stream capture.
  * ------------------------------------------------------------------------------------ */
 omq_status omq_fq_linear_fwd_noalloc(const void* Xq, const void* W_hat, omq_dtype dt, int64_t M,
                                      int64_t N, int64_t K, const float* B_tilde,

@@ -45,6 +45,8 @@ Pins (tests/test_oracle_block.py): the hand-derived backward against a float64 a
 statement of the block on tiny sizes; LET, affinity and V/o transforms leave the unquantized
 block's output unchanged; causality; RoPE's relative-position property and norm
 preservation; RMSNorm output RMS; the stage functions compose to ``block_step``.
+``block_calibrate`` against torch.optim.AdamW driving that autograd statement over two samples
+and two epochs (tests/test_oracle_calibrate.py).
 """
 from __future__ import annotations
 

@@ -48,8 +48,9 @@ Pins (tests/test_oracle_*.py): the worked affine example; gamma = beta = 1 again
 torch.fake_quantize_per_channel_affine; LET equivalence with quantization off; the
 dequantization error bound; the STE chain against an independent float64 autograd
 statement on tiny inputs; AdamW against torch.optim.AdamW; pack/unpack round trips and a
-hand-packed byte example. Parity unpinned: the multi-step trajectory of ``calibrate`` beyond
-one step (no page prints one).
+hand-packed byte example; the multi-step loop ``calibrate`` against torch.optim.AdamW (two
+parameter groups at the page's two rates) driving that autograd statement for five steps,
+where the bias corrections no longer cancel (tests/test_oracle_calibrate.py).
 """
 from __future__ import annotations
 
@@ -412,7 +413,8 @@ def fold_pack(W, s, gamma_logit, beta_logit, bits: int, group: int):
 def calibrate(X, W, B, Yref, gamma_logit, beta_logit, s, delta, bits, group, abits, let,
               steps: int):
     """The step iterated with AdamW (LWC lr 5e-3 on the logits, LET lr 1e-2 on s, delta).
-    Returns the per-step losses and the final parameters. Parity unpinned beyond step 1."""
+    Returns the per-step losses and the final parameters (pinned over several steps against
+    torch.optim.AdamW driving an independent autograd statement of the step)."""
     gl = np.asarray(gamma_logit, np.float64)
     bl = np.asarray(beta_logit, np.float64)
     sv = np.asarray(s, np.float64)

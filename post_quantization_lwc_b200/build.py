@@ -39,16 +39,34 @@ def _stale(out: str, deps) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
+def _flags_changed(cmdline) -> bool:
+    """True when the compiler and flags differ from those of the last build (recorded in a
+    stamp file beside the objects), so a flag change rebuilds everything."""
+    stamp = os.path.join(BUILD, "flags.stamp")
+    want = "\n".join(cmdline)
+    have = None
+    if os.path.exists(stamp):
+        with open(stamp) as f:
+            have = f.read()
+    if have != want:
+        with open(stamp, "w") as f:
+            f.write(want)
+        return True
+    return False
+
+
 def build(force: bool = False, verbose: bool = False, extra=()) -> str:
     os.makedirs(BUILD, exist_ok=True)
     headers = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")]
     headers.append(os.path.join(ROOT, "include", "omq.h"))
+    compiler = nvcc()
+    force = _flags_changed([compiler, *ARCH, *FLAGS, *extra]) or force
     objs, jobs = [], []
     for src in sources():
         obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
         objs.append(obj)
         if force or _stale(obj, [src, *headers]):
-            jobs.append([nvcc(), *ARCH, *FLAGS, *extra, "-dc" if False else "-c", src, "-o", obj])
+            jobs.append([compiler, *ARCH, *FLAGS, *extra, "-c", src, "-o", obj])
     def run(cmd):
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
@@ -59,7 +77,7 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
             if verbose and msg:
                 print(msg, file=sys.stderr)
     if force or jobs or _stale(LIB, objs):
-        run([nvcc(), *ARCH, "-shared", "-o", LIB, *objs])
+        run([compiler, *ARCH, "-shared", "-o", LIB, *objs])
     return LIB
 
 

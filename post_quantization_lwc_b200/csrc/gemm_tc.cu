@@ -39,12 +39,21 @@
 namespace omq {
 
 __device__ unsigned g_dev_error = 0;
+// Longest time one barrier wait may take before the waiting kernel gives up (nanoseconds).
+__device__ uint64_t g_wait_limit_ns = 2000000000ull;
 
 cudaError_t take_device_error(unsigned* flag) {
   unsigned zero = 0;
   cudaError_t e = cudaMemcpyFromSymbol(flag, g_dev_error, sizeof(unsigned));
   if (e == cudaSuccess && *flag) e = cudaMemcpyToSymbol(g_dev_error, &zero, sizeof(unsigned));
   return e;
+}
+
+cudaError_t set_wait_limit(uint64_t ns) {
+  return cudaMemcpyToSymbol(g_wait_limit_ns, &ns, sizeof(ns));
+}
+cudaError_t get_wait_limit(uint64_t* ns) {
+  return cudaMemcpyFromSymbol(ns, g_wait_limit_ns, sizeof(*ns));
 }
 
 namespace tc {
@@ -71,7 +80,6 @@ struct Cfg {
   static constexpr int WST = EV ? 32 * 64 * 2 : 0;
   static constexpr bool SLEEPY = EV != 0;
 };
-constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;   // 2 s per barrier wait
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -135,12 +143,13 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Wait until the phase with the given parity has completed, for at most WAIT_LIMIT_NS.
+// Wait until the phase with the given parity has completed, for at most g_wait_limit_ns.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned err_bit) {
   if (mbar_try(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
+  const uint64_t limit = *const_cast<volatile uint64_t*>(&g_wait_limit_ns);
   while (!mbar_try(bar, parity)) {
-    if (globaltimer() - t0 > WAIT_LIMIT_NS) {
+    if (globaltimer() - t0 > limit) {
       atomicOr(&g_dev_error, err_bit);
       return false;
     }
@@ -154,10 +163,11 @@ __device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity, u
                                                 uint32_t sleep_ns) {
   if (mbar_try(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
+  const uint64_t limit = *const_cast<volatile uint64_t*>(&g_wait_limit_ns);
   for (uint32_t n = 1;; ++n) {
     __nanosleep(sleep_ns);
     if (mbar_try(bar, parity)) return true;
-    if ((n & 15) == 0 && globaltimer() - t0 > WAIT_LIMIT_NS) {
+    if ((n & 15) == 0 && globaltimer() - t0 > limit) {
       atomicOr(&g_dev_error, err_bit);
       return false;
     }
@@ -699,6 +709,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV>::NUM_THREADS
   }
 }
 
+// Bounded-wait probe: one thread initialises a shared-memory barrier for one arrival, arrives
+// on it only when `arrive` is set, and waits for its first phase with the same bounded wait
+// the GEMM's roles use. Without the arrival nothing can complete the phase, so the wait gives
+// up after g_wait_limit_ns, raises DEV_ERR_PROBE_WAIT and the kernel returns normally: the
+// path a GEMM takes when one of its barriers never completes, without a GEMM around it.
+__global__ void wait_probe_kernel(int arrive) {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = smem_u32(&bar);
+  mbar_init(b, 1);
+  if (arrive) mbar_arrive_local(b);
+  mbar_wait(b, 0, DEV_ERR_PROBE_WAIT);
+}
+
 // ------------------------------------------------------------------------------- host side
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -803,6 +826,11 @@ cudaError_t kernel_attr(GemmKernel k, int smem) {
 }
 
 }  // namespace tc
+
+omq_status launch_wait_probe(int arrive, cudaStream_t stream) {
+  tc::wait_probe_kernel<<<1, 1, 0, stream>>>(arrive);
+  return launch_status();
+}
 
 // Loss partial slots: one per 128-row half of each 256 x 256 output tile.
 int64_t gemm_tc_tiles(int64_t rows, int64_t cols) {

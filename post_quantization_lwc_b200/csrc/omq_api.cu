@@ -217,6 +217,25 @@ int omq_last_cuda_error(void) { return t_last_cuda_error; }
 
 int omq_version(void) { return 10000; }
 
+omq_status omq_set_wait_limit_ns(uint64_t ns) {
+  if (ns < 1000000ull || ns > 60000000000ull) return OMQ_ERR_SHAPE;
+  const cudaError_t e = set_wait_limit(ns);
+  if (e != cudaSuccess) {
+    set_cuda_error(e);
+    return OMQ_ERR_CUDA;
+  }
+  return OMQ_OK;
+}
+
+uint64_t omq_wait_limit_ns(void) {
+  uint64_t ns = 0;
+  return get_wait_limit(&ns) == cudaSuccess ? ns : 0;
+}
+
+omq_status omq_wait_probe(int arrive, omq_stream_t stream) {
+  return launch_wait_probe(arrive != 0, reinterpret_cast<cudaStream_t>(stream));
+}
+
 omq_status omq_sync_check(omq_stream_t stream) {
   cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) {

@@ -18,8 +18,14 @@ namespace omq {
 // Raised (bitwise OR) by kernels whose bounded barrier waits expired; read by
 // omq_sync_check(). Bit values say which wait gave up. The flag lives in gemm_tc.cu (the
 // only translation unit with barrier waits); the host reads and clears it through this call.
-enum : unsigned { DEV_ERR_TMA_WAIT = 1u, DEV_ERR_MMA_WAIT = 2u, DEV_ERR_EPI_WAIT = 4u };
+enum : unsigned {
+  DEV_ERR_TMA_WAIT = 1u, DEV_ERR_MMA_WAIT = 2u, DEV_ERR_EPI_WAIT = 4u, DEV_ERR_PROBE_WAIT = 8u
+};
 cudaError_t take_device_error(unsigned* flag);
+// The device-side limit of one barrier wait, in nanoseconds (per device, default 2 s).
+cudaError_t set_wait_limit(uint64_t ns);
+cudaError_t get_wait_limit(uint64_t* ns);
+omq_status launch_wait_probe(int arrive, cudaStream_t stream);
 
 constexpr float H_FLOOR = 1e-8f;          // floor of the quantization step h
 constexpr int Z_LIMIT = 1 << 30;          // |z| stored as int32 is clamped to this

@@ -19,44 +19,32 @@
 //     Each call writes every slot it reads before reading it, so nothing needs clearing.
 //     Calls whose work overlaps on the GPU (different streams with no ordering between them)
 //     race on the array and may return a wrong loss; order such calls on one stream.
-//   - The first call on each device looks up the array's device address with that device
-//     current (cudaGetSymbolAddress) and keeps it; make that first call before any stream
-//     capture begins.
-#include <mutex>
-
+//   - Every call looks up the array's device address in the calling thread's current
+//     context (cudaGetSymbolAddress, a host-side lookup) instead of caching it per device
+//     ordinal: after cudaDeviceReset, or with another context current on the same device, a
+//     cached address would name memory of a context that no longer owns it. The first call in
+//     a context also loads the library's module there; make that first call before any
+//     stream capture begins.
 #include "omq_internal.cuh"
 
 namespace omq {
 namespace {
 
 constexpr int64_t kNoAllocTiles = 16384;
-constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) float g_noalloc_loss_partials[kNoAllocTiles];
 
-std::mutex g_noalloc_mu;
-float* g_noalloc_ptr[kMaxDevices] = {};
-
-// Device address of the fixed scratch array for the current device (looked up once).
+// Device address of the fixed scratch array in the current context. Looked up on every call:
+// the address belongs to the module instance of the context that is current now, which a
+// cache keyed by device ordinal cannot tell apart from one that was reset or replaced.
 omq_status noalloc_scratch(float** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) {
-    set_cuda_error(e);
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_loss_partials);
+  if (e != cudaSuccess || p == nullptr) {
+    set_cuda_error(e != cudaSuccess ? e : cudaErrorInvalidSymbol);
     return OMQ_ERR_CUDA;
   }
-  if (dev < 0 || dev >= kMaxDevices) return OMQ_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_loss_partials);
-    if (e != cudaSuccess || p == nullptr) {
-      set_cuda_error(e != cudaSuccess ? e : cudaErrorInvalidSymbol);
-      return OMQ_ERR_CUDA;
-    }
-    g_noalloc_ptr[dev] = static_cast<float*>(p);
-  }
-  *out = g_noalloc_ptr[dev];
+  *out = static_cast<float*>(p);
   return OMQ_OK;
 }
 

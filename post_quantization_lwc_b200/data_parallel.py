@@ -48,16 +48,26 @@ class DataParallelBlock:
         self.n_lwc = blk.theta_slices["s1"][0]     # the LWC logits precede the LET vectors
 
     def step(self, x, y_ref, stream=None):
+        """One data-parallel step. With ``stream`` given, the whole step (the block kernels,
+        the all-reduce and the update) is ordered on that stream: it becomes the current
+        stream for the duration, since a collective orders itself against the current stream
+        of its caller, not against the stream its inputs were produced on."""
+        if stream is not None and stream != torch.cuda.current_stream(stream.device):
+            with torch.cuda.stream(stream):
+                return self._step(x, y_ref)
+        return self._step(x, y_ref)
+
+    def _step(self, x, y_ref):
         from . import omq
         blk = self.blk
-        blk.step(x, y_ref, update=False, stream=stream)
+        blk.step(x, y_ref, update=False)
         allreduce_mean_([blk.d_theta, blk.loss], self.group)
         blk.t += 1
         n = self.n_lwc
         omq.adamw_step(blk.theta[:n], blk.d_theta[:n], blk.adam_m[:n], blk.adam_v[:n],
-                       blk.lr_lwc, blk.t, stream=stream)
+                       blk.lr_lwc, blk.t)
         omq.adamw_step(blk.theta[n:], blk.d_theta[n:], blk.adam_m[n:], blk.adam_v[n:],
-                       blk.lr_let, blk.t, stream=stream)
+                       blk.lr_let, blk.t)
         return blk.loss
 
     def calibrate(self, xs, y_refs, epochs: int):

@@ -32,7 +32,8 @@ EXPORTS = ("omq_status_str", "omq_last_cuda_error", "omq_version", "omq_sync_che
            "omq_calib_step", "omq_step_workspace_bytes", "omq_launch_count",
            "omq_fq_linear_fwd_noalloc", "omq_block_theta_range", "omq_block_buffer",
            "omq_block_workspace_bytes", "omq_block_step", "omq_block_reference",
-           "omq_block_quant_forward", "omq_block_calibrate", "omq_qgemv")
+           "omq_block_quant_forward", "omq_block_calibrate", "omq_qgemv",
+           "omq_set_wait_limit_ns", "omq_wait_limit_ns", "omq_wait_probe")
 
 _p = ctypes.c_void_p
 _i64 = ctypes.c_int64
@@ -135,6 +136,9 @@ _sig("omq_block_quant_forward", _i32, [ctypes.POINTER(BlockDims), _p, _p, _p, _p
                                        _i32, _p, _sz, _p])
 _sig("omq_block_calibrate", _i32, [ctypes.POINTER(BlockCalibArgs), _p, _sz, _p])
 _sig("omq_qgemv", _i32, [_p, _i32, _i64, _i64, _p, _p, _p, _i64, _i64, _i32, _p, _p])
+_sig("omq_set_wait_limit_ns", _i32, [ctypes.c_uint64])
+_sig("omq_wait_limit_ns", ctypes.c_uint64, [])
+_sig("omq_wait_probe", _i32, [_i32, _p])
 
 
 def _check(status: int, where: str):
@@ -184,6 +188,18 @@ def launch_count() -> int:
 
 def sync_check(stream=None):
     _check(_lib.omq_sync_check(_stream(stream)), "omq_sync_check")
+
+
+def set_wait_limit_ns(ns: int):
+    _check(_lib.omq_set_wait_limit_ns(ctypes.c_uint64(int(ns))), "omq_set_wait_limit_ns")
+
+
+def wait_limit_ns() -> int:
+    return int(_lib.omq_wait_limit_ns())
+
+
+def wait_probe(arrive: bool, stream=None):
+    _check(_lib.omq_wait_probe(1 if arrive else 0, _stream(stream)), "omq_wait_probe")
 
 
 def new_range(n: int, device) -> torch.Tensor:

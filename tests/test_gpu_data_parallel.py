@@ -70,3 +70,23 @@ def test_one_rank_calibrate_matches_the_library_loop(omq, cuda_device):
     assert _same(la, lb)
     assert _same(a.theta, b.theta)
     assert _same(a.adam_v, b.adam_v)
+
+
+def test_side_stream_step_matches_the_in_place_update(omq, cuda_device):
+    """The step given a stream that is not the current one: kernels, exchange and update all
+    run on that stream, so the result is bitwise the in-place step's."""
+    from post_quantization_lwc_b200.data_parallel import DataParallelBlock
+    (a, b), xs, ys = _blocks(omq, cuda_device)
+    dp = DataParallelBlock(b)
+    side = torch.cuda.Stream(device=cuda_device)
+    side.wait_stream(torch.cuda.current_stream())
+    for i in range(3):
+        la = a.step(xs[i], ys[i]).clone()
+        lb = dp.step(xs[i], ys[i], stream=side)
+        side.synchronize()
+        lb = lb.clone()
+        torch.cuda.synchronize()
+        omq.sync_check()
+        assert _same(la, lb)
+    for name in ("theta", "adam_m", "adam_v", "d_theta"):
+        assert _same(getattr(a, name), getattr(b, name)), name
