@@ -173,7 +173,7 @@ def phase_bytes(cfg) -> dict:
     rec = 4 + 4 + 16                             # h, z, range record
     out = {}
     # activation side of the forward: X~ (LET), per-token act quant, or the operand conversion
-    if cfg.let or cfg.abits < 16 or cfg.dtype == "bf16":   # bf16 X -> f16 operand at least
+    if cfg.let or cfg.abits < 16:   # otherwise X itself is the GEMM operand: no pass
         out["let"] = es * M * K + op * M * K + (M * rec if cfg.abits < 16 else 0)
     # W, logits (and s, delta) in; W^, h, z, ranges (and B~) out
     out["lwc"] = es * N * K + 8 * grp + op * N * K + rec * grp + (8 * K + 4 * N if cfg.let else 0)
@@ -441,6 +441,7 @@ def run_omq(args, cfg, rank: int, world: int, local_rank: int):
         return 0
 
     peaks, peak_src = load_peaks()
+    op_name = {torch.float16: "f16", torch.bfloat16: "bf16", torch.float32: "f32"}[lc.op_dtype]
     value = world * args.steps / (ms / 1e3)
     gemm_keys = ["fwd_gemm", "dw_gemm"] + (["dx_gemm"] if cfg.let else [])
     gemm_ms = sum(phases[k] for k in gemm_keys) / len(gemm_keys)
@@ -464,10 +465,10 @@ def run_omq(args, cfg, rank: int, world: int, local_rank: int):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f16" if cfg.dtype == "bf16" else "f32",
-        "dtype_detail": ("bf16 storage of W and X; float16 GEMM operands (Xq, W^, dY) with "
-                         "float32 accumulation; float32 quantizer, STE and AdamW arithmetic"
-                         if cfg.dtype == "bf16" else "float32 throughout"),
+        "scaling": "weak", "vs_baseline": None, "dtype": op_name,
+        "dtype_detail": (f"{cfg.dtype} storage of W and X; {op_name} GEMM operands (Xq, W^, "
+                         "dY) with float32 accumulation; float32 quantizer, STE and AdamW "
+                         "arithmetic" if cfg.dtype == "bf16" else "float32 throughout"),
         "data": "synthetic (seeded LLaMA-shaped weights and outlier-channel activations)",
         "config": {**workload_config(cfg),
                    "l2": "no flush: the step's working set (W, W^, X, Xq, Y*, dY, dW^, dXq) "

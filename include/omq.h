@@ -29,8 +29,9 @@
  *     OMQ_ERR_CUDA (the CUDA code is kept in omq_last_cuda_error()). No call aborts, throws
  *     or traps. Kernels that wait on barriers give up after a bounded time and raise a
  *     device error flag that omq_sync_check() reports as OMQ_ERR_TIMEOUT.
- *   - Dtypes. W and X (and their fake-quant copies, and dY) are OMQ_BF16 or OMQ_F32;
- *     all learnable parameters, scales, gradients and losses are float32.
+ *   - Dtypes. W and X are stored as OMQ_BF16, OMQ_F16 or OMQ_F32; their fake-quant copies
+ *     and dY (the GEMM operands) as OMQ_F16, OMQ_BF16 or OMQ_F32 (see omq_dtype); all
+ *     learnable parameters, scales, gradients and losses are float32.
  *   - Rounding. round() is round-half-to-even. h, z and codes follow one fixed binary32
  *     operation order (no fused multiply-add, IEEE division):
  *        W~ = W*s;  h = max(((g*M) - (b*m)) / Q, 1e-8);  z = -round((b*m)/h)
@@ -351,7 +352,8 @@ size_t omq_step_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t group);
  * The backward is the straight-through chain of every quantizer (omq_fq_linear_bwd's rule)
  * through the whole block; it fills d_theta for every learnable tensor.
  *
- * Storage: x, the weights and every GEMM operand BF16; y_ref, theta, gradients float32.
+ * Storage: x and the weights BF16; the GEMM operands of the calibration step float16 (those
+ * of omq_block_reference BF16, the weights' own type); y_ref, theta, gradients float32.
  * Weights: W_qkv [3D, D] (rows of q_proj, then k_proj, then v_proj), W_o [D, D],
  * W_gu [2I, D] (rows of gate_proj, then up_proj), W_d [D, I].
  * ==================================================================================== */
@@ -382,29 +384,31 @@ omq_status omq_block_theta_range(const omq_block_dims* dims, int id, int64_t* of
 enum {
   OMQ_BB_ROPE = 0,   /* float32 [2, M, 64]: cos, then sin, of the rotation angles */
   OMQ_BB_A,          /* float32 [M, D]  RMSNorm(x) */
-  OMQ_BB_QA,         /* BF16 [M, D]     qa */
-  OMQ_BB_WHAT_QKV,   /* BF16 [3D, D]    Ŵ_qkv (then _O, _GU, _D) */
+  OMQ_BB_QA,         /* F16 [M, D]      qa */
+  OMQ_BB_WHAT_QKV,   /* F16 [3D, D]     Ŵ_qkv (then _O, _GU, _D) */
   OMQ_BB_WHAT_O, OMQ_BB_WHAT_GU, OMQ_BB_WHAT_D,
   OMQ_BB_QKV,        /* float32 [M, 3D] q | k | v */
-  OMQ_BB_QQKV,       /* BF16 [M, 3D]    Qq | Qk | Qv */
+  OMQ_BB_QQKV,       /* F16 [M, 3D]     Qq | Qk | Qv */
   OMQ_BB_P,          /* float32 [H, M, M] softmax (zero above the diagonal) */
-  OMQ_BB_P16,        /* BF16 [H, M, M]  the same, GEMM operand */
+  OMQ_BB_P16,        /* F16 [H, M, M]   the same, GEMM operand */
   OMQ_BB_O,          /* float32 [M, D]  attention output */
-  OMQ_BB_QO,         /* BF16 [M, D]     Q_a(O) */
+  OMQ_BB_QO,         /* F16 [M, D]      Q_a(O) */
   OMQ_BB_X2,         /* float32 [M, D]  x2 */
   OMQ_BB_B,          /* float32 [M, D]  RMSNorm(x2) */
-  OMQ_BB_QB,         /* BF16 [M, D]     qb */
+  OMQ_BB_QB,         /* F16 [M, D]      qb */
   OMQ_BB_GU,         /* float32 [M, 2I] gate | up */
   OMQ_BB_MID,        /* float32 [M, I]  m = SiLU(gate) up */
-  OMQ_BB_QM,         /* BF16 [M, I]     Q_a(m) */
-  OMQ_BB_RES,        /* BF16 [M, D]     y - y_ref (the loss gradient is 2 res / (M D)) */
+  OMQ_BB_QM,         /* F16 [M, I]      Q_a(m) */
+  OMQ_BB_RES,        /* F16 [M, D]      y - y_ref (the loss gradient is 2 res / (M D)) */
+  /* The gradients below are those of (M D / 2) L, i.e. in units of res (float16 would not
+   * hold the true ones, 2 / (M D) times smaller); d_theta carries the factor 2 / (M D). */
   OMQ_BB_DMID,       /* float32 [M, I]  dL/dm */
-  OMQ_BB_DGU,        /* BF16 [M, 2I]    dL/d[gate | up] */
+  OMQ_BB_DGU,        /* F16 [M, 2I]     dL/d[gate | up] */
   OMQ_BB_DB,         /* float32 [M, D]  dL/db */
-  OMQ_BB_DX2,        /* BF16 [M, D]     dL/dx2 */
-  OMQ_BB_DO,         /* BF16 [M, D]     dL/dO */
+  OMQ_BB_DX2,        /* F16 [M, D]      dL/dx2 */
+  OMQ_BB_DO,         /* F16 [M, D]      dL/dO */
   OMQ_BB_DQQKV,      /* float32 [M, 3D] dL/d[Qq | Qk | Qv] */
-  OMQ_BB_DQKV,       /* BF16 [M, 3D]    dL/d[q | k | v] */
+  OMQ_BB_DQKV,       /* F16 [M, 3D]     dL/d[q | k | v] */
   OMQ_BB_COUNT
 };
 omq_status omq_block_buffer(const omq_block_dims* dims, int id, size_t* offset, size_t* bytes);

@@ -8,7 +8,9 @@
 // weight-side STE fused into the dW GEMM). Attention runs on the same GEMM, all heads of a
 // product in one launch, the causal structure skipping the tiles and contraction blocks the
 // mask zeroes; scores and probabilities are materialised in float32.
+#include <algorithm>
 #include <cmath>
+#include <initializer_list>
 #include <vector>
 
 #include "block_internal.cuh"
@@ -93,6 +95,7 @@ struct BlockLayout {
   size_t rstd2, tgt, o_out, loss_part, dP, dS, dxq;
   size_t gh_part, gc_part, emax, emin, dbt_part, dbt, rowstat, red;
   size_t part_sa, part_so, part_do;
+  size_t sk, sk_bytes;   // stream-K scratch of the linears' GEMMs (one at a time)
   size_t total;
   int64_t loss_tiles;
 };
@@ -175,6 +178,13 @@ BlockLayout block_layout(const omq_block_dims& d) {
   L.part_sa = take(f4 * ceil_div(M, kAttnRows) * D);
   L.part_so = take(f4 * ceil_div(M, kAttnRows) * D);
   L.part_do = take(f4 * ceil_div(M, kAttnRows) * D);
+  L.sk_bytes = 0;
+  for (int l = 0; l < L_COUNT; ++l) {
+    const LinShape s = lin_shape(d, l);
+    L.sk_bytes = std::max({L.sk_bytes, gemm_tc_sk_bytes(M, s.N), gemm_tc_sk_bytes(s.N, s.K),
+                           gemm_tc_sk_bytes(M, s.K)});
+  }
+  L.sk = take(L.sk_bytes);
   L.total = off;
   return L;
 }
@@ -199,20 +209,22 @@ struct Marks {
 };
 
 
-omq_status gemm_store(const GemmOperand& A, const GemmOperand& B, int64_t rows, int64_t cols,
-                      int64_t depth, float* out, int64_t ldo, float scale, const float* bias,
-                      cudaStream_t st) {
+omq_status gemm_store(omq_dtype op, const GemmOperand& A, const GemmOperand& B, int64_t rows,
+                      int64_t cols, int64_t depth, float* out, int64_t ldo, float scale,
+                      const float* bias, void* sk, size_t sk_bytes, cudaStream_t st) {
   GemmEpilogue e{};
+  e.sk_scratch = sk;
+  e.sk_bytes = sk_bytes;
   e.kind = Epi::StoreF32;
   e.out = out;
   e.ldo = ldo;
   e.out_scale = scale;
   e.bias = bias;
-  return gemm_tc(OMQ_BF16, A, B, rows, cols, depth, e, nullptr, st);
+  return gemm_tc(op, A, B, rows, cols, depth, e, nullptr, st);
 }
 
 // The attention products, all heads in one launch each (heads are the batch).
-omq_status gemm_heads(const GemmOperand& A, int64_t a_stride, const GemmOperand& B,
+omq_status gemm_heads(omq_dtype op, const GemmOperand& A, int64_t a_stride, const GemmOperand& B,
                       int64_t b_stride, int64_t rows, int64_t cols, int64_t depth, float* out,
                       int64_t ldo, int64_t out_stride, float scale, int64_t heads, int causal,
                       cudaStream_t st) {
@@ -222,14 +234,14 @@ omq_status gemm_heads(const GemmOperand& A, int64_t a_stride, const GemmOperand&
   e.ldo = ldo;
   e.out_scale = scale;
   const GemmBatch b{heads, a_stride, b_stride, out_stride, causal};
-  return gemm_tc(OMQ_BF16, A, B, rows, cols, depth, e, nullptr, st, &b);
+  return gemm_tc(op, A, B, rows, cols, depth, e, nullptr, st, &b);
 }
 
-omq_status act_quant(const void* X, omq_dtype xdt, int64_t M, int64_t K, const float* s,
-                     const float* d, int abits, void* Xq, float* h_a, int32_t* z_a,
+omq_status act_quant(omq_dtype op, const void* X, omq_dtype xdt, int64_t M, int64_t K,
+                     const float* s, const float* d, int abits, void* Xq, float* h_a, int32_t* z_a,
                      omq_range* range, cudaStream_t st) {
   LetParams p{X, xdt, M, K, s, d, static_cast<float>((1 << (abits < 16 ? abits : 1)) - 1), Xq,
-              OMQ_BF16, h_a, z_a, range};
+              op, h_a, z_a, range};
   return launch_let(p, abits, st);
 }
 
@@ -261,6 +273,10 @@ omq_status block_forward(const View& v, const Inputs& in, const Marks& mk, cudaS
   const int64_t M = d.M, D = d.D, H = d.H, I = d.I;
   const bool fp = in.theta == nullptr;
   const int abits = fp ? 16 : d.abits;
+  // GEMM operands: float16 for the fake-quantized block (its operands and the gradients
+  // that flow back through them keep 3 more mantissa bits than bfloat16); the full-precision
+  // block multiplies the bfloat16 weights themselves
+  const omq_dtype op = fp ? OMQ_BF16 : OMQ_F16;
   const float Qw = static_cast<float>((1 << d.wbits) - 1);
   int64_t toff[OMQ_TH_COUNT + 1], tcnt[OMQ_TH_COUNT + 1];
   theta_ranges(d, toff, tcnt);
@@ -283,7 +299,7 @@ omq_status block_forward(const View& v, const Inputs& in, const Marks& mk, cudaS
     const int64_t G = group_of(d, s.K);
     const LinScratch& c = L.lin[l];
     LwcParams p{in.W[l], OMQ_BF16, s.N, s.K, G, s.K / G, Qw, th(OMQ_TH_GAMMA_QKV + 2 * l),
-                th(OMQ_TH_BETA_QKV + 2 * l), s_w[l], v.bb<void>(what_id[l]), OMQ_BF16,
+                th(OMQ_TH_BETA_QKV + 2 * l), s_w[l], v.bb<void>(what_id[l]), op,
                 v.in<float>(c.h), v.in<int32_t>(c.z), nullptr, v.in<omq_range>(c.range), nullptr,
                 d.wbits};
     if (dl_w[l]) {   // B~ = W delta out of the same pass over W
@@ -302,11 +318,12 @@ omq_status block_forward(const View& v, const Inputs& in, const Marks& mk, cudaS
                 nullptr, nullptr};
     BLK_TRY(launch_rms(r, st));
   }
-  BLK_TRY(act_quant(v.bb<float>(OMQ_BB_A), OMQ_F32, M, D, th(OMQ_TH_S1), th(OMQ_TH_DELTA1), abits,
+  BLK_TRY(act_quant(op, v.bb<float>(OMQ_BB_A), OMQ_F32, M, D, th(OMQ_TH_S1), th(OMQ_TH_DELTA1), abits,
                     v.bb<void>(OMQ_BB_QA), v.in<float>(L.act_h[0]), v.in<int32_t>(L.act_z[0]),
                     v.in<omq_range>(L.act_range[0]), st));
-  BLK_TRY(gemm_store(GemmOperand{v.bb<void>(OMQ_BB_QA), D, false}, GemmOperand{Wop[L_QKV], D, false},
-                     M, 3 * D, D, v.bb<float>(OMQ_BB_QKV), 0, 1.f, bias(L_QKV), st));
+  BLK_TRY(gemm_store(op, GemmOperand{v.bb<void>(OMQ_BB_QA), D, false}, GemmOperand{Wop[L_QKV], D, false},
+                     M, 3 * D, D, v.bb<float>(OMQ_BB_QKV), 0, 1.f, bias(L_QKV), v.in<char>(L.sk),
+                     L.sk_bytes, st));
   {
     AttnPrepParams p{};
     p.qkv = v.bb<float>(OMQ_BB_QKV);
@@ -318,7 +335,8 @@ omq_status block_forward(const View& v, const Inputs& in, const Marks& mk, cudaS
     p.M = M; p.D = D; p.H = H;
     p.quantized = abits < 16 ? 1 : 0;
     p.Qa = static_cast<float>((1 << (abits < 16 ? abits : 1)) - 1);
-    p.out = v.bb<__nv_bfloat16>(OMQ_BB_QQKV);
+    p.out = v.bb<void>(OMQ_BB_QQKV);
+    p.dt16 = op;
     p.h_s = v.in<float>(L.head_h);
     p.z_s = v.in<int32_t>(L.head_z);
     p.range_s = v.in<omq_range>(L.head_range);
@@ -327,35 +345,39 @@ omq_status block_forward(const View& v, const Inputs& in, const Marks& mk, cudaS
   // attention, one head at a time: S = Qq Qk^T / sqrt(128), P = causal softmax, O = P Qv
   BLK_TRY(mk.mark(OMQ_BPH_ATTN));
   {
-    const __nv_bfloat16* qqkv = v.bb<__nv_bfloat16>(OMQ_BB_QQKV);
+    const uint16_t* qqkv = v.bb<uint16_t>(OMQ_BB_QQKV);
     float* P = v.bb<float>(OMQ_BB_P);
-    __nv_bfloat16* P16 = v.bb<__nv_bfloat16>(OMQ_BB_P16);
+    uint16_t* P16 = v.bb<uint16_t>(OMQ_BB_P16);
     const float scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(kHead)));
-    BLK_TRY(gemm_heads(GemmOperand{qqkv, 3 * D, false}, kHead, GemmOperand{qqkv + D, 3 * D, false},
-                       kHead, M, M, kHead, P, 0, M * M, scale, H, 1, st));
-    BLK_TRY(launch_softmax(P, P16, H * M, M, st));
-    BLK_TRY(gemm_heads(GemmOperand{P16, M, false}, M * M, GemmOperand{qqkv + 2 * D, 3 * D, true},
-                       kHead, M, kHead, M, v.bb<float>(OMQ_BB_O), D, kHead, 1.f, H, 2, st));
+    BLK_TRY(gemm_heads(op, GemmOperand{qqkv, 3 * D, false}, kHead,
+                       GemmOperand{qqkv + D, 3 * D, false}, kHead, M, M, kHead, P, 0, M * M, scale,
+                       H, 1, st));
+    BLK_TRY(launch_softmax(P, P16, op, H * M, M, st));
+    BLK_TRY(gemm_heads(op, GemmOperand{P16, M, false}, M * M,
+                       GemmOperand{qqkv + 2 * D, 3 * D, true}, kHead, M, kHead, M,
+                       v.bb<float>(OMQ_BB_O), D, kHead, 1.f, H, 2, st));
   }
   // o_proj, residual, RMSNorm, gate / up, SwiGLU, down (+ loss)
   BLK_TRY(mk.mark(OMQ_BPH_FFN));
-  BLK_TRY(act_quant(v.bb<float>(OMQ_BB_O), OMQ_F32, M, D, nullptr, nullptr, abits,
+  BLK_TRY(act_quant(op, v.bb<float>(OMQ_BB_O), OMQ_F32, M, D, nullptr, nullptr, abits,
                     v.bb<void>(OMQ_BB_QO), v.in<float>(L.act_h[1]), v.in<int32_t>(L.act_z[1]),
                     v.in<omq_range>(L.act_range[1]), st));
-  BLK_TRY(gemm_store(GemmOperand{v.bb<void>(OMQ_BB_QO), D, false}, GemmOperand{Wop[L_O], D, false},
-                     M, D, D, v.in<float>(L.o_out), 0, 1.f, bias(L_O), st));
+  BLK_TRY(gemm_store(op, GemmOperand{v.bb<void>(OMQ_BB_QO), D, false}, GemmOperand{Wop[L_O], D, false},
+                     M, D, D, v.in<float>(L.o_out), 0, 1.f, bias(L_O), v.in<char>(L.sk),
+                     L.sk_bytes, st));
   {
     RmsParams r{in.x, OMQ_BF16, v.in<float>(L.o_out), M, D, kEps, v.bb<float>(OMQ_BB_X2),
                 v.bb<float>(OMQ_BB_B), v.in<float>(L.rstd2), in.y_ref, v.in<float>(L.tgt)};
     BLK_TRY(launch_rms(r, st));
   }
-  BLK_TRY(act_quant(v.bb<float>(OMQ_BB_B), OMQ_F32, M, D, th(OMQ_TH_S2), th(OMQ_TH_DELTA2), abits,
+  BLK_TRY(act_quant(op, v.bb<float>(OMQ_BB_B), OMQ_F32, M, D, th(OMQ_TH_S2), th(OMQ_TH_DELTA2), abits,
                     v.bb<void>(OMQ_BB_QB), v.in<float>(L.act_h[2]), v.in<int32_t>(L.act_z[2]),
                     v.in<omq_range>(L.act_range[2]), st));
-  BLK_TRY(gemm_store(GemmOperand{v.bb<void>(OMQ_BB_QB), D, false}, GemmOperand{Wop[L_GU], D, false},
-                     M, 2 * I, D, v.bb<float>(OMQ_BB_GU), 0, 1.f, bias(L_GU), st));
+  BLK_TRY(gemm_store(op, GemmOperand{v.bb<void>(OMQ_BB_QB), D, false}, GemmOperand{Wop[L_GU], D, false},
+                     M, 2 * I, D, v.bb<float>(OMQ_BB_GU), 0, 1.f, bias(L_GU), v.in<char>(L.sk),
+                     L.sk_bytes, st));
   BLK_TRY(launch_swiglu(v.bb<float>(OMQ_BB_GU), v.bb<float>(OMQ_BB_MID), M, I, st));
-  BLK_TRY(act_quant(v.bb<float>(OMQ_BB_MID), OMQ_F32, M, I, nullptr, nullptr, abits,
+  BLK_TRY(act_quant(op, v.bb<float>(OMQ_BB_MID), OMQ_F32, M, I, nullptr, nullptr, abits,
                     v.bb<void>(OMQ_BB_QM), v.in<float>(L.act_h[3]), v.in<int32_t>(L.act_z[3]),
                     v.in<omq_range>(L.act_range[3]), st));
   {
@@ -365,9 +387,11 @@ omq_status block_forward(const View& v, const Inputs& in, const Marks& mk, cudaS
     e.kind = Epi::MseLoss;
     e.y_ref = v.in<float>(L.tgt);
     e.dy = in.y_ref ? v.bb<void>(OMQ_BB_RES) : in.y_out;
-    e.dy_dt = in.y_ref ? OMQ_BF16 : in.y_dt;
+    e.dy_dt = in.y_ref ? op : in.y_dt;
     e.loss_partials = v.in<float>(L.loss_part);
-    BLK_TRY(gemm_tc(OMQ_BF16, GemmOperand{v.bb<void>(OMQ_BB_QM), I, false},
+    e.sk_scratch = v.in<char>(L.sk);
+    e.sk_bytes = L.sk_bytes;
+    BLK_TRY(gemm_tc(op, GemmOperand{v.bb<void>(OMQ_BB_QM), I, false},
                     GemmOperand{Wop[L_D], I, false}, M, D, I, e, nullptr, st));
   }
   return OMQ_OK;
@@ -379,6 +403,7 @@ omq_status block_forward(const View& v, const Inputs& in, const Marks& mk, cudaS
 // and its completion (LWC logit gradients, W-side LET column partials), the dX GEMM and the
 // activation-side STE (dX~ / s_x stored in dX when asked, X-side LET column partials).
 struct LinBwd {
+  omq_dtype op;            // GEMM operand type of Xq, W_hat, dY (and dX when 16-bit)
   int64_t M, N, K, G;
   float Q;
   const void* W;
@@ -421,7 +446,7 @@ omq_status lin_bwd(const LinBwd& a, const View& v, cudaStream_t st) {
   float* emin = a.s_w ? v.in<float>(L.emin) : nullptr;
   if (a.shift) {
     float* part = v.in<float>(L.dbt_part);
-    BLK_TRY(launch_colsum(a.dY, OMQ_BF16, a.M, a.N, kRowsColsum, nullptr, part, st));
+    BLK_TRY(launch_colsum(a.dY, a.op, a.M, a.N, kRowsColsum, nullptr, part, st));
     const ColReduce r{part, ceil_div(a.M, kRowsColsum), nullptr, 0, a.dy_scale, dbt};
     BLK_TRY(launch_reduce_cols(&r, 1, a.N, v.in<double>(L.red), st));
   }
@@ -431,7 +456,9 @@ omq_status lin_bwd(const LinBwd& a, const View& v, cudaStream_t st) {
     e.out_scale = a.dy_scale;
     e.ste = SteWEpi{a.W, OMQ_BF16, a.K, a.G, a.K / a.G, a.Q, a.s_w, a.h, a.z, gh, gc,
                     a.s_w ? a.part_ws : nullptr};
-    BLK_TRY(gemm_tc(OMQ_BF16, GemmOperand{a.dY, a.N, true}, GemmOperand{a.Xq, a.K, true}, a.N, a.K,
+    e.sk_scratch = v.in<char>(L.sk);
+    e.sk_bytes = L.sk_bytes;
+    BLK_TRY(gemm_tc(a.op, GemmOperand{a.dY, a.N, true}, GemmOperand{a.Xq, a.K, true}, a.N, a.K,
                     a.M, e, nullptr, st));
   }
   {
@@ -446,8 +473,8 @@ omq_status lin_bwd(const LinBwd& a, const View& v, cudaStream_t st) {
     BLK_TRY(launch_ste_w_corr(c, st));
   }
   float* dxq = v.in<float>(L.dxq);
-  BLK_TRY(gemm_store(GemmOperand{a.dY, a.N, false}, GemmOperand{a.W_hat, a.K, true}, a.M, a.K, a.N,
-                     dxq, 0, a.dy_scale, nullptr, st));
+  BLK_TRY(gemm_store(a.op, GemmOperand{a.dY, a.N, false}, GemmOperand{a.W_hat, a.K, true}, a.M, a.K, a.N,
+                     dxq, 0, a.dy_scale, nullptr, v.in<char>(L.sk), L.sk_bytes, st));
   SteXParams p{a.X, a.xdt, a.M, a.K, a.Qa, a.quantized, a.s_x, a.d_x, a.h_a, a.z_a, a.tok_range,
                dxq, v.in<float>(L.rowstat), a.part_xs, a.part_xd, kRowsX, a.dX, a.dx_dt};
   return launch_ste_x(p, st);
@@ -465,12 +492,18 @@ omq_status block_backward(const View& v, const Inputs& in, float* d_theta, const
   const int quantized = d.abits < 16 ? 1 : 0;
   const float Qa = static_cast<float>((1 << (d.abits < 16 ? d.abits : 1)) - 1);
   const float Qw = static_cast<float>((1 << d.wbits) - 1);
+  // The activation gradients flow back unscaled: in units of the residual res = y - y*, i.e.
+  // as gradients of (M D / 2) L. They are stored as float16 GEMM operands, whose range then
+  // holds them (the true gradients, 2 / (M D) times smaller, would fall into float16's
+  // subnormals); the factor 2 / (M D) is applied once, to the parameter gradients.
   const float gscale = static_cast<float>(2.0 / (static_cast<double>(M) * static_cast<double>(D)));
+  const omq_dtype op = OMQ_F16;
   const int what_id[L_COUNT] = {OMQ_BB_WHAT_QKV, OMQ_BB_WHAT_O, OMQ_BB_WHAT_GU, OMQ_BB_WHAT_D};
   auto base = [&](int l) {
     const LinShape s = lin_shape(d, l);
     const LinScratch& c = L.lin[l];
     LinBwd a{};
+    a.op = op;
     a.M = M; a.N = s.N; a.K = s.K; a.G = group_of(d, s.K); a.Q = Qw;
     a.W = in.W[l]; a.W_hat = v.bb<void>(what_id[l]);
     a.gl = th(OMQ_TH_GAMMA_QKV + 2 * l); a.bl = th(OMQ_TH_BETA_QKV + 2 * l);
@@ -487,17 +520,17 @@ omq_status block_backward(const View& v, const Inputs& in, float* d_theta, const
     a.tok_range = v.in<omq_range>(L.act_range[k]);
   };
 
-  // down projection: dL/dy = gscale res; no LET
+  // down projection: the gradient of (M D / 2) L with respect to y is res; no LET
   BLK_TRY(mk.mark(OMQ_BPH_BWD_FFN));
   {
     LinBwd a = base(L_D);
-    a.Xq = v.bb<void>(OMQ_BB_QM); a.dY = v.bb<void>(OMQ_BB_RES); a.dy_scale = gscale;
+    a.Xq = v.bb<void>(OMQ_BB_QM); a.dY = v.bb<void>(OMQ_BB_RES); a.dy_scale = 1.f;
     a.X = v.bb<void>(OMQ_BB_MID); act(a, 3);
     a.dX = v.bb<void>(OMQ_BB_DMID);
     BLK_TRY(lin_bwd(a, v, st));
   }
   BLK_TRY(launch_swiglu_bwd(v.bb<float>(OMQ_BB_GU), v.bb<float>(OMQ_BB_DMID),
-                            v.bb<__nv_bfloat16>(OMQ_BB_DGU), M, I, st));
+                            v.bb<void>(OMQ_BB_DGU), op, M, I, st));
   {
     LinBwd a = base(L_GU);
     a.Xq = v.bb<void>(OMQ_BB_QB); a.dY = v.bb<void>(OMQ_BB_DGU); a.dy_scale = 1.f;
@@ -510,7 +543,7 @@ omq_status block_backward(const View& v, const Inputs& in, float* d_theta, const
   }
   {
     RmsBwdParams r{v.bb<float>(OMQ_BB_DB), v.bb<float>(OMQ_BB_B), v.in<float>(L.rstd2),
-                   v.bb<void>(OMQ_BB_RES), gscale, M, D, v.bb<void>(OMQ_BB_DX2)};
+                   v.bb<void>(OMQ_BB_RES), 1.f, M, D, v.bb<void>(OMQ_BB_DX2), op};
     BLK_TRY(launch_rms_bwd(r, st));
   }
   // output projection (its LET acts on V), then attention
@@ -520,28 +553,29 @@ omq_status block_backward(const View& v, const Inputs& in, float* d_theta, const
     a.Xq = v.bb<void>(OMQ_BB_QO); a.dY = v.bb<void>(OMQ_BB_DX2); a.dy_scale = 1.f;
     a.s_w = th(OMQ_TH_S_O); a.shift = true;
     a.X = v.bb<void>(OMQ_BB_O); act(a, 1);
-    a.dX = v.bb<void>(OMQ_BB_DO); a.dx_dt = OMQ_BF16;
+    a.dX = v.bb<void>(OMQ_BB_DO); a.dx_dt = op;
     BLK_TRY(lin_bwd(a, v, st));
   }
   {
-    const __nv_bfloat16* qqkv = v.bb<__nv_bfloat16>(OMQ_BB_QQKV);
-    const __nv_bfloat16* P16 = v.bb<__nv_bfloat16>(OMQ_BB_P16);
-    const __nv_bfloat16* dO = v.bb<__nv_bfloat16>(OMQ_BB_DO);
+    const uint16_t* qqkv = v.bb<uint16_t>(OMQ_BB_QQKV);
+    const uint16_t* P16 = v.bb<uint16_t>(OMQ_BB_P16);
+    const uint16_t* dO = v.bb<uint16_t>(OMQ_BB_DO);
     float* dP = v.in<float>(L.dP);
-    __nv_bfloat16* dS = v.in<__nv_bfloat16>(L.dS);
+    uint16_t* dS = v.in<uint16_t>(L.dS);
     float* dq = v.bb<float>(OMQ_BB_DQQKV);
     // dQv_h = P_h^T dO_h;  dP_h = dO_h Qv_h^T
-    BLK_TRY(gemm_heads(GemmOperand{P16, M, true}, M * M, GemmOperand{dO, D, true}, kHead, M, kHead,
-                       M, dq + 2 * D, 3 * D, kHead, 1.f, H, 3, st));
-    BLK_TRY(gemm_heads(GemmOperand{dO, D, false}, kHead, GemmOperand{qqkv + 2 * D, 3 * D, false},
-                       kHead, M, M, kHead, dP, 0, M * M, 1.f, H, 1, st));
+    BLK_TRY(gemm_heads(op, GemmOperand{P16, M, true}, M * M, GemmOperand{dO, D, true}, kHead, M,
+                       kHead, M, dq + 2 * D, 3 * D, kHead, 1.f, H, 3, st));
+    BLK_TRY(gemm_heads(op, GemmOperand{dO, D, false}, kHead,
+                       GemmOperand{qqkv + 2 * D, 3 * D, false}, kHead, M, M, kHead, dP, 0, M * M,
+                       1.f, H, 1, st));
     const float scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(kHead)));
-    BLK_TRY(launch_softmax_bwd(v.bb<float>(OMQ_BB_P), dP, dS, H * M, M, scale, st));
+    BLK_TRY(launch_softmax_bwd(v.bb<float>(OMQ_BB_P), dP, dS, op, H * M, M, scale, st));
     // dQq_h = dS_h Qk_h;  dQk_h = dS_h^T Qq_h
-    BLK_TRY(gemm_heads(GemmOperand{dS, M, false}, M * M, GemmOperand{qqkv + D, 3 * D, true}, kHead,
-                       M, kHead, M, dq, 3 * D, kHead, 1.f, H, 2, st));
-    BLK_TRY(gemm_heads(GemmOperand{dS, M, true}, M * M, GemmOperand{qqkv, 3 * D, true}, kHead, M,
-                       kHead, M, dq + D, 3 * D, kHead, 1.f, H, 3, st));
+    BLK_TRY(gemm_heads(op, GemmOperand{dS, M, false}, M * M, GemmOperand{qqkv + D, 3 * D, true},
+                       kHead, M, kHead, M, dq, 3 * D, kHead, 1.f, H, 2, st));
+    BLK_TRY(gemm_heads(op, GemmOperand{dS, M, true}, M * M, GemmOperand{qqkv, 3 * D, true}, kHead,
+                       M, kHead, M, dq + D, 3 * D, kHead, 1.f, H, 3, st));
     AttnPrepParams p{};
     p.qkv = v.bb<float>(OMQ_BB_QKV);
     p.cos_t = v.bb<float>(OMQ_BB_ROPE);
@@ -556,7 +590,8 @@ omq_status block_backward(const View& v, const Inputs& in, float* d_theta, const
     p.z_s = v.in<int32_t>(L.head_z);
     p.range_s = v.in<omq_range>(L.head_range);
     p.dq = dq;
-    p.dout = v.bb<__nv_bfloat16>(OMQ_BB_DQKV);
+    p.dout = v.bb<void>(OMQ_BB_DQKV);
+    p.dt16 = op;
     p.part_sa = v.in<float>(L.part_sa);
     p.part_so = v.in<float>(L.part_so);
     p.part_do = v.in<float>(L.part_do);
@@ -579,17 +614,20 @@ omq_status block_backward(const View& v, const Inputs& in, float* d_theta, const
                   rw_gu = ceil_div(2 * I, kRowsFusedW), rx = ceil_div(M, kRowsX),
                   ra = ceil_div(M, kAttnRows);
     const LinScratch &q = L.lin[L_QKV], &o = L.lin[L_O], &g = L.lin[L_GU];
+    const float gs = gscale;
     const ColReduce r[8] = {
-        {v.in<float>(q.part_ws), rw_qkv, v.in<float>(q.part_xs), rx, 1.f, dth(OMQ_TH_S1)},
-        {v.in<float>(q.part_wd), rw_qkv, v.in<float>(q.part_xd), rx, 1.f, dth(OMQ_TH_DELTA1)},
-        {v.in<float>(o.part_ws), rw_o, v.in<float>(L.part_so), ra, 1.f, dth(OMQ_TH_S_O)},
-        {v.in<float>(o.part_wd), rw_o, v.in<float>(L.part_do), ra, 1.f, dth(OMQ_TH_DELTA_O)},
-        {v.in<float>(g.part_ws), rw_gu, v.in<float>(g.part_xs), rx, 1.f, dth(OMQ_TH_S2)},
-        {v.in<float>(g.part_wd), rw_gu, v.in<float>(g.part_xd), rx, 1.f, dth(OMQ_TH_DELTA2)},
-        {v.in<float>(L.part_sa), ra, nullptr, 0, 1.f, dth(OMQ_TH_S_A)},
-        {v.in<float>(L.part_sa), ra, nullptr, 0, 1.f, dth(OMQ_TH_S_A)}};
+        {v.in<float>(q.part_ws), rw_qkv, v.in<float>(q.part_xs), rx, gs, dth(OMQ_TH_S1)},
+        {v.in<float>(q.part_wd), rw_qkv, v.in<float>(q.part_xd), rx, gs, dth(OMQ_TH_DELTA1)},
+        {v.in<float>(o.part_ws), rw_o, v.in<float>(L.part_so), ra, gs, dth(OMQ_TH_S_O)},
+        {v.in<float>(o.part_wd), rw_o, v.in<float>(L.part_do), ra, gs, dth(OMQ_TH_DELTA_O)},
+        {v.in<float>(g.part_ws), rw_gu, v.in<float>(g.part_xs), rx, gs, dth(OMQ_TH_S2)},
+        {v.in<float>(g.part_wd), rw_gu, v.in<float>(g.part_xd), rx, gs, dth(OMQ_TH_DELTA2)},
+        {v.in<float>(L.part_sa), ra, nullptr, 0, gs, dth(OMQ_TH_S_A)},
+        {v.in<float>(L.part_sa), ra, nullptr, 0, gs, dth(OMQ_TH_S_A)}};
     for (int k = 0; k < 7; k += 2)
       BLK_TRY(launch_reduce_cols(r + k, k == 6 ? 1 : 2, D, v.in<double>(L.red), st));
+    // the LWC logit gradients, written by the weight-side STE completion of each linear
+    BLK_TRY(launch_scale(d_theta, toff[OMQ_TH_S1], gscale, st));
   }
   return OMQ_OK;
 }

@@ -25,13 +25,14 @@ struct RmsBwdParams {
   const float* dn;      // [M, D] gradient of the normalized values
   const float* n;       // [M, D] the normalized values
   const float* rstd;    // [M]
-  const void* res;      // [M, D] BF16 residual-path gradient / res_scale
+  const void* res;      // [M, D] residual-path gradient / res_scale, in dt16
   float res_scale;
   int64_t M, D;
-  void* dx;             // [M, D] BF16
+  void* dx;             // [M, D] in dt16
+  omq_dtype dt16;       // OMQ_F16 or OMQ_BF16: the block's 16-bit GEMM operand type
 };
 
-// q | k | v [M, 3D] float32 in, Qq | Qk | Qv [M, 3D] BF16 out, per (which, token, head) stats.
+// q | k | v [M, 3D] float32 in, Qq | Qk | Qv [M, 3D] 16-bit out, per (which, token, head) stats.
 struct AttnPrepParams {
   const float* qkv;
   const float* cos_t;   // [M, 64]
@@ -42,13 +43,14 @@ struct AttnPrepParams {
   int64_t M, D, H;
   int quantized;
   float Qa;
-  __nv_bfloat16* out;   // forward: the quantized (or transformed) q~, k~, v~
+  omq_dtype dt16;       // OMQ_F16 or OMQ_BF16 for out and dout
+  void* out;            // forward: the quantized (or transformed) q~, k~, v~
   float* h_s;           // [3, M, H]
   int32_t* z_s;
   omq_range* range_s;
   // backward
   const float* dq;      // [M, 3D] gradient of the quantized values
-  __nv_bfloat16* dout;  // [M, 3D] gradient of q | k | v
+  void* dout;           // [M, 3D] gradient of q | k | v
   float* part_sa;       // [ceil(M / kAttnRows), D] or NULL
   float* part_so;
   float* part_do;
@@ -58,11 +60,14 @@ omq_status launch_rope_table(int64_t M, double base, float* cos_t, float* sin_t,
 omq_status launch_rms(const RmsParams& p, cudaStream_t st);
 omq_status launch_rms_bwd(const RmsBwdParams& p, cudaStream_t st);
 omq_status launch_attn_prep(const AttnPrepParams& p, bool backward, cudaStream_t st);
-omq_status launch_softmax(float* S, __nv_bfloat16* P16, int64_t rows, int64_t M, cudaStream_t st);
-omq_status launch_softmax_bwd(const float* P, const float* dP, __nv_bfloat16* dS, int64_t rows,
-                              int64_t M, float scale, cudaStream_t st);
+omq_status launch_softmax(float* S, void* P16, omq_dtype dt16, int64_t rows, int64_t M,
+                          cudaStream_t st);
+omq_status launch_softmax_bwd(const float* P, const float* dP, void* dS, omq_dtype dt16,
+                              int64_t rows, int64_t M, float scale, cudaStream_t st);
 omq_status launch_swiglu(const float* gu, float* mid, int64_t M, int64_t I, cudaStream_t st);
-omq_status launch_swiglu_bwd(const float* gu, const float* dmid, __nv_bfloat16* dgu, int64_t M,
-                             int64_t I, cudaStream_t st);
+omq_status launch_swiglu_bwd(const float* gu, const float* dmid, void* dgu, omq_dtype dt16,
+                             int64_t M, int64_t I, cudaStream_t st);
+// x[i] *= s for i < n (float32), in place.
+omq_status launch_scale(float* x, int64_t n, float s, cudaStream_t st);
 
 }  // namespace omq

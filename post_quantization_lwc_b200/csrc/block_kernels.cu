@@ -116,10 +116,10 @@ __global__ void __launch_bounds__(256) rms_bwd_kernel(RmsBwdParams p) {
       float dn[8], n[8], r[8], o[8];
       load_f8(p.dn, base + c * 8, dn);
       load_f8(p.n, base + c * 8, n);
-      load8(p.res, base + c * 8, OMQ_BF16, r);
+      load8(p.res, base + c * 8, p.dt16, r);
 #pragma unroll
       for (int i = 0; i < 8; ++i) o[i] = p.res_scale * r[i] + rstd * (dn[i] - n[i] * mean);
-      store8(p.dx, base + c * 8, OMQ_BF16, o);
+      store8(p.dx, base + c * 8, p.dt16, o);
     }
   }
 }
@@ -203,9 +203,21 @@ __device__ __forceinline__ void load_head4(const float* row, int lane, float (&v
   const float2 hi = *reinterpret_cast<const float2*>(row + 64 + 2 * lane);
   v[0] = lo.x; v[1] = lo.y; v[2] = hi.x; v[3] = hi.y;
 }
-__device__ __forceinline__ void store_head4_bf16(__nv_bfloat16* row, int lane, const float (&v)[4]) {
-  *reinterpret_cast<__nv_bfloat162*>(row + 2 * lane) = __floats2bfloat162_rn(v[0], v[1]);
-  *reinterpret_cast<__nv_bfloat162*>(row + 64 + 2 * lane) = __floats2bfloat162_rn(v[2], v[3]);
+// Two values rounded to the 16-bit type (nearest even), packed in one 32-bit word.
+__device__ __forceinline__ uint32_t pack2(float a, float b, bool f16) {
+  if (f16) {
+    const __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<const uint32_t*>(&h);
+  }
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+// Lane l's four columns of a head row of 16-bit values (element offset `off` from `base`).
+__device__ __forceinline__ void store_head4(void* base, int64_t off, int lane, const float (&v)[4],
+                                            bool f16) {
+  uint16_t* row = static_cast<uint16_t*>(base) + off;
+  *reinterpret_cast<uint32_t*>(row + 2 * lane) = pack2(v[0], v[1], f16);
+  *reinterpret_cast<uint32_t*>(row + 64 + 2 * lane) = pack2(v[2], v[3], f16);
 }
 __device__ __forceinline__ void load_vec4(const float* vec, int lane, float (&v)[4]) {
   load_head4(vec, lane, v);
@@ -280,7 +292,7 @@ __global__ void __launch_bounds__(256) attn_prep_kernel(AttnPrepParams p) {
         p.range_s[si] = r.rg;
       }
     }
-    store_head4_bf16(p.out + m * 3 * D + which * D + h * 128, lane, v);
+    store_head4(p.out, m * 3 * D + which * D + h * 128, lane, v, p.dt16 == OMQ_F16);
   }
 }
 
@@ -338,7 +350,7 @@ __global__ void __launch_bounds__(256) attn_prep_bwd_kernel(AttnPrepParams p) {
           d[i] = q;
         }
       }
-      store_head4_bf16(p.dout + m * 3 * D + which * D + h * 128, lane, d);
+      store_head4(p.dout, m * 3 * D + which * D + h * 128, lane, d, p.dt16 == OMQ_F16);
     }
   }
   if (!p.part_sa) return;
@@ -377,8 +389,8 @@ __device__ __forceinline__ int64_t causal_span(int64_t i, int64_t M) {
   return e < M ? e : M;
 }
 
-__global__ void __launch_bounds__(256) softmax_kernel(float* S, __nv_bfloat16* P16, int64_t rows,
-                                                      int64_t M) {
+__global__ void __launch_bounds__(256) softmax_kernel(float* S, uint16_t* P16, bool f16,
+                                                      int64_t rows, int64_t M) {
   pdl_wait();
   pdl_launch();
   const int lane = threadIdx.x & 31;
@@ -386,7 +398,7 @@ __global__ void __launch_bounds__(256) softmax_kernel(float* S, __nv_bfloat16* P
   if (r >= rows) return;
   const int64_t i = r % M;
   float* row = S + r * M;
-  __nv_bfloat16* row16 = P16 + r * M;
+  uint16_t* row16 = P16 + r * M;
   const int64_t nvalid = i + 1;
   float mx = -FLT_MAX;
   for (int64_t q = lane; q * 4 < nvalid; q += 32) {
@@ -419,11 +431,8 @@ __global__ void __launch_bounds__(256) softmax_kernel(float* S, __nv_bfloat16* P
       for (int t = 0; t < 4; ++t) e[t] = q * 4 + t < nvalid ? expf(x[t] - mx) * inv : 0.f;
       *reinterpret_cast<float4*>(row + q * 4) = make_float4(e[0], e[1], e[2], e[3]);
     }
-    __nv_bfloat162 a = __floats2bfloat162_rn(e[0], e[1]), b = __floats2bfloat162_rn(e[2], e[3]);
-    uint2 pk;
-    pk.x = *reinterpret_cast<uint32_t*>(&a);
-    pk.y = *reinterpret_cast<uint32_t*>(&b);
-    *reinterpret_cast<uint2*>(row16 + q * 4) = pk;
+    *reinterpret_cast<uint2*>(row16 + q * 4) =
+        make_uint2(pack2(e[0], e[1], f16), pack2(e[2], e[3], f16));
   }
 }
 
@@ -431,7 +440,7 @@ __global__ void __launch_bounds__(256) softmax_kernel(float* S, __nv_bfloat16* P
 // the row's 256-column tile (BF16; the causal dS Qk and dS^T Qq products read no further).
 // P and dP are read only at j <= i.
 __global__ void __launch_bounds__(256) softmax_bwd_kernel(const float* P, const float* dP,
-                                                          __nv_bfloat16* dS, int64_t rows,
+                                                          uint16_t* dS, bool f16, int64_t rows,
                                                           int64_t M, float scale) {
   pdl_wait();
   pdl_launch();
@@ -441,7 +450,7 @@ __global__ void __launch_bounds__(256) softmax_bwd_kernel(const float* P, const 
   const int64_t i = r % M;
   const float* prow = P + r * M;
   const float* drow = dP + r * M;
-  __nv_bfloat16* orow = dS + r * M;
+  uint16_t* orow = dS + r * M;
   const int64_t nvalid = i + 1;
   const int64_t nq = causal_span(i, M) / 4;
   float dot = 0.f;
@@ -464,11 +473,8 @@ __global__ void __launch_bounds__(256) softmax_bwd_kernel(const float* P, const 
 #pragma unroll
       for (int t = 0; t < 4; ++t) e[t] = q * 4 + t < nvalid ? scale * pa[t] * (pb[t] - dot) : 0.f;
     }
-    __nv_bfloat162 a = __floats2bfloat162_rn(e[0], e[1]), b = __floats2bfloat162_rn(e[2], e[3]);
-    uint2 pk;
-    pk.x = *reinterpret_cast<uint32_t*>(&a);
-    pk.y = *reinterpret_cast<uint32_t*>(&b);
-    *reinterpret_cast<uint2*>(orow + q * 4) = pk;
+    *reinterpret_cast<uint2*>(orow + q * 4) =
+        make_uint2(pack2(e[0], e[1], f16), pack2(e[2], e[3], f16));
   }
 }
 
@@ -491,9 +497,9 @@ __global__ void __launch_bounds__(256) swiglu_kernel(const float* gu, float* mid
   }
 }
 
-// d gate = dm up sigma(g) (1 + g (1 - sigma(g))), d up = dm SiLU(g)  ->  BF16 [M, 2I].
+// d gate = dm up sigma(g) (1 + g (1 - sigma(g))), d up = dm SiLU(g)  ->  16-bit [M, 2I].
 __global__ void __launch_bounds__(256) swiglu_bwd_kernel(const float* gu, const float* dmid,
-                                                         __nv_bfloat16* dgu, int64_t M,
+                                                         void* dgu, omq_dtype dt16, int64_t M,
                                                          int64_t I) {
   pdl_wait();
   pdl_launch();
@@ -511,8 +517,8 @@ __global__ void __launch_bounds__(256) swiglu_bwd_kernel(const float* gu, const 
       dg[i] = dm[i] * u[i] * sg * (1.f + g[i] * (1.f - sg));
       du[i] = dm[i] * g[i] * sg;
     }
-    store8(dgu, m * 2 * I + c, OMQ_BF16, dg);
-    store8(dgu, m * 2 * I + I + c, OMQ_BF16, du);
+    store8(dgu, m * 2 * I + c, dt16, dg);
+    store8(dgu, m * 2 * I + I + c, dt16, du);
   }
 }
 
@@ -550,16 +556,17 @@ omq_status launch_attn_prep(const AttnPrepParams& p, bool backward, cudaStream_t
   return launch_status();
 }
 
-omq_status launch_softmax(float* S, __nv_bfloat16* P16, int64_t rows, int64_t M,
+omq_status launch_softmax(float* S, void* P16, omq_dtype dt16, int64_t rows, int64_t M,
                           cudaStream_t st) {
-  launch_k(softmax_kernel, static_cast<unsigned>(ceil_div(rows, 8)), 256, 0, st, S, P16, rows, M);
+  launch_k(softmax_kernel, static_cast<unsigned>(ceil_div(rows, 8)), 256, 0, st, S,
+      static_cast<uint16_t*>(P16), dt16 == OMQ_F16, rows, M);
   return launch_status();
 }
 
-omq_status launch_softmax_bwd(const float* P, const float* dP, __nv_bfloat16* dS, int64_t rows,
-                              int64_t M, float scale, cudaStream_t st) {
+omq_status launch_softmax_bwd(const float* P, const float* dP, void* dS, omq_dtype dt16,
+                              int64_t rows, int64_t M, float scale, cudaStream_t st) {
   launch_k(softmax_bwd_kernel, static_cast<unsigned>(ceil_div(rows, 8)), 256, 0, st,
-      P, dP, dS, rows, M, scale);
+      P, dP, static_cast<uint16_t*>(dS), dt16 == OMQ_F16, rows, M, scale);
   return launch_status();
 }
 
@@ -568,9 +575,23 @@ omq_status launch_swiglu(const float* gu, float* mid, int64_t M, int64_t I, cuda
   return launch_status();
 }
 
-omq_status launch_swiglu_bwd(const float* gu, const float* dmid, __nv_bfloat16* dgu, int64_t M,
-                             int64_t I, cudaStream_t st) {
-  launch_k(swiglu_bwd_kernel, grid_for(M * I / 8, 256, 8), 256, 0, st, gu, dmid, dgu, M, I);
+omq_status launch_swiglu_bwd(const float* gu, const float* dmid, void* dgu, omq_dtype dt16,
+                             int64_t M, int64_t I, cudaStream_t st) {
+  launch_k(swiglu_bwd_kernel, grid_for(M * I / 8, 256, 8), 256, 0, st, gu, dmid, dgu, dt16, M, I);
+  return launch_status();
+}
+
+__global__ void __launch_bounds__(256) scale_kernel(float* x, int64_t n, float s) {
+  pdl_wait();
+  pdl_launch();
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    x[i] *= s;
+}
+
+omq_status launch_scale(float* x, int64_t n, float s, cudaStream_t st) {
+  if (n <= 0) return OMQ_OK;
+  launch_k(scale_kernel, grid_for(n, 256, 4), 256, 0, st, x, n, s);
   return launch_status();
 }
 

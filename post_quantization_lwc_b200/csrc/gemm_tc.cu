@@ -247,6 +247,55 @@ __device__ __forceinline__ TileWork tile_of(const TileSched& sc, int t, int nk) 
   return w;
 }
 
+// One unit of a pair's work: a whole tile, or a run of k-blocks of a stream-K tile (split
+// `split` of `nsplit`, the pairs in k order; at most two, since a run is longer than a tile's
+// contraction).
+struct Unit {
+  TileWork w;
+  int t;        // tile index (its loss partial slots are 2 t and 2 t + 1)
+  int tsk;      // index among the stream-K tiles, or -1
+  int split, nsplit;
+};
+// The pair's u-th unit: its whole tiles pair, pair + pairs, ... below dp_tiles, then its run
+// [pair sk_len, (pair + 1) sk_len) of the stream-K tiles' k-blocks (tile by tile, in order).
+template <bool BATCH>
+__device__ __forceinline__ bool next_unit(const TileSched& sc, int pair, int pairs, int u, int nk,
+                                          Unit& un) {
+  const int t = pair + u * pairs;
+  if (t < sc.dp_tiles) {
+    un.w = tile_of<BATCH>(sc, t, nk);
+    un.t = t;
+    un.tsk = -1;
+    un.split = 0;
+    un.nsplit = 1;
+    return true;
+  }
+  if (sc.sk_tiles == 0) return false;
+  const int s = u - sc.dp_tiles / pairs;            // dp_tiles is a multiple of pairs here
+  const int64_t total = static_cast<int64_t>(sc.sk_tiles) * nk;
+  const int64_t lo = static_cast<int64_t>(pair) * sc.sk_len;
+  const int64_t hi = lo + sc.sk_len < total ? lo + sc.sk_len : total;
+  const int64_t ts = lo / nk + s;
+  const int64_t a = lo > ts * nk ? lo : ts * nk;
+  const int64_t b = hi < (ts + 1) * nk ? hi : (ts + 1) * nk;
+  if (a >= b) return false;
+  un.t = sc.dp_tiles + static_cast<int>(ts);
+  un.w = tile_of<BATCH>(sc, un.t, nk);
+  un.w.kb0 = static_cast<int>(a - ts * nk);
+  un.w.kb1 = static_cast<int>(b - ts * nk);
+  un.tsk = static_cast<int>(ts);
+  const int64_t first = (ts * nk) / sc.sk_len, last = ((ts + 1) * nk - 1) / sc.sk_len;
+  un.nsplit = static_cast<int>(last - first + 1);
+  un.split = static_cast<int>(pair - first);
+  return true;
+}
+// One CTA's half of a partial accumulator: 128 rows x 256 columns, stored warp by warp as
+// [epilogue warp][column][lane] so that a warp's stores and loads are 128-byte lines.
+constexpr int64_t kSkSlot = 128 * 256;
+__device__ __forceinline__ int64_t sk_slot(int tsk, int split, uint32_t rank) {
+  return ((static_cast<int64_t>(tsk) * 2 + split) * 2 + rank) * kSkSlot;
+}
+
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -374,7 +423,8 @@ __device__ __forceinline__ void unpack8(const uint4& q, float (&w)[8]) {
 template <bool F16>
 __device__ __forceinline__ void ste_w_epilogue(const GemmEpilogue& epi, uint32_t tcol,
                                                int64_t wrow0, int64_t col0, int64_t rows,
-                                               int64_t cols, int lane, const uint8_t* wst) {
+                                               int64_t cols, int lane, const uint8_t* wst,
+                                               const float* other) {
   const SteWEpi& p = epi.ste;
   const int64_t row = wrow0 + lane;
   const bool valid = row < rows;
@@ -408,6 +458,11 @@ __device__ __forceinline__ void ste_w_epilogue(const GemmEpilogue& epi, uint32_t
       __syncwarp();
       tmem_ld16(tcol + 16 * q, r);
       tmem_ld_wait();
+      if (other) {   // a stream-K tile: add the other pair's partial (this warp's layout)
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          r[i] = __float_as_uint(__uint_as_float(r[i]) + __ldcg(other + (16 * q + i) * 32 + lane));
+      }
 #pragma unroll
       for (int v = 0; v < 2; ++v) {
         float w[8], sv[8];
@@ -448,9 +503,13 @@ struct Layout {
   // control block: barriers full[S], empty[S], acc_full[2], acc_empty[2], drain; tmem slot,
   // abort flag, the epilogue's per-warp loss partials [2][EPI_WARPS] and arrival counters [2]
   static constexpr int CTL_BYTES = 512;
+  // and, for stream-K tiles, the epilogue warps' arrival barrier, the decision barrier and
+  // the decision
   static constexpr int FULL = 0, EMPTY = 8 * STAGES, ACCF = 16 * STAGES, ACCE = ACCF + 16,
                        DRAIN = ACCE + 16, SLOT = DRAIN + 8, ABORT = SLOT + 4, RED = ABORT + 4,
-                       CNT = RED + 8 * EPI_WARPS, CTL_END = CNT + 8;
+                       CNT = RED + 8 * EPI_WARPS, SKA = CNT + 8, SKB = SKA + 8, SKF = SKB + 8,
+                       CTL_END = SKF + 8;
+  static_assert(SKA % 8 == 0, "mbarrier alignment");
   static_assert(CTL_END <= CTL_BYTES, "control block");
   static constexpr int SMEM_BYTES = 1024 /*align slack*/ + BAR_OFF + CTL_BYTES;
   static constexpr uint32_t TMEM_COLS = 2 * TILE_N;
@@ -475,6 +534,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV>::NUM_THREADS
   const uint32_t bar_accf = sbase + L::BAR_OFF + L::ACCF;
   const uint32_t bar_acce = sbase + L::BAR_OFF + L::ACCE;
   const uint32_t bar_drain = sbase + L::BAR_OFF + L::DRAIN;
+  const uint32_t bar_ska = sbase + L::BAR_OFF + L::SKA;
+  const uint32_t bar_skb = sbase + L::BAR_OFF + L::SKB;
+  volatile int* sk_flag = reinterpret_cast<volatile int*>(ctl + L::SKF);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctl + L::SLOT);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(ctl + L::ABORT);
   volatile float* red = reinterpret_cast<volatile float*>(ctl + L::RED);  // [2][EPI_WARPS]
@@ -486,7 +548,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV>::NUM_THREADS
   const int pair = static_cast<int>(cluster_id());
   const int pairs = static_cast<int>(cluster_count());
   const int nk = static_cast<int>((depth + BK - 1) / BK);
-  const int num_tiles = sc.num_tiles;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -499,6 +560,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV>::NUM_THREADS
       cnt[b] = 0;
     }
     mbar_init(bar_drain, 1);
+    mbar_init(bar_ska, EPI_WARPS);      // every epilogue warp has stored its partial
+    mbar_init(bar_skb, 1);              // the decision who finishes the tile is published
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -521,8 +584,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV>::NUM_THREADS
     // ---------------- TMA producer (both CTAs)
     int it = 0;
     bool ok = true;
-    for (int t = pair; t < num_tiles && ok; t += pairs) {
-      const TileWork tw = tile_of<BATCH>(sc, t, nk);
+    Unit un;
+    for (int u = 0; ok && next_unit<BATCH>(sc, pair, pairs, u, nk, un); ++u) {
+      const TileWork& tw = un.w;
       const int row0 = tw.row0 + static_cast<int>(rank) * HALF;
       const int col0 = tw.col0 + static_cast<int>(rank) * HALF;
       for (int kb = tw.kb0; kb < tw.kb1; ++kb, ++it) {
@@ -565,7 +629,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV>::NUM_THREADS
     const uint32_t idesc = instr_desc(TILE_M, TILE_N, a_mn != 0, b_mn != 0, fmt);
     int it = 0, lt = 0;
     bool ok = true;
-    for (int t = pair; t < num_tiles && ok; t += pairs, ++lt) {
+    Unit un;
+    for (int u = 0; ok && next_unit<BATCH>(sc, pair, pairs, u, nk, un); ++u, ++lt) {
       const int buf = lt & 1;
       const uint32_t pa = ((lt >> 1) & 1) ^ 1;
       const bool got = C::SLEEPY ? mbar_wait_sleep(bar_acce + 8 * buf, pa, DEV_ERR_MMA_WAIT, 64)
@@ -576,7 +641,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV>::NUM_THREADS
       }
       tc_fence_after();
       const uint32_t d = tmem + static_cast<uint32_t>(buf * TILE_N);
-      const TileWork tw = tile_of<BATCH>(sc, t, nk);
+      const TileWork& tw = un.w;
       for (int kb = tw.kb0; kb < tw.kb1; ++kb, ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
@@ -608,10 +673,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV>::NUM_THREADS
     const int quad = warp & 3;                       // TMEM lanes 32*quad .. 32*quad+31
     const int cq = ew >> 2;                          // columns 64*cq .. 64*cq+63 of the tile
     const uint32_t acce_leader = peer_addr(bar_acce, 0);
-    int lt = 0;
-    for (int t = pair; t < num_tiles; t += pairs, ++lt) {
+    int lt = 0, sk_n = 0;
+    Unit un;
+    for (int u = 0; next_unit<BATCH>(sc, pair, pairs, u, nk, un); ++u, ++lt) {
       const int buf = lt & 1;
-      const TileWork tw = tile_of<BATCH>(sc, t, nk);
+      const TileWork& tw = un.w;
+      const int t = un.t;
       const int64_t wrow0 = static_cast<int64_t>(tw.row0) + rank * HALF + quad * 32;
       const int64_t col0 = static_cast<int64_t>(tw.col0) + cq * EPI_COLS;
       const int64_t row = wrow0 + lane;
@@ -645,15 +712,70 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV>::NUM_THREADS
       float lsum = 0.f;
       const uint32_t tbase = tmem + (static_cast<uint32_t>(quad * 32) << 16) +
                              static_cast<uint32_t>(buf * TILE_N + cq * EPI_COLS);
+      const float* other = nullptr;
+      if (un.nsplit > 1) {
+        // A stream-K tile: both contributing pairs store their partial accumulator, then
+        // count their arrival on the tile's counter; the second to arrive adds the first's
+        // partial to its own and runs the epilogue (own + other: the same sum whichever
+        // pair comes second), the first hands its accumulator back and moves on.
+        float* mine = sc.sk_part + sk_slot(un.tsk, un.split, rank) + ew * EPI_COLS * 32;
+#pragma unroll 1
+        for (int ch = 0; ch < EPI_COLS / 32; ++ch) {
+          uint32_t r[32];
+          tmem_ld32(tbase + ch * 32, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int q = 0; q < 32; ++q) __stcg(mine + (ch * 32 + q) * 32 + lane, __uint_as_float(r[q]));
+        }
+        __threadfence();
+        __syncwarp();
+        const uint32_t ph = static_cast<uint32_t>(sk_n & 1);
+        ++sk_n;
+        if (lane == 0) mbar_arrive_local(bar_ska);
+        if (ew == 0 && lane == 0) {
+          int last = 0;
+          if (mbar_wait(bar_ska, ph, DEV_ERR_EPI_WAIT)) {
+            __threadfence();
+            int* c = sc.sk_cnt + 2 * un.tsk + static_cast<int>(rank);
+            last = atomicAdd(c, 1) == un.nsplit - 1;
+            if (last) atomicExch(c, 0);       // counters are zero again after the launch
+            __threadfence();
+          } else {
+            *abort_flag = 1;
+          }
+          *sk_flag = last;
+          mbar_arrive_local(bar_skb);
+        }
+        int fin = 0;
+        if (lane == 0)
+          fin = mbar_wait_sleep(bar_skb, ph, DEV_ERR_EPI_WAIT, 32) && *abort_flag == 0
+                    ? (*sk_flag ? 1 : 2) : 0;
+        fin = __shfl_sync(0xffffffffu, fin, 0);
+        if (fin != 1) {
+          if constexpr (EV != 0) cp_wait_all();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(acce_leader + 8 * buf);
+          if (fin == 0) break;
+          continue;
+        }
+        other = sc.sk_part + sk_slot(un.tsk, 1 - un.split, rank) + ew * EPI_COLS * 32;
+      }
       if constexpr (EV != 0) {
         ste_w_epilogue<EV == 2>(epi, tbase, wrow0, col0, rows, cols, lane,
-                                smem + L::WST_OFF + ew * C::WST);
+                                smem + L::WST_OFF + ew * C::WST, other);
       } else {
         float* const out_b = BATCH ? epi.out + static_cast<int64_t>(tw.b) * sc.out_bstride : epi.out;
         for (int ch = 0; ch < EPI_COLS / 32; ++ch) {
           uint32_t r[32];
           tmem_ld32(tbase + ch * 32, r);
           tmem_ld_wait();
+          if (other) {
+#pragma unroll
+            for (int q = 0; q < 32; ++q)
+              r[q] = __float_as_uint(__uint_as_float(r[q]) +
+                                     __ldcg(other + (ch * 32 + q) * 32 + lane));
+          }
           const int64_t cbase = col0 + ch * 32;
           if (row < rows && cbase < cols) {
             if (cbase + 32 <= cols) {
@@ -837,6 +959,25 @@ int64_t gemm_tc_tiles(int64_t rows, int64_t cols) {
   return 2 * ceil_div(rows, tc::TILE_M) * ceil_div(cols, tc::TILE_N);
 }
 
+namespace {
+// Scratch of `skt` stream-K tiles: the arrival counters (2 per tile), then the partial
+// accumulators (2 splits x 2 CTAs x 128 x 256 floats per tile).
+size_t sk_counter_bytes(int64_t skt) { return static_cast<size_t>((skt * 2 * 4 + 255) / 256 * 256); }
+size_t sk_need(int64_t skt) {
+  return sk_counter_bytes(skt) + static_cast<size_t>(skt) * 4 * tc::kSkSlot * sizeof(float);
+}
+}  // namespace
+
+// The stream-K region holds fewer than two waves of tiles (the last whole wave and the tail).
+// Sized for any contraction depth: the depth decides at launch whether the schedule is used.
+size_t gemm_tc_sk_bytes(int64_t rows, int64_t cols) {
+  const int64_t tiles = ceil_div(rows, tc::TILE_M) * ceil_div(cols, tc::TILE_N);
+  const int64_t pairs = num_sms() / 2;
+  if (tiles <= pairs) return 0;
+  const int64_t skt = tiles < 2 * pairs - 1 ? tiles : 2 * pairs - 1;
+  return sk_need(skt);
+}
+
 omq_status gemm_tc(omq_dtype dt, const GemmOperand& A, const GemmOperand& B, int64_t rows,
                    int64_t cols, int64_t depth, const GemmEpilogue& epi, int64_t* n_tiles,
                    cudaStream_t stream, const GemmBatch* batch) {
@@ -870,11 +1011,44 @@ omq_status gemm_tc(omq_dtype dt, const GemmOperand& A, const GemmOperand& B, int
     set_cuda_error(attr_err);
     return OMQ_ERR_CUDA;
   }
-  const TileSched sc{static_cast<int>(tiles_m), static_cast<int>(tiles_n), static_cast<int>(per),
-                     static_cast<int>(tiles), causal, amode, bmode,
-                     batch ? batch->out_stride : 0};
+  TileSched sc{static_cast<int>(tiles_m), static_cast<int>(tiles_n), static_cast<int>(per),
+               static_cast<int>(tiles), causal, amode, bmode,
+               batch ? batch->out_stride : 0};
   const int64_t max_pairs = num_sms() / 2;
   const int64_t pairs = tiles < max_pairs ? tiles : max_pairs;
+  // Stream-K tail: when the last wave of whole tiles would leave more than a fifth of the
+  // pairs idle, the last whole wave and the tail (fewer than 2 waves of tiles) are shared
+  // out as equal runs of k-blocks, longer than one tile's contraction, so every tile of the
+  // region has one or two contributing pairs. Only for long contractions (at least
+  // kSkMinBlocks k-blocks): measured on B200, the split tiles' partial stores and the
+  // staggered k positions of the pairs cost more than the idle tail saves when a tile's
+  // contraction is short (4096-deep: forward 78 -> 98 us at 2048 x 4096; 13824-deep:
+  // forward 287 -> 248 us at 2048 x 5120).
+  sc.dp_tiles = static_cast<int>(tiles);
+  sc.sk_tiles = 0;
+  sc.sk_len = 0;
+  sc.sk_part = nullptr;
+  sc.sk_cnt = nullptr;
+  const int64_t nk = ceil_div(depth, BK);
+  const int64_t rem = tiles % pairs;
+  constexpr int64_t kSkMinBlocks = 128;
+  if (count == 1 && !causal && epi.sk_scratch && tiles > pairs && rem != 0 && 5 * rem <= 4 * pairs &&
+      nk >= kSkMinBlocks) {
+    const int64_t dp = (tiles / pairs - 1) * pairs, skt = tiles - dp;
+    if (sk_need(skt) <= epi.sk_bytes) {
+      sc.dp_tiles = static_cast<int>(dp);
+      sc.sk_tiles = static_cast<int>(skt);
+      sc.sk_len = ceil_div(skt * nk, pairs);
+      sc.sk_cnt = static_cast<int*>(epi.sk_scratch);
+      sc.sk_part = reinterpret_cast<float*>(static_cast<char*>(epi.sk_scratch) +
+                                            sk_counter_bytes(skt));
+      const cudaError_t me = cudaMemsetAsync(sc.sk_cnt, 0, static_cast<size_t>(skt) * 2 * 4, stream);
+      if (me != cudaSuccess) {
+        set_cuda_error(me);
+        return OMQ_ERR_CUDA;
+      }
+    }
+  }
   launch_k(kc.fn, static_cast<unsigned>(2 * pairs), kc.threads, kc.smem, stream,
       ma, mb, A.mn_major ? 1 : 0, B.mn_major ? 1 : 0, dt == OMQ_F16 ? 0u : 1u, rows, cols, depth,
       epi, sc);

@@ -34,6 +34,7 @@ bool fused_ste_w(omq_dtype op_dt, omq_dtype wdt, int64_t group) {
 struct BwdLayout {
   size_t dbt_part, dbt, dwhat, dxq, part_ws, part_wd, part_xs, part_xd, rowstat, red;
   size_t gh_part, gc_part, emax, emin;   // fused weight-side STE (group a multiple of 32)
+  size_t sk_w, sk_w_bytes, sk_x, sk_x_bytes;   // stream-K scratch of the dW^ and dXq GEMMs
   size_t total;
   int64_t rb_colsum, rb_w, rb_x;
 };
@@ -62,14 +63,23 @@ BwdLayout bwd_layout(int64_t M, int64_t N, int64_t K, int64_t group) {
   L.gc_part = take(fusable ? sizeof(float) * (K / 32) * N : 0);
   L.emax = take(fusable ? sizeof(float) * N * (K / group) : 0);
   L.emin = take(fusable ? sizeof(float) * N * (K / group) : 0);
+  // the two backward GEMMs may run at the same time (two streams): one region each
+  L.sk_w_bytes = gemm_tc_sk_bytes(N, K);
+  L.sk_w = take(L.sk_w_bytes);
+  L.sk_x_bytes = gemm_tc_sk_bytes(M, K);
+  L.sk_x = take(L.sk_x_bytes);
   L.total = off;
   return L;
 }
 
-size_t fwd_bytes(int64_t M, int64_t N) {
+// Forward workspace: the per-tile loss partials, then the GEMM's stream-K scratch.
+size_t fwd_partial_bytes(int64_t M, int64_t N) {
   int64_t t = gemm_tc_tiles(M, N);
   int64_t t2 = gemm_f32_simt_tiles(M, N);
   return align256(sizeof(float) * static_cast<size_t>(t > t2 ? t : t2));
+}
+size_t fwd_bytes(int64_t M, int64_t N) {
+  return fwd_partial_bytes(M, N) + align256(gemm_tc_sk_bytes(M, N));
 }
 
 template <class T>
@@ -311,10 +321,12 @@ static omq_status run_gemm(omq_dtype dt, const GemmOperand& A, const GemmOperand
   return gemm_tc(dt, A, B, rows, cols, depth, epi, tiles, st);
 }
 
+// The forward GEMM and, unless loss_stream is given, the loss reduction after it on the same
+// stream; with loss_stream the reduction runs there (forked after the GEMM; the caller joins).
 static omq_status fwd_impl(const void* Xq, const void* W_hat, omq_dtype dt, int64_t M, int64_t N,
                            int64_t K, const float* B_tilde, const float* Y_ref, float* Y, void* dY,
                            float* loss, void* workspace, size_t ws_bytes, omq_stream_t stream,
-                           const Phases& ph) {
+                           const Phases& ph, const SideStream* loss_stream = nullptr) {
   if (!Xq || !W_hat) return OMQ_ERR_NULL;
   if (!dtype_ok(dt)) return OMQ_ERR_DTYPE;
   if (M < 1 || N < 8 || K < 8 || N % 8 || K % 8 || M > kMaxDim || N > kMaxDim || K > kMaxDim)
@@ -332,6 +344,11 @@ static omq_status fwd_impl(const void* Xq, const void* W_hat, omq_dtype dt, int6
   GemmOperand A{Xq, K, false}, B{W_hat, K, false};
   GemmEpilogue epi{};
   epi.bias = B_tilde;
+  const size_t part_bytes = fwd_partial_bytes(M, N);
+  if (workspace && ws_bytes > part_bytes) {
+    epi.sk_scratch = static_cast<char*>(workspace) + part_bytes;
+    epi.sk_bytes = ws_bytes - part_bytes;
+  }
   if (Y_ref) {
     epi.kind = Epi::MseLoss;
     epi.out = Y;
@@ -348,9 +365,15 @@ static omq_status fwd_impl(const void* Xq, const void* W_hat, omq_dtype dt, int6
   OMQ_TRY(ph.mark(OMQ_PH_FWD_GEMM));
   OMQ_TRY(run_gemm(dt, A, B, M, N, K, epi, &tiles, st));
   OMQ_TRY(ph.mark(OMQ_PH_LOSS));
-  if (Y_ref && loss)
+  if (Y_ref && loss) {
+    cudaStream_t ls = st;
+    if (loss_stream) {
+      OMQ_TRY(loss_stream->fork(st));
+      ls = loss_stream->s;
+    }
     OMQ_TRY(launch_loss_finalize(epi.loss_partials, tiles,
-                                 1.0 / (static_cast<double>(M) * static_cast<double>(N)), loss, st));
+                                 1.0 / (static_cast<double>(M) * static_cast<double>(N)), loss, ls));
+  }
   return OMQ_OK;
 }
 
@@ -424,6 +447,8 @@ static omq_status bwd_impl(const omq_bwd_args* a, void* workspace, size_t ws_byt
       GemmOperand A{a->dY, N, true}, B{a->Xq, K, true};
       GemmEpilogue epi{};
       epi.out_scale = gscale;
+      epi.sk_scratch = at<char>(workspace, L.sk_w);
+      epi.sk_bytes = L.sk_w_bytes;
       if (fused) {
         // weight-side STE in the epilogue: per-chunk partial sums and the W-side LET column
         // partials straight from the accumulator
@@ -470,6 +495,8 @@ static omq_status bwd_impl(const omq_bwd_args* a, void* workspace, size_t ws_byt
       epi.kind = Epi::StoreF32;
       epi.out = dxq;
       epi.out_scale = gscale;
+      epi.sk_scratch = at<char>(workspace, L.sk_x);
+      epi.sk_bytes = L.sk_x_bytes;
       OMQ_TRY(run_gemm(a->op_dt, A, B, M, K, N, epi, nullptr, s));
     }
     OMQ_TRY(ph.mark(OMQ_PH_STE_X));
@@ -594,8 +621,11 @@ omq_status omq_calib_step(const omq_step_args* a, void* workspace, size_t ws_byt
     OMQ_TRY(ph.mark(OMQ_PH_LWC));
     OMQ_TRY(lwc(st));
   }
+  // without phase events the loss reduction runs on the second stream, beside the backward
+  // (which does not read it); the stream is joined before AdamW
+  const SideStream* ls = ph.ev ? nullptr : side_stream();
   OMQ_TRY(fwd_impl(Xq, a->W_hat, a->op_dt, M, N, K, Bt, a->Y_ref, nullptr, a->dY, a->loss,
-                   workspace, fwd_ws, stream, ph));
+                   workspace, fwd_ws, stream, ph, ls));
   omq_bwd_args b{};
   b.M = M; b.N = N; b.K = K; b.group = G; b.bits = a->bits; b.abits = a->abits; b.dt = a->dt;
   b.op_dt = a->op_dt;
@@ -606,6 +636,7 @@ omq_status omq_calib_step(const omq_step_args* a, void* workspace, size_t ws_byt
   b.d_gamma_logit = a->d_gamma_logit; b.d_beta_logit = a->d_beta_logit;
   b.d_s = let ? a->d_s : nullptr; b.d_delta = let ? a->d_delta : nullptr;
   OMQ_TRY(bwd_impl(&b, static_cast<char*>(workspace) + fwd_ws, ws_bytes - fwd_ws, stream, ph));
+  if (ls) OMQ_TRY(ls->join(st));
   OMQ_TRY(ph.mark(OMQ_PH_ADAMW));
   const int64_t ng = N * (K / G);
   const AdamSeg segs[kMaxAdamSegs] = {

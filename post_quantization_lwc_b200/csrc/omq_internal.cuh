@@ -244,6 +244,10 @@ struct GemmEpilogue {
   float* loss_partials;    // MseLoss: one per output tile (fixed order)
   SteWEpi ste;             // SteW
   int64_t ldo;             // row stride of out / y_ref / dy in elements (0: cols)
+  // Scratch of the stream-K tail schedule of the tcgen05 GEMM (gemm_tc_sk_bytes), or NULL:
+  // partial accumulators of split tiles and their arrival counters.
+  void* sk_scratch;
+  size_t sk_bytes;
 };
 
 // Group lengths whose weight-side STE runs in the dW^ GEMM's epilogue: whole 32-column
@@ -269,6 +273,13 @@ struct TileSched {
   int causal;
   int a_bmode, b_bmode;   // operand maps: 0 2D; 1 / 2 3D, the problem index the middle / outer
   int64_t out_bstride;
+  // stream-K tail: tiles [0, dp_tiles) go whole to pairs in turn; the k-blocks of tiles
+  // [dp_tiles, dp_tiles + sk_tiles) are dealt out as contiguous runs of sk_len k-blocks per
+  // pair (sk_tiles = 0: every tile whole)
+  int dp_tiles, sk_tiles;
+  int64_t sk_len;
+  float* sk_part;         // [sk_tiles][2 splits][2 CTAs][128 x 256] partial accumulators
+  int* sk_cnt;            // [sk_tiles][2 CTAs] arrivals
 };
 
 // 16-bit operands (BF16 or F16, both the same type) on tcgen05 (sm_100a). Reports the
@@ -277,6 +288,9 @@ omq_status gemm_tc(omq_dtype dt, const GemmOperand& A, const GemmOperand& B, int
                    int64_t cols, int64_t depth, const GemmEpilogue& epi, int64_t* n_tiles,
                    cudaStream_t stream, const GemmBatch* batch = nullptr);
 int64_t gemm_tc_tiles(int64_t rows, int64_t cols);
+// Scratch that lets gemm_tc run the stream-K tail schedule on a rows x cols output (current
+// device); GemmEpilogue::sk_scratch of at least this size enables it.
+size_t gemm_tc_sk_bytes(int64_t rows, int64_t cols);
 // f32 operands on CUDA cores.
 omq_status gemm_f32_simt(const GemmOperand& A, const GemmOperand& B, int64_t rows, int64_t cols,
                          int64_t depth, const GemmEpilogue& epi, int64_t* n_tiles,

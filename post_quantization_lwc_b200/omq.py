@@ -160,10 +160,15 @@ def _dt(t) -> int:
     return _DTYPES[dtype]
 
 
-def operand_dtype(storage: torch.dtype) -> torch.dtype:
-    """GEMM operand dtype the step uses for a storage dtype: float16 for 16-bit storage
-    (3 more mantissa bits than bfloat16 at the same tensor-core rate), float32 otherwise."""
-    return torch.float32 if storage == torch.float32 else torch.float16
+def operand_dtype(storage: torch.dtype, act_pass: bool = True) -> torch.dtype:
+    """GEMM operand dtype the step uses for a storage dtype: float32 for float32 storage;
+    for 16-bit storage float16 (3 more mantissa bits than bfloat16 at the same tensor-core
+    rate) when the step writes its own activation operand anyway (LET or activation
+    quantization, ``act_pass``), else the storage type itself, so that X is the operand as
+    it stands and no conversion pass over it runs."""
+    if storage == torch.float32:
+        return torch.float32
+    return torch.float16 if act_pass else storage
 
 
 def _stream(stream=None):
@@ -392,7 +397,7 @@ class LinearCalibration:
         self.s, self.delta = f(K), f(K)
         self.moments = {k: (f(*shape), f(*shape)) for k, shape in
                         (("gamma", (N, ng)), ("beta", (N, ng)), ("s", (K,)), ("delta", (K,)))}
-        self.op_dtype = operand_dtype(self.dtype)
+        self.op_dtype = operand_dtype(self.dtype, self.let or self.abits < 16)
         need_act = self.let or self.abits < 16 or self.op_dtype != self.dtype
         self.Xq = torch.empty(M, K, dtype=self.op_dtype, device=dev) if need_act else None
         self.W_hat = torch.empty(N, K, dtype=self.op_dtype, device=dev)
@@ -489,16 +494,20 @@ class PhaseTimer:
 # theta tensors (OMQ_TH_* in include/omq.h) and workspace tensors (OMQ_BB_*), in order
 THETA = ("gamma_qkv", "beta_qkv", "gamma_o", "beta_o", "gamma_gu", "beta_gu", "gamma_d",
          "beta_d", "s1", "delta1", "s_a", "s_o", "delta_o", "s2", "delta2")
+# The block's named workspace tensors as omq_block_step leaves them: float16 GEMM operands,
+# the gradients between stages unscaled (in units of the residual y - y*, i.e. gradients of
+# (M D / 2) times the loss). omq_block_reference writes its 16-bit operands as bfloat16.
+_H = torch.float16
 BLOCK_BUFFERS = (
-    ("rope", torch.float32), ("a", torch.float32), ("qa", torch.bfloat16),
-    ("what_qkv", torch.bfloat16), ("what_o", torch.bfloat16), ("what_gu", torch.bfloat16),
-    ("what_d", torch.bfloat16), ("qkv", torch.float32), ("qqkv", torch.bfloat16),
-    ("p", torch.float32), ("p16", torch.bfloat16), ("o", torch.float32), ("qo", torch.bfloat16),
-    ("x2", torch.float32), ("b", torch.float32), ("qb", torch.bfloat16), ("gu", torch.float32),
-    ("mid", torch.float32), ("qm", torch.bfloat16), ("res", torch.bfloat16),
-    ("dmid", torch.float32), ("dgu", torch.bfloat16), ("db", torch.float32),
-    ("dx2", torch.bfloat16), ("do", torch.bfloat16), ("dqqkv", torch.float32),
-    ("dqkv", torch.bfloat16))
+    ("rope", torch.float32), ("a", torch.float32), ("qa", _H),
+    ("what_qkv", _H), ("what_o", _H), ("what_gu", _H),
+    ("what_d", _H), ("qkv", torch.float32), ("qqkv", _H),
+    ("p", torch.float32), ("p16", _H), ("o", torch.float32), ("qo", _H),
+    ("x2", torch.float32), ("b", torch.float32), ("qb", _H), ("gu", torch.float32),
+    ("mid", torch.float32), ("qm", _H), ("res", _H),
+    ("dmid", torch.float32), ("dgu", _H), ("db", torch.float32),
+    ("dx2", _H), ("do", _H), ("dqqkv", torch.float32),
+    ("dqkv", _H))
 BLOCK_PHASES = ("weights", "attn_in", "attn", "ffn", "bwd_ffn", "bwd_attn", "bwd_qkv", "reduce",
                 "adamw")
 

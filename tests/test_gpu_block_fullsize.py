@@ -67,6 +67,16 @@ def buf(r, name, *shape):
     return _f(r.blk.buffer(name)).reshape(*shape)
 
 
+def gbuf(r, name, *shape):
+    """A stored stage gradient scaled to dL (the step keeps them in units of y - y*)."""
+    return buf(r, name, *shape).astype(np.float64) * (2.0 / (r.sh.M * r.sh.D))
+
+
+def _f16(x):
+    """The float16 operand the step stores for the binary32 value x (round to nearest even)."""
+    return np.asarray(x, np.float32).astype(np.float16).astype(np.float32)
+
+
 def grad(r, name):
     o, n = r.blk.theta_slices[name]
     return r.grad[o:o + n]
@@ -83,7 +93,7 @@ def test_weights_sampled_rows(run):
         bl = r.th["beta_" + name][rows]
         _, enc, _, _ = om.lwc_quant(W, s_of[name], gl[:, None], bl[:, None], sh.wbits, W.shape[1])
         got = buf(r, "what_" + name, *shapes[name])[rows]
-        assert np.array_equal(_bits(got), _bits(om.bf16_round(enc.deq))), name
+        assert np.array_equal(_bits(got), _bits(_f16(enc.deq))), name
 
 
 def test_forward_sampled_tokens(run):
@@ -95,7 +105,7 @@ def test_forward_sampled_tokens(run):
     assert frob_rel(a[t], ob.rms_norm(r.x[t])[0]) < 1e-6
     qa_ref, _ = ob.act_encode(om.let_act(a[t], th["s1"], th["delta1"]), A, D)
     qa = buf(r, "qa", M, D)
-    assert np.array_equal(_bits(qa[t]), _bits(om.bf16_round(qa_ref)))
+    assert np.array_equal(_bits(qa[t]), _bits(_f16(qa_ref)))
     Wq = buf(r, "what_qkv", 3 * D, D).astype(np.float64)
     qkv = buf(r, "qkv", M, 3 * D)
     qkv_ref = qa[t].astype(np.float64) @ Wq.T + om.let_bias(W["qkv"], None, th["delta1"])
@@ -106,7 +116,7 @@ def test_forward_sampled_tokens(run):
     ap = ob.stage_attn_prep(qkv[t], cos[t], sin[t], th["s_a"], th["s_o"], th["delta_o"], H, A)
     qqkv = buf(r, "qqkv", M, 3 * D)
     want = np.concatenate([ap["Qq"], ap["Qk"], ap["Qv"]], axis=1)
-    assert np.array_equal(_bits(qqkv[t]), _bits(om.bf16_round(want)))
+    assert np.array_equal(_bits(qqkv[t]), _bits(_f16(want)))
     # causal softmax rows of sampled (head, query), from the GPU's quantized Q, K
     P = r.blk.buffer("p").view(H, M, M)
     P16 = r.blk.buffer("p16").view(H, M, M)
@@ -120,9 +130,9 @@ def test_forward_sampled_tokens(run):
             assert frob_rel(_f(P[h, i, :i + 1]), p) < 1e-5
             span = min((i // 256 + 1) * 256, M)
             p16 = _f(P16[h, i, :span])
-            assert np.array_equal(_bits(p16[:i + 1]), _bits(om.bf16_round(_f(P[h, i, :i + 1]))))
+            assert np.array_equal(_bits(p16[:i + 1]), _bits(_f16(_f(P[h, i, :i + 1]))))
             assert (p16[i + 1:] == 0).all()
-    # O on sampled tokens from the GPU's BF16 probabilities and Qv
+    # O on sampled tokens from the GPU's float16 probabilities and Qv
     O = buf(r, "o", M, D)
     qv = qqkv[:, 2 * D:].astype(np.float64)
     for i in t:
@@ -131,7 +141,7 @@ def test_forward_sampled_tokens(run):
         assert frob_rel(O[i], o_ref) < 1e-5
     Qo_ref, _ = ob.act_encode(O[t], A, D)
     qo = buf(r, "qo", M, D)
-    assert np.array_equal(_bits(qo[t]), _bits(om.bf16_round(Qo_ref)))
+    assert np.array_equal(_bits(qo[t]), _bits(_f16(Qo_ref)))
     x2 = buf(r, "x2", M, D)
     x2_ref = r.x[t].astype(np.float64) + qo[t].astype(np.float64) @ buf(
         r, "what_o", D, D).astype(np.float64).T + om.let_bias(W["o"], None, th["delta_o"])
@@ -140,7 +150,7 @@ def test_forward_sampled_tokens(run):
     assert frob_rel(b[t], ob.rms_norm(x2[t])[0]) < 1e-6
     qb_ref, _ = ob.act_encode(om.let_act(b[t], th["s2"], th["delta2"]), A, D)
     qb = buf(r, "qb", M, D)
-    assert np.array_equal(_bits(qb[t]), _bits(om.bf16_round(qb_ref)))
+    assert np.array_equal(_bits(qb[t]), _bits(_f16(qb_ref)))
     gu = buf(r, "gu", M, 2 * I)
     gu_ref = qb[t].astype(np.float64) @ buf(r, "what_gu", 2 * I, D).astype(np.float64).T + \
         om.let_bias(W["gu"], None, th["delta2"])
@@ -148,7 +158,7 @@ def test_forward_sampled_tokens(run):
     mid = buf(r, "mid", M, I)
     assert frob_rel(mid[t], ob.silu(gu[t, :I]) * gu[t, I:]) < 1e-5
     qm_ref, _ = ob.act_encode(mid[t], A, I)
-    assert np.array_equal(_bits(buf(r, "qm", M, I)[t]), _bits(om.bf16_round(qm_ref)))
+    assert np.array_equal(_bits(buf(r, "qm", M, I)[t]), _bits(_f16(qm_ref)))
 
 
 def test_loss_all_tokens(run):
@@ -159,7 +169,7 @@ def test_loss_all_tokens(run):
     res = y - r.y_ref
     loss_ref = float((res ** 2).mean())
     assert abs(r.loss - loss_ref) <= 1e-4 * loss_ref
-    assert frob_rel(buf(r, "res", M, D), res) < 1e-2
+    assert frob_rel(buf(r, "res", M, D), res) < 2e-3
 
 
 def test_backward_sampled(run):
@@ -176,9 +186,9 @@ def test_backward_sampled(run):
                                 th["beta_" + name][rows], sh.wbits, W[name].shape[1])
           for name, rows, s in (("d", ROWS["d"], None), ("gu", ROWS["gu"], th["s2"]),
                                 ("o", ROWS["o"], th["s_o"]), ("qkv", ROWS["qkv"], th["s1"]))}
-    dgu = buf(r, "dgu", M, 2 * I).astype(f64)
-    dx2 = buf(r, "dx2", M, D).astype(f64)
-    dqkv = buf(r, "dqkv", M, 3 * D).astype(f64)
+    dgu = gbuf(r, "dgu", M, 2 * I)
+    dx2 = gbuf(r, "dx2", M, D)
+    dqkv = gbuf(r, "dqkv", M, 3 * D)
     upstream = {"d": (dy, "qm", I), "gu": (dgu, "qb", D), "o": (dx2, "qo", D),
                 "qkv": (dqkv, "qa", D)}
     for name, (dY, xq_name, K) in upstream.items():
@@ -192,28 +202,28 @@ def test_backward_sampled(run):
     mid = buf(r, "mid", M, I)
     _, enc_m = ob.act_encode(mid[t], A, I)
     dm_ref = ob.act_backward(dy[t] @ buf(r, "what_d", D, I).astype(f64), mid[t], enc_m)
-    assert frob_rel(buf(r, "dmid", M, I)[t], dm_ref) < 1e-4
+    assert frob_rel(gbuf(r, "dmid", M, I)[t], dm_ref) < 1e-4
     gu = buf(r, "gu", M, 2 * I).astype(f64)
     g, u = gu[t, :I], gu[t, I:]
     sg = 1 / (1 + np.exp(-g))
-    dm = buf(r, "dmid", M, I)[t].astype(f64)
-    assert frob_rel(dgu[t], np.concatenate([dm * u * sg * (1 + g * (1 - sg)), dm * g * sg], 1)) < 1e-2
+    dm = gbuf(r, "dmid", M, I)[t]
+    assert frob_rel(dgu[t], np.concatenate([dm * u * sg * (1 + g * (1 - sg)), dm * g * sg], 1)) < 2e-3
     b = buf(r, "b", M, D)
     bt = om.let_act(b[t], th["s2"], th["delta2"])
     _, enc_b = ob.act_encode(bt, A, D)
     dbt = ob.act_backward(dgu[t] @ buf(r, "what_gu", 2 * I, D).astype(f64), bt, enc_b)
-    db = buf(r, "db", M, D)
+    db = gbuf(r, "db", M, D)
     assert frob_rel(db[t], dbt / th["s2"].astype(f64)) < 1e-4
     _, rstd2 = ob.rms_norm(buf(r, "x2", M, D)[t])
-    assert frob_rel(dx2[t], dy[t] + ob.rms_backward(db[t], b[t], rstd2)) < 1e-2
+    assert frob_rel(dx2[t], dy[t] + ob.rms_backward(db[t], b[t], rstd2)) < 2e-3
     O = buf(r, "o", M, D)
     _, enc_o = ob.act_encode(O[t], A, D)
     dO_ref = ob.act_backward(dx2[t] @ buf(r, "what_o", D, D).astype(f64), O[t], enc_o)
-    dO = buf(r, "do", M, D).astype(f64)
-    assert frob_rel(dO[t], dO_ref) < 1e-2
+    dO = gbuf(r, "do", M, D)
+    assert frob_rel(dO[t], dO_ref) < 2e-3
     # attention backward of sampled heads, over all tokens of the head
     qqkv = buf(r, "qqkv", M, 3 * D).astype(f64)
-    dqq = buf(r, "dqqkv", M, 3 * D)
+    dqq = gbuf(r, "dqqkv", M, 3 * D)
     Pb = r.blk.buffer("p").view(H, M, M)
     low = np.tril(np.ones((M, M), dtype=bool))
     for h in HEADS:
@@ -237,4 +247,4 @@ def test_backward_sampled(run):
     sa, so = th["s_a"].astype(f64), th["s_o"].astype(f64)
     want = np.concatenate([ob.rope_backward(dqt / sa, cos[t], sin[t], H),
                            ob.rope_backward(dkt * sa, cos[t], sin[t], H), dvt / so], axis=1)
-    assert frob_rel(dqkv[t], want) < 1e-2
+    assert frob_rel(dqkv[t], want) < 2e-3
