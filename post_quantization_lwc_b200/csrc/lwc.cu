@@ -301,55 +301,67 @@ __device__ __forceinline__ void scale8(const float* s, int64_t col, float (&v)[8
 // ---- row-staged launch shape -----------------------------------------------------------
 // 16-bit W and W^, groups of 32, 64, 128 or 256 columns or one group per row. One warp per
 // row, persistent warps: the row is copied into the warp's shared-memory buffer by 16-byte
-// cp.async copies (the next row's copies in flight while this one is encoded, when two
+// cp.async copies (the next piece's copies in flight while this one is encoded, when two
 // buffers fit), then walked in 256-column segments by a rolled loop, lane l holding columns
 // 256 i + 8 l .. + 7 of segment i. A group of G = 8 LPG columns is a sub-warp of LPG lanes;
 // one group per row (LPG = 0) takes two passes over the staged row (max / min, then the
-// encoder). B~[n] = B[n] + sum_k W[n,k] delta[k] comes out of the same pass over the row.
+// encoder), so its piece is the whole row; grouped rows are staged in pieces of `pcols`
+// columns (whole groups, whole segments), so that a long row does not take a warp's whole
+// share of shared memory and the warps per SM stay many. B~[n] = B[n] + sum_k W[n,k]
+// delta[k] comes out of the same pass over the row.
 
 constexpr int kStageSegs = 4;   // 256-column segments a grouped batch holds in registers
+constexpr int64_t kStagePiece = 2048;   // columns a grouped piece holds
 
 // Warps a block may hold: one group per row keeps few registers and takes more warps.
 constexpr int stage_max_warps(int lpg) { return lpg == 0 ? 24 : 16; }
 
 template <int LPG, bool F16>
 __global__ void __launch_bounds__(32 * stage_max_warps(LPG))
-    lwc_stage_kernel(LwcParams p, int nbuf, int64_t rows_per_warp) {
+    lwc_stage_kernel(LwcParams p, int nbuf, int64_t rows_per_warp, int64_t pcols) {
   pdl_wait();
   pdl_launch();
   extern __shared__ __align__(16) unsigned char lsm[];
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5, wpb = blockDim.x >> 5;
-  const int64_t K = p.K, ng = p.ng, chunks = K / 8;
-  uint16_t* rows = reinterpret_cast<uint16_t*>(lsm) + static_cast<int64_t>(wib) * nbuf * K;
-  // grouped: per warp, nbuf staged copies of the row's logits (gamma then beta), then the
-  // row's strengths (gamma, beta of each group interleaved)
-  float* lgb = reinterpret_cast<float*>(lsm + static_cast<size_t>(wpb) * nbuf * K * 2) +
-               static_cast<int64_t>(wib) * (nbuf + 1) * 2 * ng;
-  float* sst = lgb + nbuf * 2 * ng;
+  const int64_t K = p.K, ng = p.ng;
+  const int64_t pieces = (K + pcols - 1) / pcols, png = pcols / p.G;   // groups a piece holds
+  uint16_t* rows = reinterpret_cast<uint16_t*>(lsm) + static_cast<int64_t>(wib) * nbuf * pcols;
+  // grouped: per warp, nbuf staged copies of the piece's logits (gamma then beta), then the
+  // piece's strengths (gamma, beta of each group interleaved)
+  float* lgb = reinterpret_cast<float*>(lsm + static_cast<size_t>(wpb) * nbuf * pcols * 2) +
+               static_cast<int64_t>(wib) * (nbuf + 1) * 2 * png;
+  float* sst = lgb + nbuf * 2 * png;
   // warp w of block b is warp w * gridDim.x + b, so a partial last round of rows spreads
   // over all blocks
   const int64_t n_warps = static_cast<int64_t>(gridDim.x) * wpb;
   const int64_t wg = static_cast<int64_t>(wib) * gridDim.x + blockIdx.x;
   const bool hat_f16 = p.hat_dt == OMQ_F16;
   const bool let = p.s != nullptr, bias_on = p.Bt != nullptr && p.delta != nullptr;
+  const int64_t items = rows_per_warp * pieces;        // (row, piece) in row-major order
   auto issue = [&](int64_t it) {
-    const int64_t n = wg + it * n_warps;
-    if (it < rows_per_warp && n < p.N) {
-      const unsigned char* src = static_cast<const unsigned char*>(p.W) + n * K * 2;
-      uint16_t* dst = rows + (it % nbuf) * K;
-      for (int64_t c = lane; c < chunks; c += 32) cp_async16(dst + c * 8, src + c * 16);
+    const int64_t n = wg + (it / pieces) * n_warps;
+    if (it < items && n < p.N) {
+      const int64_t pc0 = (it % pieces) * pcols;
+      const int64_t nc = K - pc0 < pcols ? K - pc0 : pcols;
+      const unsigned char* src = static_cast<const unsigned char*>(p.W) + (n * K + pc0) * 2;
+      uint16_t* dst = rows + (it % nbuf) * pcols;
+      for (int64_t c = lane; c < nc / 8; c += 32) cp_async16(dst + c * 8, src + c * 16);
       if constexpr (LPG != 0) {
-        float* lg = lgb + (it % nbuf) * 2 * ng;
-        for (int64_t i = lane; i < 2 * ng; i += 32)
-          cp_async4(lg + i, i < ng ? p.gl + n * ng + i : p.bl + n * ng + (i - ng));
+        const int64_t g0 = pc0 / p.G, gn = nc / p.G;
+        float* lg = lgb + (it % nbuf) * 2 * png;
+        for (int64_t i = lane; i < 2 * gn; i += 32)
+          cp_async4(lg + i, i < gn ? p.gl + n * ng + g0 + i : p.bl + n * ng + g0 + (i - gn));
       }
     }
     cp_async_commit();
   };
   issue(0);
-  for (int64_t it = 0; it < rows_per_warp; ++it) {
-    const int64_t n = wg + it * n_warps;
+  float2 bias2 = make_float2(0.f, 0.f);
+  for (int64_t it = 0; it < items; ++it) {
+    const int64_t n = wg + (it / pieces) * n_warps;
     if (n >= p.N) break;                                       // warp-uniform
+    const int64_t pc = it % pieces, pc0 = pc * pcols;
+    const int64_t nc = K - pc0 < pcols ? K - pc0 : pcols;
     if (nbuf == 2) {
       issue(it + 1);
       cp_async_wait<1>();
@@ -357,11 +369,13 @@ __global__ void __launch_bounds__(32 * stage_max_warps(LPG))
       cp_async_wait<0>();
     }
     __syncwarp();
-    const uint16_t* row = rows + (it % nbuf) * K;
-    uint16_t* hat = static_cast<uint16_t*>(p.W_hat) + n * K;
-    float2 bias2 = make_float2(0.f, 0.f);
+    const uint16_t* row = rows + (it % nbuf) * pcols;        // columns pc0 .. pc0 + nc - 1
+    uint16_t* hat = static_cast<uint16_t*>(p.W_hat) + n * K + pc0;
+    if (pc == 0) bias2 = make_float2(0.f, 0.f);
     if constexpr (LPG == 0) {
-      // one group per row: max / min over the staged row, then the encoder
+      // one group per row (the piece is the whole row): max / min over the staged row, then
+      // the encoder
+      const int64_t chunks = nc / 8;
       float st = 1.f;
       if (lane < 2) st = strength((lane ? p.bl : p.gl)[n]);
       float vmax = -FLT_MAX, vmin = FLT_MAX;
@@ -450,31 +464,33 @@ __global__ void __launch_bounds__(32 * stage_max_warps(LPG))
     } else {
       // groups of 8 LPG columns: kStageSegs segments at a time; the batch's GPB groups get
       // their parameters from one lane each (lane t serves group t % GPB) and hand them back
-      // by shuffles
+      // by shuffles. Columns are local to the piece (global column pc0 + lc), groups too
+      // (group j of the piece is group pg0 + j of the row).
       constexpr int GPS = 32 / LPG, GPB = kStageSegs * GPS;
       static_assert(GPB <= 32, "one lane per group of a batch");
-      const float* lg = lgb + (it % nbuf) * 2 * ng;
-      for (int64_t i = lane; i < 2 * ng; i += 32)
-        sst[i] = strength(lg[(i & 1) * ng + (i >> 1)]);
+      const int64_t pg0 = pc0 / p.G, gn = nc / p.G;
+      const float* lg = lgb + (it % nbuf) * 2 * png;
+      for (int64_t i = lane; i < 2 * gn; i += 32)
+        sst[i] = strength(lg[(i & 1) * gn + (i >> 1)]);
       __syncwarp();
-      const int64_t nseg = (K + 255) / 256;
+      const int64_t nseg = (nc + 255) / 256;
       for (int64_t s0 = 0; s0 < nseg; s0 += kStageSegs) {
         float2 V[kStageSegs][4];
         float vmx[kStageSegs], vmn[kStageSegs], cnt[kStageSegs];
 #pragma unroll
         for (int u = 0; u < kStageSegs; ++u) {
-          const int64_t col = (s0 + u) * 256 + lane * 8;
-          if (col < K) {     // whole groups: a group's lanes are all in or all out
-            unpack16x8_x2(*reinterpret_cast<const uint4*>(row + col), F16, V[u]);
+          const int64_t lc = (s0 + u) * 256 + lane * 8;
+          if (lc < nc) {     // whole groups: a group's lanes are all in or all out
+            unpack16x8_x2(*reinterpret_cast<const uint4*>(row + lc), F16, V[u]);
             if (bias_on) {
               float2 D[4];
-              load_f8_x2(p.delta, col, D);
+              load_f8_x2(p.delta, pc0 + lc, D);
 #pragma unroll
               for (int j = 0; j < 4; ++j) bias2 = __ffma2_rn(V[u][j], D[j], bias2);
             }
             if (let) {
               float2 S[4];
-              load_f8_x2(p.s, col, S);
+              load_f8_x2(p.s, pc0 + lc, S);
 #pragma unroll
               for (int j = 0; j < 4; ++j) V[u][j] = __fmul2_rn(V[u][j], S[j]);
             }
@@ -504,13 +520,13 @@ __global__ void __launch_bounds__(32 * stage_max_warps(LPG))
           const float c = __shfl_sync(0xffffffffu, cnt[u], src);
           if (u == ut) { gmx = x; gmn = y; gc = c; }
         }
-        const int64_t j = (s0 + ut) * GPS + sg;                  // group within the row
+        const int64_t j = (s0 + ut) * GPS + sg;                  // group within the piece
         StageQ gq{H_FLOOR, 0.f, 0.f, 0.4f};
-        if (j < ng) {
+        if (j < gn) {
           const GroupQ q = group_params(sst[2 * j], sst[2 * j + 1], gmx, gmn, p.Q);
           gq = stage_q(q, gmx, gmn);
           if (lane < GPB) {
-            const int64_t gi = n * ng + j;
+            const int64_t gi = n * ng + pg0 + j;
             const int ic = static_cast<int>(gc);
             if (p.h) p.h[gi] = q.h;
             if (p.z) p.z[gi] = z_to_i32(q.z);
@@ -526,12 +542,12 @@ __global__ void __launch_bounds__(32 * stage_max_warps(LPG))
           q.z = __shfl_sync(0xffffffffu, gq.z, holder);
           q.thr = __shfl_sync(0xffffffffu, gq.thr, holder);
           const uint4 out = encode8_x2(V[u], q, p.Q, hat_f16);
-          const int64_t col = (s0 + u) * 256 + lane * 8;
-          if (col < K) *reinterpret_cast<uint4*>(hat + col) = out;
+          const int64_t lc = (s0 + u) * 256 + lane * 8;
+          if (lc < nc) *reinterpret_cast<uint4*>(hat + lc) = out;
         }
       }
     }
-    if (p.Bt) {
+    if (p.Bt && pc == pieces - 1) {
       float bias = __fadd_rn(bias2.x, bias2.y);
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) bias += __shfl_xor_sync(0xffffffffu, bias, o);
@@ -547,6 +563,7 @@ __global__ void __launch_bounds__(32 * stage_max_warps(LPG))
 struct StageShape {
   int lpg = -1;          // lanes per group (0: one group per row); -1: shape not applicable
   int nbuf = 0, wpb = 0;
+  int64_t pcols = 0;     // columns a staged piece holds (the row when one group per row)
   size_t smem = 0;
 };
 constexpr size_t kStageSmem = 200 * 1024;
@@ -564,10 +581,12 @@ StageShape stage_shape(const LwcParams& p) {
   } else {
     return s;
   }
-  const size_t row = static_cast<size_t>(p.K) * 2;
-  const size_t lg = s.lpg ? static_cast<size_t>(p.ng) * 8 : 0;   // logits or strengths, a row
+  s.pcols = s.lpg == 0 ? p.K : std::min<int64_t>((p.K + 255) / 256 * 256, kStagePiece);
+  const size_t row = static_cast<size_t>(s.pcols) * 2;
+  // logits or strengths of a piece's groups
+  const size_t lg = s.lpg ? static_cast<size_t>(s.pcols / p.G) * 8 : 0;
   const size_t cap = static_cast<size_t>(s.lpg == 0 ? stage_max_warps(0) : stage_max_warps(8));
-  // two staged rows a warp only when that still leaves room for the most warps
+  // two staged pieces a warp only when that still leaves room for the most warps
   s.nbuf = cap * (2 * row + 3 * lg) <= kStageSmem ? 2 : 1;
   const size_t per_warp = s.nbuf * (row + lg) + lg;
   s.wpb = static_cast<int>(std::min<size_t>(cap, kStageSmem / per_warp));
@@ -603,7 +622,7 @@ omq_status launch_stage(const LwcParams& p, const StageShape& s, cudaStream_t st
   const int64_t blocks = (warps + wpb - 1) / wpb;
   const size_t smem = s.smem / s.wpb * wpb;
   launch_k(kernel, static_cast<unsigned>(blocks), static_cast<unsigned>(32 * wpb), smem, stream,
-      p, s.nbuf, per);
+      p, s.nbuf, per, s.pcols);
   return launch_status();
 }
 

@@ -1,8 +1,8 @@
 """GPU parity of the row-staged LWC launch shape (16-bit W and W^, groups of 32 to 256
 columns or one group per row, no integer codes requested) against the oracle, bit for bit:
 W^, h, z and the group ranges with their tie counts. The shapes cover both buffer modes
-(two staged rows per warp, and one for long rows), persistent warps with several rows
-each, a ragged last 256-column segment, constant / zero rows and groups, ties at both
+(two staged rows per warp, and one for long rows), grouped rows staged in several pieces,
+persistent warps with several rows each, a ragged last 256-column segment, constant / zero rows and groups, ties at both
 extremes and clipping on both sides. The same pass's B~ = B + W delta is checked through
 the calibration step against the exact sum, within the binary32 summation bound."""
 import dataclasses
@@ -53,6 +53,10 @@ CASES = [
     StagedCase("bf16_g256_k2304", 150, 2304, 256, "bf16", "bf16", True, 8, 6),
     # groups of 128, one staged buffer
     StagedCase("bf16_g128_k6144_single", 64, 6144, 128, "bf16", "f16", False, 4, 7),
+    # grouped rows longer than one staged piece (2048 columns): 7 pieces with a ragged last
+    # one (K = 6.75 pieces), B~ summed across the pieces of a row; the down_proj row length
+    StagedCase("bf16_g64_k13824_pieces", 700, 13824, 64, "bf16", "bf16", True, 2, 8),
+    StagedCase("f16_g32_k2304_two_pieces", 900, 2304, 32, "f16", "f16", True, 4, 9),
 ]
 
 
@@ -113,7 +117,7 @@ def test_lwc_staged_bit_exact(omq, cuda_device, case):
     assert (enc.codes == 0).any() and (enc.codes == 2 ** case.bits - 1).any()
 
 
-@pytest.mark.parametrize("case", [CASES[0], CASES[2], CASES[4]], ids=lambda c: c.name)
+@pytest.mark.parametrize("case", [CASES[0], CASES[2], CASES[4], CASES[7]], ids=lambda c: c.name)
 def test_calib_step_fused_bias(omq, cuda_device, case):
     """B~ = B + W delta from the LWC pass of omq_calib_step (W~ = s W, LET on), with W^, h and
     z of the same pass bit for bit. (The step takes N a multiple of 8.)"""

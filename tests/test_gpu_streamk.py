@@ -47,7 +47,9 @@ def test_stream_k_forward_matches_fp64_product(omq, cuda_device, M, N, K):
     b = omq.fq_linear_fwd(*args, **kw)
     torch.cuda.synchronize()
     omq.sync_check()
-    assert frob_rel(a["Y"].cpu().numpy(), ref.numpy()) <= 2e-6
+    # float32 accumulation of K exact products: relative error about sqrt(K) 2^-24 (a
+    # missing or misplaced partial would be of order one)
+    assert frob_rel(a["Y"].cpu().numpy(), ref.numpy()) <= 3 * np.sqrt(K) * 2.0 ** -24
     res = (ref - Yref.double()).numpy()
     assert frob_rel(a["dY"].float().cpu().numpy(), res) <= 2e-3       # float16 residual
     loss = float((res ** 2).mean())
