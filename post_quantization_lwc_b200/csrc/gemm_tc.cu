@@ -424,7 +424,7 @@ template <bool F16>
 __device__ __forceinline__ void ste_w_epilogue(const GemmEpilogue& epi, uint32_t tcol,
                                                int64_t wrow0, int64_t col0, int64_t rows,
                                                int64_t cols, int lane, const uint8_t* wst,
-                                               const float* other) {
+                                               const float* other, const float (&hz)[4]) {
   const SteWEpi& p = epi.ste;
   const int64_t row = wrow0 + lane;
   const bool valid = row < rows;
@@ -437,49 +437,56 @@ __device__ __forceinline__ void ste_w_epilogue(const GemmEpilogue& epi, uint32_t
   for (int c = 0; c < 2; ++c) {
     const int64_t k0 = col0 + 32 * c;
     if (k0 >= cols) break;                           // warp-uniform
-    const int64_t gi = row * p.ng + static_cast<int>(k0) / static_cast<int>(p.G);
-    float h = 1.f, z = 0.f;
-    if (valid) {
-      h = p.h[gi];
-      z = static_cast<float>(p.z[gi]);
-    }
+    // h and z of this chunk's group (loaded before the accumulator wait)
+    const float h = hz[2 * c], z = hz[2 * c + 1];
     const float hinv = __frcp_rn(h);
     float Gh = 0.f, Gc = 0.f;
     float ps[32];
+    // the chunk's 32 accumulator columns: both 16-column loads in flight, one wait
+    uint32_t r[32];
+    __syncwarp();
+    tmem_ld16(tcol + 32 * c, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+    tmem_ld16(tcol + 32 * c + 16, *reinterpret_cast<uint32_t(*)[16]>(&r[16]));
+    tmem_ld_wait();
+    if (other) {   // a stream-K tile: add the other pair's partial (this warp's layout)
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const int q = 2 * c + hh;
-      uint4 wq[2];
-      wq[0] = valid ? *reinterpret_cast<const uint4*>(wrow + (((2 * q) ^ (lane & 7)) << 4))
-                    : make_uint4(0, 0, 0, 0);
-      wq[1] = valid ? *reinterpret_cast<const uint4*>(wrow + (((2 * q + 1) ^ (lane & 7)) << 4))
-                    : make_uint4(0, 0, 0, 0);
-      uint32_t r[16];
-      __syncwarp();
-      tmem_ld16(tcol + 16 * q, r);
-      tmem_ld_wait();
-      if (other) {   // a stream-K tile: add the other pair's partial (this warp's layout)
+      for (int i = 0; i < 32; ++i)
+        r[i] = __float_as_uint(__uint_as_float(r[i]) + __ldcg(other + (32 * c + i) * 32 + lane));
+    }
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          r[i] = __float_as_uint(__uint_as_float(r[i]) + __ldcg(other + (16 * q + i) * 32 + lane));
+    for (int v = 0; v < 4; ++v) {
+      const int q = 4 * c + v;                       // 8-column chunk of the warp's 64
+      const uint4 wq = valid ? *reinterpret_cast<const uint4*>(wrow + ((q ^ (lane & 7)) << 4))
+                             : make_uint4(0, 0, 0, 0);
+      float w[8], sv[8], wt[8], rq[8];
+      unpack8<F16>(wq, w);
+      if (p.s) load_f8(p.s, col0 + 8 * q, sv);
+      // round(W~ / h) as the forward takes it: the product with 1/h, branch-free, its
+      // distance to the nearest integer checked; one warp-wide vote sends the rare lane
+      // with a product near a half-integer (or a large quotient) to the exact quotient
+      bool slow = false;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        wt[i] = p.s ? __fmul_rn(w[i], sv[i]) : w[i];
+        const float ua = __fmul_rn(wt[i], hinv);
+        rq[i] = rne_small(ua);
+        slow |= !(fabsf(ua) < 2048.f) || !(fabsf(__fsub_rn(ua, rq[i])) <= 0.499f);
+      }
+      if (__any_sync(0xffffffffu, slow)) {
+        if (slow) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) rq[i] = round_quotient(wt[i], h, hinv);
+        }
       }
 #pragma unroll
-      for (int v = 0; v < 2; ++v) {
-        float w[8], sv[8];
-        unpack8<F16>(wq[v], w);
-        if (p.s) load_f8(p.s, col0 + 16 * q + 8 * v, sv);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float wt = p.s ? __fmul_rn(w[i], sv[i]) : w[i];
-          const float dq = epi.out_scale * __uint_as_float(r[8 * v + i]);
-          const float rq = round_quotient(wt, h, hinv);
-          const float lvl = __fadd_rn(rq, z);
-          const bool inr = lvl >= 0.f && lvl <= p.Q;
-          const float cl = fminf(fmaxf(lvl, 0.f), p.Q);
-          Gh += dq * (inr ? (rq - wt * hinv) : (cl - z));
-          Gc += inr ? 0.f : dq;
-          ps[16 * hh + 8 * v + i] = inr ? dq * w[i] : 0.f;
-        }
+      for (int i = 0; i < 8; ++i) {
+        const float dq = epi.out_scale * __uint_as_float(r[8 * v + i]);
+        const float lvl = __fadd_rn(rq[i], z);
+        const bool inr = lvl >= 0.f && lvl <= p.Q;
+        const float cl = fminf(fmaxf(lvl, 0.f), p.Q);
+        Gh += dq * (inr ? (rq[i] - wt[i] * hinv) : (cl - z));
+        Gc += inr ? 0.f : dq;
+        ps[8 * v + i] = inr ? dq * w[i] : 0.f;
       }
     }
     if (valid) {
@@ -489,6 +496,23 @@ __device__ __forceinline__ void ste_w_epilogue(const GemmEpilogue& epi, uint32_t
     if (let) {
       const float cs = warp_column_sum32(ps, lane);
       if (wrow0 < rows) p.part_s[(wrow0 >> 5) * cols + k0 + lane] = cs;
+    }
+  }
+}
+
+// h and z of the groups of a warp's two 32-column chunks of the STE epilogue (row per lane),
+// loaded ahead of the accumulator.
+__device__ __forceinline__ void ste_w_prefetch(const SteWEpi& p, int64_t row, bool valid,
+                                               int64_t col0, int64_t cols, float (&hz)[4]) {
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    const int64_t k0 = col0 + 32 * c;
+    hz[2 * c] = 1.f;
+    hz[2 * c + 1] = 0.f;
+    if (valid && k0 < cols) {
+      const int64_t gi = row * p.ng + static_cast<int>(k0) / static_cast<int>(p.G);
+      hz[2 * c] = p.h[gi];
+      hz[2 * c + 1] = static_cast<float>(p.z[gi]);
     }
   }
 }
@@ -700,6 +724,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV>::NUM_THREADS
         }
         cp_commit();
       }
+      float hz[4] = {1.f, 0.f, 1.f, 0.f};
+      if constexpr (EV != 0) ste_w_prefetch(epi.ste, row, row < rows, col0, cols, hz);
       // one lane polls; the decision is broadcast so the warp-wide tcgen05.ld stays uniform
       int go = 0;
       if (lane == 0)
@@ -763,7 +789,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV>::NUM_THREADS
       }
       if constexpr (EV != 0) {
         ste_w_epilogue<EV == 2>(epi, tbase, wrow0, col0, rows, cols, lane,
-                                smem + L::WST_OFF + ew * C::WST, other);
+                                smem + L::WST_OFF + ew * C::WST, other, hz);
       } else {
         float* const out_b = BATCH ? epi.out + static_cast<int64_t>(tw.b) * sc.out_bstride : epi.out;
         for (int ch = 0; ch < EPI_COLS / 32; ++ch) {

@@ -50,9 +50,11 @@ def test_stream_k_forward_matches_fp64_product(omq, cuda_device, M, N, K):
     # float32 accumulation of K exact products: relative error about sqrt(K) 2^-24 (a
     # missing or misplaced partial would be of order one)
     assert frob_rel(a["Y"].cpu().numpy(), ref.numpy()) <= 3 * np.sqrt(K) * 2.0 ** -24
-    res = (ref - Yref.double()).numpy()
-    assert frob_rel(a["dY"].float().cpu().numpy(), res) <= 2e-3       # float16 residual
+    # the epilogue on the GPU's own Y: the residual rounded once to float16, the loss from
+    # float32 squares summed in a fixed order
+    res = a["Y"].double().cpu().numpy() - Yref.double().numpy()
+    assert frob_rel(a["dY"].float().cpu().numpy(), res) <= 2.0 ** -11
     loss = float((res ** 2).mean())
-    assert abs(a["loss"].item() - loss) <= 1e-3 * loss
+    assert abs(a["loss"].item() - loss) <= 1e-5 * loss
     for key in ("Y", "dY", "loss"):
         assert torch.equal(a[key], b[key]), key
