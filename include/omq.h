@@ -272,13 +272,31 @@ omq_status omq_fold_pack(const void* W, omq_dtype wdt, int64_t N, int64_t K, int
  * learned transforms fold into the weights; the quantized model runs as an ordinary low-bit
  * model):  y[m, n] = sum_k x[m, k] (c[n, k] - z[n, k/group]) h[n, k/group]
  * x [M, K] in xdt (the linear's input after its folded LET, i.e. (X - delta)/s), packed /
- * h / z as written by omq_fold_pack, y [M, N] float32 (add B~ for the bias). bits in {2, 4, 8},
- * 1 <= M <= 8, group a multiple of 128/bits, K a multiple of group, M (K + K bits/128) floats
- * of shared memory at most 200 KiB. Decode-shaped: memory-bound on the codes.
+ * h / z as written by omq_fold_pack, y [M, N] float32 (add B~ for the bias). 1 <= M <= 8.
+ * bits in {2, 4, 8}: CUDA-core kernel, group a multiple of 128/bits, K a multiple of group,
+ * M (K + K bits/128) floats of shared memory at most 200 KiB; decode-shaped, memory-bound on
+ * the codes. bits 3, 5, 6, 7 (codes straddling bytes): the omq_qgemm path below (16-bit x
+ * only, its shape rules; OMQ_ERR_UNSUPPORTED for float32 x).
  * ------------------------------------------------------------------------------------ */
 omq_status omq_qgemv(const void* x, omq_dtype xdt, int64_t M, int64_t K, const uint8_t* packed,
                      const float* h, const int32_t* z, int64_t N, int64_t group, int bits,
                      float* y, omq_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
+ * omq_qgemm — the same product for any number of tokens (prefill) on the tcgen05 tensor
+ * cores ([ICLR] section 框架: the quantized model runs as an ordinary low-bit model):
+ *   y[m, n] = sum_k x[m, k] (c[n, k] - z[n, k/group]) h[n, k/group]  (+ bias[n])
+ * The packed codes, h and z are read directly: converter warps expand each 64-column block
+ * of codes into the 16-bit operand tile in shared memory ((c - z) h rounded once to xdt)
+ * while the tensor cores consume the previous ones; no dequantized weight is stored.
+ * x [M, K] F16 or BF16 (row-major, 16-byte aligned); packed [N, K bits/8] as written by
+ * omq_fold_pack (16-byte aligned); h [N, K/group] float32, z [N, K/group] int32; bias [N]
+ * float32 or NULL; y [M, N] float32. bits 2..8; K a multiple of 64; group a multiple of 8
+ * dividing K; N a multiple of 8; M >= 1. float32 accumulation.
+ * ------------------------------------------------------------------------------------ */
+omq_status omq_qgemm(const void* x, omq_dtype xdt, int64_t M, int64_t K, const uint8_t* packed,
+                     const float* h, const int32_t* z, int64_t N, int64_t group, int bits,
+                     const float* bias, float* y, omq_stream_t stream);
 
 /* ------------------------------------------------------------------------------------
  * omq_calib_step — one whole calibration step on one stream: omq_let_apply (when LET is

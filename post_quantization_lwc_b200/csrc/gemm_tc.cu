@@ -69,11 +69,18 @@ constexpr int UMMA_K = 16;
 // heaviest per-element arithmetic, with 16 epilogue warps of 64 columns (four per scheduler,
 // 96 registers a thread) and producer / MMA waits that sleep between probes, leaving issue
 // slots to the epilogue. One kernel per variant keeps each within its register budget.
-template <int EV>
+//
+// DQB (2..8): the B operand is a weight given as packed DQB-bit codes with per-group step h
+// and zero point z (omq_fold_pack's layout); four converter warps per CTA expand each
+// k-block of codes into the 16-bit values (c - z) h, written straight into the stage in the
+// layout the TMA would have produced, and only A is copied by TMA.
+template <int EV, int DQB = 0>
 struct Cfg {
   static constexpr int EPI_WARPS = EV ? 16 : 8;
   static constexpr int EPI_COLS = TILE_N * 4 / EPI_WARPS;   // accumulator columns per warp
-  static constexpr int NUM_THREADS = 32 * (2 + EPI_WARPS);
+  static constexpr int CONV_WARPS = DQB ? 8 : 0;     // two groups of four (alternate k-blocks)
+  static constexpr int CONV_ARRIVALS = DQB ? 2 * 4 : 0;   // a stage's: one group, both CTAs
+  static constexpr int NUM_THREADS = 32 * (2 + EPI_WARPS + CONV_WARPS);
   // the STE variants give two stages of the ring to a 4 KB shared slice per epilogue warp
   // (its 32 x 64 block of W, staged by coalesced copies)
   static constexpr int STAGES = EV ? 5 : 7;
@@ -517,6 +524,215 @@ __device__ __forceinline__ void ste_w_prefetch(const SteWEpi& p, int64_t row, bo
   }
 }
 
+// ---- dequantizing B producer ---------------------------------------------------------
+// The 64 DQB-bit codes of one row's k-block: 8 * DQB bytes, a little-endian bit string
+// (code j at bits j DQB .. j DQB + DQB - 1), loaded as DQB 8-byte words.
+template <int DQB>
+__device__ __forceinline__ uint32_t code_at(const uint32_t (&w)[2 * DQB + 1], int j) {
+  const int bit = j * DQB, word = bit >> 5, sh = bit & 31;
+  uint32_t v = w[word] >> sh;
+  if (sh + DQB > 32) v |= w[word + 1] << (32 - sh);
+  return v & ((1u << DQB) - 1u);
+}
+// 2^23 + code as a float, the code's byte placed in the low mantissa byte by one permute.
+__device__ __forceinline__ float magic_byte(uint32_t bytes, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(bytes), "r"(0x4B000000u), "r"(sel));
+  return __uint_as_float(r);
+}
+// The 8 codes of chunk j (columns 8 j .. 8 j + 7 of the k-block) as floats 2^23 + c, exact.
+// Byte-aligned widths take one permute a code (after a mask for 2 and 4 bits); the others
+// the generic bit-string read.
+template <int DQB>
+__device__ __forceinline__ void codes8(const uint32_t (&w)[2 * DQB + 1], int j, float (&f)[8]) {
+  if constexpr (DQB == 8) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) f[i] = magic_byte(w[2 * j + i / 4], 0x7440u + (i & 3));
+  } else if constexpr (DQB == 4) {
+    const uint32_t x = w[j];                       // codes 8 j .. 8 j + 7, two a byte
+    const uint32_t lo = x & 0x0F0F0F0Fu, hi = (x >> 4) & 0x0F0F0F0Fu;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      f[2 * i] = magic_byte(lo, 0x7440u + i);
+      f[2 * i + 1] = magic_byte(hi, 0x7440u + i);
+    }
+  } else if constexpr (DQB == 2) {
+    const uint32_t x = (w[j / 2] >> (16 * (j & 1))) & 0xFFFFu;   // 8 codes, four a byte
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t m = (x >> (2 * i)) & 0x0303u;    // codes i and i + 4 in bytes 0 and 1
+      f[i] = magic_byte(m, 0x7440u);
+      f[i + 4] = magic_byte(m, 0x7441u);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) f[i] = __uint_as_float(0x4B000000u | code_at<DQB>(w, 8 * j + i));
+  }
+}
+
+__device__ __forceinline__ uint32_t pack_pair(float a, float b, bool f16) {
+  if (f16) {
+    const __half2 x = __floats2half2_rn(a, b);
+    return *reinterpret_cast<const uint32_t*>(&x);
+  }
+  const __nv_bfloat162 x = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&x);
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Walks a pair's k-blocks in the order the producer and the MMA take them (unit by unit).
+template <bool BATCH>
+struct KbCursor {
+  Unit un;
+  int u = 0, kb = 0;
+  bool ok = false;
+  __device__ __forceinline__ void start(const TileSched& sc, int pair, int pairs, int nk) {
+    u = 0;
+    ok = next_unit<BATCH>(sc, pair, pairs, 0, nk, un);
+    kb = ok ? un.w.kb0 : 0;
+  }
+  __device__ __forceinline__ void step(const TileSched& sc, int pair, int pairs, int nk) {
+    if (!ok) return;
+    if (++kb >= un.w.kb1) {
+      ++u;
+      ok = next_unit<BATCH>(sc, pair, pairs, u, nk, un);
+      kb = ok ? un.w.kb0 : 0;
+    }
+  }
+};
+
+// One thread's inputs of a k-block: the row's 64 codes and the step / zero point of the group
+// holding its first column.
+template <int DQB>
+struct KbCodes {
+  uint32_t w[2 * DQB + 1];
+  float h, z;
+  int64_t n;
+  bool valid;
+};
+template <int DQB>
+__device__ __forceinline__ void load_kb(const QuantB& q, int64_t n, bool valid, int kb,
+                                        KbCodes<DQB>& c) {
+  c.n = n;
+  c.valid = valid;
+  c.w[2 * DQB] = 0u;
+  c.h = 0.f;
+  c.z = 0.f;
+  if (valid) {
+    const uint2* src = reinterpret_cast<const uint2*>(q.packed + n * q.row_bytes +
+                                                      static_cast<int64_t>(kb) * 8 * DQB);
+#pragma unroll
+    for (int i = 0; i < DQB; ++i) {
+      const uint2 v = __ldg(src + i);
+      c.w[2 * i] = v.x;
+      c.w[2 * i + 1] = v.y;
+    }
+    // the group of the k-block's first column (32-bit divisions by a group count)
+    const uint32_t g = q.kb_per_group ? static_cast<uint32_t>(kb) / static_cast<uint32_t>(q.kb_per_group)
+                                      : static_cast<uint32_t>(kb) * 8u /
+                                            static_cast<uint32_t>(q.chunks_per_group);
+    c.h = __ldg(q.h + n * q.ng + g);
+    c.z = static_cast<float>(__ldg(q.z + n * q.ng + g));
+  } else {
+#pragma unroll
+    for (int i = 0; i < 2 * DQB; ++i) c.w[i] = 0u;
+  }
+}
+
+// The converter warps: two groups of four, taking alternate k-blocks, so each group has two
+// stages' time for one; each thread prefetches its next k-block's codes before it waits for
+// and fills the current stage. A code c becomes float by its bits in the low mantissa of
+// 2^23 (exact), so (c - z) h = (float(2^23 + c) - (2^23 + z)) h, two full-rate operations.
+template <int DQB, bool BATCH, int STAGES>
+__device__ __forceinline__ void convert_b(const GemmEpilogue& epi, const TileSched& sc, int pair,
+                                          int pairs, int nk, uint32_t rank, int64_t cols,
+                                          uint32_t fmt, uint32_t sbase, int stage_bytes,
+                                          int a_bytes, uint32_t bar_full, uint32_t bar_empty,
+                                          volatile int* abort_flag, int cthread) {
+  const int ct = cthread & 127, grp = cthread >> 7, lane = cthread & 31;
+  const bool f16 = fmt == 0;
+  const QuantB& q = epi.qb;
+  KbCursor<BATCH> cur, nxt;
+  cur.start(sc, pair, pairs, nk);
+  int it = 0;
+  if (grp) {
+    cur.step(sc, pair, pairs, nk);
+    it = 1;
+  }
+  nxt = cur;
+  nxt.step(sc, pair, pairs, nk);
+  nxt.step(sc, pair, pairs, nk);
+  auto row_of = [&](const KbCursor<BATCH>& c, bool& valid) {
+    const int64_t n = static_cast<int64_t>(c.un.w.col0) + rank * HALF + ct;
+    valid = n < cols;
+    return n;
+  };
+  KbCodes<DQB> a, b;
+  if (cur.ok) {
+    bool v;
+    const int64_t n = row_of(cur, v);
+    load_kb<DQB>(q, n, v, cur.kb, a);
+  }
+  while (cur.ok) {
+    if (nxt.ok) {                                   // the next k-block of this group, early
+      bool v;
+      const int64_t n = row_of(nxt, v);
+      load_kb<DQB>(q, n, v, nxt.kb, b);
+    }
+    const int s = it % STAGES;
+    const uint32_t ph = (it / STAGES) & 1;
+    int ok = 1;
+    if (lane == 0)
+      ok = (mbar_wait(bar_empty + 8 * s, ph ^ 1, DEV_ERR_TMA_WAIT) && *abort_flag == 0) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (!ok) {
+      *abort_flag = 1;
+      return;
+    }
+    const uint32_t b_row = sbase + s * stage_bytes + a_bytes + ct * 128;
+    // groups narrower than a k-block (a group is a multiple of 8 columns): each 8-column
+    // chunk finds its own; otherwise the whole k-block is the group of load_kb
+    const bool split_groups = q.kb_per_group == 0;
+    const uint32_t ch0 = static_cast<uint32_t>(cur.kb) * 8u;
+    const uint32_t g0 = split_groups ? ch0 / static_cast<uint32_t>(q.chunks_per_group) : 0u;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      float hh = a.h, zz = a.z;
+      if (split_groups) {
+        const uint32_t g = (ch0 + j) / static_cast<uint32_t>(q.chunks_per_group);
+        if (g != g0 && a.valid) {
+          hh = __ldg(q.h + a.n * q.ng + g);
+          zz = static_cast<float>(__ldg(q.z + a.n * q.ng + g));
+        }
+      }
+      const float bz = 8388608.f + zz;              // exact: |z| < 2^22 for these codes
+      float f[8];
+      codes8<DQB>(a.w, j, f);
+      uint32_t o[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        // (c - z) exact, one rounding of the product: the pair on the f32x2 pipe
+        const float2 d = __fadd2_rn(make_float2(f[2 * e], f[2 * e + 1]), make_float2(-bz, -bz));
+        const float2 v = __fmul2_rn(d, make_float2(hh, hh));
+        o[e] = pack_pair(v.x, v.y, f16);
+      }
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(b_row + ((j ^ (ct & 7)) << 4)),
+                   "r"(o[0]), "r"(o[1]), "r"(o[2]), "r"(o[3])
+                   : "memory");
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive_cluster(peer_addr(bar_full + 8 * s, 0));
+    cur = nxt;
+    a = b;
+    it += 2;
+    nxt.step(sc, pair, pairs, nk);
+    nxt.step(sc, pair, pairs, nk);
+  }
+}
+
 template <int STAGES, int EPI_WARPS, int WST>
 struct Layout {
   static constexpr int A_BYTES = HALF * BK * 2;          // 16 KB
@@ -540,12 +756,12 @@ struct Layout {
 };
 
 // BATCH: a batched and / or causal schedule (attention); false compiles the plain tile loop.
-template <int EV, bool BATCH>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV>::NUM_THREADS, 1)
+template <int EV, bool BATCH, int DQB = 0>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV, DQB>::NUM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    int a_mn, int b_mn, uint32_t fmt, int64_t rows, int64_t cols, int64_t depth,
                    GemmEpilogue epi, TileSched sc) {
-  using C = Cfg<EV>;
+  using C = Cfg<EV, DQB>;
   constexpr int STAGES = C::STAGES, EPI_WARPS = C::EPI_WARPS, EPI_COLS = C::EPI_COLS;
   using L = Layout<STAGES, EPI_WARPS, C::WST>;
   extern __shared__ uint8_t smem_raw[];
@@ -575,7 +791,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV>::NUM_THREADS
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(bar_full + 8 * s, 1);     // leader's: one expect_tx arrival + both CTAs' bytes
+      // leader's: one expect_tx arrival + both CTAs' bytes (+ both CTAs' converter warps)
+      mbar_init(bar_full + 8 * s, 1 + C::CONV_ARRIVALS);
       mbar_init(bar_empty + 8 * s, 1);    // the leader's commit, multicast to both CTAs
     }
     for (int b = 0; b < 2; ++b) {
@@ -625,7 +842,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV>::NUM_THREADS
         const uint32_t a_dst = sbase + s * L::STAGE_BYTES;
         const uint32_t b_dst = a_dst + L::A_BYTES;
         const uint32_t full_leader = peer_addr(bar_full + 8 * s, 0);
-        if (rank == 0) mbar_expect_tx(bar_full + 8 * s, 2 * L::STAGE_BYTES);
+        if (rank == 0) mbar_expect_tx(bar_full + 8 * s, 2 * (DQB ? L::A_BYTES : L::STAGE_BYTES));
         const int k0 = kb * BK;
         if (a_mn) {
           for (int c = 0; c < HALF / 64; ++c)
@@ -633,7 +850,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV>::NUM_THREADS
         } else {
           tma_load_op<BATCH>(a_dst, &tmA, full_leader, k0, row0, sc.a_bmode, tw.b);
         }
-        if (b_mn) {
+        if (DQB) {
+          // B is written by the converter warps
+        } else if (b_mn) {
           for (int c = 0; c < HALF / 64; ++c)
             tma_load_op<BATCH>(b_dst + c * 8192, &tmB, full_leader, col0 + 64 * c, k0, sc.b_bmode, tw.b);
         } else {
@@ -691,6 +910,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV>::NUM_THREADS
     // every MMA issued above has completed once this commit arrives
     umma_commit_local(bar_drain);
     mbar_wait(bar_drain, 0, DEV_ERR_MMA_WAIT);
+  } else if (DQB != 0 && warp >= 2 + EPI_WARPS) {
+    // ---------------- converter warps (both CTAs): this CTA's 128 rows of B (output
+    // columns col0 + 128 rank + ct), one row a thread, each k-block's codes expanded into the
+    // stage's B half: row ct at ct * 128 bytes, its 8-value chunk j at (j ^ (ct & 7)) * 16
+    // (the 128-byte swizzle of the TMA copies), then a fence to the async proxy and one
+    // arrival per warp on the leader's full barrier
+    if constexpr (DQB != 0) convert_b<DQB, BATCH, STAGES>(epi, sc, pair, pairs, nk, rank, cols,
+                                                          fmt, sbase, L::STAGE_BYTES, L::A_BYTES,
+                                                          bar_full, bar_empty, abort_flag,
+                                                          threadIdx.x - 32 * (2 + EPI_WARPS));
   } else if (warp >= 2) {
     // ---------------- epilogue (both CTAs: this CTA's 128 rows of the tile)
     const int ew = warp - 2;                         // 0 .. EPI_WARPS-1
@@ -944,6 +1173,7 @@ bool make_map(CUtensorMap* map, omq_dtype dt, const GemmOperand& op, int64_t n_r
 
 static_assert(Layout<Cfg<0>::STAGES, Cfg<0>::EPI_WARPS, Cfg<0>::WST>::SMEM_BYTES <= 232448, "smem");
 static_assert(Layout<Cfg<1>::STAGES, Cfg<1>::EPI_WARPS, Cfg<1>::WST>::SMEM_BYTES <= 232448, "smem");
+static_assert(Cfg<0, 4>::NUM_THREADS == 576, "converter warps");
 
 using GemmKernel = void (*)(CUtensorMap, CUtensorMap, int, int, uint32_t, int64_t, int64_t,
                             int64_t, GemmEpilogue, TileSched);
@@ -953,23 +1183,24 @@ struct KernelChoice {
   int threads, smem;
 };
 
-template <int EV, bool BATCH = false>
+template <int EV, bool BATCH = false, int DQB = 0>
 KernelChoice choice() {
-  return {gemm_tc_kernel<EV, BATCH>, Cfg<EV>::NUM_THREADS,
-          Layout<Cfg<EV>::STAGES, Cfg<EV>::EPI_WARPS, Cfg<EV>::WST>::SMEM_BYTES};
+  using C = Cfg<EV, DQB>;
+  return {gemm_tc_kernel<EV, BATCH, DQB>, C::NUM_THREADS,
+          Layout<C::STAGES, C::EPI_WARPS, C::WST>::SMEM_BYTES};
 }
 
 // Opt each kernel variant into the large dynamic shared memory once.
 cudaError_t kernel_attr(GemmKernel k, int smem) {
   static std::mutex mu;
-  static GemmKernel done[8] = {};
+  static GemmKernel done[16] = {};
   static int n_done = 0;
   std::lock_guard<std::mutex> lock(mu);
   for (int i = 0; i < n_done; ++i)
     if (done[i] == k) return cudaSuccess;
   const cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(k),
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e == cudaSuccess && n_done < 8) done[n_done++] = k;
+  if (e == cudaSuccess && n_done < 16) done[n_done++] = k;
   return e;
 }
 
@@ -1078,6 +1309,51 @@ omq_status gemm_tc(omq_dtype dt, const GemmOperand& A, const GemmOperand& B, int
   launch_k(kc.fn, static_cast<unsigned>(2 * pairs), kc.threads, kc.smem, stream,
       ma, mb, A.mn_major ? 1 : 0, B.mn_major ? 1 : 0, dt == OMQ_F16 ? 0u : 1u, rows, cols, depth,
       epi, sc);
+  return launch_status();
+}
+
+omq_status gemm_tc_qb(omq_dtype dt, const GemmOperand& A, int64_t rows, int64_t cols,
+                      int64_t depth, int bits, const GemmEpilogue& epi, cudaStream_t stream) {
+  using namespace tc;
+  if (dt != OMQ_BF16 && dt != OMQ_F16) return OMQ_ERR_DTYPE;
+  if (A.mn_major || epi.kind != Epi::StoreF32 || depth % BK) return OMQ_ERR_UNSUPPORTED;
+  if (bits < 2 || bits > 8) return OMQ_ERR_BITS;
+  CUtensorMap ma;
+  int amode = 0;
+  if (!make_map(&ma, dt, A, rows, depth, 1, 0, &amode)) {
+    set_cuda_error(cudaErrorInvalidValue);
+    return OMQ_ERR_CUDA;
+  }
+  const int64_t tiles_m = ceil_div(rows, TILE_M), tiles_n = ceil_div(cols, TILE_N);
+  const int64_t tiles = tiles_m * tiles_n;
+  if (tiles > (int64_t(1) << 30)) return OMQ_ERR_SHAPE;
+  KernelChoice kc{};
+  switch (bits) {
+    case 2: kc = choice<0, false, 2>(); break;
+    case 3: kc = choice<0, false, 3>(); break;
+    case 4: kc = choice<0, false, 4>(); break;
+    case 5: kc = choice<0, false, 5>(); break;
+    case 6: kc = choice<0, false, 6>(); break;
+    case 7: kc = choice<0, false, 7>(); break;
+    default: kc = choice<0, false, 8>(); break;
+  }
+  const cudaError_t attr_err = kernel_attr(kc.fn, kc.smem);
+  if (attr_err != cudaSuccess) {
+    set_cuda_error(attr_err);
+    return OMQ_ERR_CUDA;
+  }
+  TileSched sc{static_cast<int>(tiles_m), static_cast<int>(tiles_n), static_cast<int>(tiles),
+               static_cast<int>(tiles), 0, amode, 0, 0};
+  sc.dp_tiles = static_cast<int>(tiles);
+  sc.sk_tiles = 0;
+  sc.sk_len = 0;
+  sc.sk_part = nullptr;
+  sc.sk_cnt = nullptr;
+  const int64_t max_pairs = num_sms() / 2;
+  const int64_t pairs = tiles < max_pairs ? tiles : max_pairs;
+  // the B tensor map is not read (B comes from the converter warps): A's map stands in
+  launch_k(kc.fn, static_cast<unsigned>(2 * pairs), kc.threads, kc.smem, stream,
+      ma, ma, 0, 0, dt == OMQ_F16 ? 0u : 1u, rows, cols, depth, epi, sc);
   return launch_status();
 }
 

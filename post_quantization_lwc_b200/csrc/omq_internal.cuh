@@ -233,6 +233,18 @@ struct SteWEpi {
   float* part_s;           // [ceil(N/32), K] or NULL: per 32-row block, sum (in range) dW~ W
 };
 
+// A B operand given as packed integer codes (omq_fold_pack's layout: row n of the weight is
+// a little-endian bit string of `bits`-bit codes) with per-group step h and zero point z:
+// B(n, k) = (code[n, k] - z[n, k / group]) h[n, k / group], expanded in the GEMM.
+struct QuantB {
+  const uint8_t* packed;   // [N, row_bytes]
+  const float* h;          // [N, ng]
+  const int32_t* z;        // [N, ng]
+  int64_t row_bytes, ng, group, depth;
+  int32_t kb_per_group;       // group / 64 when a group is whole 64-column k-blocks, else 0
+  int32_t chunks_per_group;   // group / 8
+};
+
 struct GemmEpilogue {
   Epi kind;
   float* out;              // StoreF32: [rows, cols] fp32 (ld = cols); MseLoss: Y or NULL
@@ -248,6 +260,7 @@ struct GemmEpilogue {
   // partial accumulators of split tiles and their arrival counters.
   void* sk_scratch;
   size_t sk_bytes;
+  QuantB qb;               // gemm_tc_qb only
 };
 
 // Group lengths whose weight-side STE runs in the dW^ GEMM's epilogue: whole 32-column
@@ -291,6 +304,10 @@ int64_t gemm_tc_tiles(int64_t rows, int64_t cols);
 // Scratch that lets gemm_tc run the stream-K tail schedule on a rows x cols output (current
 // device); GemmEpilogue::sk_scratch of at least this size enables it.
 size_t gemm_tc_sk_bytes(int64_t rows, int64_t cols);
+// C = A B^T with B expanded from packed codes in the GEMM (epi.qb; bits 2..8; epi.kind
+// StoreF32): A [rows, depth] 16-bit K-major, depth a multiple of 64, B rows = cols.
+omq_status gemm_tc_qb(omq_dtype dt, const GemmOperand& A, int64_t rows, int64_t cols,
+                      int64_t depth, int bits, const GemmEpilogue& epi, cudaStream_t stream);
 // f32 operands on CUDA cores.
 omq_status gemm_f32_simt(const GemmOperand& A, const GemmOperand& B, int64_t rows, int64_t cols,
                          int64_t depth, const GemmEpilogue& epi, int64_t* n_tiles,

@@ -142,13 +142,56 @@ __global__ void __launch_bounds__(256) qgemv_kernel(const void* x, omq_dtype xdt
 
 using namespace omq;
 
+// Tensor-core product with the folded weights (prefill, or any token count): the weight's
+// packed codes are expanded into the GEMM's B operand tiles in shared memory as they are
+// consumed (gemm_tc_qb), so the codes, h and z are the only weight bytes read.
+static omq_status qgemm_impl(const void* x, omq_dtype xdt, int64_t M, int64_t K,
+                             const uint8_t* packed, const float* h, const int32_t* z, int64_t N,
+                             int64_t group, int bits, const float* bias, float* y,
+                             cudaStream_t st) {
+  if (!x || !packed || !h || !z || !y) return OMQ_ERR_NULL;
+  if (xdt != OMQ_BF16 && xdt != OMQ_F16) return OMQ_ERR_DTYPE;
+  if (bits < 2 || bits > 8) return OMQ_ERR_BITS;
+  const int64_t kMax = (int64_t(1) << 31) - 1;
+  if (M < 1 || K < 64 || K % 64 || N < 8 || N % 8 || group < 8 || group % 8 || K % group ||
+      M > kMax || N > kMax || K > kMax)
+    return OMQ_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(packed) || !aligned16(y) || (bias && !aligned16(bias)))
+    return OMQ_ERR_ALIGN;
+  GemmEpilogue epi{};
+  epi.kind = Epi::StoreF32;
+  epi.out = y;
+  epi.out_scale = 1.f;
+  epi.bias = bias;
+  if (K / group > (int64_t(1) << 31) - 1 || (K / 8) > (int64_t(1) << 31) - 1) return OMQ_ERR_SHAPE;
+  epi.qb = QuantB{packed, h, z, K * bits / 8, K / group, group, K,
+                  static_cast<int32_t>(group % 64 == 0 ? group / 64 : 0),
+                  static_cast<int32_t>(group / 8)};
+  return gemm_tc_qb(xdt, GemmOperand{x, K, false}, M, N, K, bits, epi, st);
+}
+
+extern "C" omq_status omq_qgemm(const void* x, omq_dtype xdt, int64_t M, int64_t K,
+                                const uint8_t* packed, const float* h, const int32_t* z,
+                                int64_t N, int64_t group, int bits, const float* bias, float* y,
+                                omq_stream_t stream) {
+  return qgemm_impl(x, xdt, M, K, packed, h, z, N, group, bits, bias, y,
+                    reinterpret_cast<cudaStream_t>(stream));
+}
+
 extern "C" omq_status omq_qgemv(const void* x, omq_dtype xdt, int64_t M, int64_t K,
                                 const uint8_t* packed, const float* h, const int32_t* z,
                                 int64_t N, int64_t group, int bits, float* y,
                                 omq_stream_t stream) {
   if (!x || !packed || !h || !z || !y) return OMQ_ERR_NULL;
   if (xdt != OMQ_F32 && xdt != OMQ_BF16 && xdt != OMQ_F16) return OMQ_ERR_DTYPE;
-  if (bits != 2 && bits != 4 && bits != 8) return OMQ_ERR_UNSUPPORTED;
+  if (bits < 2 || bits > 8) return OMQ_ERR_BITS;
+  if (bits != 2 && bits != 4 && bits != 8) {
+    // codes that straddle bytes: the tensor-core path (16-bit activations)
+    if (xdt == OMQ_F32) return OMQ_ERR_UNSUPPORTED;
+    if (M < 1 || M > kGemvMaxTokens) return OMQ_ERR_SHAPE;
+    return qgemm_impl(x, xdt, M, K, packed, h, z, N, group, bits, nullptr, y,
+                      reinterpret_cast<cudaStream_t>(stream));
+  }
   const int64_t cpc = 128 / bits;
   if (M < 1 || M > kGemvMaxTokens || N < 1 || K < cpc || K % cpc || group < cpc ||
       group % cpc || K % group || N > (int64_t(1) << 31))

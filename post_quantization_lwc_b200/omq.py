@@ -33,7 +33,7 @@ EXPORTS = ("omq_status_str", "omq_last_cuda_error", "omq_version", "omq_sync_che
            "omq_fq_linear_fwd_noalloc", "omq_block_theta_range", "omq_block_buffer",
            "omq_block_workspace_bytes", "omq_block_step", "omq_block_reference",
            "omq_block_quant_forward", "omq_block_calibrate", "omq_qgemv",
-           "omq_set_wait_limit_ns", "omq_wait_limit_ns", "omq_wait_probe")
+           "omq_set_wait_limit_ns", "omq_wait_limit_ns", "omq_wait_probe", "omq_qgemm")
 
 _p = ctypes.c_void_p
 _i64 = ctypes.c_int64
@@ -139,6 +139,7 @@ _sig("omq_qgemv", _i32, [_p, _i32, _i64, _i64, _p, _p, _p, _i64, _i64, _i32, _p,
 _sig("omq_set_wait_limit_ns", _i32, [ctypes.c_uint64])
 _sig("omq_wait_limit_ns", ctypes.c_uint64, [])
 _sig("omq_wait_probe", _i32, [_i32, _p])
+_sig("omq_qgemm", _i32, [_p, _i32, _i64, _i64, _p, _p, _p, _i64, _i64, _i32, _p, _p, _p])
 
 
 def _check(status: int, where: str):
@@ -358,6 +359,18 @@ def qgemv(x, packed, h, z, group, bits, stream=None):
     y = torch.empty(M, N, dtype=torch.float32, device=x.device)
     _check(_lib.omq_qgemv(_ptr(x), _dt(x), M, K, _ptr(packed), _ptr(h), _ptr(z), N, group, bits,
                           _ptr(y), _stream(stream)), "omq_qgemv")
+    return y
+
+
+def qgemm(x, packed, h, z, group, bits, bias=None, stream=None):
+    """omq_qgemm: y = x dequant(packed, h, z)^T (+ bias) on the tensor cores, any token count.
+    x [M, K] float16 / bfloat16; returns y [M, N] float32."""
+    _dev(x, packed, h, z, bias)
+    M, K = x.shape
+    N = packed.shape[0]
+    y = torch.empty(M, N, dtype=torch.float32, device=x.device)
+    _check(_lib.omq_qgemm(_ptr(x), _dt(x), M, K, _ptr(packed), _ptr(h), _ptr(z), N, group, bits,
+                          _ptr(bias), _ptr(y), _stream(stream)), "omq_qgemm")
     return y
 
 

@@ -165,3 +165,18 @@ def test_struct_layouts_match_header(omq, tmp_path):
         for fname, _ in py._fields_:
             assert got[(cname, fname)] == getattr(py, fname).offset, (cname, fname)
     assert got[("omq_range", "sizeof")] == 16     # the binding stores ranges as int32 [n, 4]
+
+
+def test_qgemm_validation(omq):
+    """omq_qgemm rejects bad arguments before any launch."""
+    lib = omq._lib
+    P = FAKE
+    # float32 activations, 1 bit, K not a multiple of 64, N not a multiple of 8, NULL codes
+    assert lib.omq_qgemm(P, 0, 16, 256, P, P, P, 64, 64, 4, None, P, None) == 3
+    assert lib.omq_qgemm(P, 2, 16, 256, P, P, P, 64, 64, 1, None, P, None) == 5
+    assert lib.omq_qgemm(P, 2, 16, 200, P, P, P, 64, 40, 4, None, P, None) == 2
+    assert lib.omq_qgemm(P, 2, 16, 256, P, P, P, 60, 64, 4, None, P, None) == 2
+    assert lib.omq_qgemm(P, 2, 16, 256, None, P, P, 64, 64, 4, None, P, None) == 1
+    assert lib.omq_qgemm(MISALIGNED, 2, 16, 256, P, P, P, 64, 64, 4, None, P, None) == 4
+    # 3-bit decode with float32 activations has no kernel
+    assert lib.omq_qgemv(P, 0, 1, 256, P, P, P, 64, 64, 3, P, None) == 8

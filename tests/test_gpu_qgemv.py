@@ -54,6 +54,7 @@ def test_qgemv_rejects_bad_shapes(omq):
     lib = omq._lib
     P = 256
     assert lib.omq_qgemv(P, 1, 9, 256, P, P, P, 16, 128, 4, P, None) == 2      # 9 tokens
-    assert lib.omq_qgemv(P, 1, 1, 256, P, P, P, 16, 128, 3, P, None) == 8      # 3 bits
+    assert lib.omq_qgemv(P, 0, 1, 256, P, P, P, 16, 128, 3, P, None) == 8      # 3 bits, f32 x
+    assert lib.omq_qgemv(P, 1, 1, 256, P, P, P, 16, 128, 9, P, None) == 5      # 9 bits
     assert lib.omq_qgemv(P, 1, 1, 256, P, P, P, 16, 16, 4, P, None) == 2       # group < 32
     assert lib.omq_qgemv(None, 1, 1, 256, P, P, P, 16, 128, 4, P, None) == 1
