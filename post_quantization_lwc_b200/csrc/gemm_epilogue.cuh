@@ -6,33 +6,36 @@
 //           reconstruction error against the full-precision output):
 //           Y = acc + bias[j]; optionally stored; R = Y - Y_ref written as the residual
 //           (the loss gradient is 2 R / (rows cols), applied by the backward);
-//           loss partial += R^2.
+//           loss partial += R^2; optionally the column sums of R over each 32-row block
+//           (the bias gradient's partials, res_colsum).
 #pragma once
 
 #include "omq_internal.cuh"
 
 namespace omq {
 
-// `out` is e.out, or the output of this tile's problem in a batch.
-__device__ __forceinline__ void epi_element(const GemmEpilogue& e, float* out, int64_t i,
-                                            int64_t j, int64_t cols, float acc, float& lsum) {
+// `out` is e.out, or the output of this tile's problem in a batch. Returns the residual
+// (MseLoss; 0 for StoreF32).
+__device__ __forceinline__ float epi_element(const GemmEpilogue& e, float* out, int64_t i,
+                                             int64_t j, int64_t cols, float acc, float& lsum) {
   const int64_t o = i * (e.ldo ? e.ldo : cols) + j;
   if (e.kind == Epi::StoreF32) {
     out[o] = e.out_scale * acc + (e.bias ? e.bias[j] : 0.f);
-    return;
+    return 0.f;
   }
   const float y = acc + (e.bias ? e.bias[j] : 0.f);
   if (out) out[o] = y;
   const float d = y - e.y_ref[o];
   lsum += d * d;
   store_elem(e.dy, o, d, e.dy_dt);
+  return d;
 }
 
 // 8 consecutive columns j0..j0+7 of row i, all in range, j0 % 8 == 0, cols % 8 == 0 and the
 // row stride a multiple of 8.
 __device__ __forceinline__ void epi_vec8(const GemmEpilogue& e, float* out, int64_t i,
                                          int64_t j0, int64_t cols, const float (&acc)[8],
-                                         float& lsum) {
+                                         float& lsum, float (&res)[8]) {
   const int64_t o = i * (e.ldo ? e.ldo : cols) + j0;
   const float sc = e.kind == Epi::StoreF32 ? e.out_scale : 1.f;
   float y[8];
@@ -48,18 +51,19 @@ __device__ __forceinline__ void epi_vec8(const GemmEpilogue& e, float* out, int6
   }
   if (e.kind == Epi::StoreF32) {
     store8(out, o, OMQ_F32, y);
+#pragma unroll
+    for (int t = 0; t < 8; ++t) res[t] = 0.f;
     return;
   }
   if (out) store8(out, o, OMQ_F32, y);
   float r[8];
   load8(e.y_ref, o, OMQ_F32, r);
-  float d[8];
 #pragma unroll
   for (int t = 0; t < 8; ++t) {
-    d[t] = y[t] - r[t];
-    lsum += d[t] * d[t];
+    res[t] = y[t] - r[t];
+    lsum += res[t] * res[t];
   }
-  store8(e.dy, o, e.dy_dt, d);
+  store8(e.dy, o, e.dy_dt, res);
 }
 
 }  // namespace omq

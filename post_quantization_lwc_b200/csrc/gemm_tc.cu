@@ -1032,21 +1032,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV, DQB>::NUM_TH
                                      __ldcg(other + (ch * 32 + q) * 32 + lane));
           }
           const int64_t cbase = col0 + ch * 32;
+          float rc[32];                      // this row's residuals of the chunk (or zeros)
+#pragma unroll
+          for (int q = 0; q < 32; ++q) rc[q] = 0.f;
           if (row < rows && cbase < cols) {
             if (cbase + 32 <= cols) {
 #pragma unroll
               for (int v = 0; v < 4; ++v) {
-                float acc[8];
+                float acc[8], res[8];
 #pragma unroll
                 for (int q = 0; q < 8; ++q) acc[q] = __uint_as_float(r[v * 8 + q]);
-                epi_vec8(epi, out_b, row, cbase + v * 8, cols, acc, lsum);
+                epi_vec8(epi, out_b, row, cbase + v * 8, cols, acc, lsum, res);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) rc[v * 8 + q] = res[q];
               }
             } else {
 #pragma unroll
               for (int q = 0; q < 32; ++q)
                 if (cbase + q < cols)
-                  epi_element(epi, out_b, row, cbase + q, cols, __uint_as_float(r[q]), lsum);
+                  rc[q] = epi_element(epi, out_b, row, cbase + q, cols, __uint_as_float(r[q]), lsum);
             }
+          }
+          if (epi.res_colsum && cbase < cols) {   // warp-uniform: the bias gradient's partials
+            const float cs = warp_column_sum32(rc, lane);
+            if (cbase + lane < cols) epi.res_colsum[(wrow0 >> 5) * cols + cbase + lane] = cs;
           }
         }
       }

@@ -122,10 +122,13 @@ __global__ void __launch_bounds__(256) act_quant_kernel(LetParams p) {
     const GroupQ q = group_params(1.f, 1.f, vmax, vmin, p.Qa);
     const float hinv = __frcp_rn(q.h);
     for (int c = threadIdx.x; c < chunks; c += blockDim.x) {
-      float o[8];
+      float v[8], rq[8], o[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = row[c * 8 + i];
+      round_quotient8(v, q.h, hinv, rq);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const float lvl = __fadd_rn(round_quotient(row[c * 8 + i], q.h, hinv), q.z);
+        const float lvl = __fadd_rn(rq[i], q.z);
         const float cc = fminf(fmaxf(lvl, 0.f), p.Qa);
         o[i] = __fmul_rn(__fsub_rn(cc, q.z), q.h);
       }

@@ -48,7 +48,9 @@ BwdLayout bwd_layout(int64_t M, int64_t N, int64_t K, int64_t group) {
   L.rb_x = ceil_div(M, kRowsX);
   size_t off = 0;
   auto take = [&](size_t bytes) { size_t o = off; off += align256(bytes); return o; };
-  L.dbt_part = take(sizeof(float) * L.rb_colsum * N);
+  // dB~ partials: per 64-row block (colsum kernel) or per 32-row block (the forward GEMM's
+  // residual column sums)
+  L.dbt_part = take(sizeof(float) * ceil_div(M, 32) * N);
   L.dbt = take(sizeof(float) * N);
   L.dwhat = take(sizeof(float) * N * K);
   L.dxq = take(sizeof(float) * M * K);
@@ -326,7 +328,8 @@ static omq_status run_gemm(omq_dtype dt, const GemmOperand& A, const GemmOperand
 static omq_status fwd_impl(const void* Xq, const void* W_hat, omq_dtype dt, int64_t M, int64_t N,
                            int64_t K, const float* B_tilde, const float* Y_ref, float* Y, void* dY,
                            float* loss, void* workspace, size_t ws_bytes, omq_stream_t stream,
-                           const Phases& ph, const SideStream* loss_stream = nullptr) {
+                           const Phases& ph, const SideStream* loss_stream = nullptr,
+                           float* res_colsum = nullptr) {
   if (!Xq || !W_hat) return OMQ_ERR_NULL;
   if (!dtype_ok(dt)) return OMQ_ERR_DTYPE;
   if (M < 1 || N < 8 || K < 8 || N % 8 || K % 8 || M > kMaxDim || N > kMaxDim || K > kMaxDim)
@@ -356,6 +359,7 @@ static omq_status fwd_impl(const void* Xq, const void* W_hat, omq_dtype dt, int6
     epi.dy = dY;
     epi.dy_dt = dt;
     epi.loss_partials = static_cast<float*>(workspace);
+    if (dt != OMQ_F32) epi.res_colsum = res_colsum;
   } else {
     epi.kind = Epi::StoreF32;
     epi.out = Y;
@@ -390,8 +394,10 @@ size_t omq_bwd_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t group) {
   return bwd_layout(M, N, K, group).total;
 }
 
+// dbias_rows > 0: the forward already left the column sums of the residual over blocks of
+// dbias_rows rows in the dB~ partials (its MSE epilogue), so no pass over dY is needed.
 static omq_status bwd_impl(const omq_bwd_args* a, void* workspace, size_t ws_bytes,
-                           omq_stream_t stream, const Phases& ph) {
+                           omq_stream_t stream, const Phases& ph, int dbias_rows = 0) {
   if (!a) return OMQ_ERR_NULL;
   const int64_t M = a->M, N = a->N, K = a->K, G = a->group;
   if (!a->W || !a->Xq || !a->W_hat || !a->h || !a->z || !a->grp_range || !a->dY ||
@@ -437,8 +443,12 @@ static omq_status bwd_impl(const omq_bwd_args* a, void* workspace, size_t ws_byt
     // dB~ = column sums of dY (needed for d_delta, or when asked for)
     OMQ_TRY(ph.mark(OMQ_PH_DBIAS));
     if (a->d_delta || a->d_B_tilde) {
-      OMQ_TRY(launch_colsum(a->dY, a->op_dt, M, N, kRowsColsum, nullptr, dbt_part, s));
-      const ColReduce r{dbt_part, L.rb_colsum, nullptr, 0, gscale, dbt};
+      int64_t blocks = ceil_div(M, dbias_rows);
+      if (dbias_rows <= 0) {
+        OMQ_TRY(launch_colsum(a->dY, a->op_dt, M, N, kRowsColsum, nullptr, dbt_part, s));
+        blocks = L.rb_colsum;
+      }
+      const ColReduce r{dbt_part, blocks, nullptr, 0, gscale, dbt};
       OMQ_TRY(launch_reduce_cols(&r, 1, N, red, s));
     }
     // dW^ = G^T Xq   [N, K]
@@ -624,8 +634,15 @@ omq_status omq_calib_step(const omq_step_args* a, void* workspace, size_t ws_byt
   // without phase events the loss reduction runs on the second stream, beside the backward
   // (which does not read it); the stream is joined before AdamW
   const SideStream* ls = ph.ev ? nullptr : side_stream();
+  // with LET the backward needs dB~ = column sums of the residual: the forward GEMM's MSE
+  // epilogue forms them per 32-row block (tensor-core path) in the backward's partials
+  const bool fused_dbias = let && a->op_dt != OMQ_F32;
+  float* dbias_part = fused_dbias ? reinterpret_cast<float*>(
+                                        static_cast<char*>(workspace) + fwd_ws +
+                                        bwd_layout(M, N, K, G).dbt_part)
+                                  : nullptr;
   OMQ_TRY(fwd_impl(Xq, a->W_hat, a->op_dt, M, N, K, Bt, a->Y_ref, nullptr, a->dY, a->loss,
-                   workspace, fwd_ws, stream, ph, ls));
+                   workspace, fwd_ws, stream, ph, ls, dbias_part));
   omq_bwd_args b{};
   b.M = M; b.N = N; b.K = K; b.group = G; b.bits = a->bits; b.abits = a->abits; b.dt = a->dt;
   b.op_dt = a->op_dt;
@@ -635,7 +652,8 @@ omq_status omq_calib_step(const omq_step_args* a, void* workspace, size_t ws_byt
   b.h_a = a->h_a; b.z_a = a->z_a; b.tok_range = a->tok_range; b.dY = a->dY;
   b.d_gamma_logit = a->d_gamma_logit; b.d_beta_logit = a->d_beta_logit;
   b.d_s = let ? a->d_s : nullptr; b.d_delta = let ? a->d_delta : nullptr;
-  OMQ_TRY(bwd_impl(&b, static_cast<char*>(workspace) + fwd_ws, ws_bytes - fwd_ws, stream, ph));
+  OMQ_TRY(bwd_impl(&b, static_cast<char*>(workspace) + fwd_ws, ws_bytes - fwd_ws, stream, ph,
+                   fused_dbias ? 32 : 0));
   if (ls) OMQ_TRY(ls->join(st));
   OMQ_TRY(ph.mark(OMQ_PH_ADAMW));
   const int64_t ng = N * (K / G);

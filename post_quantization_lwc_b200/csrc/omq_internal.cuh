@@ -141,6 +141,26 @@ __device__ __forceinline__ float round_quotient(float v, float h, float hinv) {
   return rintf(__fdiv_rn(v, h));
 }
 
+// round(v / h) for 8 values, bitwise round_quotient's: the product with 1/h and its
+// distance to the nearest integer, branch-free; one vote among the lanes that call it sends
+// a lane holding a product near a half-integer (or a large quotient) to the exact quotient.
+__device__ __forceinline__ void round_quotient8(const float (&v)[8], float h, float hinv,
+                                                float (&r)[8]) {
+  bool slow = false;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float ua = __fmul_rn(v[i], hinv);
+    r[i] = rne_small(ua);
+    slow |= !(fabsf(ua) < 2048.f) || !(fabsf(__fsub_rn(ua, r[i])) <= 0.499f);
+  }
+  if (__any_sync(__activemask(), slow)) {
+    if (slow) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) r[i] = round_quotient(v[i], h, hinv);
+    }
+  }
+}
+
 // Integer value of an integral binary32 c in [0, 2^23): adding 2^23 leaves c in the low
 // mantissa bits.
 __device__ __forceinline__ uint32_t small_uint(float c) {
@@ -261,6 +281,9 @@ struct GemmEpilogue {
   void* sk_scratch;
   size_t sk_bytes;
   QuantB qb;               // gemm_tc_qb only
+  // MseLoss, tcgen05 path, or NULL: [ceil(rows / 32), cols] column sums of the residual over
+  // each 32-row block (its rows past the end count as zero)
+  float* res_colsum;
 };
 
 // Group lengths whose weight-side STE runs in the dW^ GEMM's epilogue: whole 32-column
@@ -452,7 +475,7 @@ omq_status launch_colsum(const void* A, omq_dtype dt, int64_t rows, int64_t cols
 // out[j] = scale * sum over the rows of p0 [r0n, cols] and p1 [r1n, cols] (p1 may be NULL),
 // binary64 in a fixed order, for one or two problems with the same cols in one launch pair;
 // scratch holds 2 * kReduceChunks * cols doubles.
-constexpr int kReduceChunks = 16;
+constexpr int kReduceChunks = 64;
 struct ColReduce {
   const float* p0;
   int64_t r0n;

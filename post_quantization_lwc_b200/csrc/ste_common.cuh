@@ -53,9 +53,11 @@ __device__ __forceinline__ bool h_active(float h, float gl, float bl, float vmax
 __device__ __forceinline__ void ste8(const float (&v)[8], const float (&dq)[8], float h,
                                      float z, float Q, bool (&inr)[8], float& Gh, float& Gz) {
   const float hinv = __frcp_rn(h);
+  float rq[8];
+  round_quotient8(v, h, hinv, rq);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const float r = round_quotient(v[i], h, hinv);
+    const float r = rq[i];
     const float lvl = __fadd_rn(r, z);
     inr[i] = lvl >= 0.f && lvl <= Q;
     const float c = fminf(fmaxf(lvl, 0.f), Q);
@@ -68,9 +70,11 @@ __device__ __forceinline__ void ste8(const float (&v)[8], const float (&dq)[8], 
 __device__ __forceinline__ void in_range8(const float (&v)[8], float h, float z, float Q,
                                           bool (&inr)[8]) {
   const float hinv = __frcp_rn(h);
+  float rq[8];
+  round_quotient8(v, h, hinv, rq);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const float lvl = __fadd_rn(round_quotient(v[i], h, hinv), z);
+    const float lvl = __fadd_rn(rq[i], z);
     inr[i] = lvl >= 0.f && lvl <= Q;
   }
 }
