@@ -65,7 +65,8 @@ constexpr int BK = 64;                    // 64 16-bit values = 128 bytes = one 
 constexpr int UMMA_K = 16;
 
 // Epilogue variants: EV = 0 the store / MSE epilogue (epi.kind), light, with 8 epilogue warps
-// of 128 columns; EV = 1 / 2 the weight-side STE epilogue (BF16 / F16 weights), the step's
+// of 128 columns; EV = 1 / 2 the weight-side STE epilogue (BF16 / F16 weights; 3 / 4 the same
+// without the LET column sums, 32 registers a thread fewer), the step's
 // heaviest per-element arithmetic, with 16 epilogue warps of 64 columns (four per scheduler,
 // 96 registers a thread) and producer / MMA waits that sleep between probes, leaving issue
 // slots to the epilogue. One kernel per variant keeps each within its register budget.
@@ -427,7 +428,7 @@ __device__ __forceinline__ void unpack8(const uint4& q, float (&w)[8]) {
 // gradients and the max / min elements' shares) are finished by ste_w_finish_kernel and
 // ste_w_corr_kernel after the GEMM. Rows past the end read as zero weights and zero
 // accumulators (the operand loads fill zeros) and store nothing.
-template <bool F16>
+template <bool F16, bool LETSUM>
 __device__ __forceinline__ void ste_w_epilogue(const GemmEpilogue& epi, uint32_t tcol,
                                                int64_t wrow0, int64_t col0, int64_t rows,
                                                int64_t cols, int lane, const uint8_t* wst,
@@ -435,7 +436,6 @@ __device__ __forceinline__ void ste_w_epilogue(const GemmEpilogue& epi, uint32_t
   const SteWEpi& p = epi.ste;
   const int64_t row = wrow0 + lane;
   const bool valid = row < rows;
-  const bool let = p.part_s != nullptr;
   // this warp's weight block was staged in wst (chunk j of row r at (j ^ (r & 7)) * 16 bytes)
   cp_wait_all();
   __syncwarp();
@@ -448,7 +448,7 @@ __device__ __forceinline__ void ste_w_epilogue(const GemmEpilogue& epi, uint32_t
     const float h = hz[2 * c], z = hz[2 * c + 1];
     const float hinv = __frcp_rn(h);
     float Gh = 0.f, Gc = 0.f;
-    float ps[32];
+    float ps[LETSUM ? 32 : 1];
     // the chunk's 32 accumulator columns: both 16-column loads in flight, one wait
     uint32_t r[32];
     __syncwarp();
@@ -465,16 +465,17 @@ __device__ __forceinline__ void ste_w_epilogue(const GemmEpilogue& epi, uint32_t
       const int q = 4 * c + v;                       // 8-column chunk of the warp's 64
       const uint4 wq = valid ? *reinterpret_cast<const uint4*>(wrow + ((q ^ (lane & 7)) << 4))
                              : make_uint4(0, 0, 0, 0);
+      // without the LET sums there is no LET at all (s is NULL): W~ = W
       float w[8], sv[8], wt[8], rq[8];
       unpack8<F16>(wq, w);
-      if (p.s) load_f8(p.s, col0 + 8 * q, sv);
+      if (LETSUM && p.s) load_f8(p.s, col0 + 8 * q, sv);
       // round(W~ / h) as the forward takes it: the product with 1/h, branch-free, its
       // distance to the nearest integer checked; one warp-wide vote sends the rare lane
       // with a product near a half-integer (or a large quotient) to the exact quotient
       bool slow = false;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        wt[i] = p.s ? __fmul_rn(w[i], sv[i]) : w[i];
+        wt[i] = (LETSUM && p.s) ? __fmul_rn(w[i], sv[i]) : w[i];
         const float ua = __fmul_rn(wt[i], hinv);
         rq[i] = rne_small(ua);
         slow |= !(fabsf(ua) < 2048.f) || !(fabsf(__fsub_rn(ua, rq[i])) <= 0.499f);
@@ -493,14 +494,14 @@ __device__ __forceinline__ void ste_w_epilogue(const GemmEpilogue& epi, uint32_t
         const float cl = fminf(fmaxf(lvl, 0.f), p.Q);
         Gh += dq * (inr ? (rq[i] - wt[i] * hinv) : (cl - z));
         Gc += inr ? 0.f : dq;
-        ps[8 * v + i] = inr ? dq * w[i] : 0.f;
+        if constexpr (LETSUM) ps[8 * v + i] = inr ? dq * w[i] : 0.f;
       }
     }
     if (valid) {
       p.gh_part[(k0 >> 5) * rows + row] = Gh;
       p.gc_part[(k0 >> 5) * rows + row] = Gc;
     }
-    if (let) {
+    if constexpr (LETSUM) {
       const float cs = warp_column_sum32(ps, lane);
       if (wrow0 < rows) p.part_s[(wrow0 >> 5) * cols + k0 + lane] = cs;
     }
@@ -968,7 +969,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV, DQB>::NUM_TH
       const uint32_t tbase = tmem + (static_cast<uint32_t>(quad * 32) << 16) +
                              static_cast<uint32_t>(buf * TILE_N + cq * EPI_COLS);
       const float* other = nullptr;
-      if (un.nsplit > 1) {
+      // (the weight-side STE variants never take the stream-K schedule: their contraction
+      // is over tokens, and the host keeps it off for them)
+      if (EV == 0 && un.nsplit > 1) {
         // A stream-K tile: both contributing pairs store their partial accumulator, then
         // count their arrival on the tile's counter; the second to arrive adds the first's
         // partial to its own and runs the epilogue (own + other: the same sum whichever
@@ -1017,7 +1020,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV, DQB>::NUM_TH
         other = sc.sk_part + sk_slot(un.tsk, 1 - un.split, rank) + ew * EPI_COLS * 32;
       }
       if constexpr (EV != 0) {
-        ste_w_epilogue<EV == 2>(epi, tbase, wrow0, col0, rows, cols, lane,
+        // EV 1 / 2: bfloat16 / float16 W with the LET column sums; 3 / 4: without
+        ste_w_epilogue<EV == 2 || EV == 4, EV <= 2>(epi, tbase, wrow0, col0, rows, cols, lane,
                                 smem + L::WST_OFF + ew * C::WST, other, hz);
       } else {
         float* const out_b = BATCH ? epi.out + static_cast<int64_t>(tw.b) * sc.out_bstride : epi.out;
@@ -1270,7 +1274,9 @@ omq_status gemm_tc(omq_dtype dt, const GemmOperand& A, const GemmOperand& B, int
   if (epi.kind == Epi::SteW) {
     if (!ste_fusable(epi.ste.G) || (epi.ste.wdt != OMQ_BF16 && epi.ste.wdt != OMQ_F16))
       return OMQ_ERR_SHAPE;
-    kc = epi.ste.wdt == OMQ_F16 ? choice<2>() : choice<1>();
+    const bool letsum = epi.ste.part_s != nullptr || epi.ste.s != nullptr;
+    kc = epi.ste.wdt == OMQ_F16 ? (letsum ? choice<2>() : choice<4>())
+                                : (letsum ? choice<1>() : choice<3>());
   }
   const cudaError_t attr_err = kernel_attr(kc.fn, kc.smem);
   if (attr_err != cudaSuccess) {
@@ -1298,8 +1304,8 @@ omq_status gemm_tc(omq_dtype dt, const GemmOperand& A, const GemmOperand& B, int
   const int64_t nk = ceil_div(depth, BK);
   const int64_t rem = tiles % pairs;
   constexpr int64_t kSkMinBlocks = 128;
-  if (count == 1 && !causal && epi.sk_scratch && tiles > pairs && rem != 0 && 5 * rem <= 4 * pairs &&
-      nk >= kSkMinBlocks) {
+  if (count == 1 && !causal && epi.kind != Epi::SteW && epi.sk_scratch && tiles > pairs &&
+      rem != 0 && 5 * rem <= 4 * pairs && nk >= kSkMinBlocks) {
     const int64_t dp = (tiles / pairs - 1) * pairs, skt = tiles - dp;
     if (sk_need(skt) <= epi.sk_bytes) {
       sc.dp_tiles = static_cast<int>(dp);

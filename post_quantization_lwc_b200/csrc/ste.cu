@@ -655,7 +655,7 @@ __global__ void __launch_bounds__(256) reduce_cols4_partial_kernel(ColReduceSet 
   const int64_t ra = static_cast<int64_t>(blockIdx.y) * rs.rpc;
   const int64_t rb = min(total, ra + rs.rpc);
   double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
-#pragma unroll 4
+#pragma unroll 8
   for (int64_t r = ra; r < rb; ++r) {
     const float* row = r < r0n ? q.p0 + r * rs.cols : q.p1 + (r - r0n) * rs.cols;
     const float4 v = __ldg(reinterpret_cast<const float4*>(row + j));
@@ -687,9 +687,17 @@ __global__ void __launch_bounds__(256) reduce_cols_final_kernel(ColReduceSet rs,
   const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (j >= rs.cols) return;
   const double* sc = scratch + static_cast<int64_t>(blockIdx.y) * rs.chunks * rs.cols;
-  double t = 0.0;
-  for (int c = 0; c < rs.chunks; ++c) t += sc[c * rs.cols + j];
-  q.out[j] = static_cast<float>(t * static_cast<double>(q.scale));
+  // four interleaved sums (chunks c = 4 i + r), then (t0 + t1) + (t2 + t3): a fixed order
+  // with four loads in flight
+  double t[4] = {0.0, 0.0, 0.0, 0.0};
+  int c = 0;
+  for (; c + 4 <= rs.chunks; c += 4) {
+#pragma unroll
+    for (int r = 0; r < 4; ++r) t[r] += sc[(c + r) * rs.cols + j];
+  }
+  for (int r = 0; c < rs.chunks; ++c, ++r) t[r] += sc[c * rs.cols + j];
+  const double sum = (t[0] + t[1]) + (t[2] + t[3]);
+  q.out[j] = static_cast<float>(sum * static_cast<double>(q.scale));
 }
 
 // loss = (sum of per-tile partials) / count, binary64, fixed order.
@@ -855,8 +863,8 @@ omq_status launch_reduce_cols(const ColReduce* probs, int nprob, int64_t cols, d
   }
   const omq_status st = launch_status();
   if (st != OMQ_OK || rs.chunks == 1) return st;
-  const dim3 g2(static_cast<unsigned>(ceil_div(cols, 256)), static_cast<unsigned>(nprob));
-  launch_k(reduce_cols_final_kernel, g2, 256, 0, stream, rs, scratch);
+  const dim3 g2(static_cast<unsigned>(ceil_div(cols, 64)), static_cast<unsigned>(nprob));
+  launch_k(reduce_cols_final_kernel, g2, 64, 0, stream, rs, scratch);
   return launch_status();
 }
 
