@@ -1292,10 +1292,12 @@ omq_status gemm_tc(omq_dtype dt, const GemmOperand& A, const GemmOperand& B, int
   // pairs idle, the last whole wave and the tail (fewer than 2 waves of tiles) are shared
   // out as equal runs of k-blocks, longer than one tile's contraction, so every tile of the
   // region has one or two contributing pairs. Only for long contractions (at least
-  // kSkMinBlocks k-blocks): measured on B200, the split tiles' partial stores and the
-  // staggered k positions of the pairs cost more than the idle tail saves when a tile's
-  // contraction is short (4096-deep: forward 78 -> 98 us at 2048 x 4096; 13824-deep:
-  // forward 287 -> 248 us at 2048 x 5120).
+  // kSkMinBlocks k-blocks) with at least one whole wave ahead of the region: measured on
+  // B200, the split tiles' partial stores and the staggered k positions of the pairs cost
+  // more than the idle tail saves when a tile's contraction is short (4096-deep: forward
+  // 78 -> 98 us at 2048 x 4096) or when every tile of the problem is in the region (the
+  // block's 22016-deep dX GEMM over 128 tiles got slower), and less on the down_proj forward
+  // (13824-deep, 160 tiles: 287 -> 248 us).
   sc.dp_tiles = static_cast<int>(tiles);
   sc.sk_tiles = 0;
   sc.sk_len = 0;
@@ -1304,7 +1306,7 @@ omq_status gemm_tc(omq_dtype dt, const GemmOperand& A, const GemmOperand& B, int
   const int64_t nk = ceil_div(depth, BK);
   const int64_t rem = tiles % pairs;
   constexpr int64_t kSkMinBlocks = 128;
-  if (count == 1 && !causal && epi.kind != Epi::SteW && epi.sk_scratch && tiles > pairs &&
+  if (count == 1 && !causal && epi.kind != Epi::SteW && epi.sk_scratch && tiles >= 2 * pairs &&
       rem != 0 && 5 * rem <= 4 * pairs && nk >= kSkMinBlocks) {
     const int64_t dp = (tiles / pairs - 1) * pairs, skt = tiles - dp;
     if (sk_need(skt) <= epi.sk_bytes) {

@@ -26,10 +26,10 @@ def omq(cuda_device):
     return m
 
 
-# (M, N, K), contractions of at least 128 k-blocks of 64 (the schedule's threshold): 80
-# tiles (one wave + 6: the whole region split), 304 tiles (4 waves + 8: the last whole wave
-# and the tail), ragged rows, columns and depth
-SHAPES = [(2048, 2560, 8192), (4096, 4864, 8192), (2000, 2504, 8200), (2304, 2368, 13824)]
+# (M, N, K), contractions of at least 128 k-blocks of 64 and at least two waves of tiles (the
+# schedule's thresholds): 160 tiles (two waves + 12: one whole wave ahead of the region, the
+# down_proj forward), 304 tiles (4 waves + 8), ragged rows, columns and depth
+SHAPES = [(2048, 5120, 13824), (4096, 4864, 8192), (2000, 5096, 8200), (2304, 4352, 8192)]
 
 
 @pytest.mark.parametrize("M,N,K", SHAPES)
