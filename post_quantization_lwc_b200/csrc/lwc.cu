@@ -308,7 +308,10 @@ __device__ __forceinline__ void scale8(const float* s, int64_t col, float (&v)[8
 // encoder), so its piece is the whole row; grouped rows are staged in pieces of `pcols`
 // columns (whole groups, whole segments), so that a long row does not take a warp's whole
 // share of shared memory and the warps per SM stay many. B~[n] = B[n] + sum_k W[n,k]
-// delta[k] comes out of the same pass over the row.
+// delta[k] comes out of the same pass over the row, so with B~ a warp takes whole rows
+// (`per` rows: all pieces of rows wg, wg + n_warps, ...); without it the (row, piece) items
+// themselves are dealt out (`per` items: wg, wg + n_warps, ...), which keeps every warp of
+// the SM busy when the rows do not divide evenly among them.
 
 constexpr int kStageSegs = 4;   // 256-column segments a grouped batch holds in registers
 constexpr int64_t kStagePiece = 2048;   // columns a grouped piece holds
@@ -318,7 +321,7 @@ constexpr int stage_max_warps(int lpg) { return lpg == 0 ? 24 : 16; }
 
 template <int LPG, bool F16>
 __global__ void __launch_bounds__(32 * stage_max_warps(LPG))
-    lwc_stage_kernel(LwcParams p, int nbuf, int64_t rows_per_warp, int64_t pcols) {
+    lwc_stage_kernel(LwcParams p, int nbuf, int64_t per, int64_t pcols, int by_rows) {
   pdl_wait();
   pdl_launch();
   extern __shared__ __align__(16) unsigned char lsm[];
@@ -337,11 +340,18 @@ __global__ void __launch_bounds__(32 * stage_max_warps(LPG))
   const int64_t wg = static_cast<int64_t>(wib) * gridDim.x + blockIdx.x;
   const bool hat_f16 = p.hat_dt == OMQ_F16;
   const bool let = p.s != nullptr, bias_on = p.Bt != nullptr && p.delta != nullptr;
-  const int64_t items = rows_per_warp * pieces;        // (row, piece) in row-major order
+  const int64_t items = by_rows ? per * pieces : per;   // this warp's (row, piece) items
+  // row and piece of this warp's item `it`
+  auto row_of = [&](int64_t it) {
+    return by_rows ? wg + (it / pieces) * n_warps : (wg + it * n_warps) / pieces;
+  };
+  auto piece_of = [&](int64_t it) {
+    return by_rows ? it % pieces : (wg + it * n_warps) % pieces;
+  };
   auto issue = [&](int64_t it) {
-    const int64_t n = wg + (it / pieces) * n_warps;
+    const int64_t n = row_of(it);
     if (it < items && n < p.N) {
-      const int64_t pc0 = (it % pieces) * pcols;
+      const int64_t pc0 = piece_of(it) * pcols;
       const int64_t nc = K - pc0 < pcols ? K - pc0 : pcols;
       const unsigned char* src = static_cast<const unsigned char*>(p.W) + (n * K + pc0) * 2;
       uint16_t* dst = rows + (it % nbuf) * pcols;
@@ -358,9 +368,9 @@ __global__ void __launch_bounds__(32 * stage_max_warps(LPG))
   issue(0);
   float2 bias2 = make_float2(0.f, 0.f);
   for (int64_t it = 0; it < items; ++it) {
-    const int64_t n = wg + (it / pieces) * n_warps;
+    const int64_t n = row_of(it);
     if (n >= p.N) break;                                       // warp-uniform
-    const int64_t pc = it % pieces, pc0 = pc * pcols;
+    const int64_t pc = piece_of(it), pc0 = pc * pcols;
     const int64_t nc = K - pc0 < pcols ? K - pc0 : pcols;
     if (nbuf == 2) {
       issue(it + 1);
@@ -614,15 +624,19 @@ omq_status launch_stage(const LwcParams& p, const StageShape& s, cudaStream_t st
     set_cuda_error(e);
     return OMQ_ERR_CUDA;
   }
-  // rows per warp from the most warps that fit, then those warps spread over every SM
+  // rows (with B~: a row's pieces stay in one warp) or (row, piece) items per warp from the
+  // most warps that fit, then those warps spread over every SM
+  const int64_t pieces = (p.K + s.pcols - 1) / s.pcols;
+  const int by_rows = p.Bt != nullptr || pieces == 1;
+  const int64_t units = by_rows ? p.N : p.N * pieces;
   const int64_t sms = num_sms();
-  const int64_t per = (p.N + sms * s.wpb - 1) / (sms * s.wpb);
-  const int64_t warps = (p.N + per - 1) / per;
+  const int64_t per = (units + sms * s.wpb - 1) / (sms * s.wpb);
+  const int64_t warps = (units + per - 1) / per;
   const int64_t wpb = std::min<int64_t>(s.wpb, (warps + sms - 1) / sms);
   const int64_t blocks = (warps + wpb - 1) / wpb;
   const size_t smem = s.smem / s.wpb * wpb;
   launch_k(kernel, static_cast<unsigned>(blocks), static_cast<unsigned>(32 * wpb), smem, stream,
-      p, s.nbuf, per, s.pcols);
+      p, s.nbuf, per, s.pcols, by_rows);
   return launch_status();
 }
 

@@ -1,8 +1,9 @@
 """GPU parity of the row-staged LWC launch shape (16-bit W and W^, groups of 32 to 256
 columns or one group per row, no integer codes requested) against the oracle, bit for bit:
 W^, h, z and the group ranges with their tie counts. The shapes cover both buffer modes
-(two staged rows per warp, and one for long rows), grouped rows staged in several pieces,
-persistent warps with several rows each, a ragged last 256-column segment, constant / zero rows and groups, ties at both
+(two staged rows per warp, and one for long rows), grouped rows staged in several pieces
+(whole rows a warp with B~, single pieces dealt out without it), persistent warps with
+several rows each, a ragged last 256-column segment, constant / zero rows and groups, ties at both
 extremes and clipping on both sides. The same pass's B~ = B + W delta is checked through
 the calibration step against the exact sum, within the binary32 summation bound."""
 import dataclasses
@@ -57,6 +58,9 @@ CASES = [
     # one (K = 6.75 pieces), B~ summed across the pieces of a row; the down_proj row length
     StagedCase("bf16_g64_k13824_pieces", 700, 13824, 64, "bf16", "bf16", True, 2, 8),
     StagedCase("f16_g32_k2304_two_pieces", 900, 2304, 32, "f16", "f16", True, 4, 9),
+    # without B~ the (row, piece) items are dealt out one by one: 3 pieces a row (the last
+    # 256 columns), 15000 items, several per warp and a partial last round
+    StagedCase("bf16_g128_k4352_items", 5000, 4352, 128, "bf16", "bf16", False, 3, 10),
 ]
 
 
