@@ -68,8 +68,7 @@ constexpr int UMMA_K = 16;
 // of 128 columns; EV = 1 / 2 the weight-side STE epilogue (BF16 / F16 weights; 3 / 4 the same
 // without the LET column sums, 32 registers a thread fewer), the step's
 // heaviest per-element arithmetic, with 16 epilogue warps of 64 columns (four per scheduler,
-// 96 registers a thread) and producer / MMA waits that sleep between probes, leaving issue
-// slots to the epilogue. One kernel per variant keeps each within its register budget.
+// 96 registers a thread). One kernel per variant keeps each within its register budget.
 //
 // DQB (2..8): the B operand is a weight given as packed DQB-bit codes with per-group step h
 // and zero point z (omq_fold_pack's layout); four converter warps per CTA expand each
@@ -82,11 +81,13 @@ struct Cfg {
   static constexpr int CONV_WARPS = DQB ? 8 : 0;     // two groups of four (alternate k-blocks)
   static constexpr int CONV_ARRIVALS = DQB ? 2 * 4 : 0;   // a stage's: one group, both CTAs
   static constexpr int NUM_THREADS = 32 * (2 + EPI_WARPS + CONV_WARPS);
-  // the STE variants give two stages of the ring to a 4 KB shared slice per epilogue warp
-  // (its 32 x 64 block of W, staged by coalesced copies)
-  static constexpr int STAGES = EV ? 5 : 7;
+  // The STE variants give a 4 KB shared slice to each epilogue warp (its 32 x 64 block of W,
+  // staged by coalesced copies). Ring depth, measured on B200: 6 stages (EV 0) and 4 (STE)
+  // ran the GEMMs 1-5% faster than 7 and 5, the smaller shared-memory carve-out leaving the
+  // L1 room for the epilogue's row-per-thread accesses; a shared-memory transpose of the
+  // accumulator chunks (coalesced global accesses) was slower again on the forward.
+  static constexpr int STAGES = EV ? 4 : 6;
   static constexpr int WST = EV ? 32 * 64 * 2 : 0;
-  static constexpr bool SLEEPY = EV != 0;
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -834,8 +835,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV, DQB>::NUM_TH
       for (int kb = tw.kb0; kb < tw.kb1; ++kb, ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
-        const bool got = C::SLEEPY ? mbar_wait_sleep(bar_empty + 8 * s, ph ^ 1, DEV_ERR_TMA_WAIT, 64)
-                                   : mbar_wait(bar_empty + 8 * s, ph ^ 1, DEV_ERR_TMA_WAIT);
+        const bool got = mbar_wait(bar_empty + 8 * s, ph ^ 1, DEV_ERR_TMA_WAIT);
         if (*abort_flag || !got) {
           ok = false;
           break;
@@ -877,8 +877,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV, DQB>::NUM_TH
     for (int u = 0; ok && next_unit<BATCH>(sc, pair, pairs, u, nk, un); ++u, ++lt) {
       const int buf = lt & 1;
       const uint32_t pa = ((lt >> 1) & 1) ^ 1;
-      const bool got = C::SLEEPY ? mbar_wait_sleep(bar_acce + 8 * buf, pa, DEV_ERR_MMA_WAIT, 64)
-                                 : mbar_wait(bar_acce + 8 * buf, pa, DEV_ERR_MMA_WAIT);
+      const bool got = mbar_wait(bar_acce + 8 * buf, pa, DEV_ERR_MMA_WAIT);
       if (*abort_flag || !got) {
         ok = false;
         break;
@@ -1057,7 +1056,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<EV, DQB>::NUM_TH
                   rc[q] = epi_element(epi, out_b, row, cbase + q, cols, __uint_as_float(r[q]), lsum);
             }
           }
-          if (epi.res_colsum && cbase < cols) {   // warp-uniform: the bias gradient's partials
+          // warp-uniform: the bias gradient's partials, for row blocks that hold rows
+          if (epi.res_colsum && cbase < cols && wrow0 < rows) {
             const float cs = warp_column_sum32(rc, lane);
             if (cbase + lane < cols) epi.res_colsum[(wrow0 >> 5) * cols + cbase + lane] = cs;
           }
