@@ -303,7 +303,9 @@ omq_status omq_qgemm(const void* x, omq_dtype xdt, int64_t M, int64_t K, const u
  * on or abits < 16), omq_lwc_quant, omq_fq_linear_fwd, omq_fq_linear_bwd, then AdamW on
  * the logits (lr_lwc) and, with LET, on s and delta (lr_let). `step` counts from 1.
  * All buffers are caller-owned device memory. When LET is off and abits == 16, X itself is
- * the GEMM operand and Xq is not used. Workspace: omq_step_workspace_bytes(M, N, K, group).
+ * the GEMM operand and Xq is not used. When LET is off the step leaves the tie counts
+ * (nmax, nmin) of grp_range at 0 where its row-staged LWC pass runs (16-bit W and W_hat):
+ * only the LET gradients read them. Workspace: omq_step_workspace_bytes(M, N, K, group).
  *
  * Per-phase timing: `events` is NULL or an array of OMQ_PH_COUNT + 1 cudaEvent_t (passed
  * as void*). Event i is recorded on `stream` when phase i starts and event OMQ_PH_COUNT

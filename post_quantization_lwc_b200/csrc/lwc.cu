@@ -448,7 +448,7 @@ __global__ void __launch_bounds__(32 * stage_max_warps(LPG))
         }
         // ties are counted only in the rare rounds where some lane's 8 values reach an
         // extreme of the row
-        const bool ext = ok && (max8(V, V[0].x) == vmax || min8(V, V[0].x) == vmin);
+        const bool ext = ok && !p.no_ties && (max8(V, V[0].x) == vmax || min8(V, V[0].x) == vmin);
         if (__any_sync(0xffffffffu, ext)) {
           if (ext) {
 #pragma unroll
@@ -515,10 +515,13 @@ __global__ void __launch_bounds__(32 * stage_max_warps(LPG))
             vmx[u] = fmaxf(vmx[u], __shfl_xor_sync(0xffffffffu, vmx[u], o));
             vmn[u] = fminf(vmn[u], __shfl_xor_sync(0xffffffffu, vmn[u], o));
           }
-          cnt[u] = ties8(V[u], vmx[u], vmn[u]);
+          cnt[u] = 0.f;
+          if (!p.no_ties) {                                  // uniform
+            cnt[u] = ties8(V[u], vmx[u], vmn[u]);
 #pragma unroll
-          for (int o = LPG / 2; o > 0; o >>= 1)
-            cnt[u] = __fadd_rn(cnt[u], __shfl_xor_sync(0xffffffffu, cnt[u], o));
+            for (int o = LPG / 2; o > 0; o >>= 1)
+              cnt[u] = __fadd_rn(cnt[u], __shfl_xor_sync(0xffffffffu, cnt[u], o));
+          }
         }
         // this lane's group of the batch: segment ut, sub-warp sg
         const int gb = lane % GPB, ut = gb / GPS, sg = gb % GPS, src = sg * LPG;

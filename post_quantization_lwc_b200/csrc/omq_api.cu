@@ -612,6 +612,7 @@ omq_status omq_calib_step(const omq_step_args* a, void* workspace, size_t ws_byt
       p.B = a->B;
       p.Bt = a->B_tilde;
     }
+    p.no_ties = !let;     // without LET no gradient reads the tie counts
     return launch_lwc(p, s);
   };
   // The activation and weight sides of the forward are independent: without phase events

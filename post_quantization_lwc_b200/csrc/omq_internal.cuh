@@ -360,6 +360,9 @@ struct LwcParams {
   const float* delta;
   const float* B;
   float* Bt;
+  // the row-staged kernel leaves the tie counts of `range` at 0 (they feed only the LET
+  // gradients, through the extremes' shares)
+  bool no_ties;
 };
 
 struct LetParams {

@@ -202,6 +202,33 @@ def test_calib_step_through_one_call(omq, cuda_device, case):
         check_update(lc.delta, p.delta.numpy(), r.d_delta, om.LR_LET)
 
 
+@pytest.mark.parametrize("case", [c for c in SMALL_CASES if c.dtype != "f32"],
+                         ids=lambda c: c.name)
+def test_calib_step_group_records(omq, cuda_device, case):
+    """The step's group records: ranges bit for bit; the tie counts as the oracle's with LET
+    (the extremes' gradient shares need them) and 0 without (nothing reads them there)."""
+    p = prepare(case)
+    d = _dev(p, cuda_device)
+    lc = omq.LinearCalibration(M=case.M, N=case.N, K=case.K, group=case.group, bits=case.bits,
+                               abits=case.abits, let=case.let, dtype=torch.bfloat16,
+                               device=cuda_device)
+    lc.load(d["W"], d["gl"], d["bl"], s=d["s"], delta=d["d"], B=d["B"])
+    lc.step(d["X"], d["Yref"])
+    torch.cuda.synchronize()
+    omq.sync_check()
+    s = p.s.numpy() if case.let else None
+    _, enc, _, _ = om.lwc_quant(p.W.float().numpy(), s, p.gl.numpy(), p.bl.numpy(), case.bits,
+                                case.group)
+    vmax, vmin, nmax, nmin = (x.cpu().numpy() for x in omq.range_fields(lc.grp_range))
+    assert np.array_equal(vmax, enc.vmax.reshape(-1))
+    assert np.array_equal(vmin, enc.vmin.reshape(-1))
+    if case.let:
+        assert np.array_equal(nmax, enc.nmax.reshape(-1))
+        assert np.array_equal(nmin, enc.nmin.reshape(-1))
+    else:
+        assert not nmax.any() and not nmin.any()
+
+
 @pytest.mark.parametrize("case", SMALL_CASES, ids=lambda c: c.name)
 def test_fold_pack_bit_exact(omq, cuda_device, case):
     p = prepare(case)
