@@ -274,8 +274,8 @@ omq_status omq_fold_pack(const void* W, omq_dtype wdt, int64_t N, int64_t K, int
  * x [M, K] in xdt (the linear's input after its folded LET, i.e. (X - delta)/s), packed /
  * h / z as written by omq_fold_pack, y [M, N] float32 (add B~ for the bias). 1 <= M <= 8.
  * bits in {2, 4, 8}: CUDA-core kernel, group a multiple of 128/bits, K a multiple of group,
- * M (K + K bits/128) floats of shared memory at most 200 KiB; decode-shaped, memory-bound on
- * the codes. bits 3, 5, 6, 7 (codes straddling bytes): the omq_qgemm path below (16-bit x
+ * min(M, 4) (K + K bits/128) floats of shared memory at most 200 KiB (more than four tokens
+ * run as two launches of at most four); decode-shaped, memory-bound on the codes. bits 3, 5, 6, 7 (codes straddling bytes): the omq_qgemm path below (16-bit x
  * only, its shape rules; OMQ_ERR_UNSUPPORTED for float32 x).
  * ------------------------------------------------------------------------------------ */
 omq_status omq_qgemv(const void* x, omq_dtype xdt, int64_t M, int64_t K, const uint8_t* packed,

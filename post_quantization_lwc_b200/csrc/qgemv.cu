@@ -196,11 +196,18 @@ extern "C" omq_status omq_qgemv(const void* x, omq_dtype xdt, int64_t M, int64_t
   if (M < 1 || M > kGemvMaxTokens || N < 1 || K < cpc || K % cpc || group < cpc ||
       group % cpc || K % group || N > (int64_t(1) << 31))
     return OMQ_ERR_SHAPE;
-  const size_t smem = sizeof(float) * static_cast<size_t>(M) * (K + K / cpc);
-  if (smem > 200 * 1024) return OMQ_ERR_SHAPE;
+  // more than four tokens go as two launches of at most four (the eight-token variant needs
+  // twice the registers, runs one block an SM and took 95 us for the q_proj fold against 27
+  // for four tokens)
+  const int64_t m_launch = M > 4 ? 4 : M;
+  if (sizeof(float) * static_cast<size_t>(m_launch) * (K + K / cpc) > 200 * 1024)
+    return OMQ_ERR_SHAPE;
   if (!aligned16(packed) || ((K * bits / 8) % 16)) return OMQ_ERR_ALIGN;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  auto launch = [&](auto kernel) -> omq_status {
+  const size_t xes = xdt == OMQ_F32 ? 4 : 2;
+  // tokens [m0, m0 + mt) of x and y
+  auto launch = [&](auto kernel, int64_t m0, int64_t mt) -> omq_status {
+    const size_t smem = sizeof(float) * static_cast<size_t>(mt) * (K + K / cpc);
     if (smem > 48 * 1024) {
       const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  static_cast<int>(smem));
@@ -214,15 +221,20 @@ extern "C" omq_status omq_qgemv(const void* x, omq_dtype xdt, int64_t M, int64_t
     const int64_t per = (N + max_warps - 1) / max_warps;
     const int64_t warps = (N + per - 1) / per;
     launch_k(kernel, static_cast<unsigned>((warps + 7) / 8), 256, smem, st,
-        x, xdt, static_cast<int>(M), K, packed, h, z, N, group, y, per);
+        static_cast<const void*>(static_cast<const char*>(x) + m0 * K * xes), xdt,
+        static_cast<int>(mt), K, packed, h, z, N, group, y + m0 * N, per);
     return launch_status();
   };
   auto pick = [&](auto bits_c) -> omq_status {
     constexpr int B = decltype(bits_c)::value;
-    if (M == 1) return launch(qgemv_kernel<B, 1>);
-    if (M == 2) return launch(qgemv_kernel<B, 2>);
-    if (M <= 4) return launch(qgemv_kernel<B, 4>);
-    return launch(qgemv_kernel<B, 8>);
+    for (int64_t m0 = 0; m0 < M; m0 += 4) {
+      const int64_t mt = M - m0 < 4 ? M - m0 : 4;
+      const omq_status st_m = mt == 1   ? launch(qgemv_kernel<B, 1>, m0, mt)
+                              : mt == 2 ? launch(qgemv_kernel<B, 2>, m0, mt)
+                                        : launch(qgemv_kernel<B, 4>, m0, mt);
+      if (st_m != OMQ_OK) return st_m;
+    }
+    return OMQ_OK;
   };
   if (bits == 4) return pick(std::integral_constant<int, 4>{});
   if (bits == 2) return pick(std::integral_constant<int, 2>{});

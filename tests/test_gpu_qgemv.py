@@ -28,6 +28,7 @@ CASES = [  # M tokens, N, K, group, bits
     (5, 72, 384, 384, 4),
     (1, 4096, 4096, 128, 4),     # LLaMA-7B q_proj, g128 (the fold of the bench workload)
     (4, 11008, 4096, 4096, 4),   # LLaMA-7B gate/up, per channel
+    (7, 4096, 4096, 128, 2),     # more than four tokens: two launches (4 + 3)
 ]
 
 
