@@ -24,21 +24,26 @@ struct GroupGrad {
   float dg, db;       // gradient of the strengths
 };
 
+// (gradient values only: the quotients by h and Q are taken as products with the correctly
+// rounded reciprocals, one rounding more than a division)
 __device__ __forceinline__ GroupGrad group_grad(float Gh, float Gz, float g, float b, float h,
                                                 float vmax, float vmin, float Q, bool active) {
-  const float t = b * vmin / h;
-  const float dh = active ? Gh + Gz * t / h : 0.f;
+  const float rh = __frcp_rn(h), rQ = __frcp_rn(Q);
+  const float t = b * vmin * rh;
+  const float dh = active ? Gh + Gz * t * rh : 0.f;
+  const float dhq = dh * rQ, gzh = Gz * rh;
   GroupGrad r;
-  r.dg = dh * vmax / Q;
-  r.db = -dh * vmin / Q - Gz * vmin / h;
-  r.dM = dh * g / Q;
-  r.dm = -dh * b / Q - Gz * b / h;
+  r.dg = dhq * vmax;
+  r.db = -dhq * vmin - gzh * vmin;
+  r.dM = dhq * g;
+  r.dm = -dhq * b - gzh * b;
   return r;
 }
 
-// Clipping strength used in gradient values (never in an integer decision).
+// Clipping strength used in gradient values (never in an integer decision); the correctly
+// rounded reciprocal is the quotient 1 / (1 + e^-x) itself.
 __device__ __forceinline__ float strength_value(float logit) {
-  return 1.f / (1.f + __expf(-logit));
+  return __frcp_rn(1.f + __expf(-logit));
 }
 
 // Whether h's own gradient reaches g, b and the range: the stored h is max(h_raw, floor),
